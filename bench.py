@@ -1,0 +1,319 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-MoE decode path on B200.
+
+One step = one token through the whole hot path of a 40-layer stack shaped
+like Qwen3.6-35B-A3B (H=2048, 256 experts, top-8, I=Is=512, 4-bit affine
+groups of 64 with bf16 scales/biases, packed gate/up): router + softmax
+top-k, the 8 selected experts' gate/up + SwiGLU + down, the sigmoid-gated
+shared expert, the weighted combine and the residual/RMSNorm glue, for all
+40 layers (moe_stack_forward, T=1). Each step feeds a new token, so the
+selected experts change every step; the 18.1 GB expert stack is far larger
+than L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0). With N > 1 (torchrun) every rank runs an
+independent replica on its own tokens: the path has no exchange step.
+`--impl reference` times the CPU oracle instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_routed_expert_bit_b200 import moe, synth  # noqa: E402
+
+METRIC = "MoE-layer decode tokens/s and achieved HBM GB/s (% of 8 TB/s) at 1 B200"
+SHAPE_KEY = "35b"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def touched_bytes_per_token(shape: synth.MoEShape) -> int:
+    """Algorithmic bytes of one token through the stack: per layer the k
+    selected experts and the shared expert (packed codes + bf16 scales and
+    biases), the router E*H*2, the shared gate H*2 and the router bias E*4."""
+    per_layer = shape.top_k * shape.expert_bytes() + shape.expert_bytes(shape.shared_inter)
+    per_layer += shape.num_experts * shape.hidden * 2 + shape.hidden * 2
+    if shape.router_bias:
+        per_layer += shape.num_experts * 4
+    return per_layer * shape.layers
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 8:
+                self.rows.append(parts)
+
+    def __exit__(self, *a):
+        time.sleep(0.2)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+        return dist, dist.get_rank(), world, local
+    return None, 0, 1, 0
+
+
+def barrier_max(dist, value: float) -> float:
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_tokens_per_s(shape, layers_dev, x_tokens, n_layers_sample: int, threads: int):
+    """The oracle (as it stands) on a bounded sample: the first tokens through
+    the first `n_layers_sample` layers, scaled to the full stack."""
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from parity import DeviceLayer  # host view of device weights (copies outside the timing)
+    hosts = [DeviceLayer(shape, layers_dev[l]) for l in range(n_layers_sample)]
+    xs = [synth.bf16_bits(x_tokens[i:i + 1]) for i in range(x_tokens.shape[0])]
+    # route once untimed to know the experts, and copy them to the host
+    for h in hosts:
+        for x in xs:
+            lg = oracle.router_logits(x, h.router_w, h.router_bias)
+            for e in oracle.softmax_topk(lg[0], shape.top_k)[0]:
+                h.expert(int(e))
+    t0 = time.perf_counter()
+    for x in xs:
+        for h in hosts:
+            oracle.layer_forward(h, x, threads=threads)
+    dt = time.perf_counter() - t0
+    per_token = dt / len(xs) * (shape.layers / n_layers_sample)
+    return 1.0 / per_token, dt
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle timed on this host (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    shape = synth.SHAPES[SHAPE_KEY]
+    threads = os.cpu_count() or 1
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    n_layers = 2
+    layers = [synth.make_layer(shape, l, dev) for l in range(n_layers)]
+    tokens = synth.make_tokens(shape, list(range(args.warmup + args.steps)), dev)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from parity import DeviceLayer
+    hosts = [DeviceLayer(shape, lw) for lw in layers]
+    xs = [synth.bf16_bits(tokens[i:i + 1]) for i in range(tokens.shape[0])]
+    for h in hosts:
+        for x in xs:
+            lg = oracle.router_logits(x, h.router_w, h.router_bias)
+            for e in oracle.softmax_topk(lg[0], shape.top_k)[0]:
+                h.expert(int(e))
+    for i in range(args.warmup):
+        for h in hosts:
+            oracle.layer_forward(h, xs[i], threads=threads)
+    t0 = time.perf_counter()
+    for i in range(args.warmup, args.warmup + args.steps):
+        for h in hosts:
+            oracle.layer_forward(h, xs[i], threads=threads)
+    dt = time.perf_counter() - t0
+    sec_per_token = dt / args.steps * (shape.layers / n_layers)
+    value = 1.0 / sec_per_token
+    sample = f"1 token x {n_layers} of {shape.layers} layers per step, scaled to {shape.layers}"
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec_per_token * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(shape),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def workload_config(shape):
+    return {"workload": f"{shape.name}: decode T=1 through {shape.layers} stacked MoE layers "
+                        f"(H={shape.hidden}, E={shape.num_experts}, top-{shape.top_k}, I=Is={shape.inter}, "
+                        f"{shape.bits}-bit affine g{shape.group}, bf16 scale/bias, packed gate/up)",
+            "tokens_per_step": 1, "layers": shape.layers,
+            "l2": "inputs larger than L2: 18.1 GB resident expert stack, a new token (new experts) every step"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    dist, rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    shape = synth.SHAPES[SHAPE_KEY]
+    cfg = moe.make_config(shape)
+    layers = [synth.make_layer(shape, l, "cuda") for l in range(shape.layers)]
+    arr = moe.make_layer_array([moe.make_layer_weights(lw) for lw in layers])
+    ws = moe.Workspace(cfg, 1, L=shape.layers)
+    nsteps = args.warmup + args.steps
+    # each rank its own tokens (independent replicas)
+    tokens = synth.make_tokens(shape, [rank * 100000 + i for i in range(nsteps)], "cuda")
+    xout = torch.empty(1, shape.hidden, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        moe.moe_stack_forward(cfg, arr, tokens[i:i + 1], xout, ws, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == moe.MOE_OK
+
+    # ---- device-timed region: inputs resident in HBM
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for i in range(args.warmup, nsteps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    ms = barrier_max(dist, ms)
+    status = moe.moe_get_device_status(ws)
+
+    # ---- end to end: host tokens in pinned memory, result read back every step
+    host_tok = tokens.cpu().pin_memory()
+    host_out = torch.empty(1, shape.hidden, dtype=torch.bfloat16).pin_memory()
+    xin = torch.empty(1, shape.hidden, dtype=torch.bfloat16, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(args.warmup, nsteps):
+        xin.copy_(host_tok[i:i + 1], non_blocking=True)
+        moe.moe_stack_forward(cfg, arr, xin, xout, ws, stream=stream)
+        host_out.copy_(xout, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = barrier_max(dist, e0.elapsed_time(e1))
+
+    launches_per_step = moe.kernel_launches_per_stack(cfg, shape.layers, 1)
+    bytes_tok = touched_bytes_per_token(shape)
+    total_tokens = args.steps * world
+    tok_s = total_tokens / (ms / 1e3)
+    per_step_s = ms / 1e3 / args.steps
+    gbs = bytes_tok / per_step_s / 1e9
+    peak, peak_src = peaks()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        v, dt = cpu_oracle_tokens_per_s(shape, layers, tokens[:2], 4, threads)
+        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"2 tokens x 4 of {shape.layers} layers ({dt:.1f} s of CPU work), scaled to "
+                         f"{shape.layers} layers; expert copies to the host outside the timing"}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "weights": f"u{shape.bits} affine g{shape.group}, bf16 scale/bias",
+            "data": "synthetic", "config": workload_config(shape),
+            "hbm_gbs": gbs, "hbm_frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
+            "roofline": {"bound": "hbm", "kernel": moe.dominant_kernel_name(),
+                         "achieved": gbs, "peak": peak, "peak_source": peak_src, "unit": "GB/s",
+                         "frac": gbs / peak, "traffic": None,
+                         "bytes_per_launch": bytes_tok,
+                         "note": "achieved = algorithmic bytes per step / device time per step"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": total_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": shape.hidden * 2, "d2h_bytes_per_step": shape.hidden * 2},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+            "device_status": moe.status_string(status),
+        }
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+/*
+ * moe_b200.h -- C ABI of the routed Mixture-of-Experts FFN for NVIDIA B200
+ * (sm_100a), at decode time and for batches of tokens.
+ *
+ * What the library computes, per token x (bf16, hidden size H):
+ *   1. router logits   l_e = x . Wr[e] (+ bias[e]) for all E experts;
+ *   2. routing         softmax over all E, keep the k largest, renormalise
+ *                      the k weights to sum to 1 (ties: lower expert index);
+ *   3. per selected expert e: gu = dequant(GU_e) x with GU_e the packed
+ *                      [2I][H] gate/up matrix (gate rows [0,I), up rows
+ *                      [I,2I)), h = silu(gu[0:I]) * gu[I:2I], o_e = dequant(D_e) h;
+ *   4. shared expert   o_s the same way with its own [2Is][H] and [H][Is]
+ *                      matrices, gated by s = sigmoid(x . w_sg);
+ *   5. combine         y = sum_j w_j o_{e_j} + s o_s, rounded once to bf16.
+ * Sources: the routing fan-out (8 of 256 experts for the 35B model, 10 of
+ * 512 for the 80B model; routers and shared experts resident) is in the
+ * Swiftlet article (xix.ai, "Pacotes de Swiftlet 80B Qwen no Mac ..."),
+ * paragraph 4, and the Runnel README, section "Target" (256 routed
+ * experts, top-8, plus one shared expert); the MLX-style int4/int8 group
+ * quantisation and the sparse MoE with shared experts are in the same
+ * article, paragraph 8; the packed routed gate/up projection is in the
+ * Runnel README, introduction and "Streaming CLI". The pages give no
+ * formula; the steps above are the plain reading of them.
+ *
+ * Quantised matrices ("moe_qtensor"): E matrices [rows][K] at fixed
+ * strides, one expert after the other (fixed-stride expert blocks: the
+ * Swiftlet article, paragraph 4). Element k of a row belongs to group
+ * k / group; its weight is  w = scale[g] * q + bias[g]  (bf16 scale and
+ * bias, no zero-point). Codes run along K: 8-bit is one byte per element;
+ * 4-bit is two elements per byte, the even element in the low nibble.
+ * Row r of expert e starts at  q + e*q_expert_stride + r*K*bits/8  and its
+ * scales/biases at  scales + e*sb_expert_stride + r*(K/group).
+ *
+ * Conventions for every call:
+ *   - Tensor pointers are DEVICE pointers owned by the caller. The library
+ *     allocates nothing; its scratch is the caller's workspace (`ws`,
+ *     sized by moe_workspace_size and set up once by moe_workspace_init).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous; outputs are valid once the stream has
+ *     reached that point.
+ *   - Argument errors return at once, before anything is enqueued. Errors
+ *     the device finds (an expert index outside [0,E) in the caller's
+ *     topk_idx, a bounded wait that ran out) are recorded in a status word
+ *     inside the workspace and read with moe_get_device_status; the kernel
+ *     that found one skips the offending work and returns.
+ *   - T = 0 is a no-op returning MOE_OK.
+ *   - Calls that share a workspace must not run concurrently on the GPU.
+ * Limits (else MOE_ERR_UNSUPPORTED): bits in {4, 8}; group in {32, 64};
+ * H, I and Is multiples of group; 64 <= H <= 8192; I, Is <= 2048;
+ * 1 <= k <= 16; k <= E <= 512; renorm in {0, 1}.
+ * Alignment (else MOE_ERR_INVALID_ARG): x, y, router_w, shared_gate_w,
+ * q, scales and biases 16-byte aligned; q_expert_stride a multiple of 16
+ * bytes and sb_expert_stride a multiple of 8 elements, each at least one
+ * expert's size.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ABI-identical to cudaStream_t; spelled out so this header needs no CUDA headers. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, bad stride */
+  MOE_ERR_UNSUPPORTED = 2, /* shape or format outside the limits above */
+  MOE_ERR_WORKSPACE = 3,   /* workspace missing or smaller than moe_workspace_size */
+  MOE_ERR_CUDA = 4,        /* a CUDA runtime call failed; see moe_last_error_string */
+  MOE_ERR_TIMEOUT = 5,     /* (device) a bounded wait gave up */
+  MOE_ERR_BOUNDS = 6       /* (device) an expert index outside [0, E) was skipped */
+} moe_status;
+
+/* Shape of one MoE layer. */
+typedef struct {
+  int32_t hidden;       /* H */
+  int32_t num_experts;  /* E routed experts */
+  int32_t top_k;        /* k experts per token */
+  int32_t inter;        /* I, routed expert intermediate size */
+  int32_t shared_inter; /* Is, shared expert intermediate size; 0 = no shared expert */
+  int32_t bits;         /* 4 or 8 */
+  int32_t group;        /* 32 or 64 elements per (scale, bias) along K */
+  int32_t renorm;       /* 1: renormalise the k weights; 0: keep softmax probabilities */
+} moe_config;
+
+/* E quantised matrices [rows][K]; see the layout above. */
+typedef struct {
+  const uint8_t* q;          /* codes */
+  const uint16_t* scales;    /* bf16 bit patterns [E][rows][K/group] */
+  const uint16_t* biases;    /* bf16 bit patterns [E][rows][K/group] */
+  int64_t q_expert_stride;   /* bytes from expert e to e+1 (64-bit: stacks exceed 2 GiB) */
+  int64_t sb_expert_stride;  /* elements from expert e to e+1, scales and biases */
+} moe_qtensor;
+
+/* One layer's weights (all device memory). */
+typedef struct {
+  const uint16_t* router_w;      /* bf16 [E][H] */
+  const float* router_bias;      /* fp32 [E] added to the logits before the softmax, or NULL */
+  moe_qtensor gate_up;           /* E matrices [2I][H]: gate rows [0,I), up rows [I,2I) */
+  moe_qtensor down;              /* E matrices [H][I] */
+  moe_qtensor shared_gate_up;    /* 1 matrix [2Is][H] (ignored when shared_inter == 0) */
+  moe_qtensor shared_down;       /* 1 matrix [H][Is] */
+  const uint16_t* shared_gate_w; /* bf16 [H], the shared expert's sigmoid gate */
+} moe_layer_weights;
+
+/* Per-layer record of a stack run; any member may be NULL (not recorded). */
+typedef struct {
+  uint16_t* x;   /* bf16 [L][T][H] input of each layer */
+  int32_t* idx;  /* [L][T][k] selected experts */
+  float* w;      /* [L][T][k] routing weights */
+  uint16_t* y;   /* bf16 [L][T][H] output of each layer */
+} moe_trace;
+
+/* Bytes of workspace the calls below need for T tokens (L is unused and
+ * kept for callers that size one workspace per stack). 0 on bad config. */
+MOE_API size_t moe_workspace_size(const moe_config* cfg, int32_t T, int32_t L);
+
+/* Zeroes the workspace's status word and counters (asynchronously on
+ * `stream`). Call once per new workspace before its first use. */
+MOE_API moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Steps 1-2 for T tokens. x bf16 [T][H]; router_w bf16 [E][H];
+ * router_bias fp32 [E] or NULL. Writes topk_idx [T][k] and topk_w [T][k]
+ * (fp32), each token's experts in descending weight. */
+MOE_API moe_status moe_route_topk(const moe_config* cfg, const uint16_t* x, int32_t T,
+                          const uint16_t* router_w, const float* router_bias,
+                          int32_t* topk_idx, float* topk_w,
+                          void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Steps 3-5 for T tokens given a selection: x bf16 [T][H], topk_idx [T][k],
+ * topk_w [T][k] (fp32) -> y bf16 [T][H]. Indices outside [0, E) are
+ * skipped and reported as MOE_ERR_BOUNDS by moe_get_device_status. */
+MOE_API moe_status moe_expert_ffn(const moe_config* cfg, const moe_layer_weights* w,
+                          const uint16_t* x, int32_t T,
+                          const int32_t* topk_idx, const float* topk_w, uint16_t* y,
+                          void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Steps 1-5: x bf16 [T][H] -> y bf16 [T][H], plus the selection
+ * (topk_idx, topk_w [T][k]; either may be NULL if not wanted). */
+MOE_API moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w,
+                             const uint16_t* x, int32_t T, uint16_t* y,
+                             int32_t* topk_idx, float* topk_w,
+                             void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* L stacked layers (`layers` is a HOST array of L moe_layer_weights, one
+ * configuration for all) joined by a residual stream with a parameter-free
+ * RMSNorm, the pre-norm decoder the MoE block sits in:
+ *   r_0 = x_0;  y_l = MoE_l(x_l);  r_{l+1} = r_l + y_l (fp32);
+ *   x_{l+1} = bf16(r_{l+1} / sqrt(mean(r_{l+1}^2) + 1e-6)).
+ * x0 bf16 [T][H] in, x_out = x_L bf16 [T][H] out. `trace` (host struct of
+ * device pointers, may be NULL) records every layer. */
+MOE_API moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weights* layers, int32_t L,
+                             const uint16_t* x0, int32_t T, uint16_t* x_out,
+                             const moe_trace* trace, void* ws, size_t ws_bytes,
+                             moe_stream_t stream);
+
+/* The batched path's grouping step on its own: the T*k (token, slot) pairs
+ * of topk_idx [T][k] grouped by expert, stable in (token, slot) order, with
+ * the shared expert (if cfg->shared_inter > 0) as expert E taken by every
+ * token. perm [T*k (+T)] receives pair ids (t*k + slot; T*k + t for shared
+ * pairs); offsets [E+2] (or [E+1] without a shared expert) the first
+ * position of each expert and, last, the pair count. */
+MOE_API moe_status moe_sort_by_expert(const moe_config* cfg, const int32_t* topk_idx, int32_t T,
+                              int32_t* perm, int32_t* offsets,
+                              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Waits for `stream`, then returns and clears the workspace's device status
+ * (MOE_OK if no kernel reported an error since the last read). */
+MOE_API moe_status moe_get_device_status(void* ws, moe_stream_t stream);
+
+/* Static text for a status code. */
+MOE_API const char* moe_status_string(moe_status s);
+
+/* Text of the last error raised in this thread by a library call. */
+MOE_API const char* moe_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

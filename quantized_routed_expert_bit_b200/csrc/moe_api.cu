@@ -1,0 +1,350 @@
+// C ABI of the routed-MoE library (declared in include/moe_b200.h):
+// argument validation, the workspace layout, and the stream-ordered launch
+// sequence of each call. Nothing here allocates device memory.
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "moe_b200.h"
+#include "moe_common.cuh"
+#include "moe_launch.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+moe_status fail(moe_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+moe_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr size_t kAlign = 256;
+size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+// Byte offsets of the workspace regions for T tokens.
+struct Layout {
+  size_t hdr, counters, logits, sgate, h, r, xa, xb, y, idx, w, total;
+};
+
+Layout layout(const moe_config& c, int64_t T) {
+  Layout L{};
+  const int64_t imax = c.inter > c.shared_inter ? c.inter : c.shared_inter;
+  const int64_t tiles = (T + moe::kRouteTokTile - 1) / moe::kRouteTokTile;
+  size_t o = 0;
+  L.hdr = o;      o += up(sizeof(moe::WsHeader));
+  L.counters = o; o += up(static_cast<size_t>(tiles) * 4);
+  L.logits = o;   o += up(static_cast<size_t>(T) * c.num_experts * 4);
+  L.sgate = o;    o += up(static_cast<size_t>(T) * 4);
+  L.h = o;        o += up(static_cast<size_t>(T) * (c.top_k + 1) * imax * 4);
+  L.r = o;        o += up(static_cast<size_t>(T) * c.hidden * 4);
+  L.xa = o;       o += up(static_cast<size_t>(T) * c.hidden * 2);
+  L.xb = o;       o += up(static_cast<size_t>(T) * c.hidden * 2);
+  L.y = o;        o += up(static_cast<size_t>(T) * c.hidden * 2);
+  L.idx = o;      o += up(static_cast<size_t>(T) * c.top_k * 4);
+  L.w = o;        o += up(static_cast<size_t>(T) * c.top_k * 4);
+  L.total = o;
+  return L;
+}
+
+moe::WsView view(void* ws, const Layout& L) {
+  char* b = static_cast<char*>(ws);
+  moe::WsView v;
+  v.hdr = reinterpret_cast<moe::WsHeader*>(b + L.hdr);
+  v.counters = reinterpret_cast<uint32_t*>(b + L.counters);
+  v.logits = reinterpret_cast<float*>(b + L.logits);
+  v.sgate = reinterpret_cast<float*>(b + L.sgate);
+  v.h = reinterpret_cast<float*>(b + L.h);
+  return v;
+}
+
+moe_status check_cfg(const moe_config* c) {
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->bits != 4 && c->bits != 8) return fail(MOE_ERR_UNSUPPORTED, "bits=%d (need 4 or 8)", c->bits);
+  if (c->group != 32 && c->group != 64) return fail(MOE_ERR_UNSUPPORTED, "group=%d (need 32 or 64)", c->group);
+  if (c->hidden < 64 || c->hidden > 8192 || c->hidden % c->group)
+    return fail(MOE_ERR_UNSUPPORTED, "hidden=%d (64..8192, multiple of group)", c->hidden);
+  if (c->top_k < 1 || c->top_k > 16) return fail(MOE_ERR_UNSUPPORTED, "top_k=%d (1..16)", c->top_k);
+  if (c->num_experts < c->top_k || c->num_experts > 512)
+    return fail(MOE_ERR_UNSUPPORTED, "num_experts=%d (top_k..512)", c->num_experts);
+  if (c->inter < c->group || c->inter > 2048 || c->inter % c->group)
+    return fail(MOE_ERR_UNSUPPORTED, "inter=%d (group..2048, multiple of group)", c->inter);
+  if (c->shared_inter != 0 &&
+      (c->shared_inter < c->group || c->shared_inter > 2048 || c->shared_inter % c->group))
+    return fail(MOE_ERR_UNSUPPORTED, "shared_inter=%d (0, or group..2048, multiple of group)", c->shared_inter);
+  if (c->renorm != 0 && c->renorm != 1) return fail(MOE_ERR_UNSUPPORTED, "renorm=%d (0 or 1)", c->renorm);
+  return MOE_OK;
+}
+
+moe_status check_ptr(const void* p, size_t a, const char* what) {
+  if (!p) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", what);
+  if (!aligned(p, a)) return fail(MOE_ERR_INVALID_ARG, "%s is not %zu-byte aligned", what, a);
+  return MOE_OK;
+}
+
+moe_status check_qt(const moe_qtensor& q, int64_t rows, int64_t K, int bits, int group, int64_t n,
+                    const char* what) {
+  char name[64];
+  snprintf(name, sizeof(name), "%s.q", what);
+  moe_status s = check_ptr(q.q, 16, name);
+  if (s) return s;
+  snprintf(name, sizeof(name), "%s.scales", what);
+  if ((s = check_ptr(q.scales, 16, name))) return s;
+  snprintf(name, sizeof(name), "%s.biases", what);
+  if ((s = check_ptr(q.biases, 16, name))) return s;
+  if (n > 1) {
+    if (q.q_expert_stride < rows * K * bits / 8 || q.q_expert_stride % 16)
+      return fail(MOE_ERR_INVALID_ARG, "%s.q_expert_stride=%lld (>= %lld, multiple of 16)", what,
+                  static_cast<long long>(q.q_expert_stride), static_cast<long long>(rows * K * bits / 8));
+    if (q.sb_expert_stride < rows * (K / group) || q.sb_expert_stride % 8)
+      return fail(MOE_ERR_INVALID_ARG, "%s.sb_expert_stride=%lld (>= %lld, multiple of 8)", what,
+                  static_cast<long long>(q.sb_expert_stride), static_cast<long long>(rows * (K / group)));
+  }
+  return MOE_OK;
+}
+
+moe_status check_weights(const moe_config& c, const moe_layer_weights* w, bool need_router) {
+  if (!w) return fail(MOE_ERR_INVALID_ARG, "weights is NULL");
+  moe_status s;
+  if (need_router && (s = check_ptr(w->router_w, 16, "router_w"))) return s;
+  if (w->router_bias && !aligned(w->router_bias, 4)) return fail(MOE_ERR_INVALID_ARG, "router_bias misaligned");
+  if ((s = check_qt(w->gate_up, 2LL * c.inter, c.hidden, c.bits, c.group, c.num_experts, "gate_up"))) return s;
+  if ((s = check_qt(w->down, c.hidden, c.inter, c.bits, c.group, c.num_experts, "down"))) return s;
+  if (c.shared_inter > 0) {
+    if ((s = check_qt(w->shared_gate_up, 2LL * c.shared_inter, c.hidden, c.bits, c.group, 1, "shared_gate_up")))
+      return s;
+    if ((s = check_qt(w->shared_down, c.hidden, c.shared_inter, c.bits, c.group, 1, "shared_down"))) return s;
+    if ((s = check_ptr(w->shared_gate_w, 16, "shared_gate_w"))) return s;
+  }
+  return MOE_OK;
+}
+
+moe_status check_ws(const moe_config& c, void* ws, size_t ws_bytes, int64_t T, Layout* L) {
+  if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+  if (!aligned(ws, kAlign)) return fail(MOE_ERR_WORKSPACE, "workspace is not %zu-byte aligned", kAlign);
+  *L = layout(c, T);
+  if (ws_bytes < L->total)
+    return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L->total);
+  return MOE_OK;
+}
+
+moe::QMat qmat(const moe_qtensor& q) {
+  return moe::QMat{q.q, q.scales, q.biases, q.q_expert_stride, q.sb_expert_stride};
+}
+
+moe_status route(const moe_config& c, const uint16_t* x, int T, const uint16_t* wr, const float* rbias,
+                 int32_t* idx, float* w, const moe::WsView& v, cudaStream_t st) {
+  moe::RouteParams p{x, wr, rbias, T, c.hidden, c.num_experts, c.top_k, c.renorm, idx, w, v};
+  cudaError_t e = moe::launch_route_topk(p, st);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "route_topk launch");
+}
+
+moe_status ffn(const moe_config& c, const moe_layer_weights& wt, const uint16_t* x, int T, const int32_t* idx,
+               const float* w, uint16_t* y, const moe::WsView& v, cudaStream_t st) {
+  moe::FfnParams p{};
+  p.x = x;
+  p.idx = idx;
+  p.w = w;
+  p.y = y;
+  p.gate_up = qmat(wt.gate_up);
+  p.down = qmat(wt.down);
+  if (c.shared_inter > 0) {
+    p.sh_gate_up = qmat(wt.shared_gate_up);
+    p.sh_down = qmat(wt.shared_down);
+    p.wsg = wt.shared_gate_w;
+  }
+  p.T = T;
+  p.H = c.hidden;
+  p.E = c.num_experts;
+  p.k = c.top_k;
+  p.I = c.inter;
+  p.Is = c.shared_inter;
+  p.group = c.group;
+  p.Imax = c.inter > c.shared_inter ? c.inter : c.shared_inter;
+  p.ws = v;
+  cudaError_t e = moe::launch_expert_ffn(p, c.bits, st);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "expert_ffn launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_config* cfg, int32_t T, int32_t L) {
+  (void)L;
+  if (check_cfg(cfg) != MOE_OK || T < 0) return 0;
+  return layout(*cfg, T < 1 ? 1 : T).total;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!ws || !aligned(ws, kAlign)) return fail(MOE_ERR_WORKSPACE, "workspace NULL or misaligned");
+  if (ws_bytes < 2 * kAlign) return fail(MOE_ERR_WORKSPACE, "workspace too small");
+  cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "workspace memset");
+}
+
+moe_status moe_route_topk(const moe_config* cfg, const uint16_t* x, int32_t T, const uint16_t* router_w,
+                          const float* router_bias, int32_t* topk_idx, float* topk_w, void* ws,
+                          size_t ws_bytes, moe_stream_t stream) {
+  moe_status s;
+  if ((s = check_cfg(cfg))) return s;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d", T);
+  if (T == 0) return MOE_OK;
+  if ((s = check_ptr(x, 16, "x")) || (s = check_ptr(router_w, 16, "router_w")) ||
+      (s = check_ptr(topk_idx, 4, "topk_idx")) || (s = check_ptr(topk_w, 4, "topk_w")))
+    return s;
+  if (router_bias && !aligned(router_bias, 4)) return fail(MOE_ERR_INVALID_ARG, "router_bias misaligned");
+  Layout L;
+  if ((s = check_ws(*cfg, ws, ws_bytes, T, &L))) return s;
+  return route(*cfg, x, T, router_w, router_bias, topk_idx, topk_w, view(ws, L),
+               reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_ffn(const moe_config* cfg, const moe_layer_weights* w, const uint16_t* x, int32_t T,
+                          const int32_t* topk_idx, const float* topk_w, uint16_t* y, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+  moe_status s;
+  if ((s = check_cfg(cfg))) return s;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d", T);
+  if (T == 0) return MOE_OK;
+  if ((s = check_weights(*cfg, w, false))) return s;
+  if ((s = check_ptr(x, 16, "x")) || (s = check_ptr(y, 16, "y")) || (s = check_ptr(topk_idx, 4, "topk_idx")) ||
+      (s = check_ptr(topk_w, 4, "topk_w")))
+    return s;
+  Layout L;
+  if ((s = check_ws(*cfg, ws, ws_bytes, T, &L))) return s;
+  return ffn(*cfg, *w, x, T, topk_idx, topk_w, y, view(ws, L), reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, const uint16_t* x, int32_t T,
+                             uint16_t* y, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
+  moe_status s;
+  if ((s = check_cfg(cfg))) return s;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d", T);
+  if (T == 0) return MOE_OK;
+  if ((s = check_weights(*cfg, w, true))) return s;
+  if ((s = check_ptr(x, 16, "x")) || (s = check_ptr(y, 16, "y"))) return s;
+  if ((topk_idx && !aligned(topk_idx, 4)) || (topk_w && !aligned(topk_w, 4)))
+    return fail(MOE_ERR_INVALID_ARG, "topk_idx/topk_w misaligned");
+  Layout L;
+  if ((s = check_ws(*cfg, ws, ws_bytes, T, &L))) return s;
+  char* b = static_cast<char*>(ws);
+  int32_t* idx = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(b + L.idx);
+  float* wt = topk_w ? topk_w : reinterpret_cast<float*>(b + L.w);
+  const moe::WsView v = view(ws, L);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if ((s = route(*cfg, x, T, w->router_w, w->router_bias, idx, wt, v, st))) return s;
+  return ffn(*cfg, *w, x, T, idx, wt, y, v, st);
+}
+
+moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weights* layers, int32_t L, const uint16_t* x0,
+                             int32_t T, uint16_t* x_out, const moe_trace* trace, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
+  moe_status s;
+  if ((s = check_cfg(cfg))) return s;
+  if (T < 0 || L < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d L=%d", T, L);
+  if (T == 0 || L == 0) return MOE_OK;
+  if (!layers) return fail(MOE_ERR_INVALID_ARG, "layers is NULL");
+  for (int l = 0; l < L; ++l)
+    if ((s = check_weights(*cfg, &layers[l], true))) return fail(s, "layer %d: %s", l, g_last_error.c_str());
+  if ((s = check_ptr(x0, 16, "x0")) || (s = check_ptr(x_out, 16, "x_out"))) return s;
+  if (trace && ((trace->x && !aligned(trace->x, 16)) || (trace->y && !aligned(trace->y, 16)) ||
+                (trace->idx && !aligned(trace->idx, 4)) || (trace->w && !aligned(trace->w, 4))))
+    return fail(MOE_ERR_INVALID_ARG, "trace buffers misaligned");
+  Layout Ly;
+  if ((s = check_ws(*cfg, ws, ws_bytes, T, &Ly))) return s;
+  char* b = static_cast<char*>(ws);
+  const moe::WsView v = view(ws, Ly);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t TH = static_cast<size_t>(T) * cfg->hidden;
+  const size_t Tk = static_cast<size_t>(T) * cfg->top_k;
+  float* r = reinterpret_cast<float*>(b + Ly.r);
+  uint16_t* xbuf[2] = {reinterpret_cast<uint16_t*>(b + Ly.xa), reinterpret_cast<uint16_t*>(b + Ly.xb)};
+
+  if (trace && trace->x) {
+    cudaError_t e = cudaMemcpyAsync(trace->x, x0, TH * 2, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "trace copy");
+  }
+  moe::GlueParams g0{r, nullptr, x0, nullptr, T, cfg->hidden, 1e-6f};
+  cudaError_t e = moe::launch_glue(g0, st);
+  if (e != cudaSuccess) return cuda_fail(e, "glue launch");
+  const uint16_t* xcur = x0;
+  for (int l = 0; l < L; ++l) {
+    int32_t* idx = (trace && trace->idx) ? trace->idx + l * Tk : reinterpret_cast<int32_t*>(b + Ly.idx);
+    float* wt = (trace && trace->w) ? trace->w + l * Tk : reinterpret_cast<float*>(b + Ly.w);
+    uint16_t* y = (trace && trace->y) ? trace->y + l * TH : reinterpret_cast<uint16_t*>(b + Ly.y);
+    if ((s = route(*cfg, xcur, T, layers[l].router_w, layers[l].router_bias, idx, wt, v, st))) return s;
+    if ((s = ffn(*cfg, layers[l], xcur, T, idx, wt, y, v, st))) return s;
+    uint16_t* xnext;
+    if (l == L - 1) xnext = x_out;
+    else if (trace && trace->x) xnext = trace->x + (l + 1) * TH;
+    else xnext = xbuf[l & 1];
+    moe::GlueParams g{r, y, nullptr, xnext, T, cfg->hidden, 1e-6f};
+    if ((e = moe::launch_glue(g, st)) != cudaSuccess) return cuda_fail(e, "glue launch");
+    xcur = xnext;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_sort_by_expert(const moe_config* cfg, const int32_t* topk_idx, int32_t T, int32_t* perm,
+                              int32_t* offsets, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status s;
+  if ((s = check_cfg(cfg))) return s;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d", T);
+  if ((s = check_ptr(offsets, 4, "offsets"))) return s;
+  if (T > 0 && ((s = check_ptr(topk_idx, 4, "topk_idx")) || (s = check_ptr(perm, 4, "perm")))) return s;
+  Layout L;
+  if ((s = check_ws(*cfg, ws, ws_bytes, T, &L))) return s;
+  moe::SortParams p{topk_idx, T, cfg->top_k, cfg->num_experts, cfg->shared_inter > 0 ? 1 : 0, perm, offsets,
+                    view(ws, L).hdr};
+  cudaError_t e = moe::launch_sort_by_expert(p, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "sort_by_expert launch");
+}
+
+moe_status moe_get_device_status(void* ws, moe_stream_t stream) {
+  if (!ws || !aligned(ws, kAlign)) return fail(MOE_ERR_WORKSPACE, "workspace NULL or misaligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t hdr[2] = {0, 0};
+  cudaError_t e = cudaMemcpyAsync(hdr, ws, sizeof(hdr), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (hdr[0] != 0) {
+    fail(static_cast<moe_status>(hdr[0]), "device reported %s (detail %d)",
+         moe_status_string(static_cast<moe_status>(hdr[0])), hdr[1]);
+    e = cudaMemsetAsync(ws, 0, sizeof(hdr), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "status clear");
+    return static_cast<moe_status>(hdr[0]);
+  }
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_BOUNDS: return "MOE_ERR_BOUNDS";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+const char* moe_last_error_string(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

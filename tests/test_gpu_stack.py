@@ -1,0 +1,101 @@
+"""GPU parity of full-size stacked layers against the CPU oracle.
+
+Decode stacks (T=1, the launch configuration the benchmark times):
+  35b   40 layers, H=2048, E=256, top-8, I=Is=512, 4-bit g64
+  80b   48 layers, H=2048, E=512, top-10, I=Is=512, 4-bit g64
+  35b8  40 layers, the 35b shape in 8-bit g64 with a per-expert router bias
+Batched stacks: the 35b shape with T=64 and T=512 tokens.
+
+Every layer is checked teacher-forced: the oracle gets the GPU's own bf16
+input of that layer (recorded by the stack's trace), so one-ulp
+differences do not compound through later routing. The residual/RMSNorm
+glue between layers is checked separately (within one bf16 ulp).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_routed_expert_bit_b200 import moe, synth
+
+from parity import DeviceLayer, ParityStats, bits, check_tokens
+
+pytestmark = pytest.mark.gpu
+
+
+def run_stack(shape, layers, x0):
+    T, L, H, k = x0.shape[0], len(layers), shape.hidden, shape.top_k
+    cfg = moe.make_config(shape)
+    ws = moe.Workspace(cfg, T, L=L)
+    arr = moe.make_layer_array([moe.make_layer_weights(lw) for lw in layers])
+    tx = torch.empty(L, T, H, dtype=torch.bfloat16, device="cuda")
+    ti = torch.empty(L, T, k, dtype=torch.int32, device="cuda")
+    tw = torch.empty(L, T, k, dtype=torch.float32, device="cuda")
+    ty = torch.empty(L, T, H, dtype=torch.bfloat16, device="cuda")
+    xo = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    tr = moe.Trace(tx.data_ptr(), ti.data_ptr(), tw.data_ptr(), ty.data_ptr())
+    moe.moe_stack_forward(cfg, arr, x0, xo, ws, trace=tr)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == moe.MOE_OK
+    return bits(tx), ti.cpu().numpy(), tw.cpu().numpy(), bits(ty), bits(xo)
+
+
+def check_glue(x0_bits, tx, ty, xo):
+    """x_{l+1} = bf16(rmsnorm(x_0 + sum_{m<=l} y_m)) within one bf16 ulp."""
+    L = ty.shape[0]
+    r = oracle.bf16_to_f32(x0_bits).astype(np.float64)
+    worst, flips = 0, 0
+    for l in range(L):
+        r, x_ref = oracle.residual_rmsnorm(r, ty[l])
+        got = xo if l == L - 1 else tx[l + 1]
+        d = np.abs(got.astype(np.int32) - x_ref.astype(np.int32))
+        worst = max(worst, int(d.max()))
+        flips += int((d > 0).sum())
+    assert worst <= 1, f"glue differs by {worst} bf16 ulps"
+    return flips
+
+
+@pytest.mark.parametrize("key", ["35b", "80b", "35b8"])
+def test_decode_stack_parity(key):
+    shape = synth.SHAPES[key]
+    layers = [synth.make_layer(shape, l, "cuda") for l in range(shape.layers)]
+    total = ParityStats()
+    for tok in (0, 1):
+        x0 = synth.make_tokens(shape, [tok], "cuda")
+        tx, ti, tw, ty, xo = run_stack(shape, layers, x0)
+        for l in range(shape.layers):
+            host = DeviceLayer(shape, layers[l])
+            total.merge(check_tokens(host, tx[l], ti[l], tw[l], ty[l], [0], f"{key} tok {tok} layer {l}"))
+        flips = check_glue(bits(x0), tx, ty, xo)
+    print(f"{key}: {total.checked} (token, layer) pairs, {total.excluded} gap-excluded, "
+          f"max-abs {total.max_abs:.2e}, rel-L2 {total.max_rel_l2:.2e} "
+          f"(unrounded {total.max_rel_l2_unrounded:.2e}), w-err {total.max_w_err:.2e}, glue flips {flips}")
+    assert total.excluded <= max(2, total.checked // 20)
+    del layers
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("key", ["35b_t64", "35b_t512"])
+def test_batched_stack_parity(key):
+    shape = synth.SHAPES[key]
+    T = shape.tokens
+    layers = [synth.make_layer(shape, l, "cuda") for l in range(shape.layers)]
+    x0 = synth.make_batch(shape, T, 0, "cuda")
+    tx, ti, tw, ty, xo = run_stack(shape, layers, x0)
+    total = ParityStats()
+    rng = np.random.default_rng(T)
+    for l in range(shape.layers):
+        host = DeviceLayer(shape, layers[l])
+        toks = sorted(rng.choice(T, size=2, replace=False).tolist())
+        total.merge(check_tokens(host, tx[l], ti[l], tw[l], ty[l], toks, f"{key} layer {l}"))
+    flips = check_glue(bits(x0), tx, ty, xo)
+    print(f"{key}: {total.checked} sampled (token, layer) pairs, {total.excluded} gap-excluded, "
+          f"max-abs {total.max_abs:.2e}, rel-L2 {total.max_rel_l2:.2e}, glue flips {flips}")
+    # every token's selection is a valid set of k distinct experts
+    assert np.all((ti >= 0) & (ti < shape.num_experts))
+    s = np.sort(ti, axis=-1)
+    assert np.all(s[..., 1:] != s[..., :-1])
+    assert np.allclose(tw.sum(axis=-1), 1.0, atol=1e-5)
+    del layers
+    torch.cuda.empty_cache()
