@@ -131,27 +131,43 @@ def barrier_max(dist, value: float) -> float:
     return float(t.item())
 
 
-def cpu_oracle_tokens_per_s(shape, layers_dev, x_tokens, n_layers_sample: int, threads: int):
-    """The oracle (as it stands) on a bounded sample: the first tokens through
-    the first `n_layers_sample` layers, scaled to the full stack."""
+def host_layers_for(shape, layers_dev, tokens_bits):
+    """Host copies (outside any timing) of what the oracle needs for these tokens."""
     import oracle
     sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from parity import DeviceLayer  # host view of device weights (copies outside the timing)
-    hosts = [DeviceLayer(shape, layers_dev[l]) for l in range(n_layers_sample)]
-    xs = [synth.bf16_bits(x_tokens[i:i + 1]) for i in range(x_tokens.shape[0])]
-    # route once untimed to know the experts, and copy them to the host
-    for h in hosts:
-        for x in xs:
+    from parity import DeviceLayer  # host view of device weights
+    hosts = []
+    for lw in layers_dev:
+        h = DeviceLayer(shape, lw)
+        for x in tokens_bits:
             lg = oracle.router_logits(x, h.router_w, h.router_bias)
             for e in oracle.softmax_topk(lg[0], shape.top_k)[0]:
                 h.expert(int(e))
-    t0 = time.perf_counter()
-    for x in xs:
-        for h in hosts:
-            oracle.layer_forward(h, x, threads=threads)
-    dt = time.perf_counter() - t0
-    per_token = dt / len(xs) * (shape.layers / n_layers_sample)
-    return 1.0 / per_token, dt
+        hosts.append(h)
+    return hosts
+
+
+def cpu_oracle_tokens_per_s(shape, layers_dev, x_tokens, threads: int, budget_s: float = 12.0):
+    """The oracle (as it stands) on a bounded sample of the workload: tokens
+    through all layers, one layer at a time, until `budget_s` of CPU time is
+    spent. Only the oracle calls are timed. Returns (tokens/s, evaluations, seconds)."""
+    import oracle
+    spent, evals = 0.0, 0
+    for i in range(x_tokens.shape[0]):
+        x = synth.bf16_bits(x_tokens[i:i + 1])
+        for l0 in range(0, shape.layers, 8):
+            hosts = host_layers_for(shape, layers_dev[l0:l0 + 8], [x])
+            for h in hosts:
+                t0 = time.perf_counter()
+                oracle.layer_forward(h, x, threads=threads)
+                spent += time.perf_counter() - t0
+                evals += 1
+            if spent >= budget_s:
+                break
+        if spent >= budget_s:
+            break
+    per_token = spent / evals * shape.layers
+    return 1.0 / per_token, evals, spent
 
 
 def run_reference(args):
@@ -163,18 +179,12 @@ def run_reference(args):
     shape = synth.SHAPES[SHAPE_KEY]
     threads = os.cpu_count() or 1
     dev = "cuda" if torch.cuda.is_available() else "cpu"
+    threads = min(threads, shape.top_k + 1)  # the oracle runs one expert per thread
     n_layers = 2
     layers = [synth.make_layer(shape, l, dev) for l in range(n_layers)]
     tokens = synth.make_tokens(shape, list(range(args.warmup + args.steps)), dev)
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from parity import DeviceLayer
-    hosts = [DeviceLayer(shape, lw) for lw in layers]
     xs = [synth.bf16_bits(tokens[i:i + 1]) for i in range(tokens.shape[0])]
-    for h in hosts:
-        for x in xs:
-            lg = oracle.router_logits(x, h.router_w, h.router_bias)
-            for e in oracle.softmax_topk(lg[0], shape.top_k)[0]:
-                h.expert(int(e))
+    hosts = host_layers_for(shape, layers, xs)
     for i in range(args.warmup):
         for h in hosts:
             oracle.layer_forward(h, xs[i], threads=threads)
@@ -284,11 +294,11 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        threads = os.cpu_count() or 1
-        v, dt = cpu_oracle_tokens_per_s(shape, layers, tokens[:2], 4, threads)
+        threads = min(os.cpu_count() or 1, shape.top_k + 1)  # one expert per thread
+        v, evals, dt = cpu_oracle_tokens_per_s(shape, layers, tokens, threads)
         cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"2 tokens x 4 of {shape.layers} layers ({dt:.1f} s of CPU work), scaled to "
-                         f"{shape.layers} layers; expert copies to the host outside the timing"}
+               "sample": f"{evals} (token, layer) evaluations of the bench tokens, {dt:.1f} s of oracle time, "
+                         f"scaled to {shape.layers} layers per token; expert copies to the host untimed"}
 
     if rank == 0:
         out = {

@@ -88,8 +88,13 @@ def y_errors(y_gpu_bits: np.ndarray, ref: dict, row: int = 0):
 
 
 def check_tokens(layer: oracle.HostLayer, x_bits: np.ndarray, gpu_idx: np.ndarray, gpu_w: np.ndarray,
-                 gpu_y_bits: np.ndarray, tokens, where: str = "", threads: int = 4) -> ParityStats:
-    """Checks (1)-(3) for the given token rows; raises AssertionError on a violation."""
+                 gpu_y_bits: np.ndarray, tokens, where: str = "", threads: int = 4,
+                 ulp_floor: bool = False) -> ParityStats:
+    """Checks (1)-(3) for the given token rows; raises AssertionError on a violation.
+
+    ulp_floor (for shapes beyond the measured workloads, whose outputs grow
+    past |y| ~ 2): the max-abs bound becomes max(2e-2, one bf16 ulp of the
+    largest |y|), since a single rounding flip there already exceeds 2e-2."""
     st = ParityStats()
     for t in tokens:
         ref = oracle.layer_forward(layer, x_bits[t:t + 1], threads=threads)
@@ -105,7 +110,11 @@ def check_tokens(layer: oracle.HostLayer, x_bits: np.ndarray, gpu_idx: np.ndarra
             st.excluded += 1
             ref = oracle.layer_forward(layer, x_bits[t:t + 1], force_idx=gpu_idx[t:t + 1], threads=threads)
         max_abs, rel, rel32 = y_errors(gpu_y_bits[t], ref)
-        assert max_abs <= Y_MAX_ABS and rel <= Y_REL_L2, \
+        lim = Y_MAX_ABS
+        if ulp_floor:
+            ymax = float(np.max(np.abs(oracle.bf16_to_f32(ref["y16"][0]))))
+            lim = max(lim, 2.0 ** (np.floor(np.log2(max(ymax, 1e-30))) - 7))
+        assert max_abs <= lim and rel <= Y_REL_L2, \
             f"{where} token {t}: max-abs {max_abs:.3e}, rel-L2 {rel:.3e}"
         st.checked += 1
         st.max_abs = max(st.max_abs, max_abs)
