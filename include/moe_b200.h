@@ -175,6 +175,30 @@ MOE_API moe_status moe_sort_by_expert(const moe_config* cfg, const int32_t* topk
                               int32_t* perm, int32_t* offsets,
                               void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_layer_forward without a workspace, for callers that cannot allocate
+ * device memory or pass a scratch buffer of their own: code inside a host
+ * framework that owns all device memory and forbids allocation after
+ * start-up, plugins that are handed only their inputs and outputs, and
+ * latency-critical paths where an allocation (which may synchronise the
+ * device) is not allowed. The pages have no counterpart of this call; it
+ * exists for those callers only.
+ * Its scratch is a fixed 2 MiB array inside the library that every GPU that
+ * loads the library holds until the process exits; calls whose
+ * moe_workspace_size(cfg, T, 1) exceeds 2 MiB (T above about 50 tokens at
+ * H=2048, E=256, k=8, I=512) return MOE_ERR_WORKSPACE. The call allocates
+ * nothing. The first call on a device looks up the array's device address
+ * (with that device current) and keeps it; make that first call before any
+ * stream capture. Every call shares the one array: calls that overlap on the
+ * GPU (other streams, other threads) race and must be serialised by the
+ * caller. Each call clears the status word and counters it needs. Arguments
+ * as moe_layer_forward; device_status (optional, device int32) receives the
+ * call's device status (0 = MOE_OK, else a moe_status) when the stream gets
+ * there. */
+MOE_API moe_status moe_layer_forward_static(const moe_config* cfg, const moe_layer_weights* w,
+                                            const uint16_t* x, int32_t T, uint16_t* y,
+                                            int32_t* topk_idx, float* topk_w, int32_t* device_status,
+                                            moe_stream_t stream);
+
 /* Waits for `stream`, then returns and clears the workspace's device status
  * (MOE_OK if no kernel reported an error since the last read). */
 MOE_API moe_status moe_get_device_status(void* ws, moe_stream_t stream);

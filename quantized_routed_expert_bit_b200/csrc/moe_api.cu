@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "moe_b200.h"
@@ -348,3 +349,81 @@ const char* moe_status_string(moe_status s) {
 const char* moe_last_error_string(void) { return g_last_error.c_str(); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free layer call
+//
+// moe_layer_forward_static runs the same kernels as moe_layer_forward but
+// takes no workspace: its scratch (status word, routing counters, logits,
+// gate activations) lives in the fixed array below, which every GPU that
+// loads this library holds until the process exits. It serves callers that
+// cannot call cudaMalloc or hand the library a buffer of their own: code
+// running inside a host framework that owns all device memory and forbids
+// allocation after start-up, plugins that are handed only their inputs and
+// outputs, and latency-critical paths where an allocation (which may
+// synchronise the device) is not allowed.
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(2) << 20;  // 2 MiB per GPU
+constexpr int kMaxDevices = 128;
+
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_mu;
+void* g_static_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device. In host code the
+// symbol's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and kept.
+moe_status static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_layer_forward_static(const moe_config* cfg, const moe_layer_weights* w,
+                                               const uint16_t* x, int32_t T, uint16_t* y, int32_t* topk_idx,
+                                               float* topk_w, int32_t* device_status, moe_stream_t stream) {
+  moe_status s;
+  if ((s = check_cfg(cfg))) return s;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d", T);
+  if (T == 0) return MOE_OK;
+  if ((s = check_weights(*cfg, w, true))) return s;
+  if ((s = check_ptr(x, 16, "x")) || (s = check_ptr(y, 16, "y"))) return s;
+  if ((topk_idx && !aligned(topk_idx, 4)) || (topk_w && !aligned(topk_w, 4)) ||
+      (device_status && !aligned(device_status, 4)))
+    return fail(MOE_ERR_INVALID_ARG, "topk_idx/topk_w/device_status misaligned");
+  const Layout L = layout(*cfg, T);
+  if (L.total > kStaticScratchBytes)
+    return fail(MOE_ERR_WORKSPACE, "T=%d needs %zu bytes of scratch; the static scratch holds %zu", T, L.total,
+                kStaticScratchBytes);
+  void* ws = nullptr;
+  if ((s = static_scratch(&ws))) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // Status word and arrival counters must start at zero; the rest is overwritten.
+  cudaError_t e = cudaMemsetAsync(ws, 0, L.logits, st);
+  if (e != cudaSuccess) return cuda_fail(e, "static scratch clear");
+  char* b = static_cast<char*>(ws);
+  int32_t* idx = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(b + L.idx);
+  float* wt = topk_w ? topk_w : reinterpret_cast<float*>(b + L.w);
+  const moe::WsView v = view(ws, L);
+  if ((s = route(*cfg, x, T, w->router_w, w->router_bias, idx, wt, v, st))) return s;
+  if ((s = ffn(*cfg, *w, x, T, idx, wt, y, v, st))) return s;
+  if (device_status) {
+    e = cudaMemcpyAsync(device_status, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "device status copy");
+  }
+  return MOE_OK;
+}

@@ -68,13 +68,15 @@ def lib() -> ctypes.CDLL:
         L.moe_layer_forward.argtypes = [CP, LP, P, I32, P, P, P, P, ctypes.c_size_t, P]
         L.moe_stack_forward.argtypes = [CP, LP, I32, P, I32, P, ctypes.POINTER(Trace), P, ctypes.c_size_t, P]
         L.moe_sort_by_expert.argtypes = [CP, P, I32, P, P, P, ctypes.c_size_t, P]
+        L.moe_layer_forward_static.argtypes = [CP, LP, P, I32, P, P, P, P, P]
         L.moe_get_device_status.argtypes = [P, P]
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_last_error_string.argtypes = []
         L.moe_last_error_string.restype = ctypes.c_char_p
         for f in ("moe_workspace_init", "moe_route_topk", "moe_expert_ffn", "moe_layer_forward",
-                  "moe_stack_forward", "moe_sort_by_expert", "moe_get_device_status"):
+                  "moe_stack_forward", "moe_sort_by_expert", "moe_get_device_status",
+                  "moe_layer_forward_static"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -168,6 +170,15 @@ def moe_layer_forward(cfg: Config, w: LayerWeights, x: torch.Tensor, y: torch.Te
                       stream=None):
     _check(lib().moe_layer_forward(ctypes.byref(cfg), ctypes.byref(w), x.data_ptr(), x.shape[0], y.data_ptr(),
                                    _p(topk_idx), _p(topk_w), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def moe_layer_forward_static(cfg: Config, w: LayerWeights, x: torch.Tensor, y: torch.Tensor,
+                             topk_idx: Optional[torch.Tensor], topk_w: Optional[torch.Tensor],
+                             device_status: Optional[torch.Tensor] = None, stream=None):
+    """moe_layer_forward with the library's fixed scratch instead of a workspace."""
+    _check(lib().moe_layer_forward_static(ctypes.byref(cfg), ctypes.byref(w), x.data_ptr(), x.shape[0],
+                                          y.data_ptr(), _p(topk_idx), _p(topk_w), _p(device_status),
+                                          _stream(stream)))
 
 
 def make_layer_array(layers: Sequence[LayerWeights]):
