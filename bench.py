@@ -212,7 +212,8 @@ def workload_config(shape):
                         f"(H={shape.hidden}, E={shape.num_experts}, top-{shape.top_k}, I=Is={shape.inter}, "
                         f"{shape.bits}-bit affine g{shape.group}, bf16 scale/bias, packed gate/up)",
             "tokens_per_step": 1, "layers": shape.layers,
-            "l2": "inputs larger than L2: 18.1 GB resident expert stack, a new token (new experts) every step"}
+            "l2": f"inputs larger than L2: {shape.layers * shape.num_experts * shape.expert_bytes() / 1e9:.1f} GB "
+                  "resident expert stack, a new token (new experts) every step"}
 
 
 def main():
@@ -222,6 +223,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profile a shorter stack (small ncu case); the default is the full 40 layers")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -232,13 +235,18 @@ def main():
     dist, rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
     shape = synth.SHAPES[SHAPE_KEY]
+    if args.layers:
+        import dataclasses
+        shape = dataclasses.replace(shape, layers=args.layers, name=shape.name + f"-first{args.layers}")
     cfg = moe.make_config(shape)
-    layers = [synth.make_layer(shape, l, "cuda") for l in range(shape.layers)]
+    layers = [synth.make_layer(shape, l, "cuda", seed_id=synth.SHAPE_SEED_ID[SHAPE_KEY])
+              for l in range(shape.layers)]
     arr = moe.make_layer_array([moe.make_layer_weights(lw) for lw in layers])
     ws = moe.Workspace(cfg, 1, L=shape.layers)
     nsteps = args.warmup + args.steps
     # each rank its own tokens (independent replicas)
-    tokens = synth.make_tokens(shape, [rank * 100000 + i for i in range(nsteps)], "cuda")
+    tokens = synth.make_tokens(shape, [rank * 100000 + i for i in range(nsteps)], "cuda",
+                               seed_id=synth.SHAPE_SEED_ID[SHAPE_KEY])
     xout = torch.empty(1, shape.hidden, dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
 
@@ -284,7 +292,8 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = barrier_max(dist, e0.elapsed_time(e1))
 
-    launches_per_step = moe.kernel_launches_per_stack(cfg, shape.layers, 1)
+    launches_per_step = moe.moe_stack_kernel_launches(cfg, 1, shape.layers)
+    persistent = launches_per_step < shape.layers
     bytes_tok = touched_bytes_per_token(shape)
     total_tokens = args.steps * world
     tok_s = total_tokens / (ms / 1e3)
@@ -307,11 +316,14 @@ def main():
             "vs_baseline": None, "dtype": "f32", "weights": f"u{shape.bits} affine g{shape.group}, bf16 scale/bias",
             "data": "synthetic", "config": workload_config(shape),
             "hbm_gbs": gbs, "hbm_frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
-            "roofline": {"bound": "hbm", "kernel": moe.dominant_kernel_name(),
+            "roofline": {"bound": "hbm",
+                         "kernel": ("decode_stack_kernel (the whole stack, one launch per step)" if persistent
+                                    else "moe_stack_forward step (router, gate/up, down, glue kernels)"),
                          "achieved": gbs, "peak": peak, "peak_source": peak_src, "unit": "GB/s",
                          "frac": gbs / peak, "traffic": None,
                          "bytes_per_launch": bytes_tok,
-                         "note": "achieved = algorithmic bytes per step / device time per step"},
+                         "note": "achieved = algorithmic bytes per step / device time per step (CUDA events "
+                                 "on the launch stream around the timed steps)"},
             "cpu_baseline": cpu,
             "e2e": {"value": total_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": shape.hidden * 2, "d2h_bytes_per_step": shape.hidden * 2},

@@ -120,6 +120,9 @@ typedef struct {
   int32_t* idx;  /* [L][T][k] selected experts */
   float* w;      /* [L][T][k] routing weights */
   uint16_t* y;   /* bf16 [L][T][H] output of each layer */
+  uint64_t* t;   /* [L][8] device clock (ns) at the phase boundaries of each layer, single-token
+                    persistent path only: 0 layer start, 1 router done, 2 routing barrier passed,
+                    3 top-k done, 4 gate/up done, 5 h barrier passed, 6 down done, 7 y barrier passed */
 } moe_trace;
 
 /* Bytes of workspace the calls below need for T tokens (L is unused and
@@ -164,6 +167,12 @@ MOE_API moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weig
                              const uint16_t* x0, int32_t T, uint16_t* x_out,
                              const moe_trace* trace, void* ws, size_t ws_bytes,
                              moe_stream_t stream);
+
+/* Number of kernel launches moe_stack_forward makes for T tokens and L
+ * layers on the current device: a single token runs the whole stack as one
+ * persistent kernel (one launch per 128 layers) when the shape fits it;
+ * otherwise 1 + 4*L. -1 on a bad configuration. */
+MOE_API int32_t moe_stack_kernel_launches(const moe_config* cfg, int32_t T, int32_t L);
 
 /* The batched path's grouping step on its own: the T*k (token, slot) pairs
  * of topk_idx [T][k] grouped by expert, stable in (token, slot) order, with

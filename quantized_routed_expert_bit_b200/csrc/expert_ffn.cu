@@ -15,8 +15,8 @@
 // staged into shared memory by bulk copies (TMA engine) completing on an
 // mbarrier, overlapping the code loads. A group's share of a dot product is
 // s * sum(q x) + b * sum(x), with sum(x) over each 16-byte segment computed
-// once per CTA; codes become floats in registers without int->float
-// conversion (see dot_seg in moe_common.cuh).
+// once per CTA; codes become exact fp32 integers in registers without
+// int->float conversion (see dot_seg in moe_common.cuh).
 
 #include "moe_common.cuh"
 #include "moe_launch.h"
@@ -77,7 +77,6 @@ __global__ void __launch_bounds__(kWarps * 32)
     gateup_swiglu_kernel(FfnParams p) {
   using CT = CodeTraits<BITS>;
   constexpr int PS = CT::kPerSeg;
-  constexpr float D = CT::kD;
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ __align__(8) uint64_t bar;
 
@@ -191,10 +190,10 @@ __global__ void __launch_bounds__(kWarps * 32)
 #pragma unroll
         for (int rr = 0; rr < kRowsPerWarp; ++rr) {
           const int il = warp * kRowsPerWarp + rr;
-          const float sg = D * bf16_to_f32(sb[0 * sb_elems + il * ng + g]);
-          const float su = D * bf16_to_f32(sb[1 * sb_elems + il * ng + g]);
-          const float bg = bf16_to_f32(sb[2 * sb_elems + il * ng + g]) - sg;
-          const float bu = bf16_to_f32(sb[3 * sb_elems + il * ng + g]) - su;
+          const float sg = bf16_to_f32(sb[0 * sb_elems + il * ng + g]);
+          const float su = bf16_to_f32(sb[1 * sb_elems + il * ng + g]);
+          const float bg = bf16_to_f32(sb[2 * sb_elems + il * ng + g]);
+          const float bu = bf16_to_f32(sb[3 * sb_elems + il * ng + g]);
           ag[rr] = fmaf(sg, dot_seg<BITS>(cg[rr][c], xv), fmaf(bg, xsm, ag[rr]));
           au[rr] = fmaf(su, dot_seg<BITS>(cu[rr][c], xv), fmaf(bu, xsm, au[rr]));
         }
@@ -219,7 +218,6 @@ __global__ void __launch_bounds__(kWarps * 32)
     down_combine_kernel(FfnParams p) {
   using CT = CodeTraits<BITS>;
   constexpr int PS = CT::kPerSeg;
-  constexpr float D = CT::kD;
   constexpr int kMaxSlots = 17;
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ __align__(8) uint64_t bar;
@@ -340,8 +338,8 @@ __global__ void __launch_bounds__(kWarps * 32)
 #pragma unroll
           for (int rr = 0; rr < kRowsPerWarp; ++rr) {
             const int il = warp * kRowsPerWarp + rr;
-            const float sc = D * bf16_to_f32(sb[j * sb_slot + il * ng + g]);
-            const float bi = bf16_to_f32(sb[j * sb_slot + kRB * ng + il * ng + g]) - sc;
+            const float sc = bf16_to_f32(sb[j * sb_slot + il * ng + g]);
+            const float bi = bf16_to_f32(sb[j * sb_slot + kRB * ng + il * ng + g]);
             const float part = fmaf(sc, dot_seg<BITS>(cd[rr][c], xv), bi * hsm);
             acc[rr] = fmaf(wj, part, acc[rr]);
           }

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <memory>
 #include <mutex>
 #include <string>
 
@@ -37,8 +38,12 @@ size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // Byte offsets of the workspace regions for T tokens.
 struct Layout {
-  size_t hdr, counters, logits, sgate, h, r, xa, xb, y, idx, w, total;
+  size_t hdr, counters, logits, sgate, h, r, xa, xb, y, idx, w;
+  size_t flags, dlogits, dh, dy, dr, dx;  // persistent single-token decode
+  size_t total;
 };
+
+constexpr int kMaxGrid = 1024;  // barrier flags reserved for the persistent decode grid
 
 Layout layout(const moe_config& c, int64_t T) {
   Layout L{};
@@ -56,6 +61,12 @@ Layout layout(const moe_config& c, int64_t T) {
   L.y = o;        o += up(static_cast<size_t>(T) * c.hidden * 2);
   L.idx = o;      o += up(static_cast<size_t>(T) * c.top_k * 4);
   L.w = o;        o += up(static_cast<size_t>(T) * c.top_k * 4);
+  L.flags = o;    o += up(static_cast<size_t>(kMaxGrid) * 4);
+  L.dlogits = o;  o += up(static_cast<size_t>(c.num_experts + 1) * 4);
+  L.dh = o;       o += up(static_cast<size_t>(c.top_k + 1) * imax * 4);
+  L.dy = o;       o += up(static_cast<size_t>(c.hidden) * 2);
+  L.dr = o;       o += up(static_cast<size_t>(c.hidden) * 4);
+  L.dx = o;       o += up(static_cast<size_t>(c.hidden) * 2);
   L.total = o;
   return L;
 }
@@ -179,9 +190,114 @@ moe_status ffn(const moe_config& c, const moe_layer_weights& wt, const uint16_t*
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "expert_ffn launch");
 }
 
+// Device facts the persistent decode needs, looked up once per device.
+struct DevInfo {
+  bool ok = false;
+  int sms = 0, coop = 0, smem_optin = 0;
+};
+
+std::mutex g_dev_mu;
+DevInfo g_dev[128];
+
+bool dev_info(DevInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return false;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.ok) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return false;
+    d.ok = true;
+  }
+  *out = d;
+  return true;
+}
+
+// Whether one token through a stack runs as the persistent kernel (one
+// launch per up to kMaxDecodeLayers layers) rather than four kernels per layer.
+bool decode_eligible(const moe_config& c, int* grid) {
+  DevInfo d;
+  if (!dev_info(&d) || !d.coop || d.sms < 1 || d.sms > kMaxGrid) return false;
+  if (!moe::decode_stack_supported(c.hidden, c.num_experts, c.top_k, c.inter, c.shared_inter, c.group, c.bits))
+    return false;
+  const size_t smem =
+      moe::decode_stack_smem(c.hidden, c.num_experts, c.top_k, c.inter, c.shared_inter, c.group, c.bits, d.sms);
+  if (smem + 1024 > static_cast<size_t>(d.smem_optin)) return false;
+  *grid = d.sms;
+  return true;
+}
+
+moe::LayerDesc layer_desc(const moe_layer_weights& w) {
+  moe::LayerDesc d{};
+  d.wr = w.router_w;
+  d.rbias = w.router_bias;
+  d.wsg = w.shared_gate_w;
+  d.gu = qmat(w.gate_up);
+  d.dn = qmat(w.down);
+  d.sgu = qmat(w.shared_gate_up);
+  d.sdn = qmat(w.shared_down);
+  return d;
+}
+
+moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, int L, const uint16_t* x0,
+                        uint16_t* x_out, const moe_trace* trace, void* ws, const Layout& Ly, int grid,
+                        cudaStream_t st) {
+  char* b = static_cast<char*>(ws);
+  auto P = std::make_unique<moe::DecodeParams>();
+  P->H = c.hidden;
+  P->E = c.num_experts;
+  P->k = c.top_k;
+  P->I = c.inter;
+  P->Is = c.shared_inter;
+  P->group = c.group;
+  P->renorm = c.renorm;
+  P->layer_mode = 0;
+  P->epoch0 = 0;
+  P->eps = 1e-6f;
+  P->tr_x = trace ? trace->x : nullptr;
+  P->tr_idx = trace ? trace->idx : nullptr;
+  P->tr_w = trace ? trace->w : nullptr;
+  P->tr_y = trace ? trace->y : nullptr;
+  P->tr_t = trace ? trace->t : nullptr;
+  P->logits = reinterpret_cast<float*>(b + Ly.dlogits);
+  P->hbuf = reinterpret_cast<float*>(b + Ly.dh);
+  P->ybuf = reinterpret_cast<uint16_t*>(b + Ly.dy);
+  P->flags = reinterpret_cast<unsigned*>(b + Ly.flags);
+  P->hdr = reinterpret_cast<moe::WsHeader*>(b + Ly.hdr);
+  uint16_t* xmid = reinterpret_cast<uint16_t*>(b + Ly.dx);
+  float* rmid = reinterpret_cast<float*>(b + Ly.dr);
+  for (int l0 = 0; l0 < L; l0 += moe::kMaxDecodeLayers) {
+    const int n = (L - l0 < moe::kMaxDecodeLayers) ? L - l0 : moe::kMaxDecodeLayers;
+    const bool last = (l0 + n == L);
+    P->L = n;
+    P->l0 = l0;
+    P->x0 = (l0 == 0) ? x0 : xmid;
+    P->r_in = (l0 == 0) ? nullptr : rmid;
+    P->out = last ? x_out : xmid;
+    P->r_out = last ? nullptr : rmid;
+    for (int i = 0; i < n; ++i) P->layers[i] = layer_desc(layers[l0 + i]);
+    cudaError_t e = cudaMemsetAsync(P->flags, 0, static_cast<size_t>(grid) * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "barrier flag reset");
+    e = moe::launch_decode_stack(*P, c.bits, grid, st);
+    if (e != cudaSuccess) return cuda_fail(e, "decode_stack launch");
+  }
+  return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+int32_t moe_stack_kernel_launches(const moe_config* cfg, int32_t T, int32_t L) {
+  if (check_cfg(cfg) != MOE_OK || T < 0 || L < 0) return -1;
+  if (T == 0 || L == 0) return 0;
+  int grid = 0;
+  if (T == 1 && decode_eligible(*cfg, &grid))
+    return (L + moe::kMaxDecodeLayers - 1) / moe::kMaxDecodeLayers;
+  return 1 + 4 * L;
+}
 
 size_t moe_workspace_size(const moe_config* cfg, int32_t T, int32_t L) {
   (void)L;
@@ -270,6 +386,8 @@ moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weights* lay
   char* b = static_cast<char*>(ws);
   const moe::WsView v = view(ws, Ly);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int grid = 0;
+  if (T == 1 && decode_eligible(*cfg, &grid)) return stack_decode(*cfg, layers, L, x0, x_out, trace, ws, Ly, grid, st);
   const size_t TH = static_cast<size_t>(T) * cfg->hidden;
   const size_t Tk = static_cast<size_t>(T) * cfg->top_k;
   float* r = reinterpret_cast<float*>(b + Ly.r);

@@ -142,31 +142,41 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
 // ---------------------------------------------------------------- dequant dot products
 //
 // The weight of a code q in group g is s_g*q + b_g, so a group's share of a
-// dot product is  s_g * sum(q x) + b_g * sum(x).  The kernels build each code
-// as the fp32 number 1 + q/16 (4-bit) or 1 + q/256 (8-bit) by placing it in
-// the top mantissa bits of 1.0 (exact, no int->float conversion), so that
-//   sum((1 + q/D) x) = sum(x) + sum(q x)/D
-// and the group's share becomes  (D s) * acc + (b - D s) * sum(x).
+// dot product is  s_g * sum(q x) + b_g * sum(x),  with sum(x) per 16-byte
+// segment of codes computed once. sum(q x) is formed from exact integers:
+// a code sitting at bits [p, p+w) of a word becomes the fp32 number M + q,
+// M = 2^(23-p), by OR-ing the masked word into the bits of M (one lop3/prmt,
+// no int->float conversion); subtracting M gives q exactly, and q*x is an
+// exact product accumulated in fp32. Pairs of codes go through the packed
+// fp32x2 add and fma of sm_100.
 
-// sum over the 8 codes of one 32-bit word of 4-bit codes of (1 + q/16) * x.
-__device__ __forceinline__ float dot8_u4(uint32_t w, const float* x, float acc) {
-#pragma unroll
-  for (int n = 0; n < 8; ++n) {
-    const int sh = 19 - 4 * n;  // move nibble n to mantissa bits 19..22
-    const uint32_t m = (sh >= 0) ? (w << sh) : (w >> (-sh));
-    acc = fmaf(__uint_as_float((m & 0x00780000u) | 0x3f800000u), x[n], acc);
-  }
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float fb(uint32_t u) { return __uint_as_float(u); }
+
+// sum over the 8 codes of one 32-bit word of 4-bit codes of q * x (x: 8 floats),
+// accumulated into the pair acc.
+__device__ __forceinline__ float2 dot8_u4(uint32_t w, const float* x, float2 acc) {
+  const uint32_t v = w >> 12;  // codes 5, 6, 7 move to bits 8, 12, 16
+  // M + q for code positions 0, 4, 8, 12, 16: M = 2^23, 2^19, 2^15, 2^11, 2^7
+  const float2 f01 = f2(fb((w & 0xFu) | 0x4B000000u), fb((w & 0xF0u) | 0x49000000u));
+  const float2 f23 = f2(fb((w & 0xF00u) | 0x47000000u), fb((w & 0xF000u) | 0x45000000u));
+  const float2 f45 = f2(fb((w & 0xF0000u) | 0x43000000u), fb((v & 0xF00u) | 0x47000000u));
+  const float2 f67 = f2(fb((v & 0xF000u) | 0x45000000u), fb((v & 0xF0000u) | 0x43000000u));
+  acc = __ffma2_rn(__fadd2_rn(f01, f2(-8388608.f, -524288.f)), f2(x[0], x[1]), acc);
+  acc = __ffma2_rn(__fadd2_rn(f23, f2(-32768.f, -2048.f)), f2(x[2], x[3]), acc);
+  acc = __ffma2_rn(__fadd2_rn(f45, f2(-128.f, -32768.f)), f2(x[4], x[5]), acc);
+  acc = __ffma2_rn(__fadd2_rn(f67, f2(-2048.f, -128.f)), f2(x[6], x[7]), acc);
   return acc;
 }
 
-// sum over the 4 codes of one 32-bit word of 8-bit codes of (1 + q/256) * x.
-__device__ __forceinline__ float dot4_u8(uint32_t w, const float* x, float acc) {
-#pragma unroll
-  for (int n = 0; n < 4; ++n) {
-    const int sh = 15 - 8 * n;  // move byte n to mantissa bits 15..22
-    const uint32_t m = (sh >= 0) ? (w << sh) : (w >> (-sh));
-    acc = fmaf(__uint_as_float((m & 0x007f8000u) | 0x3f800000u), x[n], acc);
-  }
+// sum over the 4 codes of one 32-bit word of 8-bit codes of q * x (x: 4 floats).
+// Each byte is permuted into bits 8..15 under the exponent of 2^15.
+__device__ __forceinline__ float2 dot4_u8(uint32_t w, const float* x, float2 acc) {
+  constexpr uint32_t kM = 0x47000000u;  // 2^15, exponent byte in byte 3
+  const float2 f01 = f2(fb(__byte_perm(w, kM, 0x7504)), fb(__byte_perm(w, kM, 0x7514)));
+  const float2 f23 = f2(fb(__byte_perm(w, kM, 0x7524)), fb(__byte_perm(w, kM, 0x7534)));
+  acc = __ffma2_rn(__fadd2_rn(f01, f2(-32768.f, -32768.f)), f2(x[0], x[1]), acc);
+  acc = __ffma2_rn(__fadd2_rn(f23, f2(-32768.f, -32768.f)), f2(x[2], x[3]), acc);
   return acc;
 }
 
@@ -174,19 +184,17 @@ template <int BITS>
 struct CodeTraits;
 template <>
 struct CodeTraits<4> {
-  static constexpr int kPerSeg = 32;     // codes per 16-byte segment
-  static constexpr float kD = 16.0f;     // code scale in the 1 + q/D trick
+  static constexpr int kPerSeg = 32;  // codes per 16-byte segment
 };
 template <>
 struct CodeTraits<8> {
   static constexpr int kPerSeg = 16;
-  static constexpr float kD = 256.0f;
 };
 
-// sum over one 16-byte segment of codes of (1 + q/D) * x[i] (x: kPerSeg floats).
+// sum over one 16-byte segment of codes of q * x[i] (x: kPerSeg floats).
 template <int BITS>
 __device__ __forceinline__ float dot_seg(const uint4& c, const float* x) {
-  float acc = 0.f;
+  float2 acc = f2(0.f, 0.f);
   if constexpr (BITS == 4) {
     acc = dot8_u4(c.x, x + 0, acc);
     acc = dot8_u4(c.y, x + 8, acc);
@@ -198,7 +206,7 @@ __device__ __forceinline__ float dot_seg(const uint4& c, const float* x) {
     acc = dot4_u8(c.z, x + 8, acc);
     acc = dot4_u8(c.w, x + 12, acc);
   }
-  return acc;
+  return acc.x + acc.y;
 }
 
 }  // namespace moe

@@ -58,9 +58,46 @@ struct SortParams {
   WsHeader* hdr;
 };
 
+// One layer's weights for the persistent decode kernel.
+struct LayerDesc {
+  const uint16_t* wr;    // bf16 [E][H]
+  const float* rbias;    // fp32 [E] or null
+  const uint16_t* wsg;   // bf16 [H] shared-expert gate vector (when Is > 0)
+  QMat gu, dn, sgu, sdn;
+};
+
+constexpr int kMaxDecodeLayers = 128;  // layers per launch (kernel parameter space)
+
+struct DecodeParams {
+  int L, l0;             // layers in this launch; index of its first layer in the stack
+  int H, E, k, I, Is, group, renorm;
+  int layer_mode;        // 1: one layer, y -> out (no residual/norm); 0: stack, x_L -> out
+  unsigned epoch0;       // barrier epochs start above this value
+  float eps;
+  const uint16_t* x0;    // bf16 [H] input of the first layer
+  const float* r_in;     // fp32 [H] residual at the first layer, or null (= x0)
+  uint16_t* out;         // bf16 [H]
+  float* r_out;          // fp32 [H] residual after the last layer, or null
+  uint16_t* tr_x;        // bf16 [layers][H] or null
+  int32_t* tr_idx;       // [layers][k] or null
+  float* tr_w;           // [layers][k] or null
+  uint16_t* tr_y;        // bf16 [layers][H] or null
+  uint64_t* tr_t;        // [layers][8] phase timestamps of CTA 0, or null
+  float* logits;         // fp32 [E+1] (workspace)
+  float* hbuf;           // fp32 [k+1][Imax] (workspace)
+  uint16_t* ybuf;        // bf16 [H] (workspace)
+  unsigned* flags;       // [grid] barrier flags, zero at launch (workspace)
+  WsHeader* hdr;
+  LayerDesc layers[kMaxDecodeLayers];
+};
+
 cudaError_t launch_route_topk(const RouteParams& p, cudaStream_t stream);
 cudaError_t launch_expert_ffn(const FfnParams& p, int bits, cudaStream_t stream);
 cudaError_t launch_glue(const GlueParams& p, cudaStream_t stream);
 cudaError_t launch_sort_by_expert(const SortParams& p, cudaStream_t stream);
+
+bool decode_stack_supported(int H, int E, int k, int I, int Is, int group, int bits);
+size_t decode_stack_smem(int H, int E, int k, int I, int Is, int group, int bits, int grid);
+cudaError_t launch_decode_stack(const DecodeParams& p, int bits, int grid, cudaStream_t stream);
 
 }  // namespace moe

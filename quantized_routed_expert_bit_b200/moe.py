@@ -48,7 +48,7 @@ class LayerWeights(ctypes.Structure):
 
 
 class Trace(ctypes.Structure):
-    _fields_ = [("x", P), ("idx", P), ("w", P), ("y", P)]
+    _fields_ = [("x", P), ("idx", P), ("w", P), ("y", P), ("t", P)]
 
 
 def lib() -> ctypes.CDLL:
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.moe_stack_forward.argtypes = [CP, LP, I32, P, I32, P, ctypes.POINTER(Trace), P, ctypes.c_size_t, P]
         L.moe_sort_by_expert.argtypes = [CP, P, I32, P, P, P, ctypes.c_size_t, P]
         L.moe_layer_forward_static.argtypes = [CP, LP, P, I32, P, P, P, P, P]
+        L.moe_stack_kernel_launches.argtypes = [CP, I32, I32]
+        L.moe_stack_kernel_launches.restype = I32
         L.moe_get_device_status.argtypes = [P, P]
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
@@ -207,12 +209,6 @@ def moe_get_device_status(ws: Workspace, stream=None) -> int:
 # ---------------------------------------------------------------- launch plan (for reporting)
 
 
-def kernel_launches_per_stack(cfg: Config, L: int, T: int) -> int:
-    """Kernels the library launches for one moe_stack_forward call: one
-    residual initialisation, then per layer the router/top-k, the gate/up +
-    SwiGLU, the down + combine and the residual/RMSNorm kernels."""
-    return 1 + 4 * L
-
-
-def dominant_kernel_name() -> str:
-    return "moe_stack_forward step (router, gate/up+SwiGLU, down+combine, glue kernels)"
+def moe_stack_kernel_launches(cfg: Config, T: int, L: int) -> int:
+    """Kernels one moe_stack_forward call launches on the current device."""
+    return int(lib().moe_stack_kernel_launches(ctypes.byref(cfg), int(T), int(L)))

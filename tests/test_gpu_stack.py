@@ -99,3 +99,41 @@ def test_batched_stack_parity(key):
     assert np.allclose(tw.sum(axis=-1), 1.0, atol=1e-5)
     del layers
     torch.cuda.empty_cache()
+
+
+def test_decode_stack_longer_than_one_launch():
+    """130 layers: the persistent path splits the stack over two launches and
+    carries the residual stream between them."""
+    shape = synth.MoEShape("chunk-h256-e16", 256, 16, 2, 128, 128, 4, 32, 130, False, 1)
+    cfg = moe.make_config(shape)
+    assert moe.moe_stack_kernel_launches(cfg, 1, shape.layers) == 2
+    layers = [synth.make_layer(shape, l, "cuda", seed_id=400) for l in range(shape.layers)]
+    x0 = synth.make_tokens(shape, [3], "cuda", seed_id=400)
+    tx, ti, tw, ty, xo = run_stack(shape, layers, x0)
+    total = ParityStats()
+    for l in (0, 1, 63, 126, 127, 128, 129):
+        total.merge(check_tokens(DeviceLayer(shape, layers[l]), tx[l], ti[l], tw[l], ty[l], [0], f"layer {l}"))
+    check_glue(bits(x0), tx, ty, xo)
+    assert total.checked == 7
+
+
+def test_single_token_path_matches_multi_kernel_path():
+    """One token through the persistent kernel against the same token run
+    twice in a batch of two (the multi-kernel path): same experts, outputs
+    within the parity tolerance of each other, layer by layer."""
+    shape = synth.SHAPES["35b"]
+    import dataclasses
+    shape = dataclasses.replace(shape, layers=4)
+    layers = [synth.make_layer(shape, l, "cuda", seed_id=2) for l in range(shape.layers)]
+    cfg = moe.make_config(shape)
+    assert moe.moe_stack_kernel_launches(cfg, 1, 4) == 1
+    assert moe.moe_stack_kernel_launches(cfg, 2, 4) == 17
+    x1 = synth.make_tokens(shape, [7], "cuda", seed_id=2)
+    a = run_stack(shape, layers, x1)
+    b = run_stack(shape, layers, torch.cat([x1, x1]))
+    for l in range(shape.layers):
+        assert set(a[1][l][0].tolist()) == set(b[1][l][0].tolist()) == set(b[1][l][1].tolist())
+        ya = oracle.bf16_to_f32(a[3][l][0]).astype(np.float64)
+        yb = oracle.bf16_to_f32(b[3][l][0]).astype(np.float64)
+        assert np.max(np.abs(ya - yb)) <= 2e-2
+        assert np.linalg.norm(ya - yb) <= 1e-3 * np.linalg.norm(yb)
