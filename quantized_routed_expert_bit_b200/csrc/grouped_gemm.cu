@@ -1,0 +1,497 @@
+// Kernel (c): the batched path. Tokens are grouped by expert (counting sort,
+// sort_by_expert.cu), so each selected expert's weights are read once for
+// all of its tokens, and each expert's gate/up and down products become
+// small GEMMs run on the tensor cores (tcgen05, accumulators in TMEM).
+//
+//   gather   x (bf16) of every (token, expert) pair, in expert order, as
+//            fp16 rows: the B operand of the gate/up GEMM; also the shared
+//            expert's sigmoid gate per token;
+//   GEMM gu  per (expert chunk of <=128 pairs, 64 intermediate indices):
+//            A = the 64 gate rows and 64 up rows, dequantised in shared
+//            memory to fp16, B = the chunk's gathered tokens; epilogue
+//            h = silu(gate) * up, stored as an fp16 hi/lo pair;
+//   GEMM dn  per (expert chunk, 128 output rows): A = down rows dequantised,
+//            B = h hi and h lo (two MMAs, so h keeps ~22 bits); epilogue
+//            writes each pair's output row (fp32);
+//   combine  y = sum_j w_j o_j + sigmoid-gate * o_shared, in rank order,
+//            one bf16 rounding.
+// MLX-style affine groups (Swiftlet article on xix.ai, paragraph 8), packed
+// routed gate/up (Runnel README, introduction and "Streaming CLI"), shared
+// expert (same article, paragraph 8; Runnel README, "Target").
+//
+// GEMM CTA (one per SM, persistent over tiles), 16 warps:
+//   warp 0      TMA producer: codes (3D map over the expert stack), scales
+//               and biases (per tile), B tiles (128-byte swizzled);
+//   warp 1      TMEM owner; lane 0 issues tcgen05.mma (M=128, N=16..128, K=16);
+//   warps 4-11  dequantisers: codes -> fp16 A tiles in the swizzled layout;
+//   warps 12-15 epilogue: TMEM -> registers -> global.
+// A stage ring of NS k-blocks (64 K each) decouples the roles; every wait
+// is bounded and an abort drains copies and MMAs before TMEM is freed.
+//
+// Dequantisation: w = s*q + b rounded once to fp16. 4-bit codes become fp16
+// (1024 + q) / (64 + q) by one lop3 per pair of codes; subtracting the
+// offset is exact; one fp16 fma applies scale and bias. For 4-bit the pairs
+// come out as (k, k+4) within each 8 codes, so the A tile holds K in the
+// order 0,4,1,5,2,6,3,7 inside every 8; the B operands (gathered x, h) are
+// written in the same order (the dot product does not depend on the order).
+
+#include <cuda_fp16.h>
+
+#include "moe_common.cuh"
+#include "moe_launch.h"
+#include "tc.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kBM = 128;           // tile rows
+constexpr int kBK = 64;            // K per k-block (128 bytes of fp16: one swizzle row)
+constexpr int kDequantWarp0 = 4;   // warps 4..11
+constexpr int kEpiWarp0 = 12;      // warps 12..15
+constexpr int kAccCols = 128;      // TMEM columns per accumulator buffer
+
+__host__ __device__ constexpr uint32_t al1k(uint32_t v) { return (v + 1023u) & ~1023u; }
+
+// Position p of an 8-block of K holds element kPerm8[p] (4-bit codes only).
+__host__ __device__ constexpr int perm8_pos(int k) {  // position of element k
+  return (k & 4) ? ((k & 3) * 2 + 1) : ((k & 3) * 2);
+}
+
+struct GemmSmem {
+  uint32_t a, b, codes, sc, bar, total;
+  int ns, b_stage_bytes, codes_stage_bytes, sc_buf_bytes;
+};
+
+__host__ __device__ inline GemmSmem gemm_smem(int mode, int bits, int K, int group, int ns) {
+  GemmSmem s{};
+  s.ns = ns;
+  const int ng = K / group;
+  s.b_stage_bytes = (mode == 0 ? 1 : 2) * kAccCols * 128;  // up to 128 rows x 128 B (x2: h hi and lo)
+  s.codes_stage_bytes = kBM * (kBK * bits / 8);
+  s.sc_buf_bytes = 2 * kBM * ng * 2;                         // scales and biases of 128 rows
+  uint32_t o = 0;
+  s.a = o;     o = al1k(o + ns * kBM * kBK * 2);
+  s.b = o;     o = al1k(o + ns * s.b_stage_bytes);
+  s.codes = o; o = al1k(o + ns * s.codes_stage_bytes);
+  s.sc = o;    o = al1k(o + 2 * s.sc_buf_bytes);
+  s.bar = o;   o += 256;
+  s.total = o + 1024;  // slack to align the dynamic base to 1 KiB
+  return s;
+}
+
+__device__ __forceinline__ int b_box_index(int n) { return n <= 16 ? 0 : n <= 32 ? 1 : n <= 64 ? 2 : 3; }
+__device__ __forceinline__ int b_box_rows(int i) { return 16 << i; }
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.f + expf(-z)); }
+
+// Bounded wait that also gives up as soon as another role has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, WsHeader* hdr, volatile int* abort,
+                                              int where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0; it < kWaitIters; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitNs) break;
+    }
+  }
+  report(hdr, MOE_ERR_TIMEOUT, where);
+  *abort = 1;
+  return false;
+}
+
+// Warp-uniform wait: lane 0 waits, every lane gets the same answer.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, WsHeader* hdr, volatile int* abort,
+                                         int where) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = wait_or_abort(bar, parity, hdr, abort, where);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+__device__ __forceinline__ bool warp_aborted(volatile int* abort) {
+  return __shfl_sync(0xffffffffu, ((threadIdx.x & 31) == 0) ? *abort : 0, 0) != 0;
+}
+
+// Dequantise 32 codes (4-bit: 16 bytes) of one row into 4 swizzled 16-byte fp16 chunks.
+__device__ __forceinline__ void dequant32_u4(const uint4 c, __half2 s2, __half2 b2, uint4* out) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  const __half2 k1024 = __half2half2(__ushort_as_half(0x6400));
+  const __half2 k64 = __half2half2(__ushort_as_half(0x5400));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t x = w[i], y = w[i] >> 8;
+    uint32_t v0 = (x & 0x000F000Fu) | 0x64006400u;  // (1024 + q0, 1024 + q4)
+    uint32_t v1 = (x & 0x00F000F0u) | 0x54005400u;  // (  64 + q1,   64 + q5)
+    uint32_t v2 = (y & 0x000F000Fu) | 0x64006400u;  // (1024 + q2, 1024 + q6)
+    uint32_t v3 = (y & 0x00F000F0u) | 0x54005400u;  // (  64 + q3,   64 + q7)
+    const __half2 q0 = __hsub2(*reinterpret_cast<__half2*>(&v0), k1024);
+    const __half2 q1 = __hsub2(*reinterpret_cast<__half2*>(&v1), k64);
+    const __half2 q2 = __hsub2(*reinterpret_cast<__half2*>(&v2), k1024);
+    const __half2 q3 = __hsub2(*reinterpret_cast<__half2*>(&v3), k64);
+    __half2 d0 = __hfma2(q0, s2, b2), d1 = __hfma2(q1, s2, b2), d2 = __hfma2(q2, s2, b2), d3 = __hfma2(q3, s2, b2);
+    out[i] = make_uint4(*reinterpret_cast<uint32_t*>(&d0), *reinterpret_cast<uint32_t*>(&d1),
+                        *reinterpret_cast<uint32_t*>(&d2), *reinterpret_cast<uint32_t*>(&d3));
+  }
+}
+
+// Dequantise 32 codes (8-bit: 32 bytes) of one row into 4 16-byte fp16 chunks (natural K order).
+__device__ __forceinline__ void dequant32_u8(const uint4 c0, const uint4 c1, __half2 s2, __half2 b2, uint4* out) {
+  const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  const __half2 k1024 = __half2half2(__ushort_as_half(0x6400));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t r[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t x = w[2 * i + h];
+      uint32_t v0 = __byte_perm(x, 0x64646464u, 0x5140);  // (1024 + b0, 1024 + b1)
+      uint32_t v1 = __byte_perm(x, 0x64646464u, 0x5342);  // (1024 + b2, 1024 + b3)
+      __half2 d0 = __hfma2(__hsub2(*reinterpret_cast<__half2*>(&v0), k1024), s2, b2);
+      __half2 d1 = __hfma2(__hsub2(*reinterpret_cast<__half2*>(&v1), k1024), s2, b2);
+      r[2 * h] = *reinterpret_cast<uint32_t*>(&d0);
+      r[2 * h + 1] = *reinterpret_cast<uint32_t*>(&d1);
+    }
+    out[i] = make_uint4(r[0], r[1], r[2], r[3]);
+  }
+}
+
+// ------------------------------------------------------------------ GEMM kernel
+
+template <int MODE, int BITS, int NS>
+__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const GemmSmem L = gemm_smem(MODE, BITS, p.K, p.group, NS);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bar);  // [NS] TMA landed (codes + B)
+  uint64_t* afull = full + NS;                               // [NS] A tile written
+  uint64_t* empty = afull + NS;                              // [NS] MMAs done with the stage
+  uint64_t* scfull = empty + NS;                             // [2] scales of a tile landed
+  uint64_t* scempty = scfull + 2;                            // [2] dequantisers done with them
+  uint64_t* accfull = scempty + 2;                           // [2] accumulator ready
+  uint64_t* accempty = accfull + 2;                          // [2] epilogue done with it
+  uint64_t* drain = accempty + 2;                            // MMA issuer: everything issued has finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int CB = kBK * BITS / 8;          // code bytes per row per k-block
+  const int ng = p.K / p.group;           // groups per row
+  const int nkb = p.K / kBK;              // k-blocks per tile
+  const int MT = (MODE == 0) ? p.I / 64 : p.H / kBM;
+  const int nchunks = *p.nchunks;
+  const int ntiles = nchunks * MT;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&afull[i], 8);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&scfull[i], 1);
+      mbar_init(&scempty[i], 8);
+      mbar_init(&accfull[i], 1);
+      mbar_init(&accempty[i], 4);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, 2 * kAccCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      for (int i = 0; i < 2; ++i) {
+        tc::prefetch_tmap(&p.tm_codes[i]);
+        tc::prefetch_tmap(&p.tm_scales[i]);
+        tc::prefetch_tmap(&p.tm_biases[i]);
+      }
+      int kbg = 0, it = 0;
+      int armed[NS];
+      for (int s = 0; s < NS; ++s) armed[s] = -1;
+      int sc_armed[2] = {-1, -1};
+      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++it) {
+        const int ci = t / MT, mt = t % MT;
+        const int e = p.chunks[3 * ci], start = p.chunks[3 * ci + 1], cnt = p.chunks[3 * ci + 2];
+        const bool shared = (e == p.E);
+        const int ez = shared ? 0 : e;
+        const int mi = shared ? 1 : 0;  // which codes / scales maps
+        const int bi = b_box_index(cnt);
+        const int brows = b_box_rows(bi);
+        // scales and biases of the tile's 128 rows
+        const int tb = it & 1, tu = it >> 1;
+        if (tu >= 1 && !wait_or_abort(&scempty[tb], (tu - 1) & 1, p.hdr, abort, 30)) break;
+        unsigned char* scb = sm + L.sc + tb * L.sc_buf_bytes;
+        const uint32_t half_bytes = 64u * ng * 2u;
+        tc::mbar_expect_tx(&scfull[tb], 4u * half_bytes);
+        const int r0 = (MODE == 0) ? mt * 64 : mt * kBM;
+        const int r1 = (MODE == 0) ? p.rows / 2 + mt * 64 : mt * kBM + 64;
+        tc::tma_load_3d(scb, &p.tm_scales[mi], 0, r0, ez, &scfull[tb]);
+        tc::tma_load_3d(scb + half_bytes, &p.tm_scales[mi], 0, r1, ez, &scfull[tb]);
+        tc::tma_load_3d(scb + 2 * half_bytes, &p.tm_biases[mi], 0, r0, ez, &scfull[tb]);
+        tc::tma_load_3d(scb + 3 * half_bytes, &p.tm_biases[mi], 0, r1, ez, &scfull[tb]);
+        tc::mbar_arrive(&scfull[tb]);
+        sc_armed[tb] = tu;
+        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+          const int s = kbg % NS, u = kbg / NS;
+          if (u >= 1 && !wait_or_abort(&empty[s], (u - 1) & 1, p.hdr, abort, 31)) break;
+          unsigned char* cs = sm + L.codes + s * L.codes_stage_bytes;
+          unsigned char* bs = sm + L.b + s * L.b_stage_bytes;
+          const uint32_t bbytes = static_cast<uint32_t>(brows) * 128u * (MODE == 0 ? 1u : 2u);
+          tc::mbar_expect_tx(&full[s], static_cast<uint32_t>(L.codes_stage_bytes) + bbytes);
+          tc::tma_load_3d(cs, &p.tm_codes[mi], kb * CB, r0, ez, &full[s]);
+          tc::tma_load_3d(cs + 64 * CB, &p.tm_codes[mi], kb * CB, r1, ez, &full[s]);
+          tc::tma_load_2d(bs, &p.tm_b[bi], kb * kBK, start, &full[s]);
+          if (MODE == 1) tc::tma_load_2d(bs + kAccCols * 128, &p.tm_b2[bi], kb * kBK, start, &full[s]);
+          tc::mbar_arrive(&full[s]);
+          armed[s] = u;
+        }
+      }
+      // leave no copy in flight: wait for the last phase armed on every barrier
+      for (int s = 0; s < NS; ++s)
+        if (armed[s] >= 0) mbar_wait(&full[s], armed[s] & 1, p.hdr, 39);
+      for (int b = 0; b < 2; ++b)
+        if (sc_armed[b] >= 0) mbar_wait(&scfull[b], sc_armed[b] & 1, p.hdr, 38);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int kbg = 0, it = 0, last_commit_acc = -1;
+      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++it) {
+        const int ci = t / MT;
+        const int cnt = p.chunks[3 * ci + 2];
+        const int npad = (cnt + 15) & ~15;
+        const uint32_t idesc = tc::idesc_f16_f32(kBM, npad);
+        const int ab = it & 1, au = it >> 1;
+        if (au >= 1 && !wait_or_abort(&accempty[ab], (au - 1) & 1, p.hdr, abort, 40)) break;
+        tc::fence_after_sync();
+        const uint32_t dt = tmem + ab * kAccCols;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+          const int s = kbg % NS, u = kbg / NS;
+          if (!wait_or_abort(&full[s], u & 1, p.hdr, abort, 41) || !wait_or_abort(&afull[s], u & 1, p.hdr, abort, 42)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t a0 = smem_addr(sm + L.a + s * kBM * kBK * 2);
+          const uint32_t b0 = smem_addr(sm + L.b + s * L.b_stage_bytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = tc::smem_desc_sw128(a0 + kk * 32);
+            tc::mma_f16(dt, ad, tc::smem_desc_sw128(b0 + kk * 32), idesc, (kb | kk) != 0);
+            if (MODE == 1) tc::mma_f16(dt, ad, tc::smem_desc_sw128(b0 + kAccCols * 128 + kk * 32), idesc, 1);
+          }
+          tc::commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc::commit(&accfull[ab]);
+        last_commit_acc = it;
+      }
+      // every MMA issued must be finished before TMEM is released
+      (void)last_commit_acc;
+      tc::commit(drain);
+      mbar_wait(drain, 0, p.hdr, 49);
+    }
+  } else if (warp >= kDequantWarp0 && warp < kEpiWarp0) {
+    // ------------------------------------------------ dequantisers: 2 threads per row
+    const int d = threadIdx.x - kDequantWarp0 * 32;  // 0..255
+    const int m = d >> 1, half = d & 1;              // A-tile row, which 32 codes of the 64
+    // A row m <- staging row: gate/up interleaved for mode 0, identity for mode 1
+    const int srow = (MODE == 0) ? ((m & 1) * 64 + (m >> 1)) : m;
+    int kbg = 0, it = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+      if (warp_aborted(abort)) break;
+      const int tb = it & 1, tu = it >> 1;
+      if (!warp_wait(&scfull[tb], tu & 1, p.hdr, abort, 50)) break;
+      const uint16_t* scs = reinterpret_cast<const uint16_t*>(sm + L.sc + tb * L.sc_buf_bytes);
+      const uint16_t* bis = scs + 2 * 64 * ng;
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+        const int s = kbg % NS, u = kbg / NS;
+        if (!warp_wait(&full[s], u & 1, p.hdr, abort, 51)) { ok = false; break; }
+        if (u >= 1 && !warp_wait(&empty[s], (u - 1) & 1, p.hdr, abort, 52)) { ok = false; break; }
+        const int g = (kb * kBK + 32 * half) / p.group;
+        const __half2 s2 = __half2half2(__float2half_rn(bf16_to_f32(scs[srow * ng + g])));
+        const __half2 b2 = __half2half2(__float2half_rn(bf16_to_f32(bis[srow * ng + g])));
+        const unsigned char* crow = sm + L.codes + s * L.codes_stage_bytes + srow * CB + half * (CB / 2);
+        uint4 outv[4];
+        if (BITS == 4) {
+          dequant32_u4(*reinterpret_cast<const uint4*>(crow), s2, b2, outv);
+        } else {
+          dequant32_u8(*reinterpret_cast<const uint4*>(crow), *reinterpret_cast<const uint4*>(crow + 16), s2, b2, outv);
+        }
+        unsigned char* arow = sm + L.a + s * kBM * kBK * 2 + (m >> 3) * 1024 + (m & 7) * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int chunk = half * 4 + q;
+          *reinterpret_cast<uint4*>(arow + ((chunk ^ (m & 7)) << 4)) = outv[q];
+        }
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&afull[s]);
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&scempty[tb]);
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;         // TMEM lane quarter
+    const int m = 32 * q + lane;    // accumulator row held by this thread
+    int it = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+      if (warp_aborted(abort)) break;
+      const int ci = t / MT, mt = t % MT;
+      const int start = p.chunks[3 * ci + 1], cnt = p.chunks[3 * ci + 2];
+      const int ab = it & 1, au = it >> 1;
+      if (!warp_wait(&accfull[ab], au & 1, p.hdr, abort, 60)) break;
+      tc::fence_after_sync();
+      const uint32_t ta = tmem + (static_cast<uint32_t>(32 * q) << 16) + ab * kAccCols;
+      for (int c0 = 0; c0 < cnt; c0 += 32) {
+        uint32_t v[32];
+        tc::tmem_ld32(ta + c0, v);
+        tc::tmem_wait_ld();
+        if (MODE == 0) {
+          // rows 2i (gate) and 2i+1 (up) of intermediate index mt*64 + i
+          const int i = mt * 64 + (m >> 1);
+          const int ip = (BITS == 4) ? ((i & ~7) | perm8_pos(i & 7)) : i;
+#pragma unroll
+          for (int n = 0; n < 32; ++n) {
+            const float a = __uint_as_float(v[n]);
+            const float u = __shfl_xor_sync(0xffffffffu, a, 1);
+            if (!(m & 1) && c0 + n < cnt) {
+              const float h = silu_f(a) * u;
+              const __half hi = __float2half_rn(h);
+              const __half lo = __float2half_rn(h - __half2float(hi));
+              const size_t o = static_cast<size_t>(start + c0 + n) * p.ldh + ip;
+              p.h_hi[o] = __half_as_ushort(hi);
+              p.h_lo[o] = __half_as_ushort(lo);
+            }
+          }
+        } else {
+          const int r = mt * kBM + m;
+#pragma unroll
+          for (int n = 0; n < 32; ++n) {
+            if (c0 + n < cnt) {
+              const int pid = __ldg(p.perm + start + c0 + n);
+              p.out[static_cast<size_t>(pid) * p.H + r] = __uint_as_float(v[n]);
+            }
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&accempty[ab]);
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 2 * kAccCols);
+  }
+}
+
+// ------------------------------------------------------------------ gather, combine
+
+// X16[pos][:] = fp16(x[token(pos)][:]) for every sorted pair, K order permuted for
+// 4-bit codes; gate[t] = sigmoid(x[t] . w_sg) for the shared expert.
+__global__ void __launch_bounds__(256) gather_kernel(BatchParams p) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int npairs = p.T * p.k + (p.Is > 0 ? p.T : 0);
+  for (int pos = warp; pos < npairs; pos += nwarps) {
+    const int pid = p.perm[pos];
+    const int t = (pid < p.T * p.k) ? pid / p.k : pid - p.T * p.k;
+    const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t) * p.H);
+    uint4* dst = reinterpret_cast<uint4*>(p.x16 + static_cast<size_t>(pos) * p.H);
+    for (int s = lane; s < p.H / 8; s += 32) {
+      const uint4 v = xr[s];
+      const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                          bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+      __half o[8];
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) o[p.perm8 ? perm8_pos(kk) : kk] = __float2half_rn(f[kk]);
+      dst[s] = *reinterpret_cast<const uint4*>(o);
+    }
+  }
+  if (p.Is > 0) {
+    for (int t = warp; t < p.T; t += nwarps) {
+      const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t) * p.H);
+      const uint4* wr = reinterpret_cast<const uint4*>(p.wsg);
+      float a = 0.f;
+      for (int s = lane; s < p.H / 8; s += 32) {
+        const uint4 xa = xr[s], wa = wr[s];
+        a = fmaf(bf16_lo(xa.x), bf16_lo(wa.x), a);
+        a = fmaf(bf16_hi(xa.x), bf16_hi(wa.x), a);
+        a = fmaf(bf16_lo(xa.y), bf16_lo(wa.y), a);
+        a = fmaf(bf16_hi(xa.y), bf16_hi(wa.y), a);
+        a = fmaf(bf16_lo(xa.z), bf16_lo(wa.z), a);
+        a = fmaf(bf16_hi(xa.z), bf16_hi(wa.z), a);
+        a = fmaf(bf16_lo(xa.w), bf16_lo(wa.w), a);
+        a = fmaf(bf16_hi(xa.w), bf16_hi(wa.w), a);
+      }
+      a = warp_sum(a);
+      if (lane == 0) p.sgate[t] = 1.f / (1.f + expf(-a));
+    }
+  }
+}
+
+// y[t][r] = bf16( sum_j w[t][j] * O[t*k+j][r] + gate[t] * O[T*k+t][r] ), rank order, shared last.
+__global__ void __launch_bounds__(256) combine_kernel(BatchParams p) {
+  const size_t n = static_cast<size_t>(p.T) * p.H;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>(i / p.H), r = static_cast<int>(i % p.H);
+    float acc = 0.f;
+    for (int j = 0; j < p.k; ++j)
+      acc = fmaf(p.w[static_cast<size_t>(t) * p.k + j], p.o[(static_cast<size_t>(t) * p.k + j) * p.H + r], acc);
+    if (p.Is > 0) acc = fmaf(p.sgate[t], p.o[(static_cast<size_t>(p.T) * p.k + t) * p.H + r], acc);
+    p.y[i] = f32_to_bf16(acc);
+  }
+}
+
+template <int MODE, int BITS, int NS>
+cudaError_t launch_gemm_t(const GemmParams& g, int grid, cudaStream_t st) {
+  const GemmSmem L = gemm_smem(MODE, BITS, g.K, g.group, NS);
+  auto kern = grouped_gemm_kernel<MODE, BITS, NS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, L.total, st>>>(g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t grouped_gemm_smem(int mode, int bits, int K, int group) {
+  return gemm_smem(mode, bits, K, group, mode == 0 ? 4 : 3).total;
+}
+
+cudaError_t launch_grouped_gemm(const GemmParams& g, int mode, int bits, int grid, cudaStream_t st) {
+  if (mode == 0) return bits == 4 ? launch_gemm_t<0, 4, 4>(g, grid, st) : launch_gemm_t<0, 8, 4>(g, grid, st);
+  return bits == 4 ? launch_gemm_t<1, 4, 3>(g, grid, st) : launch_gemm_t<1, 8, 3>(g, grid, st);
+}
+
+cudaError_t launch_gather(const BatchParams& p, int grid, cudaStream_t st) {
+  gather_kernel<<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const BatchParams& p, int grid, cudaStream_t st) {
+  combine_kernel<<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -4,10 +4,13 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <memory>
 #include <mutex>
 #include <string>
+
+#include <cudaTypedefs.h>
 
 #include "moe_b200.h"
 #include "moe_common.cuh"
@@ -39,9 +42,13 @@ size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 // Byte offsets of the workspace regions for T tokens.
 struct Layout {
   size_t hdr, counters, logits, sgate, h, r, xa, xb, y, idx, w;
-  size_t flags, dlogits, dh, dy, dr, dx;  // persistent single-token decode
+  size_t flags, dlogits, dh, dy, dr, dx;                  // persistent single-token decode
+  size_t base_total;                                      // end of the regions above
+  size_t perm, offs, chunks, nchunks, x16, hhi, hlo, o;   // batched tensor-core path
   size_t total;
 };
+
+constexpr int kBatchMinTokens = 8;  // from this many tokens the grouped tensor-core path runs
 
 constexpr int kMaxGrid = 1024;  // barrier flags reserved for the persistent decode grid
 
@@ -67,6 +74,16 @@ Layout layout(const moe_config& c, int64_t T) {
   L.dy = o;       o += up(static_cast<size_t>(c.hidden) * 2);
   L.dr = o;       o += up(static_cast<size_t>(c.hidden) * 4);
   L.dx = o;       o += up(static_cast<size_t>(c.hidden) * 2);
+  L.base_total = o;
+  const size_t np = static_cast<size_t>(T) * (c.top_k + 1);
+  L.perm = o;     o += up(np * 4);
+  L.offs = o;     o += up(static_cast<size_t>(c.num_experts + 2) * 4);
+  L.chunks = o;   o += up((static_cast<size_t>(c.num_experts) + 2 + np / moe::kChunkTokens + 1) * 12);
+  L.nchunks = o;  o += up(4);
+  L.x16 = o;      o += up(np * c.hidden * 2);
+  L.hhi = o;      o += up(np * imax * 2);
+  L.hlo = o;      o += up(np * imax * 2);
+  L.o = o;        o += up(np * c.hidden * 4);
   L.total = o;
   return L;
 }
@@ -190,6 +207,161 @@ moe_status ffn(const moe_config& c, const moe_layer_weights& wt, const uint16_t*
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "expert_ffn launch");
 }
 
+// ---------------------------------------------------------------- batched tensor-core path
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::call_once(g_encode_once, []() {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// 3D map over E matrices [rows][inner] (inner contiguous, `esize` bytes per element),
+// box = (box_inner, 64 rows, 1 expert).
+bool map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int64_t inner, int64_t rows,
+            int64_t E, int64_t expert_stride_bytes, int box_inner) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(E)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner * esize), static_cast<cuuint64_t>(expert_stride_bytes)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 64u, 1u};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  return encode_fn()(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2D fp16 map over [rows][K] with a (64 x box_rows) box in the 128-byte swizzle.
+bool map_b(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * 2)};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1u, 1u};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return n;
+}
+
+bool batched_eligible(const moe_config& c, int T) {
+  if (T < kBatchMinTokens) return false;
+  if (c.shared_inter != 0 && c.shared_inter != c.inter) return false;
+  if ((c.hidden / c.group) % 8 || (c.inter / c.group) % 8 || c.hidden % 128 || c.inter % 64) return false;
+  if (!encode_fn()) return false;
+  int dev = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return false;
+  const size_t need = std::max(moe::grouped_gemm_smem(0, c.bits, c.hidden, c.group),
+                               moe::grouped_gemm_smem(1, c.bits, c.inter, c.group));
+  return need <= static_cast<size_t>(optin);
+}
+
+// Experts' gate/up and down for T tokens given their selection, on the tensor cores.
+moe_status batched_ffn(const moe_config& c, const moe_layer_weights& wt, const uint16_t* x, int T, const int32_t* idx,
+                       const float* w, uint16_t* y, void* ws, const Layout& Ly, cudaStream_t st) {
+  char* b = static_cast<char*>(ws);
+  const moe::WsView v = view(ws, Ly);
+  const int H = c.hidden, I = c.inter, k = c.top_k, E = c.num_experts;
+  const bool shared = c.shared_inter > 0;
+  const int np = T * k + (shared ? T : 0);
+  int32_t* perm = reinterpret_cast<int32_t*>(b + Ly.perm);
+  int32_t* offs = reinterpret_cast<int32_t*>(b + Ly.offs);
+  int32_t* chunks = reinterpret_cast<int32_t*>(b + Ly.chunks);
+  int32_t* nchunks = reinterpret_cast<int32_t*>(b + Ly.nchunks);
+  uint16_t* x16 = reinterpret_cast<uint16_t*>(b + Ly.x16);
+  uint16_t* hhi = reinterpret_cast<uint16_t*>(b + Ly.hhi);
+  uint16_t* hlo = reinterpret_cast<uint16_t*>(b + Ly.hlo);
+  float* o = reinterpret_cast<float*>(b + Ly.o);
+  const int sms = device_sms();
+  if (sms < 1) return fail(MOE_ERR_CUDA, "no device");
+
+  moe::SortParams sp{idx, T, k, E, shared ? 1 : 0, perm, offs, chunks, nchunks, moe::kChunkTokens, v.hdr};
+  cudaError_t e = moe::launch_sort_by_expert(sp, st);
+  if (e != cudaSuccess) return cuda_fail(e, "sort launch");
+  moe::BatchParams bp{};
+  bp.x = x;
+  bp.wsg = wt.shared_gate_w;
+  bp.perm = perm;
+  bp.T = T;
+  bp.k = k;
+  bp.H = H;
+  bp.Is = c.shared_inter;
+  bp.perm8 = (c.bits == 4) ? 1 : 0;
+  bp.x16 = x16;
+  bp.sgate = v.sgate;
+  bp.w = w;
+  bp.o = o;
+  bp.y = y;
+  if ((e = moe::launch_gather(bp, sms * 4, st)) != cudaSuccess) return cuda_fail(e, "gather launch");
+
+  auto gp = std::make_unique<moe::GemmParams>();
+  const int bits = c.bits, g = c.group;
+  const moe_qtensor& sgu = shared ? wt.shared_gate_up : wt.gate_up;
+  const moe_qtensor& sdn = shared ? wt.shared_down : wt.down;
+  // gate/up: K = H, rows = 2I
+  bool ok = map_3d(&gp->tm_codes[0], wt.gate_up.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H * bits / 8, 2 * I, E,
+                   wt.gate_up.q_expert_stride, 64 * bits / 8) &&
+            map_3d(&gp->tm_codes[1], sgu.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H * bits / 8, 2 * I, 1,
+                   static_cast<int64_t>(2) * I * H * bits / 8, 64 * bits / 8) &&
+            map_3d(&gp->tm_scales[0], wt.gate_up.scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, H / g, 2 * I, E,
+                   wt.gate_up.sb_expert_stride * 2, H / g) &&
+            map_3d(&gp->tm_scales[1], sgu.scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, H / g, 2 * I, 1,
+                   static_cast<int64_t>(2) * I * (H / g) * 2, H / g) &&
+            map_3d(&gp->tm_biases[0], wt.gate_up.biases, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, H / g, 2 * I, E,
+                   wt.gate_up.sb_expert_stride * 2, H / g) &&
+            map_3d(&gp->tm_biases[1], sgu.biases, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, H / g, 2 * I, 1,
+                   static_cast<int64_t>(2) * I * (H / g) * 2, H / g);
+  for (int i = 0; i < 4 && ok; ++i) ok = map_b(&gp->tm_b[i], x16, H, np, 16 << i) && map_b(&gp->tm_b2[i], x16, H, np, 16 << i);
+  if (!ok) return fail(MOE_ERR_CUDA, "tensor map encoding failed (gate/up)");
+  gp->chunks = chunks;
+  gp->nchunks = nchunks;
+  gp->perm = perm;
+  gp->K = H;
+  gp->rows = 2 * I;
+  gp->I = I;
+  gp->H = H;
+  gp->E = E;
+  gp->group = g;
+  gp->ldh = I;
+  gp->h_hi = hhi;
+  gp->h_lo = hlo;
+  gp->out = o;
+  gp->hdr = v.hdr;
+  if ((e = moe::launch_grouped_gemm(*gp, 0, bits, sms, st)) != cudaSuccess) return cuda_fail(e, "gate/up GEMM launch");
+  // down: K = I, rows = H
+  ok = map_3d(&gp->tm_codes[0], wt.down.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, I * bits / 8, H, E,
+              wt.down.q_expert_stride, 64 * bits / 8) &&
+       map_3d(&gp->tm_codes[1], sdn.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, I * bits / 8, H, 1,
+              static_cast<int64_t>(H) * I * bits / 8, 64 * bits / 8) &&
+       map_3d(&gp->tm_scales[0], wt.down.scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, I / g, H, E,
+              wt.down.sb_expert_stride * 2, I / g) &&
+       map_3d(&gp->tm_scales[1], sdn.scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, I / g, H, 1,
+              static_cast<int64_t>(H) * (I / g) * 2, I / g) &&
+       map_3d(&gp->tm_biases[0], wt.down.biases, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, I / g, H, E,
+              wt.down.sb_expert_stride * 2, I / g) &&
+       map_3d(&gp->tm_biases[1], sdn.biases, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, I / g, H, 1,
+              static_cast<int64_t>(H) * (I / g) * 2, I / g);
+  for (int i = 0; i < 4 && ok; ++i) ok = map_b(&gp->tm_b[i], hhi, I, np, 16 << i) && map_b(&gp->tm_b2[i], hlo, I, np, 16 << i);
+  if (!ok) return fail(MOE_ERR_CUDA, "tensor map encoding failed (down)");
+  gp->K = I;
+  gp->rows = H;
+  if ((e = moe::launch_grouped_gemm(*gp, 1, bits, sms, st)) != cudaSuccess) return cuda_fail(e, "down GEMM launch");
+  if ((e = moe::launch_combine(bp, sms * 4, st)) != cudaSuccess) return cuda_fail(e, "combine launch");
+  return MOE_OK;
+}
+
 // Device facts the persistent decode needs, looked up once per device.
 struct DevInfo {
   bool ok = false;
@@ -296,6 +468,7 @@ int32_t moe_stack_kernel_launches(const moe_config* cfg, int32_t T, int32_t L) {
   int grid = 0;
   if (T == 1 && decode_eligible(*cfg, &grid))
     return (L + moe::kMaxDecodeLayers - 1) / moe::kMaxDecodeLayers;
+  if (batched_eligible(*cfg, T)) return 1 + 7 * L;  // route, sort, gather, 2 GEMMs, combine, glue
   return 1 + 4 * L;
 }
 
@@ -342,6 +515,8 @@ moe_status moe_expert_ffn(const moe_config* cfg, const moe_layer_weights* w, con
     return s;
   Layout L;
   if ((s = check_ws(*cfg, ws, ws_bytes, T, &L))) return s;
+  if (batched_eligible(*cfg, T))
+    return batched_ffn(*cfg, *w, x, T, topk_idx, topk_w, y, ws, L, reinterpret_cast<cudaStream_t>(stream));
   return ffn(*cfg, *w, x, T, topk_idx, topk_w, y, view(ws, L), reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -364,6 +539,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, 
   const moe::WsView v = view(ws, L);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if ((s = route(*cfg, x, T, w->router_w, w->router_bias, idx, wt, v, st))) return s;
+  if (batched_eligible(*cfg, T)) return batched_ffn(*cfg, *w, x, T, idx, wt, y, ws, L, st);
   return ffn(*cfg, *w, x, T, idx, wt, y, v, st);
 }
 
@@ -388,6 +564,7 @@ moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weights* lay
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int grid = 0;
   if (T == 1 && decode_eligible(*cfg, &grid)) return stack_decode(*cfg, layers, L, x0, x_out, trace, ws, Ly, grid, st);
+  const bool batched = batched_eligible(*cfg, T);
   const size_t TH = static_cast<size_t>(T) * cfg->hidden;
   const size_t Tk = static_cast<size_t>(T) * cfg->top_k;
   float* r = reinterpret_cast<float*>(b + Ly.r);
@@ -406,7 +583,9 @@ moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weights* lay
     float* wt = (trace && trace->w) ? trace->w + l * Tk : reinterpret_cast<float*>(b + Ly.w);
     uint16_t* y = (trace && trace->y) ? trace->y + l * TH : reinterpret_cast<uint16_t*>(b + Ly.y);
     if ((s = route(*cfg, xcur, T, layers[l].router_w, layers[l].router_bias, idx, wt, v, st))) return s;
-    if ((s = ffn(*cfg, layers[l], xcur, T, idx, wt, y, v, st))) return s;
+    if (batched) s = batched_ffn(*cfg, layers[l], xcur, T, idx, wt, y, ws, Ly, st);
+    else s = ffn(*cfg, layers[l], xcur, T, idx, wt, y, v, st);
+    if (s) return s;
     uint16_t* xnext;
     if (l == L - 1) xnext = x_out;
     else if (trace && trace->x) xnext = trace->x + (l + 1) * TH;
@@ -428,7 +607,7 @@ moe_status moe_sort_by_expert(const moe_config* cfg, const int32_t* topk_idx, in
   Layout L;
   if ((s = check_ws(*cfg, ws, ws_bytes, T, &L))) return s;
   moe::SortParams p{topk_idx, T, cfg->top_k, cfg->num_experts, cfg->shared_inter > 0 ? 1 : 0, perm, offsets,
-                    view(ws, L).hdr};
+                    nullptr, nullptr, 0, view(ws, L).hdr};
   cudaError_t e = moe::launch_sort_by_expert(p, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "sort_by_expert launch");
 }
@@ -524,8 +703,8 @@ extern "C" moe_status moe_layer_forward_static(const moe_config* cfg, const moe_
       (device_status && !aligned(device_status, 4)))
     return fail(MOE_ERR_INVALID_ARG, "topk_idx/topk_w/device_status misaligned");
   const Layout L = layout(*cfg, T);
-  if (L.total > kStaticScratchBytes)
-    return fail(MOE_ERR_WORKSPACE, "T=%d needs %zu bytes of scratch; the static scratch holds %zu", T, L.total,
+  if (L.base_total > kStaticScratchBytes)
+    return fail(MOE_ERR_WORKSPACE, "T=%d needs %zu bytes of scratch; the static scratch holds %zu", T, L.base_total,
                 kStaticScratchBytes);
   void* ws = nullptr;
   if ((s = static_scratch(&ws))) return s;

@@ -2,6 +2,7 @@
 // kernels. Parameter blocks are passed by value to the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -55,6 +56,41 @@ struct SortParams {
   int T, k, E, with_shared;
   int32_t* perm;         // [T*k (+T)]
   int32_t* offsets;      // [E+1 (+1)]
+  int32_t* chunks;       // optional [max][3]: expert, first sorted position, pair count (<= chunk_tokens)
+  int32_t* nchunks;      // optional scalar
+  int chunk_tokens;
+  WsHeader* hdr;
+};
+
+constexpr int kChunkTokens = 128;  // pairs per GEMM chunk (the MMA N dimension)
+
+// Batched path: gather of the sorted pairs' activations and the final combine.
+struct BatchParams {
+  const uint16_t* x;     // bf16 [T][H]
+  const uint16_t* wsg;   // bf16 [H] shared-expert gate vector (when Is > 0)
+  const int32_t* perm;   // [npairs] sorted position -> pair id
+  int T, k, H, Is, perm8;
+  uint16_t* x16;         // fp16 [npairs][H], K permuted in blocks of 8 when perm8
+  float* sgate;          // [T]
+  const float* w;        // [T][k] routing weights
+  const float* o;        // fp32 [npairs by pair id][H] expert outputs
+  uint16_t* y;           // bf16 [T][H]
+};
+
+// One grouped GEMM launch (gate/up + SwiGLU, or down) over expert chunks.
+struct GemmParams {
+  CUtensorMap tm_codes[2];   // 3D codes maps: [0] routed experts, [1] shared expert
+  CUtensorMap tm_scales[2];
+  CUtensorMap tm_biases[2];
+  CUtensorMap tm_b[4];       // B operand [npairs][K] fp16, box rows 16/32/64/128, 128-byte swizzle
+  CUtensorMap tm_b2[4];      // second B operand (h lo) of the down GEMM
+  const int32_t* chunks;
+  const int32_t* nchunks;
+  const int32_t* perm;
+  int K, rows, I, H, E, group, ldh;
+  uint16_t* h_hi;            // gate/up output [npairs][ldh] fp16 hi / lo
+  uint16_t* h_lo;
+  float* out;                // down output [pair id][H] fp32
   WsHeader* hdr;
 };
 
@@ -86,7 +122,7 @@ struct DecodeParams {
   float* logits;         // fp32 [E+1] (workspace)
   float* hbuf;           // fp32 [k+1][Imax] (workspace)
   uint16_t* ybuf;        // bf16 [H] (workspace)
-  unsigned* flags;       // [grid] barrier flags, zero at launch (workspace)
+  unsigned* flags;       // grid barrier counter, zero at launch (workspace)
   WsHeader* hdr;
   LayerDesc layers[kMaxDecodeLayers];
 };
@@ -95,6 +131,11 @@ cudaError_t launch_route_topk(const RouteParams& p, cudaStream_t stream);
 cudaError_t launch_expert_ffn(const FfnParams& p, int bits, cudaStream_t stream);
 cudaError_t launch_glue(const GlueParams& p, cudaStream_t stream);
 cudaError_t launch_sort_by_expert(const SortParams& p, cudaStream_t stream);
+
+size_t grouped_gemm_smem(int mode, int bits, int K, int group);
+cudaError_t launch_grouped_gemm(const GemmParams& g, int mode, int bits, int grid, cudaStream_t st);
+cudaError_t launch_gather(const BatchParams& p, int grid, cudaStream_t st);
+cudaError_t launch_combine(const BatchParams& p, int grid, cudaStream_t st);
 
 bool decode_stack_supported(int H, int E, int k, int I, int Is, int group, int bits);
 size_t decode_stack_smem(int H, int E, int k, int I, int Is, int group, int bits, int grid);

@@ -55,6 +55,32 @@ __global__ void __launch_bounds__(kThreads) sort_by_expert_kernel(SortParams p) 
       run += c;
     }
     if (lane == 31) p.offsets[nbins] = incl;
+    if (p.chunks) {
+      // GEMM work list: every expert's run of pairs cut into chunks of <= chunk_tokens
+      __syncwarp();
+      int nloc = 0;
+      for (int b = b0; b < b1; ++b) {
+        const int cnt = (b + 1 < nbins ? sh[b + 1] : incl) - sh[b];
+        nloc += (cnt + p.chunk_tokens - 1) / p.chunk_tokens;
+      }
+      int cin = nloc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, cin, o);
+        if (lane >= o) cin += v;
+      }
+      int ci = cin - nloc;
+      for (int b = b0; b < b1; ++b) {
+        const int first = sh[b];
+        const int cnt = (b + 1 < nbins ? sh[b + 1] : incl) - first;
+        for (int s0 = 0; s0 < cnt; s0 += p.chunk_tokens, ++ci) {
+          p.chunks[3 * ci] = b;
+          p.chunks[3 * ci + 1] = first + s0;
+          p.chunks[3 * ci + 2] = min(p.chunk_tokens, cnt - s0);
+        }
+      }
+      if (lane == 31) *p.nchunks = cin;
+    }
   }
   __syncthreads();
   if (threadIdx.x >= 32) return;

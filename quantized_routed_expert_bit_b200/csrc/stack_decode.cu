@@ -90,47 +90,35 @@ __device__ __forceinline__ void copy_tx(void* dst, const void* src, uint32_t byt
   bulk_g2s(dst, src, bytes, bar);
 }
 
-__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void fence_acq_rel() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-
 __device__ __forceinline__ float silu_f(float z) { return z / (1.f + expf(-z)); }
 
 // All CTAs reach `epoch`. Returns false if this CTA must stop (a wait ran
-// out here or elsewhere).
+// out here or elsewhere). One counter in global memory: every CTA adds 1
+// with release semantics after __syncthreads; thread 0 alone polls it with
+// acquire loads and a short sleep, so the barrier puts almost no load on the
+// L2 slice that holds it.
 __device__ bool grid_barrier(const DecodeParams& p, unsigned epoch, volatile int* s_abort) {
   __syncthreads();
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    if (lane == 0) {
-      __threadfence();
-      st_release(p.flags + blockIdx.x, epoch);
-    }
-    __syncwarp();
+  if (threadIdx.x == 0) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.flags) : "memory");
+    const unsigned target = epoch * gridDim.x;
     bool ok = false;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0; it < kWaitIters; ++it) {
-      bool mine = true;
-      for (int i = lane; i < (int)gridDim.x; i += 32) mine &= (ld_relaxed(p.flags + i) >= epoch);
-      if (__all_sync(0xffffffffu, mine)) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.flags) : "memory");
+      if (v >= target) {
         ok = true;
         break;
       }
-      if ((it & 31u) == 0) {
+      __nanosleep(32);
+      if ((it & 15u) == 0) {
         const int st = *reinterpret_cast<volatile int*>(&p.hdr->status);
         if (st != 0 || globaltimer_ns() - t0 > kWaitNs) break;
       }
     }
-    fence_acq_rel();
-    if (!ok && lane == 0) {
+    __threadfence();
+    if (!ok) {
       report(p.hdr, MOE_ERR_TIMEOUT, 1000 + static_cast<int>(epoch));
       *s_abort = 1;
     }

@@ -134,3 +134,15 @@ def gap_filtered_tokens(shape: synth.MoEShape, layer: oracle.HostLayer, n: int, 
             ids.append(i)
         i += 1
     return ids, synth.make_tokens(shape, ids, device)
+
+
+def oracle_ffn_given_selection(layer: oracle.HostLayer, x_bits_row, idx_row, w_row, threads: int = 4):
+    """Oracle expert part for one token under a given selection and weights
+    (as moe_expert_ffn receives them): returns the oracle dict for y."""
+    mats = [layer.expert(int(e)) for e in idx_row]
+    sgu, sdn = layer.shared()
+    gate = oracle.shared_gate(x_bits_row, layer.shared_gate_w) if sgu is not None else 0.0
+    y64, y32, y16 = oracle.moe_token(layer.H, layer.I, layer.Is, layer.bits, layer.group, x_bits_row,
+                                     [m[0] for m in mats], [m[1] for m in mats],
+                                     np.asarray(w_row, dtype=np.float64), sgu, sdn, gate, threads)
+    return dict(y64=y64[None], y32=y32[None], y16=y16[None])
