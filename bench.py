@@ -52,6 +52,27 @@ def touched_bytes_per_token(shape: synth.MoEShape) -> int:
     return per_layer * shape.layers
 
 
+def touched_bytes_batched(shape, layers_dev, tokens, T, steps):
+    """Algorithmic bytes of a batched step: per layer every distinct expert the
+    batch selects (read once), the shared expert, the router and w_sg. The
+    selection is recomputed per layer on the host side from the library's
+    own routing of the stack (trace), averaged over the timed steps."""
+    cfg = moe.make_config(shape)
+    ws = moe.Workspace(cfg, T, L=shape.layers)
+    arr = moe.make_layer_array([moe.make_layer_weights(lw) for lw in layers_dev])
+    ti = torch.empty(shape.layers, T, shape.top_k, dtype=torch.int32, device="cuda")
+    xo = torch.empty(T, shape.hidden, dtype=torch.bfloat16, device="cuda")
+    distinct = 0
+    for s in range(steps):
+        tr = moe.Trace(0, ti.data_ptr(), 0, 0, 0)
+        moe.moe_stack_forward(cfg, arr, tokens[s * T:(s + 1) * T], xo, ws, trace=tr)
+        torch.cuda.synchronize()
+        for l in range(shape.layers):
+            distinct += int(torch.unique(ti[l]).numel())
+    per_layer_fixed = shape.expert_bytes(shape.shared_inter) + shape.num_experts * shape.hidden * 2 + shape.hidden * 2
+    return (distinct / steps) * shape.expert_bytes() + shape.layers * per_layer_fixed
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -208,10 +229,10 @@ def run_reference(args):
 
 
 def workload_config(shape):
-    return {"workload": f"{shape.name}: decode T=1 through {shape.layers} stacked MoE layers "
+    return {"workload": f"{shape.name}: T={shape.tokens} through {shape.layers} stacked MoE layers "
                         f"(H={shape.hidden}, E={shape.num_experts}, top-{shape.top_k}, I=Is={shape.inter}, "
                         f"{shape.bits}-bit affine g{shape.group}, bf16 scale/bias, packed gate/up)",
-            "tokens_per_step": 1, "layers": shape.layers,
+            "tokens_per_step": shape.tokens, "layers": shape.layers,
             "l2": f"inputs larger than L2: {shape.layers * shape.num_experts * shape.expert_bytes() / 1e9:.1f} GB "
                   "resident expert stack, a new token (new experts) every step"}
 
@@ -224,7 +245,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0,
-                    help="profile a shorter stack (small ncu case); the default is the full 40 layers")
+                    help="profile a shorter stack (small ncu case); the default is the full stack")
+    ap.add_argument("--workload", default=SHAPE_KEY, choices=sorted(synth.SHAPES),
+                    help="35b (default, the headline), 80b, 35b8, or the batched 35b_t64 / 35b_t512")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -234,24 +257,30 @@ def main():
 
     dist, rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
-    shape = synth.SHAPES[SHAPE_KEY]
+    key = args.workload
+    shape = synth.SHAPES[key]
     if args.layers:
         import dataclasses
         shape = dataclasses.replace(shape, layers=args.layers, name=shape.name + f"-first{args.layers}")
     cfg = moe.make_config(shape)
-    layers = [synth.make_layer(shape, l, "cuda", seed_id=synth.SHAPE_SEED_ID[SHAPE_KEY])
+    layers = [synth.make_layer(shape, l, "cuda", seed_id=synth.SHAPE_SEED_ID[key])
               for l in range(shape.layers)]
     arr = moe.make_layer_array([moe.make_layer_weights(lw) for lw in layers])
-    ws = moe.Workspace(cfg, 1, L=shape.layers)
+    T = shape.tokens
+    ws = moe.Workspace(cfg, T, L=shape.layers)
     nsteps = args.warmup + args.steps
-    # each rank its own tokens (independent replicas)
-    tokens = synth.make_tokens(shape, [rank * 100000 + i for i in range(nsteps)], "cuda",
-                               seed_id=synth.SHAPE_SEED_ID[SHAPE_KEY])
-    xout = torch.empty(1, shape.hidden, dtype=torch.bfloat16, device="cuda")
+    # each rank its own tokens (independent replicas); a step is one batch of T tokens
+    if T == 1:
+        tokens = synth.make_tokens(shape, [rank * 100000 + i for i in range(nsteps)], "cuda",
+                                   seed_id=synth.SHAPE_SEED_ID[key])
+    else:
+        tokens = torch.cat([synth.make_batch(shape, T, rank * 100000 + i, "cuda", seed_id=synth.SHAPE_SEED_ID[key])
+                            for i in range(nsteps)])
+    xout = torch.empty(T, shape.hidden, dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step(i):
-        moe.moe_stack_forward(cfg, arr, tokens[i:i + 1], xout, ws, stream=stream)
+        moe.moe_stack_forward(cfg, arr, tokens[i * T:(i + 1) * T], xout, ws, stream=stream)
 
     for i in range(args.warmup):
         step(i)
@@ -277,32 +306,35 @@ def main():
 
     # ---- end to end: host tokens in pinned memory, result read back every step
     host_tok = tokens.cpu().pin_memory()
-    host_out = torch.empty(1, shape.hidden, dtype=torch.bfloat16).pin_memory()
-    xin = torch.empty(1, shape.hidden, dtype=torch.bfloat16, device="cuda")
+    host_out = torch.empty(T, shape.hidden, dtype=torch.bfloat16).pin_memory()
+    xin = torch.empty(T, shape.hidden, dtype=torch.bfloat16, device="cuda")
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     e0.record(stream)
     for i in range(args.warmup, nsteps):
-        xin.copy_(host_tok[i:i + 1], non_blocking=True)
+        xin.copy_(host_tok[i * T:(i + 1) * T], non_blocking=True)
         moe.moe_stack_forward(cfg, arr, xin, xout, ws, stream=stream)
         host_out.copy_(xout, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = barrier_max(dist, e0.elapsed_time(e1))
 
-    launches_per_step = moe.moe_stack_kernel_launches(cfg, 1, shape.layers)
+    launches_per_step = moe.moe_stack_kernel_launches(cfg, T, shape.layers)
     persistent = launches_per_step < shape.layers
-    bytes_tok = touched_bytes_per_token(shape)
-    total_tokens = args.steps * world
+    if T == 1:
+        bytes_step = touched_bytes_per_token(shape)
+    else:
+        bytes_step = touched_bytes_batched(shape, layers, tokens[args.warmup * T:nsteps * T], T, args.steps)
+    total_tokens = args.steps * world * T
     tok_s = total_tokens / (ms / 1e3)
     per_step_s = ms / 1e3 / args.steps
-    gbs = bytes_tok / per_step_s / 1e9
+    gbs = bytes_step / per_step_s / 1e9
     peak, peak_src = peaks()
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and T == 1:
         threads = min(os.cpu_count() or 1, shape.top_k + 1)  # one expert per thread
         v, evals, dt = cpu_oracle_tokens_per_s(shape, layers, tokens, threads)
         cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -321,12 +353,12 @@ def main():
                                     else "moe_stack_forward step (router, gate/up, down, glue kernels)"),
                          "achieved": gbs, "peak": peak, "peak_source": peak_src, "unit": "GB/s",
                          "frac": gbs / peak, "traffic": None,
-                         "bytes_per_launch": bytes_tok,
+                         "bytes_per_step": bytes_step,
                          "note": "achieved = algorithmic bytes per step / device time per step (CUDA events "
                                  "on the launch stream around the timed steps)"},
             "cpu_baseline": cpu,
             "e2e": {"value": total_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": shape.hidden * 2, "d2h_bytes_per_step": shape.hidden * 2},
+                    "h2d_bytes_per_step": T * shape.hidden * 2, "d2h_bytes_per_step": T * shape.hidden * 2},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "device_status": moe.status_string(status),

@@ -6,11 +6,12 @@
 //   gather   x (bf16) of every (token, expert) pair, in expert order, as
 //            fp16 rows: the B operand of the gate/up GEMM; also the shared
 //            expert's sigmoid gate per token;
-//   GEMM gu  per (expert chunk of <=128 pairs, 64 intermediate indices):
-//            A = the 64 gate rows and 64 up rows, dequantised in shared
-//            memory to fp16, B = the chunk's gathered tokens; epilogue
-//            h = silu(gate) * up, stored as an fp16 hi/lo pair;
-//   GEMM dn  per (expert chunk, 128 output rows): A = down rows dequantised,
+//   GEMM gu  per (expert chunk of <=64 pairs, 64 intermediate indices):
+//            A = the integer codes of the 64 gate rows and 64 up rows, as
+//            exact fp16 integers, B = the chunk's gathered tokens; epilogue
+//            h = silu(gate) * up, stored as an fp16 hi/lo pair, plus the
+//            sum of h over each group of 64 intermediate indices;
+//   GEMM dn  per (expert chunk, 128 output rows): A = the down rows' codes,
 //            B = h hi and h lo (two MMAs, so h keeps ~22 bits); epilogue
 //            writes each pair's output row (fp32);
 //   combine  y = sum_j w_j o_j + sigmoid-gate * o_shared, in rank order,
@@ -22,18 +23,24 @@
 // GEMM CTA (one per SM, persistent over tiles), 16 warps:
 //   warp 0      TMA producer: codes (3D map over the expert stack), scales
 //               and biases (per tile), B tiles (128-byte swizzled);
-//   warp 1      TMEM owner; lane 0 issues tcgen05.mma (M=128, N=16..128, K=16);
-//   warps 4-11  dequantisers: codes -> fp16 A tiles in the swizzled layout;
-//   warps 12-15 epilogue: TMEM -> registers -> global.
-// A stage ring of NS k-blocks (64 K each) decouples the roles; every wait
-// is bounded and an abort drains copies and MMAs before TMEM is freed.
+//   warp 1      TMEM owner; lane 0 issues tcgen05.mma (M=128, N=16..64, K=16);
+//   warps 4-11  unpack codes into exact fp16 integers, swizzled A tiles;
+//   warps 12-15 scale and accumulate, then the epilogue.
+// The weight of code q in group g is s*q + b (MLX-style affine groups), so
+// a row's dot product with a column x is  sum_g ( s_g * P_g + b_g * X_g ),
+// P_g = sum_{k in g} q_k x_k,  X_g = sum_{k in g} x_k.  One k-block is one
+// group of 64: the tensor cores form P_g from exact integer codes and exact
+// fp16 activations with fp32 accumulation, each group into its own TMEM
+// buffer (4 in rotation), and the scaling warps add s_g * P_g + b_g * X_g
+// into fp32 registers. No weight is ever rounded to 16 bits. A stage ring
+// of NS k-blocks decouples the roles; every wait is bounded and an abort
+// drains copies and MMAs before TMEM is freed.
 //
-// Dequantisation: w = s*q + b rounded once to fp16. 4-bit codes become fp16
-// (1024 + q) / (64 + q) by one lop3 per pair of codes; subtracting the
-// offset is exact; one fp16 fma applies scale and bias. For 4-bit the pairs
-// come out as (k, k+4) within each 8 codes, so the A tile holds K in the
-// order 0,4,1,5,2,6,3,7 inside every 8; the B operands (gathered x, h) are
-// written in the same order (the dot product does not depend on the order).
+// Unpacking: 4-bit codes become fp16 (1024 + q) / (64 + q) by one lop3 per
+// pair of codes and subtracting the offset gives q exactly. The pairs come
+// out as (k, k+4) within each 8 codes, so the A tile holds K in the order
+// 0,4,1,5,2,6,3,7 inside every 8; the B operands (gathered x, h) are
+// written in the same order (a dot product does not depend on the order).
 
 #include <cuda_fp16.h>
 
@@ -47,10 +54,11 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kBM = 128;           // tile rows
-constexpr int kBK = 64;            // K per k-block (128 bytes of fp16: one swizzle row)
+constexpr int kBK = 64;            // K per k-block: one quantisation group, one 128-byte swizzle row
+constexpr int kNT = kChunkTokens;  // columns (pairs) per tile
+constexpr int kPBuf = 4;           // TMEM buffers of per-group products in rotation
 constexpr int kDequantWarp0 = 4;   // warps 4..11
 constexpr int kEpiWarp0 = 12;      // warps 12..15
-constexpr int kAccCols = 128;      // TMEM columns per accumulator buffer
 
 __host__ __device__ constexpr uint32_t al1k(uint32_t v) { return (v + 1023u) & ~1023u; }
 
@@ -60,7 +68,7 @@ __host__ __device__ constexpr int perm8_pos(int k) {  // position of element k
 }
 
 struct GemmSmem {
-  uint32_t a, b, codes, sc, bar, total;
+  uint32_t a, b, codes, sc, xs, bar, total;
   int ns, b_stage_bytes, codes_stage_bytes, sc_buf_bytes;
 };
 
@@ -68,20 +76,21 @@ __host__ __device__ inline GemmSmem gemm_smem(int mode, int bits, int K, int gro
   GemmSmem s{};
   s.ns = ns;
   const int ng = K / group;
-  s.b_stage_bytes = (mode == 0 ? 1 : 2) * kAccCols * 128;  // up to 128 rows x 128 B (x2: h hi and lo)
+  s.b_stage_bytes = (mode == 0 ? 1 : 2) * kNT * 128;  // up to kNT rows x 128 B (x2: h hi and lo)
   s.codes_stage_bytes = kBM * (kBK * bits / 8);
-  s.sc_buf_bytes = 2 * kBM * ng * 2;                         // scales and biases of 128 rows
+  s.sc_buf_bytes = 2 * kBM * ng * 2;                    // scales and biases of 128 rows
   uint32_t o = 0;
   s.a = o;     o = al1k(o + ns * kBM * kBK * 2);
   s.b = o;     o = al1k(o + ns * s.b_stage_bytes);
   s.codes = o; o = al1k(o + ns * s.codes_stage_bytes);
   s.sc = o;    o = al1k(o + 2 * s.sc_buf_bytes);
+  s.xs = o;    o = al1k(o + 4 * ng * kNT * 4);          // group sums of the tile's columns, one copy per scaling warp
   s.bar = o;   o += 256;
   s.total = o + 1024;  // slack to align the dynamic base to 1 KiB
   return s;
 }
 
-__device__ __forceinline__ int b_box_index(int n) { return n <= 16 ? 0 : n <= 32 ? 1 : n <= 64 ? 2 : 3; }
+__device__ __forceinline__ int b_box_index(int n) { return n <= 16 ? 0 : n <= 32 ? 1 : 2; }
 __device__ __forceinline__ int b_box_rows(int i) { return 16 << i; }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.f + expf(-z)); }
@@ -115,8 +124,8 @@ __device__ __forceinline__ bool warp_aborted(volatile int* abort) {
   return __shfl_sync(0xffffffffu, ((threadIdx.x & 31) == 0) ? *abort : 0, 0) != 0;
 }
 
-// Dequantise 32 codes (4-bit: 16 bytes) of one row into 4 swizzled 16-byte fp16 chunks.
-__device__ __forceinline__ void dequant32_u4(const uint4 c, __half2 s2, __half2 b2, uint4* out) {
+// 32 4-bit codes (16 bytes) of one row -> 4 16-byte chunks of exact fp16 integers.
+__device__ __forceinline__ void unpack32_u4(const uint4 c, uint4* out) {
   const uint32_t w[4] = {c.x, c.y, c.z, c.w};
   const __half2 k1024 = __half2half2(__ushort_as_half(0x6400));
   const __half2 k64 = __half2half2(__ushort_as_half(0x5400));
@@ -127,18 +136,17 @@ __device__ __forceinline__ void dequant32_u4(const uint4 c, __half2 s2, __half2 
     uint32_t v1 = (x & 0x00F000F0u) | 0x54005400u;  // (  64 + q1,   64 + q5)
     uint32_t v2 = (y & 0x000F000Fu) | 0x64006400u;  // (1024 + q2, 1024 + q6)
     uint32_t v3 = (y & 0x00F000F0u) | 0x54005400u;  // (  64 + q3,   64 + q7)
-    const __half2 q0 = __hsub2(*reinterpret_cast<__half2*>(&v0), k1024);
-    const __half2 q1 = __hsub2(*reinterpret_cast<__half2*>(&v1), k64);
-    const __half2 q2 = __hsub2(*reinterpret_cast<__half2*>(&v2), k1024);
-    const __half2 q3 = __hsub2(*reinterpret_cast<__half2*>(&v3), k64);
-    __half2 d0 = __hfma2(q0, s2, b2), d1 = __hfma2(q1, s2, b2), d2 = __hfma2(q2, s2, b2), d3 = __hfma2(q3, s2, b2);
+    __half2 d0 = __hsub2(*reinterpret_cast<__half2*>(&v0), k1024);
+    __half2 d1 = __hsub2(*reinterpret_cast<__half2*>(&v1), k64);
+    __half2 d2 = __hsub2(*reinterpret_cast<__half2*>(&v2), k1024);
+    __half2 d3 = __hsub2(*reinterpret_cast<__half2*>(&v3), k64);
     out[i] = make_uint4(*reinterpret_cast<uint32_t*>(&d0), *reinterpret_cast<uint32_t*>(&d1),
                         *reinterpret_cast<uint32_t*>(&d2), *reinterpret_cast<uint32_t*>(&d3));
   }
 }
 
-// Dequantise 32 codes (8-bit: 32 bytes) of one row into 4 16-byte fp16 chunks (natural K order).
-__device__ __forceinline__ void dequant32_u8(const uint4 c0, const uint4 c1, __half2 s2, __half2 b2, uint4* out) {
+// 32 8-bit codes (32 bytes) of one row -> 4 16-byte chunks of exact fp16 integers (natural K order).
+__device__ __forceinline__ void unpack32_u8(const uint4 c0, const uint4 c1, uint4* out) {
   const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
   const __half2 k1024 = __half2half2(__ushort_as_half(0x6400));
 #pragma unroll
@@ -149,13 +157,25 @@ __device__ __forceinline__ void dequant32_u8(const uint4 c0, const uint4 c1, __h
       const uint32_t x = w[2 * i + h];
       uint32_t v0 = __byte_perm(x, 0x64646464u, 0x5140);  // (1024 + b0, 1024 + b1)
       uint32_t v1 = __byte_perm(x, 0x64646464u, 0x5342);  // (1024 + b2, 1024 + b3)
-      __half2 d0 = __hfma2(__hsub2(*reinterpret_cast<__half2*>(&v0), k1024), s2, b2);
-      __half2 d1 = __hfma2(__hsub2(*reinterpret_cast<__half2*>(&v1), k1024), s2, b2);
+      __half2 d0 = __hsub2(*reinterpret_cast<__half2*>(&v0), k1024);
+      __half2 d1 = __hsub2(*reinterpret_cast<__half2*>(&v1), k1024);
       r[2 * h] = *reinterpret_cast<uint32_t*>(&d0);
       r[2 * h + 1] = *reinterpret_cast<uint32_t*>(&d1);
     }
     out[i] = make_uint4(r[0], r[1], r[2], r[3]);
   }
+}
+
+// acc[c0 + n] += s * P[n] + b * X[g][c0 + n] for the columns n < cnt - c0 of one 32-column slice.
+template <int C0>
+__device__ __forceinline__ void scale_slice(float* acc, uint32_t ta, float sc, float bi, const float* xs_g, int cnt) {
+  if (cnt <= C0) return;
+  uint32_t v[32];
+  tc::tmem_ld32(ta + C0, v);
+  tc::tmem_wait_ld();
+#pragma unroll
+  for (int n = 0; n < 32; ++n)
+    if (C0 + n < cnt) acc[C0 + n] = fmaf(sc, __uint_as_float(v[n]), fmaf(bi, xs_g[C0 + n], acc[C0 + n]));
 }
 
 // ------------------------------------------------------------------ GEMM kernel
@@ -164,22 +184,22 @@ template <int MODE, int BITS, int NS>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const GemmSmem L = gemm_smem(MODE, BITS, p.K, p.group, NS);
+  const GemmSmem L = gemm_smem(MODE, BITS, p.K, kBK, NS);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bar);  // [NS] TMA landed (codes + B)
   uint64_t* afull = full + NS;                               // [NS] A tile written
   uint64_t* empty = afull + NS;                              // [NS] MMAs done with the stage
   uint64_t* scfull = empty + NS;                             // [2] scales of a tile landed
-  uint64_t* scempty = scfull + 2;                            // [2] dequantisers done with them
-  uint64_t* accfull = scempty + 2;                           // [2] accumulator ready
-  uint64_t* accempty = accfull + 2;                          // [2] epilogue done with it
-  uint64_t* drain = accempty + 2;                            // MMA issuer: everything issued has finished
+  uint64_t* scempty = scfull + 2;                            // [2] unpackers and scalers done with them
+  uint64_t* pfull = scempty + 2;                             // [kPBuf] a group's products are in TMEM
+  uint64_t* pempty = pfull + kPBuf;                          // [kPBuf] scalers have read them
+  uint64_t* drain = pempty + kPBuf;                          // MMA issuer: everything issued has finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int CB = kBK * BITS / 8;          // code bytes per row per k-block
-  const int ng = p.K / p.group;           // groups per row
-  const int nkb = p.K / kBK;              // k-blocks per tile
+  const int ng = p.K / kBK;               // groups per row (one per k-block)
+  const int nkb = ng;
   const int MT = (MODE == 0) ? p.I / 64 : p.H / kBM;
   const int nchunks = *p.nchunks;
   const int ntiles = nchunks * MT;
@@ -192,16 +212,18 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&scfull[i], 1);
-      mbar_init(&scempty[i], 8);
-      mbar_init(&accfull[i], 1);
-      mbar_init(&accempty[i], 4);
+      mbar_init(&scempty[i], 12);
+    }
+    for (int i = 0; i < kPBuf; ++i) {
+      mbar_init(&pfull[i], 1);
+      mbar_init(&pempty[i], 4);
     }
     mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tc::tmem_alloc(tmem_slot, 2 * kAccCols);
+    tc::tmem_alloc(tmem_slot, kPBuf * kNT);
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
@@ -229,7 +251,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         const int mi = shared ? 1 : 0;  // which codes / scales maps
         const int bi = b_box_index(cnt);
         const int brows = b_box_rows(bi);
-        // scales and biases of the tile's 128 rows
         const int tb = it & 1, tu = it >> 1;
         if (tu >= 1 && !wait_or_abort(&scempty[tb], (tu - 1) & 1, p.hdr, abort, 30)) break;
         unsigned char* scb = sm + L.sc + tb * L.sc_buf_bytes;
@@ -253,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
           tc::tma_load_3d(cs, &p.tm_codes[mi], kb * CB, r0, ez, &full[s]);
           tc::tma_load_3d(cs + 64 * CB, &p.tm_codes[mi], kb * CB, r1, ez, &full[s]);
           tc::tma_load_2d(bs, &p.tm_b[bi], kb * kBK, start, &full[s]);
-          if (MODE == 1) tc::tma_load_2d(bs + kAccCols * 128, &p.tm_b2[bi], kb * kBK, start, &full[s]);
+          if (MODE == 1) tc::tma_load_2d(bs + kNT * 128, &p.tm_b2[bi], kb * kBK, start, &full[s]);
           tc::mbar_arrive(&full[s]);
           armed[s] = u;
         }
@@ -265,47 +286,44 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         if (sc_armed[b] >= 0) mbar_wait(&scfull[b], sc_armed[b] & 1, p.hdr, 38);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer
+    // ------------------------------------------------ MMA issuer: one group per k-block into its own TMEM buffer
     if (lane == 0) {
-      int kbg = 0, it = 0, last_commit_acc = -1;
-      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++it) {
+      int kbg = 0;
+      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
         const int ci = t / MT;
         const int cnt = p.chunks[3 * ci + 2];
         const int npad = (cnt + 15) & ~15;
         const uint32_t idesc = tc::idesc_f16_f32(kBM, npad);
-        const int ab = it & 1, au = it >> 1;
-        if (au >= 1 && !wait_or_abort(&accempty[ab], (au - 1) & 1, p.hdr, abort, 40)) break;
-        tc::fence_after_sync();
-        const uint32_t dt = tmem + ab * kAccCols;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb, ++kbg) {
           const int s = kbg % NS, u = kbg / NS;
-          if (!wait_or_abort(&full[s], u & 1, p.hdr, abort, 41) || !wait_or_abort(&afull[s], u & 1, p.hdr, abort, 42)) {
+          const int pb = kbg % kPBuf, pu = kbg / kPBuf;
+          if (!wait_or_abort(&full[s], u & 1, p.hdr, abort, 41) || !wait_or_abort(&afull[s], u & 1, p.hdr, abort, 42) ||
+              (pu >= 1 && !wait_or_abort(&pempty[pb], (pu - 1) & 1, p.hdr, abort, 43))) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
           const uint32_t a0 = smem_addr(sm + L.a + s * kBM * kBK * 2);
           const uint32_t b0 = smem_addr(sm + L.b + s * L.b_stage_bytes);
+          const uint32_t dt = tmem + pb * kNT;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t ad = tc::smem_desc_sw128(a0 + kk * 32);
-            tc::mma_f16(dt, ad, tc::smem_desc_sw128(b0 + kk * 32), idesc, (kb | kk) != 0);
-            if (MODE == 1) tc::mma_f16(dt, ad, tc::smem_desc_sw128(b0 + kAccCols * 128 + kk * 32), idesc, 1);
+            tc::mma_f16(dt, ad, tc::smem_desc_sw128(b0 + kk * 32), idesc, kk != 0);
+            if (MODE == 1) tc::mma_f16(dt, ad, tc::smem_desc_sw128(b0 + kNT * 128 + kk * 32), idesc, 1);
           }
           tc::commit(&empty[s]);
+          tc::commit(&pfull[pb]);
         }
         if (!ok) break;
-        tc::commit(&accfull[ab]);
-        last_commit_acc = it;
       }
       // every MMA issued must be finished before TMEM is released
-      (void)last_commit_acc;
       tc::commit(drain);
       mbar_wait(drain, 0, p.hdr, 49);
     }
   } else if (warp >= kDequantWarp0 && warp < kEpiWarp0) {
-    // ------------------------------------------------ dequantisers: 2 threads per row
+    // ------------------------------------------------ unpackers: 2 threads per row
     const int d = threadIdx.x - kDequantWarp0 * 32;  // 0..255
     const int m = d >> 1, half = d & 1;              // A-tile row, which 32 codes of the 64
     // A row m <- staging row: gate/up interleaved for mode 0, identity for mode 1
@@ -313,24 +331,18 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     int kbg = 0, it = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
       if (warp_aborted(abort)) break;
-      const int tb = it & 1, tu = it >> 1;
-      if (!warp_wait(&scfull[tb], tu & 1, p.hdr, abort, 50)) break;
-      const uint16_t* scs = reinterpret_cast<const uint16_t*>(sm + L.sc + tb * L.sc_buf_bytes);
-      const uint16_t* bis = scs + 2 * 64 * ng;
+      const int tb = it & 1;
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb, ++kbg) {
         const int s = kbg % NS, u = kbg / NS;
         if (!warp_wait(&full[s], u & 1, p.hdr, abort, 51)) { ok = false; break; }
         if (u >= 1 && !warp_wait(&empty[s], (u - 1) & 1, p.hdr, abort, 52)) { ok = false; break; }
-        const int g = (kb * kBK + 32 * half) / p.group;
-        const __half2 s2 = __half2half2(__float2half_rn(bf16_to_f32(scs[srow * ng + g])));
-        const __half2 b2 = __half2half2(__float2half_rn(bf16_to_f32(bis[srow * ng + g])));
         const unsigned char* crow = sm + L.codes + s * L.codes_stage_bytes + srow * CB + half * (CB / 2);
         uint4 outv[4];
         if (BITS == 4) {
-          dequant32_u4(*reinterpret_cast<const uint4*>(crow), s2, b2, outv);
+          unpack32_u4(*reinterpret_cast<const uint4*>(crow), outv);
         } else {
-          dequant32_u8(*reinterpret_cast<const uint4*>(crow), *reinterpret_cast<const uint4*>(crow + 16), s2, b2, outv);
+          unpack32_u8(*reinterpret_cast<const uint4*>(crow), *reinterpret_cast<const uint4*>(crow + 16), outv);
         }
         unsigned char* arow = sm + L.a + s * kBM * kBK * 2 + (m >> 3) * 1024 + (m & 7) * 128;
 #pragma unroll
@@ -344,63 +356,95 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       }
       if (!ok) break;
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&scempty[tb]);
+      if (lane == 0) tc::mbar_arrive(&scempty[tb]);  // this role does not read the scales; it keeps the count
     }
   } else if (warp >= kEpiWarp0) {
-    // ------------------------------------------------ epilogue
+    // ------------------------------------------------ scalers + epilogue (four independent warps)
     const int q = warp & 3;         // TMEM lane quarter
     const int m = 32 * q + lane;    // accumulator row held by this thread
-    int it = 0;
+    const int srow = (MODE == 0) ? ((m & 1) * 64 + (m >> 1)) : m;
+    float* xs = reinterpret_cast<float*>(sm + L.xs) + q * ng * kNT;  // this warp's [ng][kNT]
+    int kbg = 0, it = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
       if (warp_aborted(abort)) break;
       const int ci = t / MT, mt = t % MT;
       const int start = p.chunks[3 * ci + 1], cnt = p.chunks[3 * ci + 2];
-      const int ab = it & 1, au = it >> 1;
-      if (!warp_wait(&accfull[ab], au & 1, p.hdr, abort, 60)) break;
-      tc::fence_after_sync();
-      const uint32_t ta = tmem + (static_cast<uint32_t>(32 * q) << 16) + ab * kAccCols;
-      for (int c0 = 0; c0 < cnt; c0 += 32) {
-        uint32_t v[32];
-        tc::tmem_ld32(ta + c0, v);
-        tc::tmem_wait_ld();
+      const int tb = it & 1, tu = it >> 1;
+      // group sums of the tile's columns (the down GEMM's come as 4 partial sums, added in order)
+      __syncwarp();
+      for (int i = lane; i < ng * cnt; i += 32) {
+        const int n = i / ng, g = i % ng;
+        float v;
         if (MODE == 0) {
-          // rows 2i (gate) and 2i+1 (up) of intermediate index mt*64 + i
-          const int i = mt * 64 + (m >> 1);
-          const int ip = (BITS == 4) ? ((i & ~7) | perm8_pos(i & 7)) : i;
-#pragma unroll
-          for (int n = 0; n < 32; ++n) {
-            const float a = __uint_as_float(v[n]);
-            const float u = __shfl_xor_sync(0xffffffffu, a, 1);
-            if (!(m & 1) && c0 + n < cnt) {
-              const float h = silu_f(a) * u;
-              const __half hi = __float2half_rn(h);
-              const __half lo = __float2half_rn(h - __half2float(hi));
-              const size_t o = static_cast<size_t>(start + c0 + n) * p.ldh + ip;
-              p.h_hi[o] = __half_as_ushort(hi);
-              p.h_lo[o] = __half_as_ushort(lo);
-            }
-          }
+          v = __ldg(p.xs_in + static_cast<size_t>(start + n) * ng + g);
         } else {
-          const int r = mt * kBM + m;
+          const float* ps = p.xs_in + (static_cast<size_t>(start + n) * ng + g) * 4;
+          v = (__ldg(ps) + __ldg(ps + 1)) + (__ldg(ps + 2) + __ldg(ps + 3));
+        }
+        xs[g * kNT + n] = v;
+      }
+      __syncwarp();
+      if (!warp_wait(&scfull[tb], tu & 1, p.hdr, abort, 60)) break;
+      const uint16_t* scs = reinterpret_cast<const uint16_t*>(sm + L.sc + tb * L.sc_buf_bytes);
+      const uint16_t* bis = scs + 2 * 64 * ng;
+      float acc[kNT];
 #pragma unroll
-          for (int n = 0; n < 32; ++n) {
-            if (c0 + n < cnt) {
-              const int pid = __ldg(p.perm + start + c0 + n);
-              p.out[static_cast<size_t>(pid) * p.H + r] = __uint_as_float(v[n]);
-            }
+      for (int n = 0; n < kNT; ++n) acc[n] = 0.f;
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+        const int pb = kbg % kPBuf, pu = kbg / kPBuf;
+        if (!warp_wait(&pfull[pb], pu & 1, p.hdr, abort, 61)) { ok = false; break; }
+        tc::fence_after_sync();
+        const float sc = bf16_to_f32(scs[srow * ng + kb]);
+        const float bi = bf16_to_f32(bis[srow * ng + kb]);
+        const uint32_t ta = tmem + (static_cast<uint32_t>(32 * q) << 16) + pb * kNT;
+        const float* xg = xs + kb * kNT;
+        scale_slice<0>(acc, ta, sc, bi, xg, cnt);
+        scale_slice<32>(acc, ta, sc, bi, xg, cnt);
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&pempty[pb]);
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&scempty[tb]);
+      if (MODE == 0) {
+        // rows 2i (gate) and 2i+1 (up) of intermediate index mt*64 + i
+        const int i = mt * 64 + (m >> 1);
+        const int ip = (BITS == 4) ? ((i & ~7) | perm8_pos(i & 7)) : i;
+#pragma unroll
+        for (int n = 0; n < kNT; ++n) {
+          const float u = __shfl_xor_sync(0xffffffffu, acc[n], 1);
+          float h = 0.f;
+          if (!(m & 1) && n < cnt) {
+            h = silu_f(acc[n]) * u;
+            const __half hi = __float2half_rn(h);
+            const __half lo = __float2half_rn(h - __half2float(hi));
+            const size_t o = static_cast<size_t>(start + n) * p.ldh + ip;
+            p.h_hi[o] = __half_as_ushort(hi);
+            p.h_lo[o] = __half_as_ushort(lo);
+          }
+          // this warp's share (16 intermediate indices) of the group sum of h
+          const float ws = warp_sum(h);
+          if (lane == 0 && n < cnt) p.hsum_out[(static_cast<size_t>(start + n) * (p.I / 64) + mt) * 4 + q] = ws;
+        }
+      } else {
+        const int r = mt * kBM + m;
+#pragma unroll
+        for (int n = 0; n < kNT; ++n) {
+          if (n < cnt) {
+            const int pid = __ldg(p.perm + start + n);
+            p.out[static_cast<size_t>(pid) * p.H + r] = acc[n];
           }
         }
       }
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&accempty[ab]);
     }
   }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 2 * kAccCols);
+    tc::tmem_dealloc(tmem, kPBuf * kNT);
   }
 }
 
@@ -417,7 +461,7 @@ __global__ void __launch_bounds__(256) gather_kernel(BatchParams p) {
     const int t = (pid < p.T * p.k) ? pid / p.k : pid - p.T * p.k;
     const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t) * p.H);
     uint4* dst = reinterpret_cast<uint4*>(p.x16 + static_cast<size_t>(pos) * p.H);
-    for (int s = lane; s < p.H / 8; s += 32) {
+    for (int s = lane; s < p.H / 8; s += 32) {  // H % 256 == 0: every lane has a segment
       const uint4 v = xr[s];
       const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
                           bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
@@ -425,6 +469,12 @@ __global__ void __launch_bounds__(256) gather_kernel(BatchParams p) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) o[p.perm8 ? perm8_pos(kk) : kk] = __float2half_rn(f[kk]);
       dst[s] = *reinterpret_cast<const uint4*>(o);
+      // sum of each group of 64 (8 segments, 8 consecutive lanes)
+      float g = ((f[0] + f[1]) + (f[2] + f[3])) + ((f[4] + f[5]) + (f[6] + f[7]));
+      g += __shfl_xor_sync(0xffffffffu, g, 1);
+      g += __shfl_xor_sync(0xffffffffu, g, 2);
+      g += __shfl_xor_sync(0xffffffffu, g, 4);
+      if ((lane & 7) == 0) p.xs[static_cast<size_t>(pos) * (p.H / 64) + s / 8] = g;
     }
   }
   if (p.Is > 0) {
@@ -465,7 +515,7 @@ __global__ void __launch_bounds__(256) combine_kernel(BatchParams p) {
 
 template <int MODE, int BITS, int NS>
 cudaError_t launch_gemm_t(const GemmParams& g, int grid, cudaStream_t st) {
-  const GemmSmem L = gemm_smem(MODE, BITS, g.K, g.group, NS);
+  const GemmSmem L = gemm_smem(MODE, BITS, g.K, kBK, NS);
   auto kern = grouped_gemm_kernel<MODE, BITS, NS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
   if (e != cudaSuccess) return e;
@@ -476,7 +526,8 @@ cudaError_t launch_gemm_t(const GemmParams& g, int grid, cudaStream_t st) {
 }  // namespace
 
 size_t grouped_gemm_smem(int mode, int bits, int K, int group) {
-  return gemm_smem(mode, bits, K, group, mode == 0 ? 4 : 3).total;
+  (void)group;
+  return gemm_smem(mode, bits, K, kBK, mode == 0 ? 4 : 3).total;
 }
 
 cudaError_t launch_grouped_gemm(const GemmParams& g, int mode, int bits, int grid, cudaStream_t st) {

@@ -45,6 +45,7 @@ struct Layout {
   size_t flags, dlogits, dh, dy, dr, dx;                  // persistent single-token decode
   size_t base_total;                                      // end of the regions above
   size_t perm, offs, chunks, nchunks, x16, hhi, hlo, o;   // batched tensor-core path
+  size_t xsx, xsh;                                        // group sums of x and of h
   size_t total;
 };
 
@@ -84,6 +85,8 @@ Layout layout(const moe_config& c, int64_t T) {
   L.hhi = o;      o += up(np * imax * 2);
   L.hlo = o;      o += up(np * imax * 2);
   L.o = o;        o += up(np * c.hidden * 4);
+  L.xsx = o;      o += up(np * (c.hidden / 64 + 1) * 4);
+  L.xsh = o;      o += up(np * (imax / 64 + 1) * 4 * 4);
   L.total = o;
   return L;
 }
@@ -256,8 +259,9 @@ int device_sms() {
 
 bool batched_eligible(const moe_config& c, int T) {
   if (T < kBatchMinTokens) return false;
+  if (c.group != 64) return false;  // one quantisation group per GEMM k-block
   if (c.shared_inter != 0 && c.shared_inter != c.inter) return false;
-  if ((c.hidden / c.group) % 8 || (c.inter / c.group) % 8 || c.hidden % 128 || c.inter % 64) return false;
+  if ((c.hidden / c.group) % 8 || (c.inter / c.group) % 8 || c.hidden % 256 || c.inter % 64) return false;
   if (!encode_fn()) return false;
   int dev = 0, optin = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -284,6 +288,8 @@ moe_status batched_ffn(const moe_config& c, const moe_layer_weights& wt, const u
   uint16_t* hhi = reinterpret_cast<uint16_t*>(b + Ly.hhi);
   uint16_t* hlo = reinterpret_cast<uint16_t*>(b + Ly.hlo);
   float* o = reinterpret_cast<float*>(b + Ly.o);
+  float* xsx = reinterpret_cast<float*>(b + Ly.xsx);
+  float* xsh = reinterpret_cast<float*>(b + Ly.xsh);
   const int sms = device_sms();
   if (sms < 1) return fail(MOE_ERR_CUDA, "no device");
 
@@ -300,6 +306,7 @@ moe_status batched_ffn(const moe_config& c, const moe_layer_weights& wt, const u
   bp.Is = c.shared_inter;
   bp.perm8 = (c.bits == 4) ? 1 : 0;
   bp.x16 = x16;
+  bp.xs = xsx;
   bp.sgate = v.sgate;
   bp.w = w;
   bp.o = o;
@@ -323,11 +330,13 @@ moe_status batched_ffn(const moe_config& c, const moe_layer_weights& wt, const u
                    wt.gate_up.sb_expert_stride * 2, H / g) &&
             map_3d(&gp->tm_biases[1], sgu.biases, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, H / g, 2 * I, 1,
                    static_cast<int64_t>(2) * I * (H / g) * 2, H / g);
-  for (int i = 0; i < 4 && ok; ++i) ok = map_b(&gp->tm_b[i], x16, H, np, 16 << i) && map_b(&gp->tm_b2[i], x16, H, np, 16 << i);
+  for (int i = 0; i < 4 && ok; ++i) ok = map_b(&gp->tm_b[i], x16, H, np, i < 3 ? 16 << i : 64) && map_b(&gp->tm_b2[i], x16, H, np, i < 3 ? 16 << i : 64);
   if (!ok) return fail(MOE_ERR_CUDA, "tensor map encoding failed (gate/up)");
   gp->chunks = chunks;
   gp->nchunks = nchunks;
   gp->perm = perm;
+  gp->xs_in = xsx;
+  gp->hsum_out = xsh;
   gp->K = H;
   gp->rows = 2 * I;
   gp->I = I;
@@ -353,10 +362,11 @@ moe_status batched_ffn(const moe_config& c, const moe_layer_weights& wt, const u
               wt.down.sb_expert_stride * 2, I / g) &&
        map_3d(&gp->tm_biases[1], sdn.biases, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, I / g, H, 1,
               static_cast<int64_t>(H) * (I / g) * 2, I / g);
-  for (int i = 0; i < 4 && ok; ++i) ok = map_b(&gp->tm_b[i], hhi, I, np, 16 << i) && map_b(&gp->tm_b2[i], hlo, I, np, 16 << i);
+  for (int i = 0; i < 4 && ok; ++i) ok = map_b(&gp->tm_b[i], hhi, I, np, i < 3 ? 16 << i : 64) && map_b(&gp->tm_b2[i], hlo, I, np, i < 3 ? 16 << i : 64);
   if (!ok) return fail(MOE_ERR_CUDA, "tensor map encoding failed (down)");
   gp->K = I;
   gp->rows = H;
+  gp->xs_in = xsh;
   if ((e = moe::launch_grouped_gemm(*gp, 1, bits, sms, st)) != cudaSuccess) return cuda_fail(e, "down GEMM launch");
   if ((e = moe::launch_combine(bp, sms * 4, st)) != cudaSuccess) return cuda_fail(e, "combine launch");
   return MOE_OK;

@@ -62,7 +62,7 @@ struct SortParams {
   WsHeader* hdr;
 };
 
-constexpr int kChunkTokens = 128;  // pairs per GEMM chunk (the MMA N dimension)
+constexpr int kChunkTokens = 64;  // pairs per GEMM chunk (the MMA N dimension)
 
 // Batched path: gather of the sorted pairs' activations and the final combine.
 struct BatchParams {
@@ -71,6 +71,7 @@ struct BatchParams {
   const int32_t* perm;   // [npairs] sorted position -> pair id
   int T, k, H, Is, perm8;
   uint16_t* x16;         // fp16 [npairs][H], K permuted in blocks of 8 when perm8
+  float* xs;             // fp32 [npairs][H/64] sums of x over each group of 64
   float* sgate;          // [T]
   const float* w;        // [T][k] routing weights
   const float* o;        // fp32 [npairs by pair id][H] expert outputs
@@ -87,9 +88,11 @@ struct GemmParams {
   const int32_t* chunks;
   const int32_t* nchunks;
   const int32_t* perm;
+  const float* xs_in;        // group sums of the B operand: x [npairs][K/64], or h as 4 partials [npairs][K/64][4]
   int K, rows, I, H, E, group, ldh;
   uint16_t* h_hi;            // gate/up output [npairs][ldh] fp16 hi / lo
   uint16_t* h_lo;
+  float* hsum_out;           // gate/up output [npairs][I/64][4] partial group sums of h (one per epilogue warp)
   float* out;                // down output [pair id][H] fp32
   WsHeader* hdr;
 };

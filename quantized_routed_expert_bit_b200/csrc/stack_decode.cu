@@ -45,7 +45,7 @@ __host__ __device__ constexpr int al8(int v) { return (v + 7) & ~7; }
 // Shared-memory carve-up; identical on host (sizing) and device.
 struct Carve {
   int PS, nseg_x, nslots, Imax, npc_max, ng, nr_max, ng_dmax, rowb_dmax, d_sc_el, rr_max;
-  uint32_t xs, xsum, xn, r, hs, hsum, gsb, dbuf, d_slot_bytes, rbuf, total;
+  uint32_t xs, xsum, xn, r, dred, gsb, dbuf, d_slot_bytes, rbuf, total;
 };
 
 __host__ __device__ inline Carve carve(int H, int E, int k, int I, int Is, int group, int bits, int G) {
@@ -67,8 +67,7 @@ __host__ __device__ inline Carve carve(int H, int E, int k, int I, int Is, int g
   c.xsum = o;  o = al128(o + c.nseg_x * 4);
   c.xn = o;    o = al128(o + H * 4);
   c.r = o;     o = al128(o + H * 4);
-  c.hs = o;    o = al128(o + c.nslots * c.Imax * 4);
-  c.hsum = o;  o = al128(o + c.nslots * (c.Imax / c.PS) * 4);
+  c.dred = o;  o = al128(o + c.nslots * c.nr_max * 4);
   c.gsb = o;   o = al128(o + 4 * c.npc_max * c.ng * 2);
   c.d_slot_bytes = al128(c.nr_max * c.rowb_dmax + 2 * c.d_sc_el * 2);
   c.dbuf = o;  o = al128(o + c.nslots * c.d_slot_bytes);
@@ -133,57 +132,67 @@ __device__ __forceinline__ unsigned fkey(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+__device__ __forceinline__ float fkey_inv(unsigned k) {
+  return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
+}
+
 // Softmax + top-k of one token by one warp: larger logit first, equal
 // logits to the lower expert index; weights renormalised over the k (or the
-// plain softmax probabilities when renorm == 0).
+// plain softmax probabilities when renorm == 0). Each lane sorts its PER
+// logits once (largest first, then lower index); every round one warp-wide
+// max over the lanes' heads picks the winner, whose lane pops its head.
+template <int PER>
 __device__ void topk_warp(const float* lg, int E, int k, int renorm, int* s_idx, float* s_w) {
-  constexpr int kPer = 16;
   const int lane = threadIdx.x & 31;
-  float v[kPer];
-  unsigned key[kPer];
+  unsigned key[PER];
+  int idx[PER];
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
+  for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
-    v[i] = (e < E) ? __ldcg(lg + e) : -FLT_MAX;
-    key[i] = (e < E) ? fkey(v[i]) : 0u;
+    key[i] = (e < E) ? fkey(__ldcg(lg + e)) : 0u;
+    idx[i] = e;
   }
-  float mx = -FLT_MAX;
+  // odd-even transposition sort: key descending, index ascending among equal keys
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) mx = fmaxf(mx, v[i]);
-  mx = warp_max(mx);
+  for (int r = 0; r < PER; ++r) {
+#pragma unroll
+    for (int i = (r & 1); i + 1 < PER; i += 2) {
+      const bool sw = key[i + 1] > key[i] || (key[i + 1] == key[i] && idx[i + 1] < idx[i]);
+      const unsigned k0 = key[i], k1 = key[i + 1];
+      const int i0 = idx[i], i1 = idx[i + 1];
+      key[i] = sw ? k1 : k0;
+      key[i + 1] = sw ? k0 : k1;
+      idx[i] = sw ? i1 : i0;
+      idx[i + 1] = sw ? i0 : i1;
+    }
+  }
+  const float mx = fkey_inv(__reduce_max_sync(0xffffffffu, key[0]));
   float z = 0.f;
   if (!renorm) {
 #pragma unroll
-    for (int i = 0; i < kPer; ++i)
-      if (lane + 32 * i < E) z += expf(v[i] - mx);
+    for (int i = 0; i < PER; ++i)
+      if (key[i] != 0u) z += expf(fkey_inv(key[i]) - mx);
     z = warp_sum(z);
   }
-  float my_v = 0.f;
+  unsigned my_k = 0u;
   int my_e = 0;
   for (int j = 0; j < k; ++j) {
-    unsigned bk = 0u;
-    int be = INT_MAX;
-    float bv = 0.f;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      if (key[i] > bk) {  // strict: lowest index among equal keys of this lane
-        bk = key[i];
-        be = lane + 32 * i;
-        bv = v[i];
-      }
-    }
-    const unsigned wk = __reduce_max_sync(0xffffffffu, bk);
-    const unsigned we = __reduce_min_sync(0xffffffffu, bk == wk ? static_cast<unsigned>(be) : 0xffffffffu);
-    const float wv = __shfl_sync(0xffffffffu, bv, static_cast<int>(we & 31u));
-#pragma unroll
-    for (int i = 0; i < kPer; ++i)
-      if (lane + 32 * i == static_cast<int>(we)) key[i] = 0u;
+    const unsigned wk = __reduce_max_sync(0xffffffffu, key[0]);
+    const unsigned we = __reduce_min_sync(0xffffffffu, key[0] == wk ? static_cast<unsigned>(idx[0]) : 0xffffffffu);
     if (lane == j) {
-      my_v = wv;
+      my_k = wk;
       my_e = static_cast<int>(we);
     }
+    if (idx[0] == static_cast<int>(we) && key[0] == wk) {  // pop the head
+#pragma unroll
+      for (int i = 0; i + 1 < PER; ++i) {
+        key[i] = key[i + 1];
+        idx[i] = idx[i + 1];
+      }
+      key[PER - 1] = 0u;
+    }
   }
-  const float ex = (lane < k) ? expf(my_v - mx) : 0.f;
+  const float ex = (lane < k) ? expf(fkey_inv(my_k) - mx) : 0.f;
   const float den = renorm ? warp_sum(ex) : z;
   if (lane < k) {
     s_idx[lane] = my_e;
@@ -236,8 +245,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
   float* xsum = reinterpret_cast<float*>(sm + cv.xsum);
   float* xn = reinterpret_cast<float*>(sm + cv.xn);
   float* rr = reinterpret_cast<float*>(sm + cv.r);
-  float* hs = reinterpret_cast<float*>(sm + cv.hs);
-  float* hsum = reinterpret_cast<float*>(sm + cv.hsum);
   uint16_t* gsb = reinterpret_cast<uint16_t*>(sm + cv.gsb);
   unsigned char* dbuf = sm + cv.dbuf;
   uint16_t* rbuf = reinterpret_cast<uint16_t*>(sm + cv.rbuf);
@@ -342,7 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
 
     // ---------------- 2. softmax + top-k (every CTA)
     if (warp == 0) {
-      topk_warp(p.logits, E, k, p.renorm, s_idx, s_w);
+      if (E <= 256) topk_warp<8>(p.logits, E, k, p.renorm, s_idx, s_w);
+      else topk_warp<16>(p.logits, E, k, p.renorm, s_idx, s_w);
       if (lane == 0) s_sg = (Is > 0) ? 1.f / (1.f + expf(-__ldcg(p.logits + E))) : 0.f;
       __syncwarp();
       if (c == 0 && lane < k) {
@@ -354,30 +362,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
     stamp(3);
 
     // ---------------- 3. bulk copies: gate/up scales+biases of this CTA's pairs, down rows
-    if (tid == 0) {
+    // (issued by the 32 lanes of warp 0 in parallel; lane 0 arrives once all are armed)
+    if (warp == 0) {
       const int ng = cv.ng;
-      int P = gp0;
+      // gate/up scale and bias rows: the CTA's pairs fall in at most 3 slots
+      int P = gp0, seg = 0;
       while (P < gp1) {
         const bool routed = P < k * I;
         const int j = routed ? P / I : k;
         const int sstart = routed ? j * I : k * I;
         const int send = routed ? (j + 1) * I : k * I + Is;
         const int n = min(gp1, send) - P;
-        const int i0 = P - sstart;
-        const int q0 = P - gp0;
-        const QMat m = routed ? Ld.gu : Ld.sgu;
-        const int Ij = routed ? I : Is;
-        const size_t eoff = static_cast<size_t>(routed ? s_idx[j] : 0) * m.sb_stride;
-        const uint32_t nb = static_cast<uint32_t>(n * ng) * 2u;
-        copy_tx(gsb + (0 * cv.npc_max + q0) * ng, m.s + eoff + static_cast<size_t>(i0) * ng, nb, &bar_g);
-        copy_tx(gsb + (1 * cv.npc_max + q0) * ng, m.s + eoff + static_cast<size_t>(Ij + i0) * ng, nb, &bar_g);
-        copy_tx(gsb + (2 * cv.npc_max + q0) * ng, m.b + eoff + static_cast<size_t>(i0) * ng, nb, &bar_g);
-        copy_tx(gsb + (3 * cv.npc_max + q0) * ng, m.b + eoff + static_cast<size_t>(Ij + i0) * ng, nb, &bar_g);
+        if (lane >= 4 * seg && lane < 4 * seg + 4) {
+          const int which = lane - 4 * seg;  // 0 gate scales, 1 up scales, 2 gate biases, 3 up biases
+          const int i0 = P - sstart;
+          const int q0 = P - gp0;
+          const QMat m = routed ? Ld.gu : Ld.sgu;
+          const int Ij = routed ? I : Is;
+          const size_t eoff = static_cast<size_t>(routed ? s_idx[j] : 0) * m.sb_stride;
+          const uint16_t* src = ((which & 2) ? m.b : m.s) + eoff + static_cast<size_t>((which & 1) ? Ij + i0 : i0) * ng;
+          copy_tx(gsb + (which * cv.npc_max + q0) * ng, src, static_cast<uint32_t>(n * ng) * 2u, &bar_g);
+        }
         P += n;
+        ++seg;
       }
-      mbar_arrive(&bar_g);
-      s_pend[2] = l & 1;
-      for (int j = 0; j < nslots; ++j) {
+      // down rows of every slot: codes, scales, biases (3 copies per slot)
+      for (int c3 = lane; c3 < 3 * nslots && nr > 0; c3 += 32) {
+        const int j = c3 / 3, which = c3 % 3;
         const bool routed = j < k;
         const QMat m = routed ? Ld.dn : Ld.sdn;
         const int Ij = routed ? I : Is;
@@ -385,19 +396,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         const size_t rowbd = static_cast<size_t>(Ij) * BITS / 8;
         const int e = routed ? s_idx[j] : 0;
         unsigned char* slot = dbuf + static_cast<size_t>(j) * cv.d_slot_bytes;
-        if (nr > 0) {
+        if (which == 0) {
           copy_tx(slot, m.q + static_cast<size_t>(e) * m.q_stride + static_cast<size_t>(r0) * rowbd,
                   static_cast<uint32_t>(nr * rowbd), &bar_d);
+        } else {
           const int el0 = (r0 * ngd) & ~7;
           const int el1 = al8(r1 * ngd);
           uint16_t* sc = reinterpret_cast<uint16_t*>(slot + static_cast<size_t>(cv.nr_max) * cv.rowb_dmax);
           const size_t eo = static_cast<size_t>(e) * m.sb_stride + el0;
-          copy_tx(sc, m.s + eo, static_cast<uint32_t>(el1 - el0) * 2u, &bar_d);
-          copy_tx(sc + cv.d_sc_el, m.b + eo, static_cast<uint32_t>(el1 - el0) * 2u, &bar_d);
+          copy_tx(sc + (which == 2 ? cv.d_sc_el : 0), (which == 2 ? m.b : m.s) + eo,
+                  static_cast<uint32_t>(el1 - el0) * 2u, &bar_d);
         }
       }
-      mbar_arrive(&bar_d);
-      s_pend[3] = l & 1;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar_g);
+        mbar_arrive(&bar_d);
+        s_pend[2] = l & 1;
+        s_pend[3] = l & 1;
+      }
+      __syncwarp();
     }
 
     // ---------------- 4. gate/up + SwiGLU of this CTA's row pairs
@@ -490,75 +508,59 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
     if (!grid_barrier(p, ++epoch, &s_abort)) { drain(); return; }
     stamp(5);
 
-    // ---------------- 5. all h into shared memory (permuted) + segment sums
-    for (int j = 0; j < nslots; ++j) {
-      const int Ij = (j < k) ? I : Is;
-      const int nsg = Ij / PS;
-      const float4* hg = reinterpret_cast<const float4*>(p.hbuf + static_cast<size_t>(j) * cv.Imax);
-      float* hj = hs + static_cast<size_t>(j) * cv.Imax;
-      for (int i4 = tid; i4 < Ij / 4; i4 += kThreads) {
-        const int s = (4 * i4) / PS, q4 = ((4 * i4) % PS) / 4;
-        reinterpret_cast<float4*>(hj)[q4 * nsg + s] = __ldcg(hg + i4);
-      }
-    }
-    __syncthreads();
-    for (int j = 0; j < nslots; ++j) {
-      const int Ij = (j < k) ? I : Is;
-      const int nsg = Ij / PS;
-      const float* hj = hs + static_cast<size_t>(j) * cv.Imax;
-      for (int s = tid; s < nsg; s += kThreads) {
-        float a = 0.f;
-#pragma unroll
-        for (int q4 = 0; q4 < PS / 4; ++q4) {
-          const float4 f = reinterpret_cast<const float4*>(hj)[q4 * nsg + s];
-          a += (f.x + f.y) + (f.z + f.w);
-        }
-        hsum[j * (cv.Imax / PS) + s] = a;
-      }
-    }
-    __syncthreads();
-
-    // ---------------- 6. down rows + weighted combine + shared expert
+    // ---------------- 5+6. down rows + weighted combine + shared expert
+    // Warp w owns slots w, w+16: its lanes keep one 16-byte code segment's
+    // worth of that slot's h (read once from L2) and walk the CTA's rows; the
+    // per-slot row sums meet in shared memory and are combined in slot order.
     if (!mbar_wait(&bar_d, l & 1, p.hdr, 13)) s_abort = 1;
-    __syncthreads();
     if (tid == 0) s_pend[3] = -1;
     const bool last_layer_out = p.layer_mode && (l == p.L - 1);
-    for (int rl = warp; rl < nr; rl += kWarps) {
-      const int row = r0 + rl;
-      const int nseg_r = I / PS, nseg_s = Is / PS;
-      const int nflat = k * nseg_r + nseg_s;
-      float acc = 0.f;
-      for (int f = lane; f < nflat; f += 32) {
-        const bool routed = f < k * nseg_r;
-        const int j = routed ? f / nseg_r : k;
-        const int s = routed ? f - j * nseg_r : f - k * nseg_r;
+    {
+      float* dred = reinterpret_cast<float*>(sm + cv.dred);  // [nslots][nr_max]
+      for (int j = warp; j < nslots; j += kWarps) {
+        const bool routed = j < k;
         const int Ij = routed ? I : Is;
+        const int nsg = Ij / PS;                   // code segments per row (16 or 32 at I = 512)
+        const int rows_per_step = 32 / nsg;        // 2 rows at a time for 16 segments
+        const int s = lane % nsg;
+        const int sub = lane / nsg;                // which of the rows of this step
         const int ngd = Ij / group;
         const int rowbd = Ij * BITS / 8;
+        const float* hg = p.hbuf + static_cast<size_t>(j) * cv.Imax + s * PS;
+        float hv[PS];
+        float hsm = 0.f;
+#pragma unroll
+        for (int q4 = 0; q4 < PS / 4; ++q4) {
+          const float4 f = __ldcg(reinterpret_cast<const float4*>(hg) + q4);
+          hv[4 * q4] = f.x;
+          hv[4 * q4 + 1] = f.y;
+          hv[4 * q4 + 2] = f.z;
+          hv[4 * q4 + 3] = f.w;
+          hsm += (f.x + f.y) + (f.z + f.w);
+        }
         const unsigned char* slot = dbuf + static_cast<size_t>(j) * cv.d_slot_bytes;
-        const uint4 cd = *reinterpret_cast<const uint4*>(slot + static_cast<size_t>(rl) * rowbd + 16 * s);
         const uint16_t* sc = reinterpret_cast<const uint16_t*>(slot + static_cast<size_t>(cv.nr_max) * cv.rowb_dmax);
         const int off = r0 * ngd - ((r0 * ngd) & ~7);
         const int g = s * PS / group;
-        const int ei = off + rl * ngd + g;
-        const float scl = bf16_to_f32(sc[ei]);
-        const float bia = bf16_to_f32(sc[cv.d_sc_el + ei]);
-        const int nsg = Ij / PS;
-        float xv[PS];
-        const float* hj = hs + static_cast<size_t>(j) * cv.Imax;
-#pragma unroll
-        for (int q4 = 0; q4 < PS / 4; ++q4) {
-          const float4 v4 = reinterpret_cast<const float4*>(hj)[q4 * nsg + s];
-          xv[4 * q4] = v4.x;
-          xv[4 * q4 + 1] = v4.y;
-          xv[4 * q4 + 2] = v4.z;
-          xv[4 * q4 + 3] = v4.w;
+        for (int rl0 = 0; rl0 < nr; rl0 += rows_per_step) {
+          const int rl = rl0 + sub;
+          float part = 0.f;
+          if (rl < nr) {
+            const uint4 cd = *reinterpret_cast<const uint4*>(slot + static_cast<size_t>(rl) * rowbd + 16 * s);
+            const int ei = off + rl * ngd + g;
+            part = fmaf(bf16_to_f32(sc[ei]), dot_seg<BITS>(cd, hv), bf16_to_f32(sc[cv.d_sc_el + ei]) * hsm);
+          }
+          // sum over the nsg lanes of each row
+          for (int o = nsg >> 1; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+          if (s == 0 && rl < nr) dred[j * cv.nr_max + rl] = part;
         }
-        const float part = fmaf(scl, dot_seg<BITS>(cd, xv), bia * hsum[j * (cv.Imax / PS) + s]);
-        acc = fmaf(routed ? s_w[j] : s_sg, part, acc);
       }
-      acc = warp_sum(acc);
-      if (lane == 0) {
+      __syncthreads();
+      if (tid < nr) {
+        const int row = r0 + tid;
+        float acc = 0.f;
+        for (int j = 0; j < k; ++j) acc = fmaf(s_w[j], dred[j * cv.nr_max + tid], acc);
+        if (Is > 0) acc = fmaf(s_sg, dred[k * cv.nr_max + tid], acc);
         const uint16_t yb = f32_to_bf16(acc);
         if (last_layer_out) {
           p.out[row] = yb;
