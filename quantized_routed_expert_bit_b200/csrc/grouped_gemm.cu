@@ -57,6 +57,7 @@ constexpr int kBM = 128;           // tile rows
 constexpr int kBK = 64;            // K per k-block: one quantisation group, one 128-byte swizzle row
 constexpr int kNT = kChunkTokens;  // columns (pairs) per tile
 constexpr int kPBuf = 4;           // TMEM buffers of per-group products in rotation
+constexpr int kNA = 4;             // unpacked A tiles in flight
 constexpr int kDequantWarp0 = 4;   // warps 4..11
 constexpr int kEpiWarp0 = 12;      // warps 12..15
 
@@ -69,28 +70,32 @@ __host__ __device__ constexpr int perm8_pos(int k) {  // position of element k
 
 struct GemmSmem {
   uint32_t a, b, codes, sc, xs, bar, total;
-  int ns, b_stage_bytes, codes_stage_bytes, sc_buf_bytes;
+  int na, nb, nc, b_stage_bytes, codes_stage_bytes, sc_buf_bytes;
 };
 
-__host__ __device__ inline GemmSmem gemm_smem(int mode, int bits, int K, int group, int ns) {
+// Rings: codes (nc k-blocks, freed once unpacked), B tiles (nb, freed by the
+// MMAs), unpacked A tiles (na, freed by the MMAs).
+__host__ __device__ inline GemmSmem gemm_smem(int mode, int bits, int K, int group, int na) {
   GemmSmem s{};
-  s.ns = ns;
   const int ng = K / group;
-  s.b_stage_bytes = (mode == 0 ? 1 : 2) * kNT * 128;  // up to kNT rows x 128 B (x2: h hi and lo)
+  s.na = na;
+  s.nb = 8;
+  s.b_stage_bytes = (mode == 0 ? 1 : 2) * kNT * 128;  // kNT rows x 128 B (x2: h hi and lo)
   s.codes_stage_bytes = kBM * (kBK * bits / 8);
-  s.sc_buf_bytes = 2 * kBM * ng * 2;                    // scales and biases of 128 rows
+  s.nc = (64 * 1024) / s.codes_stage_bytes;           // 64 KiB of codes in flight
+  s.sc_buf_bytes = 2 * kBM * ng * 2;                  // scales and biases of 128 rows
   uint32_t o = 0;
-  s.a = o;     o = al1k(o + ns * kBM * kBK * 2);
-  s.b = o;     o = al1k(o + ns * s.b_stage_bytes);
-  s.codes = o; o = al1k(o + ns * s.codes_stage_bytes);
+  s.a = o;     o = al1k(o + na * kBM * kBK * 2);
+  s.b = o;     o = al1k(o + s.nb * s.b_stage_bytes);
+  s.codes = o; o = al1k(o + s.nc * s.codes_stage_bytes);
   s.sc = o;    o = al1k(o + 2 * s.sc_buf_bytes);
-  s.xs = o;    o = al1k(o + 4 * ng * kNT * 4);          // group sums of the tile's columns, one copy per scaling warp
-  s.bar = o;   o += 256;
+  s.xs = o;    o = al1k(o + 4 * ng * kNT * 4);        // group sums of the tile's columns, one copy per scaling warp
+  s.bar = o;   o += 1024;  // up to ~70 mbarriers, the TMEM slot and the abort flag
   s.total = o + 1024;  // slack to align the dynamic base to 1 KiB
   return s;
 }
 
-__device__ __forceinline__ int b_box_index(int n) { return n <= 16 ? 0 : n <= 32 ? 1 : 2; }
+__device__ __forceinline__ int b_box_index(int n) { return n <= 16 ? 0 : 1; }
 __device__ __forceinline__ int b_box_rows(int i) { return 16 << i; }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.f + expf(-z)); }
@@ -102,10 +107,8 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ws
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0; it < kWaitIters; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitNs) break;
-    }
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitNs) break;
   }
   report(hdr, MOE_ERR_TIMEOUT, where);
   *abort = 1;
@@ -180,19 +183,23 @@ __device__ __forceinline__ void scale_slice(float* acc, uint32_t ta, float sc, f
 
 // ------------------------------------------------------------------ GEMM kernel
 
-template <int MODE, int BITS, int NS>
+template <int MODE, int BITS, int NA>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const GemmSmem L = gemm_smem(MODE, BITS, p.K, kBK, NS);
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bar);  // [NS] TMA landed (codes + B)
-  uint64_t* afull = full + NS;                               // [NS] A tile written
-  uint64_t* empty = afull + NS;                              // [NS] MMAs done with the stage
-  uint64_t* scfull = empty + NS;                             // [2] scales of a tile landed
-  uint64_t* scempty = scfull + 2;                            // [2] unpackers and scalers done with them
-  uint64_t* pfull = scempty + 2;                             // [kPBuf] a group's products are in TMEM
-  uint64_t* pempty = pfull + kPBuf;                          // [kPBuf] scalers have read them
-  uint64_t* drain = pempty + kPBuf;                          // MMA issuer: everything issued has finished
+  const GemmSmem L = gemm_smem(MODE, BITS, p.K, kBK, NA);
+  const int NC = L.nc, NB = L.nb;
+  uint64_t* cfull = reinterpret_cast<uint64_t*>(sm + L.bar);  // [NC] codes landed
+  uint64_t* cempty = cfull + NC;                              // [NC] codes unpacked
+  uint64_t* bfull = cempty + NC;                              // [NB] B tile landed
+  uint64_t* bempty = bfull + NB;                              // [NB] MMAs done with the B tile
+  uint64_t* afull = bempty + NB;                              // [NA] A tile written
+  uint64_t* aempty = afull + NA;                              // [NA] MMAs done with the A tile
+  uint64_t* scfull = aempty + NA;                             // [2] scales of a tile landed
+  uint64_t* scempty = scfull + 2;                             // [2] scalers done with them
+  uint64_t* pfull = scempty + 2;                              // [kPBuf] a group's products are in TMEM
+  uint64_t* pempty = pfull + kPBuf;                           // [kPBuf] scalers have read them
+  uint64_t* drain = pempty + kPBuf;                           // MMA issuer: everything issued has finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -205,14 +212,21 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   const int ntiles = nchunks * MT;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&full[i], 1);
+    for (int i = 0; i < NC; ++i) {
+      mbar_init(&cfull[i], 1);
+      mbar_init(&cempty[i], 8);
+    }
+    for (int i = 0; i < NB; ++i) {
+      mbar_init(&bfull[i], 1);
+      mbar_init(&bempty[i], 1);
+    }
+    for (int i = 0; i < NA; ++i) {
       mbar_init(&afull[i], 8);
-      mbar_init(&empty[i], 1);
+      mbar_init(&aempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&scfull[i], 1);
-      mbar_init(&scempty[i], 12);
+      mbar_init(&scempty[i], 4);
     }
     for (int i = 0; i < kPBuf; ++i) {
       mbar_init(&pfull[i], 1);
@@ -232,23 +246,47 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------ TMA producer
+    // ------------------------------------------------ codes producer (deep ring, freed by the unpackers)
+    if (lane == 0) {
+      for (int i = 0; i < 2; ++i) tc::prefetch_tmap(&p.tm_codes[i]);
+      int kbg = 0, last = -1;
+      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+        const int ci = t / MT, mt = t % MT;
+        const int e = p.chunks[3 * ci];
+        const bool shared = (e == p.E);
+        const int ez = shared ? 0 : e, mi = shared ? 1 : 0;
+        const int r0 = (MODE == 0) ? mt * 64 : mt * kBM;
+        const int r1 = (MODE == 0) ? p.rows / 2 + mt * 64 : mt * kBM + 64;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+          const int s = kbg % NC, u = kbg / NC;
+          if (u >= 1 && !wait_or_abort(&cempty[s], (u - 1) & 1, p.hdr, abort, 31)) { ok = false; break; }
+          unsigned char* cs = sm + L.codes + s * L.codes_stage_bytes;
+          tc::mbar_expect_tx(&cfull[s], static_cast<uint32_t>(L.codes_stage_bytes));
+          tc::tma_load_3d(cs, &p.tm_codes[mi], kb * CB, r0, ez, &cfull[s]);
+          tc::tma_load_3d(cs + 64 * CB, &p.tm_codes[mi], kb * CB, r1, ez, &cfull[s]);
+          tc::mbar_arrive(&cfull[s]);
+          last = kbg;
+        }
+        if (!ok) break;
+      }
+      // leave no copy in flight
+      for (int j = (last - NC + 1 > 0 ? last - NC + 1 : 0); j <= last; ++j) mbar_wait(&cfull[j % NC], (j / NC) & 1, p.hdr, 39);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------ B tiles and scales producer (freed by MMAs / scalers)
     if (lane == 0) {
       for (int i = 0; i < 2; ++i) {
-        tc::prefetch_tmap(&p.tm_codes[i]);
         tc::prefetch_tmap(&p.tm_scales[i]);
         tc::prefetch_tmap(&p.tm_biases[i]);
       }
-      int kbg = 0, it = 0;
-      int armed[NS];
-      for (int s = 0; s < NS; ++s) armed[s] = -1;
+      int kbg = 0, it = 0, last = -1;
       int sc_armed[2] = {-1, -1};
       for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++it) {
         const int ci = t / MT, mt = t % MT;
         const int e = p.chunks[3 * ci], start = p.chunks[3 * ci + 1], cnt = p.chunks[3 * ci + 2];
         const bool shared = (e == p.E);
-        const int ez = shared ? 0 : e;
-        const int mi = shared ? 1 : 0;  // which codes / scales maps
+        const int ez = shared ? 0 : e, mi = shared ? 1 : 0;
         const int bi = b_box_index(cnt);
         const int brows = b_box_rows(bi);
         const int tb = it & 1, tu = it >> 1;
@@ -264,24 +302,20 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         tc::tma_load_3d(scb + 3 * half_bytes, &p.tm_biases[mi], 0, r1, ez, &scfull[tb]);
         tc::mbar_arrive(&scfull[tb]);
         sc_armed[tb] = tu;
+        bool ok = true;
         for (int kb = 0; kb < nkb; ++kb, ++kbg) {
-          const int s = kbg % NS, u = kbg / NS;
-          if (u >= 1 && !wait_or_abort(&empty[s], (u - 1) & 1, p.hdr, abort, 31)) break;
-          unsigned char* cs = sm + L.codes + s * L.codes_stage_bytes;
+          const int s = kbg % NB, u = kbg / NB;
+          if (u >= 1 && !wait_or_abort(&bempty[s], (u - 1) & 1, p.hdr, abort, 32)) { ok = false; break; }
           unsigned char* bs = sm + L.b + s * L.b_stage_bytes;
-          const uint32_t bbytes = static_cast<uint32_t>(brows) * 128u * (MODE == 0 ? 1u : 2u);
-          tc::mbar_expect_tx(&full[s], static_cast<uint32_t>(L.codes_stage_bytes) + bbytes);
-          tc::tma_load_3d(cs, &p.tm_codes[mi], kb * CB, r0, ez, &full[s]);
-          tc::tma_load_3d(cs + 64 * CB, &p.tm_codes[mi], kb * CB, r1, ez, &full[s]);
-          tc::tma_load_2d(bs, &p.tm_b[bi], kb * kBK, start, &full[s]);
-          if (MODE == 1) tc::tma_load_2d(bs + kNT * 128, &p.tm_b2[bi], kb * kBK, start, &full[s]);
-          tc::mbar_arrive(&full[s]);
-          armed[s] = u;
+          tc::mbar_expect_tx(&bfull[s], static_cast<uint32_t>(brows) * 128u * (MODE == 0 ? 1u : 2u));
+          tc::tma_load_2d(bs, &p.tm_b[bi], kb * kBK, start, &bfull[s]);
+          if (MODE == 1) tc::tma_load_2d(bs + kNT * 128, &p.tm_b2[bi], kb * kBK, start, &bfull[s]);
+          tc::mbar_arrive(&bfull[s]);
+          last = kbg;
         }
+        if (!ok) break;
       }
-      // leave no copy in flight: wait for the last phase armed on every barrier
-      for (int s = 0; s < NS; ++s)
-        if (armed[s] >= 0) mbar_wait(&full[s], armed[s] & 1, p.hdr, 39);
+      for (int j = (last - NB + 1 > 0 ? last - NB + 1 : 0); j <= last; ++j) mbar_wait(&bfull[j % NB], (j / NB) & 1, p.hdr, 37);
       for (int b = 0; b < 2; ++b)
         if (sc_armed[b] >= 0) mbar_wait(&scfull[b], sc_armed[b] & 1, p.hdr, 38);
     }
@@ -296,16 +330,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         const uint32_t idesc = tc::idesc_f16_f32(kBM, npad);
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb, ++kbg) {
-          const int s = kbg % NS, u = kbg / NS;
+          const int as = kbg % NA, au = kbg / NA;
+          const int bs = kbg % NB, bu = kbg / NB;
           const int pb = kbg % kPBuf, pu = kbg / kPBuf;
-          if (!wait_or_abort(&full[s], u & 1, p.hdr, abort, 41) || !wait_or_abort(&afull[s], u & 1, p.hdr, abort, 42) ||
+          if (!wait_or_abort(&afull[as], au & 1, p.hdr, abort, 41) || !wait_or_abort(&bfull[bs], bu & 1, p.hdr, abort, 42) ||
               (pu >= 1 && !wait_or_abort(&pempty[pb], (pu - 1) & 1, p.hdr, abort, 43))) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
-          const uint32_t a0 = smem_addr(sm + L.a + s * kBM * kBK * 2);
-          const uint32_t b0 = smem_addr(sm + L.b + s * L.b_stage_bytes);
+          const uint32_t a0 = smem_addr(sm + L.a + as * kBM * kBK * 2);
+          const uint32_t b0 = smem_addr(sm + L.b + bs * L.b_stage_bytes);
           const uint32_t dt = tmem + pb * kNT;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
@@ -313,7 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             tc::mma_f16(dt, ad, tc::smem_desc_sw128(b0 + kk * 32), idesc, kk != 0);
             if (MODE == 1) tc::mma_f16(dt, ad, tc::smem_desc_sw128(b0 + kNT * 128 + kk * 32), idesc, 1);
           }
-          tc::commit(&empty[s]);
+          tc::commit(&aempty[as]);
+          tc::commit(&bempty[bs]);
           tc::commit(&pfull[pb]);
         }
         if (!ok) break;
@@ -328,23 +364,25 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     const int m = d >> 1, half = d & 1;              // A-tile row, which 32 codes of the 64
     // A row m <- staging row: gate/up interleaved for mode 0, identity for mode 1
     const int srow = (MODE == 0) ? ((m & 1) * 64 + (m >> 1)) : m;
-    int kbg = 0, it = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+    int kbg = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       if (warp_aborted(abort)) break;
-      const int tb = it & 1;
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb, ++kbg) {
-        const int s = kbg % NS, u = kbg / NS;
-        if (!warp_wait(&full[s], u & 1, p.hdr, abort, 51)) { ok = false; break; }
-        if (u >= 1 && !warp_wait(&empty[s], (u - 1) & 1, p.hdr, abort, 52)) { ok = false; break; }
-        const unsigned char* crow = sm + L.codes + s * L.codes_stage_bytes + srow * CB + half * (CB / 2);
+        const int cs = kbg % NC, cu = kbg / NC;
+        const int as = kbg % NA, au = kbg / NA;
+        if (!warp_wait(&cfull[cs], cu & 1, p.hdr, abort, 51)) { ok = false; break; }
+        if (au >= 1 && !warp_wait(&aempty[as], (au - 1) & 1, p.hdr, abort, 52)) { ok = false; break; }
+        const unsigned char* crow = sm + L.codes + cs * L.codes_stage_bytes + srow * CB + half * (CB / 2);
         uint4 outv[4];
         if (BITS == 4) {
           unpack32_u4(*reinterpret_cast<const uint4*>(crow), outv);
         } else {
           unpack32_u8(*reinterpret_cast<const uint4*>(crow), *reinterpret_cast<const uint4*>(crow + 16), outv);
         }
-        unsigned char* arow = sm + L.a + s * kBM * kBK * 2 + (m >> 3) * 1024 + (m & 7) * 128;
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&cempty[cs]);  // codes read: the slot can be refilled
+        unsigned char* arow = sm + L.a + as * kBM * kBK * 2 + (m >> 3) * 1024 + (m & 7) * 128;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int chunk = half * 4 + q;
@@ -352,11 +390,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         }
         tc::fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&afull[s]);
+        if (lane == 0) tc::mbar_arrive(&afull[as]);
       }
       if (!ok) break;
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&scempty[tb]);  // this role does not read the scales; it keeps the count
     }
   } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------ scalers + epilogue (four independent warps)
@@ -398,9 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         const float sc = bf16_to_f32(scs[srow * ng + kb]);
         const float bi = bf16_to_f32(bis[srow * ng + kb]);
         const uint32_t ta = tmem + (static_cast<uint32_t>(32 * q) << 16) + pb * kNT;
-        const float* xg = xs + kb * kNT;
-        scale_slice<0>(acc, ta, sc, bi, xg, cnt);
-        scale_slice<32>(acc, ta, sc, bi, xg, cnt);
+        scale_slice<0>(acc, ta, sc, bi, xs + kb * kNT, cnt);
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&pempty[pb]);
@@ -513,10 +547,10 @@ __global__ void __launch_bounds__(256) combine_kernel(BatchParams p) {
   }
 }
 
-template <int MODE, int BITS, int NS>
+template <int MODE, int BITS, int NA>
 cudaError_t launch_gemm_t(const GemmParams& g, int grid, cudaStream_t st) {
-  const GemmSmem L = gemm_smem(MODE, BITS, g.K, kBK, NS);
-  auto kern = grouped_gemm_kernel<MODE, BITS, NS>;
+  const GemmSmem L = gemm_smem(MODE, BITS, g.K, kBK, NA);
+  auto kern = grouped_gemm_kernel<MODE, BITS, NA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, L.total, st>>>(g);
@@ -527,12 +561,12 @@ cudaError_t launch_gemm_t(const GemmParams& g, int grid, cudaStream_t st) {
 
 size_t grouped_gemm_smem(int mode, int bits, int K, int group) {
   (void)group;
-  return gemm_smem(mode, bits, K, kBK, mode == 0 ? 4 : 3).total;
+  return gemm_smem(mode, bits, K, kBK, kNA).total;
 }
 
 cudaError_t launch_grouped_gemm(const GemmParams& g, int mode, int bits, int grid, cudaStream_t st) {
-  if (mode == 0) return bits == 4 ? launch_gemm_t<0, 4, 4>(g, grid, st) : launch_gemm_t<0, 8, 4>(g, grid, st);
-  return bits == 4 ? launch_gemm_t<1, 4, 3>(g, grid, st) : launch_gemm_t<1, 8, 3>(g, grid, st);
+  if (mode == 0) return bits == 4 ? launch_gemm_t<0, 4, kNA>(g, grid, st) : launch_gemm_t<0, 8, kNA>(g, grid, st);
+  return bits == 4 ? launch_gemm_t<1, 4, kNA>(g, grid, st) : launch_gemm_t<1, 8, kNA>(g, grid, st);
 }
 
 cudaError_t launch_gather(const BatchParams& p, int grid, cudaStream_t st) {

@@ -406,7 +406,7 @@ bool decode_eligible(const moe_config& c, int* grid) {
     return false;
   const size_t smem =
       moe::decode_stack_smem(c.hidden, c.num_experts, c.top_k, c.inter, c.shared_inter, c.group, c.bits, d.sms);
-  if (smem + 1024 > static_cast<size_t>(d.smem_optin)) return false;
+  if (d.smem_optin < 1024 || smem > static_cast<size_t>(d.smem_optin) - 1024) return false;
   *grid = d.sms;
   return true;
 }

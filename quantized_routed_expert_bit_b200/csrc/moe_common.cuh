@@ -95,14 +95,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// One test of phase `parity`; if it is not complete the thread may be
+// suspended (up to the hint, 0.5 ms) until it completes, instead of spinning
+// and taking issue slots from the warps doing the work.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(500000u)
       : "memory");
   return ok != 0;
 }
@@ -114,7 +117,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, WsHead
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0; it < kWaitIters; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitNs) break;
+    if (globaltimer_ns() - t0 > kWaitNs) break;
   }
   report(hdr, MOE_ERR_TIMEOUT, where);
   return false;

@@ -44,7 +44,7 @@ __host__ __device__ constexpr int al8(int v) { return (v + 7) & ~7; }
 
 // Shared-memory carve-up; identical on host (sizing) and device.
 struct Carve {
-  int PS, nseg_x, nslots, Imax, npc_max, ng, nr_max, ng_dmax, rowb_dmax, d_sc_el, rr_max;
+  int PS, nseg_x, nslots, Imax, npc_max, ng, nr_max, ng_dmax, rowb_dmax, d_sc_el, rr_max, rowb;
   uint32_t xs, xsum, xn, r, dred, gsb, dbuf, d_slot_bytes, rbuf, total;
 };
 
@@ -70,7 +70,12 @@ __host__ __device__ inline Carve carve(int H, int E, int k, int I, int Is, int g
   c.dred = o;  o = al128(o + c.nslots * c.nr_max * 4);
   c.gsb = o;   o = al128(o + 4 * c.npc_max * c.ng * 2);
   c.d_slot_bytes = al128(c.nr_max * c.rowb_dmax + 2 * c.d_sc_el * 2);
-  c.dbuf = o;  o = al128(o + c.nslots * c.d_slot_bytes);
+  c.rowb = H * bits / 8;
+  // one buffer, used first for this CTA's gate/up code rows ([gate rows][up rows]),
+  // then for its down rows of every slot
+  const uint32_t gu_bytes = 2u * c.npc_max * c.rowb;
+  const uint32_t dn_bytes = c.nslots * c.d_slot_bytes;
+  c.dbuf = o;  o = al128(o + (gu_bytes > dn_bytes ? gu_bytes : dn_bytes));
   c.rbuf = o;  o = al128(o + 2 * c.rr_max * H * 2);
   c.total = o;
   return c;
@@ -230,12 +235,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
   extern __shared__ __align__(128) unsigned char sm[];
   __shared__ __align__(8) uint64_t bar_r[2];
   __shared__ __align__(8) uint64_t bar_g, bar_d;
+  __shared__ __align__(8) uint64_t bar_gc[3];  // gate/up code rows of pairs [0,16), [16,32), [32,48)
   __shared__ int s_idx[16];
   __shared__ float s_w[16];
   __shared__ float s_sg;
   __shared__ int s_abort;
   __shared__ float s_red[kWarps];
-  __shared__ int s_pend[4];  // outstanding copy phases: router[0], router[1], gate/up scales, down rows
+  __shared__ int s_pend[5];  // outstanding copy phases: router[0], router[1], gate/up scales, down rows, gate/up codes
 
   const int H = p.H, E = p.E, k = p.k, I = p.I, Is = p.Is, group = p.group;
   const int G = gridDim.x, c = blockIdx.x;
@@ -268,9 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
     mbar_init(&bar_r[1], 1);
     mbar_init(&bar_g, 1);
     mbar_init(&bar_d, 1);
+    for (int b = 0; b < 3; ++b) mbar_init(&bar_gc[b], 1);
     fence_mbar_init();
     s_abort = 0;
-    s_pend[0] = s_pend[1] = s_pend[2] = s_pend[3] = -1;
+    s_pend[0] = s_pend[1] = s_pend[2] = s_pend[3] = s_pend[4] = -1;
   }
   __syncthreads();
 
@@ -293,6 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
       if (s_pend[1] >= 0) mbar_wait(&bar_r[1], s_pend[1], p.hdr, 91);
       if (s_pend[2] >= 0) mbar_wait(&bar_g, s_pend[2], p.hdr, 92);
       if (s_pend[3] >= 0) mbar_wait(&bar_d, s_pend[3], p.hdr, 93);
+      if (s_pend[4] >= 0)
+        for (int b = 0; b < 3; ++b) mbar_wait(&bar_gc[b], s_pend[4], p.hdr, 94);
     }
     __syncthreads();
   };
@@ -386,34 +395,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         P += n;
         ++seg;
       }
-      // down rows of every slot: codes, scales, biases (3 copies per slot)
-      for (int c3 = lane; c3 < 3 * nslots && nr > 0; c3 += 32) {
-        const int j = c3 / 3, which = c3 % 3;
-        const bool routed = j < k;
-        const QMat m = routed ? Ld.dn : Ld.sdn;
-        const int Ij = routed ? I : Is;
-        const int ngd = Ij / group;
-        const size_t rowbd = static_cast<size_t>(Ij) * BITS / 8;
-        const int e = routed ? s_idx[j] : 0;
-        unsigned char* slot = dbuf + static_cast<size_t>(j) * cv.d_slot_bytes;
-        if (which == 0) {
-          copy_tx(slot, m.q + static_cast<size_t>(e) * m.q_stride + static_cast<size_t>(r0) * rowbd,
-                  static_cast<uint32_t>(nr * rowbd), &bar_d);
-        } else {
-          const int el0 = (r0 * ngd) & ~7;
-          const int el1 = al8(r1 * ngd);
-          uint16_t* sc = reinterpret_cast<uint16_t*>(slot + static_cast<size_t>(cv.nr_max) * cv.rowb_dmax);
-          const size_t eo = static_cast<size_t>(e) * m.sb_stride + el0;
-          copy_tx(sc + (which == 2 ? cv.d_sc_el : 0), (which == 2 ? m.b : m.s) + eo,
-                  static_cast<uint32_t>(el1 - el0) * 2u, &bar_d);
+      // gate/up code rows of this CTA's pairs, in batches of 16 pairs (one
+      // mbarrier each): per batch and slot segment one copy of gate rows, one of up rows
+      {
+        int c2 = 0;
+        for (int b = 0; b < 3; ++b) {
+          const int q_lo = 16 * b, q_hi = min(npc, 16 * b + 16);
+          int P2 = gp0 + q_lo;
+          while (P2 < gp0 + q_hi) {
+            const bool routed = P2 < k * I;
+            const int j = routed ? P2 / I : k;
+            const int sstart = routed ? j * I : k * I;
+            const int send = routed ? (j + 1) * I : k * I + Is;
+            const int n = min(gp0 + q_hi, send) - P2;
+            const int qq = P2 - gp0;
+            for (int gu = 0; gu < 2; ++gu, ++c2) {
+              if (lane == 16 + (c2 & 15)) {
+                const QMat m = routed ? Ld.gu : Ld.sgu;
+                const int Ij = routed ? I : Is;
+                const uint8_t* src = m.q + static_cast<size_t>(routed ? s_idx[j] : 0) * m.q_stride +
+                                     static_cast<size_t>(gu * Ij + (P2 - sstart)) * rowb;
+                copy_tx(dbuf + (static_cast<size_t>(gu) * cv.npc_max + qq) * rowb, src,
+                        static_cast<uint32_t>(n * rowb), &bar_gc[b]);
+              }
+            }
+            P2 += n;
+          }
         }
       }
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bar_g);
-        mbar_arrive(&bar_d);
+        for (int b = 0; b < 3; ++b) mbar_arrive(&bar_gc[b]);
         s_pend[2] = l & 1;
-        s_pend[3] = l & 1;
+        s_pend[4] = l & 1;
       }
       __syncwarp();
     }
@@ -425,33 +440,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
       for (int m0 = warp; m0 < npc; m0 += kWarps * RB) {
         uint4 cg[RB][CH], cu[RB][CH];
         int qv[RB];
+        if (!waited) {
+          if (!mbar_wait(&bar_g, l & 1, p.hdr, 11)) s_abort = 1;
+          waited = true;
+        }
 #pragma unroll
         for (int b = 0; b < RB; ++b) {
           const int q = m0 + b * kWarps;
           qv[b] = q;
           if (q < npc) {
-            const int P = gp0 + q;
-            const bool routed = P < k * I;
-            const int j = routed ? P / I : k;
-            const int i = routed ? P - j * I : P - k * I;
-            const QMat m = routed ? Ld.gu : Ld.sgu;
-            const int Ij = routed ? I : Is;
-            const uint8_t* base = m.q + static_cast<size_t>(routed ? s_idx[j] : 0) * m.q_stride;
-            const uint8_t* qg = base + static_cast<size_t>(i) * rowb;
-            const uint8_t* qu = base + static_cast<size_t>(Ij + i) * rowb;
+            if (!mbar_wait(&bar_gc[q >> 4], l & 1, p.hdr, 14)) s_abort = 1;
+            const unsigned char* qg = dbuf + static_cast<size_t>(q) * rowb;
+            const unsigned char* qu = dbuf + (static_cast<size_t>(cv.npc_max) + q) * rowb;
 #pragma unroll
             for (int ch = 0; ch < CH; ++ch) {
               const int s = lane + 32 * ch;
               if (s < nseg_x) {
-                cg[b][ch] = ldg_stream(qg + 16 * static_cast<size_t>(s));
-                cu[b][ch] = ldg_stream(qu + 16 * static_cast<size_t>(s));
+                cg[b][ch] = *reinterpret_cast<const uint4*>(qg + 16 * s);
+                cu[b][ch] = *reinterpret_cast<const uint4*>(qu + 16 * s);
               }
             }
           }
-        }
-        if (!waited) {
-          if (!mbar_wait(&bar_g, l & 1, p.hdr, 11)) s_abort = 1;
-          waited = true;
         }
         float ag[RB], au[RB];
 #pragma unroll
@@ -503,7 +512,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
       }
     }
     __syncthreads();
-    if (tid == 0) s_pend[2] = -1;
+    if (tid == 0) {
+      s_pend[2] = -1;
+      s_pend[4] = -1;
+    }
+    // down rows of every slot into the same buffer (codes, scales, biases: 3 copies
+    // per slot, by warp 0's lanes); they travel while the grid waits on h
+    if (warp == 0) {
+      for (int c3 = lane; c3 < 3 * nslots && nr > 0; c3 += 32) {
+        const int j = c3 / 3, which = c3 % 3;
+        const bool routed = j < k;
+        const QMat m = routed ? Ld.dn : Ld.sdn;
+        const int Ij = routed ? I : Is;
+        const int ngd = Ij / group;
+        const size_t rowbd = static_cast<size_t>(Ij) * BITS / 8;
+        const int e = routed ? s_idx[j] : 0;
+        unsigned char* slot = dbuf + static_cast<size_t>(j) * cv.d_slot_bytes;
+        if (which == 0) {
+          copy_tx(slot, m.q + static_cast<size_t>(e) * m.q_stride + static_cast<size_t>(r0) * rowbd,
+                  static_cast<uint32_t>(nr * rowbd), &bar_d);
+        } else {
+          const int el0 = (r0 * ngd) & ~7;
+          const int el1 = al8(r1 * ngd);
+          uint16_t* sc = reinterpret_cast<uint16_t*>(slot + static_cast<size_t>(cv.nr_max) * cv.rowb_dmax);
+          const size_t eo = static_cast<size_t>(e) * m.sb_stride + el0;
+          copy_tx(sc + (which == 2 ? cv.d_sc_el : 0), (which == 2 ? m.b : m.s) + eo,
+                  static_cast<uint32_t>(el1 - el0) * 2u, &bar_d);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar_d);
+        s_pend[3] = l & 1;
+      }
+    }
     stamp(4);
     if (!grid_barrier(p, ++epoch, &s_abort)) { drain(); return; }
     stamp(5);
@@ -623,6 +665,8 @@ cudaError_t launch_t(const DecodeParams& p, size_t smem, int grid, cudaStream_t 
 }  // namespace
 
 size_t decode_stack_smem(int H, int E, int k, int I, int Is, int group, int bits, int grid) {
+  // the gate/up code rows of a CTA are staged in three batches of 16 pairs
+  if (cdiv(k * I + Is, grid) > 48) return ~size_t(0);
   return carve(H, E, k, I, Is, group, bits, grid).total;
 }
 
