@@ -42,7 +42,7 @@ size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 // Byte offsets of the workspace regions for T tokens.
 struct Layout {
   size_t hdr, counters, logits, sgate, h, r, xa, xb, y, idx, w;
-  size_t flags, dlogits, dh, dy, dr, dx;                  // persistent single-token decode
+  size_t dlogits, dh, dy, dr, dx;                         // persistent single-token decode
   size_t base_total;                                      // end of the regions above
   size_t perm, offs, chunks, nchunks, x16, hhi, hlo, o;   // batched tensor-core path
   size_t xsx, xsh;                                        // group sums of x and of h
@@ -51,7 +51,7 @@ struct Layout {
 
 constexpr int kBatchMinTokens = 8;  // from this many tokens the grouped tensor-core path runs
 
-constexpr int kMaxGrid = 1024;  // barrier flags reserved for the persistent decode grid
+constexpr int kMaxGrid = 1024;  // largest persistent decode grid
 
 Layout layout(const moe_config& c, int64_t T) {
   Layout L{};
@@ -69,10 +69,9 @@ Layout layout(const moe_config& c, int64_t T) {
   L.y = o;        o += up(static_cast<size_t>(T) * c.hidden * 2);
   L.idx = o;      o += up(static_cast<size_t>(T) * c.top_k * 4);
   L.w = o;        o += up(static_cast<size_t>(T) * c.top_k * 4);
-  L.flags = o;    o += up(static_cast<size_t>(kMaxGrid) * 4);
-  L.dlogits = o;  o += up(static_cast<size_t>(c.num_experts + 1) * 4);
-  L.dh = o;       o += up(static_cast<size_t>(c.top_k + 1) * imax * 4);
-  L.dy = o;       o += up(static_cast<size_t>(c.hidden) * 2);
+  L.dlogits = o;  o += up(static_cast<size_t>(c.num_experts + 1) * 4);   // decode exchange words:
+  L.dh = o;       o += up(static_cast<size_t>(c.top_k + 1) * imax * 4);  //   logits, h, y (contiguous,
+  L.dy = o;       o += up(static_cast<size_t>(c.hidden) * 4);             //   zeroed before each launch)
   L.dr = o;       o += up(static_cast<size_t>(c.hidden) * 4);
   L.dx = o;       o += up(static_cast<size_t>(c.hidden) * 2);
   L.base_total = o;
@@ -435,18 +434,15 @@ moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, in
   P->Is = c.shared_inter;
   P->group = c.group;
   P->renorm = c.renorm;
-  P->layer_mode = 0;
-  P->epoch0 = 0;
   P->eps = 1e-6f;
   P->tr_x = trace ? trace->x : nullptr;
   P->tr_idx = trace ? trace->idx : nullptr;
   P->tr_w = trace ? trace->w : nullptr;
   P->tr_y = trace ? trace->y : nullptr;
   P->tr_t = trace ? trace->t : nullptr;
-  P->logits = reinterpret_cast<float*>(b + Ly.dlogits);
-  P->hbuf = reinterpret_cast<float*>(b + Ly.dh);
-  P->ybuf = reinterpret_cast<uint16_t*>(b + Ly.dy);
-  P->flags = reinterpret_cast<unsigned*>(b + Ly.flags);
+  P->logits = reinterpret_cast<uint32_t*>(b + Ly.dlogits);
+  P->hbuf = reinterpret_cast<uint32_t*>(b + Ly.dh);
+  P->ybuf = reinterpret_cast<uint32_t*>(b + Ly.dy);
   P->hdr = reinterpret_cast<moe::WsHeader*>(b + Ly.hdr);
   uint16_t* xmid = reinterpret_cast<uint16_t*>(b + Ly.dx);
   float* rmid = reinterpret_cast<float*>(b + Ly.dr);
@@ -460,8 +456,8 @@ moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, in
     P->out = last ? x_out : xmid;
     P->r_out = last ? nullptr : rmid;
     for (int i = 0; i < n; ++i) P->layers[i] = layer_desc(layers[l0 + i]);
-    cudaError_t e = cudaMemsetAsync(P->flags, 0, static_cast<size_t>(grid) * 4, st);
-    if (e != cudaSuccess) return cuda_fail(e, "barrier flag reset");
+    cudaError_t e = cudaMemsetAsync(b + Ly.dlogits, 0, Ly.dr - Ly.dlogits, st);
+    if (e != cudaSuccess) return cuda_fail(e, "exchange word reset");
     e = moe::launch_decode_stack(*P, c.bits, grid, st);
     if (e != cudaSuccess) return cuda_fail(e, "decode_stack launch");
   }

@@ -110,8 +110,6 @@ constexpr int kMaxDecodeLayers = 128;  // layers per launch (kernel parameter sp
 struct DecodeParams {
   int L, l0;             // layers in this launch; index of its first layer in the stack
   int H, E, k, I, Is, group, renorm;
-  int layer_mode;        // 1: one layer, y -> out (no residual/norm); 0: stack, x_L -> out
-  unsigned epoch0;       // barrier epochs start above this value
   float eps;
   const uint16_t* x0;    // bf16 [H] input of the first layer
   const float* r_in;     // fp32 [H] residual at the first layer, or null (= x0)
@@ -122,10 +120,10 @@ struct DecodeParams {
   float* tr_w;           // [layers][k] or null
   uint16_t* tr_y;        // bf16 [layers][H] or null
   uint64_t* tr_t;        // [layers][8] phase timestamps of CTA 0, or null
-  float* logits;         // fp32 [E+1] (workspace)
-  float* hbuf;           // fp32 [k+1][Imax] (workspace)
-  uint16_t* ybuf;        // bf16 [H] (workspace)
-  unsigned* flags;       // grid barrier counter, zero at launch (workspace)
+  // exchange words between CTAs (workspace), zero at launch
+  uint32_t* logits;      // [E+1] fp32 logits, last mantissa bit = layer parity
+  uint32_t* hbuf;        // [k+1][I] fp32 SwiGLU outputs, last mantissa bit = layer parity
+  uint32_t* ybuf;        // [H] bf16 layer output << 16 | 16-bit layer tag
   WsHeader* hdr;
   LayerDesc layers[kMaxDecodeLayers];
 };

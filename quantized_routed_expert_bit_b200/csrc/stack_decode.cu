@@ -1,29 +1,37 @@
 // Persistent single-token decode of a whole MoE stack in one launch.
 //
 // One CTA per SM, all co-resident (cooperative launch), walks every layer:
-//   1. router rows: each CTA owns E/G rows of the router (plus the shared
+//   1. residual + parameter-free RMSNorm of the previous layer's output
+//      (every CTA redundantly, identical arithmetic), giving this layer's x;
+//   2. router rows: each CTA owns E/G rows of the router (plus the shared
 //      expert's gate vector as row E), prefetched into shared memory by bulk
-//      copies one layer ahead, and writes their logits;
-//   2. grid barrier, then every CTA runs softmax + top-k itself (one warp);
-//   3. the CTA's share of the selected experts' packed gate/up row pairs
-//      (k*I + Is pairs split evenly over the grid) streams through registers
-//      with 128-bit loads while one thread issues bulk copies of their scales
-//      and biases and of the CTA's down-projection rows of every selected
-//      expert (fetched now, used after the next barrier);
-//   4. grid barrier on h, then every CTA computes its H/G output rows: the
-//      weighted combine of the k routed experts and the gated shared expert;
-//   5. grid barrier on y, then every CTA applies the residual and the
-//      parameter-free RMSNorm to the full vector itself (identical arithmetic
-//      in every CTA), giving the next layer's input without another pass.
+//      copies one layer ahead, and publishes their logits;
+//   3. softmax + top-k in every CTA from all published logits (one warp);
+//   4. the CTA's share of the selected experts' packed gate/up row pairs
+//      (k*I + Is pairs split evenly over the grid) lands in shared memory by
+//      bulk copies in batches of 8 pairs; the dot products dequantize in
+//      registers; SwiGLU of each pair is published as h;
+//   5. every CTA computes its H/G output rows from all published h: the
+//      weighted combine of the k routed down projections and the gated shared
+//      expert, and publishes them as y.
 // Routing fan-out and shared experts: Swiftlet article (xix.ai), paragraphs
 // 4 and 8; Runnel README, "Target". Low-bit groups: same article, paragraph
 // 8. Packed gate/up: Runnel README, introduction and "Streaming CLI".
 //
-// Grid barriers are per-CTA flags in global memory holding a rising epoch:
-// a CTA publishes its epoch with a release store after __syncthreads, and
-// waits until every flag has reached it. Every wait is bounded (time and
-// polls); a CTA that gives up records MOE_ERR_TIMEOUT, and the others see the
-// status word and leave too, after draining their own bulk copies.
+// Exchanges between CTAs carry their own layer tag, so no grid barrier and no
+// memory fence is needed: every exchanged value is one 32-bit word written
+// once per layer with a relaxed store, and a reader polls the words
+// themselves until every one carries the current layer's tag.
+//  - logits and h are fp32 whose least significant mantissa bit is replaced
+//    by the layer parity (a change of at most one unit in the last place);
+//  - y is a bf16 in the high half with a 16-bit layer tag in the low half.
+// One bit of parity is enough for logits and h: every word is rewritten in
+// every layer, a writer of layer l+1 has necessarily seen all of layer l's
+// exchanges (so every reader of layer l is done with it), and the host
+// zeroes the exchange words before each launch (layer tags start at 1).
+// Every poll and every mbarrier wait is bounded (time and polls); a CTA that
+// gives up records MOE_ERR_TIMEOUT, the others see the status word and leave
+// too, each after draining its own bulk copies.
 
 #include <cfloat>
 #include <climits>
@@ -37,6 +45,10 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
+constexpr int kBatch = 8;        // gate/up pairs per code batch (one mbarrier each)
+constexpr int kMaxBatches = 8;   // at most 64 pairs per CTA
+constexpr int kHChunks = 4;      // 16-byte chunks of h each thread reads: (k+1)*I <= 4*4*512
+constexpr int kTopPer = 16;      // logits per lane in the top-k warp: E <= 512
 
 __host__ __device__ constexpr uint32_t al128(uint32_t v) { return (v + 127u) & ~127u; }
 __host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -44,33 +56,33 @@ __host__ __device__ constexpr int al8(int v) { return (v + 7) & ~7; }
 
 // Shared-memory carve-up; identical on host (sizing) and device.
 struct Carve {
-  int PS, nseg_x, nslots, Imax, npc_max, ng, nr_max, ng_dmax, rowb_dmax, d_sc_el, rr_max, rowb;
-  uint32_t xs, xsum, xn, r, dred, gsb, dbuf, d_slot_bytes, rbuf, total;
+  int PS, nsg, nsgd, nslots, npc_max, ng, nr_max, ngd, rowb, rowbd, d_sc_el, rr_max;
+  uint32_t xs, xn, rr, hs, dred, guv, gsb, dbuf, d_slot_bytes, rbuf, total;
 };
 
 __host__ __device__ inline Carve carve(int H, int E, int k, int I, int Is, int group, int bits, int G) {
   Carve c{};
   c.PS = 128 / bits;
-  c.nseg_x = H / c.PS;
+  c.nsg = H / c.PS;
+  c.nsgd = I / c.PS;
   c.nslots = k + (Is > 0 ? 1 : 0);
-  c.Imax = I > Is ? I : Is;
-  const int NP = k * I + Is;
-  c.npc_max = cdiv(NP, G) + 1;
+  c.npc_max = cdiv(k * I + Is, G) + 1;
   c.ng = H / group;
   c.nr_max = cdiv(H, G) + 1;
-  c.ng_dmax = c.Imax / group;
-  c.rowb_dmax = c.Imax * bits / 8;
-  c.d_sc_el = al8(c.nr_max * c.ng_dmax + 16);
+  c.ngd = I / group;
+  c.rowb = H * bits / 8;
+  c.rowbd = I * bits / 8;
+  c.d_sc_el = al8(c.nr_max * c.ngd + 16);
   c.rr_max = cdiv(E + (Is > 0 ? 1 : 0), G);
   uint32_t o = 0;
   c.xs = o;    o = al128(o + H * 4);
-  c.xsum = o;  o = al128(o + c.nseg_x * 4);
   c.xn = o;    o = al128(o + H * 4);
-  c.r = o;     o = al128(o + H * 4);
+  c.rr = o;    o = al128(o + H * 4);
+  c.hs = o;    o = al128(o + c.nslots * I * 4);
   c.dred = o;  o = al128(o + c.nslots * c.nr_max * 4);
+  c.guv = o;   o = al128(o + 2 * c.npc_max * 4);
   c.gsb = o;   o = al128(o + 4 * c.npc_max * c.ng * 2);
-  c.d_slot_bytes = al128(c.nr_max * c.rowb_dmax + 2 * c.d_sc_el * 2);
-  c.rowb = H * bits / 8;
+  c.d_slot_bytes = al128(c.nr_max * c.rowbd + 2 * c.d_sc_el * 2);
   // one buffer, used first for this CTA's gate/up code rows ([gate rows][up rows]),
   // then for its down rows of every slot
   const uint32_t gu_bytes = 2u * c.npc_max * c.rowb;
@@ -81,55 +93,77 @@ __host__ __device__ inline Carve carve(int H, int E, int k, int I, int Is, int g
   return c;
 }
 
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
 __device__ __forceinline__ void copy_tx(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  mbar_expect_tx(bar, bytes);
+  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
   bulk_g2s(dst, src, bytes, bar);
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.f + expf(-z)); }
-
-// All CTAs reach `epoch`. Returns false if this CTA must stop (a wait ran
-// out here or elsewhere). One counter in global memory: every CTA adds 1
-// with release semantics after __syncthreads; thread 0 alone polls it with
-// acquire loads and a short sleep, so the barrier puts almost no load on the
-// L2 slice that holds it.
-__device__ bool grid_barrier(const DecodeParams& p, unsigned epoch, volatile int* s_abort) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.flags) : "memory");
-    const unsigned target = epoch * gridDim.x;
-    bool ok = false;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 0; it < kWaitIters; ++it) {
-      unsigned v;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.flags) : "memory");
-      if (v >= target) {
-        ok = true;
-        break;
-      }
-      __nanosleep(32);
-      if ((it & 15u) == 0) {
-        const int st = *reinterpret_cast<volatile int*>(&p.hdr->status);
-        if (st != 0 || globaltimer_ns() - t0 > kWaitNs) break;
-      }
-    }
-    __threadfence();
-    if (!ok) {
-      report(p.hdr, MOE_ERR_TIMEOUT, 1000 + static_cast<int>(epoch));
-      *s_abort = 1;
-    }
-  }
-  __syncthreads();
-  return *s_abort == 0;
+__device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
+
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void st_word(uint32_t* a, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_word(const uint32_t* a) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint4 ld_words4(const uint32_t* a) {
+  uint4 v;
+  asm volatile("ld.relaxed.gpu.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(a)
+               : "memory");
+  return v;
+}
+
+// fp32 with its last mantissa bit replaced by the layer parity.
+__device__ __forceinline__ uint32_t tag_f32(float v, uint32_t par) {
+  return (__float_as_uint(v) & ~1u) | par;
+}
+
+// Checked every 16 polls of a tagged-word wait that started at t0: true once
+// the wait must end, because its time or poll limit ran out here
+// (MOE_ERR_TIMEOUT recorded) or some CTA has already recorded an error.
+__device__ __noinline__ bool give_up(uint64_t t0, uint32_t it, WsHeader* hdr, int where) {
+  if (*reinterpret_cast<volatile int*>(&hdr->status) != 0) return true;
+  if (globaltimer_ns() - t0 > kWaitNs || it >= kWaitIters) {
+    report(hdr, MOE_ERR_TIMEOUT, where);
+    return true;
+  }
+  return false;
+}
+
+// Between two polls that found a word not yet written: sleep a little; every
+// 16 polls ask give_up.
+#define MOE_POLL_BACKOFF(it, t0, hdr, where, fail) \
+  {                                                \
+    if ((it) == 0) (t0) = globaltimer_ns();        \
+    __nanosleep(128);                              \
+    if (((it) & 15u) == 15u && give_up((t0), (it), (hdr), (where))) { \
+      fail = true;                                 \
+      break;                                       \
+    }                                              \
+  }
+
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, WsHeader* hdr, int where) {
+  return mbar_wait(bar, parity, hdr, where);
+}
+
+__device__ __forceinline__ bool mbar_ready(uint64_t* bar, uint32_t parity, WsHeader* hdr, int where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, hdr, where);
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.f + expf(-z)); }
 
 // Order-preserving map of a float to an unsigned key (larger float, larger key).
 __device__ __forceinline__ unsigned fkey(float f) {
@@ -141,116 +175,51 @@ __device__ __forceinline__ float fkey_inv(unsigned k) {
   return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
 }
 
-// Softmax + top-k of one token by one warp: larger logit first, equal
-// logits to the lower expert index; weights renormalised over the k (or the
-// plain softmax probabilities when renorm == 0). Each lane sorts its PER
-// logits once (largest first, then lower index); every round one warp-wide
-// max over the lanes' heads picks the winner, whose lane pops its head.
-template <int PER>
-__device__ void topk_warp(const float* lg, int E, int k, int renorm, int* s_idx, float* s_w) {
-  const int lane = threadIdx.x & 31;
-  unsigned key[PER];
-  int idx[PER];
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int e = lane + 32 * i;
-    key[i] = (e < E) ? fkey(__ldcg(lg + e)) : 0u;
-    idx[i] = e;
+// Copy-phase bookkeeping for leaving early: parities of the phases this CTA
+// still has bulk copies in flight on (-1 = none).
+struct Pending {
+  int r[2], g, d, gc;
+};
+
+__device__ __noinline__ void drain(Pending* pend, uint64_t* bar_r, uint64_t* bar_g, uint64_t* bar_d,
+                                   uint64_t* bar_gc, int nb, WsHeader* hdr) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (pend->r[0] >= 0) mbar_wait(&bar_r[0], pend->r[0], hdr, 90);
+    if (pend->r[1] >= 0) mbar_wait(&bar_r[1], pend->r[1], hdr, 91);
+    if (pend->g >= 0) mbar_wait(bar_g, pend->g, hdr, 92);
+    if (pend->d >= 0) mbar_wait(bar_d, pend->d, hdr, 93);
+    if (pend->gc >= 0)
+      for (int b = 0; b < nb; ++b) mbar_wait(&bar_gc[b], pend->gc, hdr, 94);
   }
-  // odd-even transposition sort: key descending, index ascending among equal keys
-#pragma unroll
-  for (int r = 0; r < PER; ++r) {
-#pragma unroll
-    for (int i = (r & 1); i + 1 < PER; i += 2) {
-      const bool sw = key[i + 1] > key[i] || (key[i + 1] == key[i] && idx[i + 1] < idx[i]);
-      const unsigned k0 = key[i], k1 = key[i + 1];
-      const int i0 = idx[i], i1 = idx[i + 1];
-      key[i] = sw ? k1 : k0;
-      key[i + 1] = sw ? k0 : k1;
-      idx[i] = sw ? i1 : i0;
-      idx[i + 1] = sw ? i0 : i1;
-    }
-  }
-  const float mx = fkey_inv(__reduce_max_sync(0xffffffffu, key[0]));
-  float z = 0.f;
-  if (!renorm) {
-#pragma unroll
-    for (int i = 0; i < PER; ++i)
-      if (key[i] != 0u) z += expf(fkey_inv(key[i]) - mx);
-    z = warp_sum(z);
-  }
-  unsigned my_k = 0u;
-  int my_e = 0;
-  for (int j = 0; j < k; ++j) {
-    const unsigned wk = __reduce_max_sync(0xffffffffu, key[0]);
-    const unsigned we = __reduce_min_sync(0xffffffffu, key[0] == wk ? static_cast<unsigned>(idx[0]) : 0xffffffffu);
-    if (lane == j) {
-      my_k = wk;
-      my_e = static_cast<int>(we);
-    }
-    if (idx[0] == static_cast<int>(we) && key[0] == wk) {  // pop the head
-#pragma unroll
-      for (int i = 0; i + 1 < PER; ++i) {
-        key[i] = key[i + 1];
-        idx[i] = idx[i + 1];
-      }
-      key[PER - 1] = 0u;
-    }
-  }
-  const float ex = (lane < k) ? expf(fkey_inv(my_k) - mx) : 0.f;
-  const float den = renorm ? warp_sum(ex) : z;
-  if (lane < k) {
-    s_idx[lane] = my_e;
-    s_w[lane] = ex / den;
-  }
+  __syncthreads();
 }
 
-// x (bf16 bits, natural order) into the three shared views the layer uses.
-template <int PS>
-__device__ void set_x(float* xn, float* xs, float* xsum, int H, int i, float v) {
-  const int nseg = H / PS;
-  xn[i] = v;
-  const int s = i / PS, q = (i % PS) / 4, c4 = i % 4;
-  xs[(q * nseg + s) * 4 + c4] = v;
-}
-
-template <int PS>
-__device__ void finish_xsum(const float* xs, float* xsum, int H) {
-  const int nseg = H / PS;
-  for (int s = threadIdx.x; s < nseg; s += blockDim.x) {
-    float a = 0.f;
-#pragma unroll
-    for (int q = 0; q < PS / 4; ++q) {
-      const float4 f = reinterpret_cast<const float4*>(xs)[q * nseg + s];
-      a += (f.x + f.y) + (f.z + f.w);
-    }
-    xsum[s] = a;
-  }
-}
-
-template <int BITS, int CH, int RB>
+template <int BITS, int CH>
 __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_constant__ DecodeParams p) {
-  using CT = CodeTraits<BITS>;
-  constexpr int PS = CT::kPerSeg;
+  constexpr int PS = 128 / BITS;  // codes per 16-byte segment
   extern __shared__ __align__(128) unsigned char sm[];
   __shared__ __align__(8) uint64_t bar_r[2];
   __shared__ __align__(8) uint64_t bar_g, bar_d;
-  __shared__ __align__(8) uint64_t bar_gc[3];  // gate/up code rows of pairs [0,16), [16,32), [32,48)
+  __shared__ __align__(8) uint64_t bar_gc[kMaxBatches];
+  __shared__ __align__(16) LayerDesc s_ld[2];
   __shared__ int s_idx[16];
   __shared__ float s_w[16];
   __shared__ float s_sg;
-  __shared__ int s_abort;
   __shared__ float s_red[kWarps];
-  __shared__ int s_pend[5];  // outstanding copy phases: router[0], router[1], gate/up scales, down rows, gate/up codes
+  __shared__ Pending s_pend;
 
   const int H = p.H, E = p.E, k = p.k, I = p.I, Is = p.Is, group = p.group;
   const int G = gridDim.x, c = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  bool ab = false;  // a wait of this thread gave up; combined over the CTA at each phase end
   const Carve cv = carve(H, E, k, I, Is, group, BITS, G);
-  float* xs = reinterpret_cast<float*>(sm + cv.xs);
-  float* xsum = reinterpret_cast<float*>(sm + cv.xsum);
-  float* xn = reinterpret_cast<float*>(sm + cv.xn);
-  float* rr = reinterpret_cast<float*>(sm + cv.r);
+  float* xs = reinterpret_cast<float*>(sm + cv.xs);  // x by 16-byte code segment (conflict-free float4 reads)
+  float* xn = reinterpret_cast<float*>(sm + cv.xn);  // x in natural order
+  float* rr = reinterpret_cast<float*>(sm + cv.rr);  // residual stream, fp32
+  float* hs = reinterpret_cast<float*>(sm + cv.hs);  // h of every slot, by down code segment
+  float* dred = reinterpret_cast<float*>(sm + cv.dred);
+  float* guv = reinterpret_cast<float*>(sm + cv.guv);
   uint16_t* gsb = reinterpret_cast<uint16_t*>(sm + cv.gsb);
   unsigned char* dbuf = sm + cv.dbuf;
   uint16_t* rbuf = reinterpret_cast<uint16_t*>(sm + cv.rbuf);
@@ -260,82 +229,145 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
   const int gp0 = static_cast<int>(static_cast<int64_t>(c) * NP / G);
   const int gp1 = static_cast<int>(static_cast<int64_t>(c + 1) * NP / G);
   const int npc = gp1 - gp0;
+  const int nb = cdiv(npc, kBatch);
+  // the pair range covers at most two slots: [0, nA) in slot jA from slot row iA, then [nA, npc) in slot jA + 1
+  const int jA = gp0 < k * I ? gp0 / I : k;
+  const int endA = jA < k ? (jA + 1) * I : NP;
+  const int nA = min(gp1, endA) - gp0;
+  const int iA = gp0 - (jA < k ? jA * I : k * I);
   const int r0 = static_cast<int>(static_cast<int64_t>(c) * H / G);
   const int r1 = static_cast<int>(static_cast<int64_t>(c + 1) * H / G);
   const int nr = r1 - r0;
   const int nrows_rt = E + (Is > 0 ? 1 : 0);
   const int rr_cnt = (c < nrows_rt) ? cdiv(nrows_rt - c, G) : 0;
-  const int nseg_x = cv.nseg_x;
   const int nslots = cv.nslots;
-  const size_t rowb = static_cast<size_t>(H) * BITS / 8;
+  const int rowb = cv.rowb, rowbd = cv.rowbd, ng = cv.ng, ngd = cv.ngd;
+  const int lgI = 31 - __clz(I);          // I and group are powers of two
+  const int lgG = 31 - __clz(group);
 
   if (tid == 0) {
     mbar_init(&bar_r[0], 1);
     mbar_init(&bar_r[1], 1);
     mbar_init(&bar_g, 1);
     mbar_init(&bar_d, 1);
-    for (int b = 0; b < 3; ++b) mbar_init(&bar_gc[b], 1);
+    for (int b = 0; b < kMaxBatches; ++b) mbar_init(&bar_gc[b], 1);
     fence_mbar_init();
-    s_abort = 0;
-    s_pend[0] = s_pend[1] = s_pend[2] = s_pend[3] = s_pend[4] = -1;
+    s_pend.r[0] = s_pend.r[1] = s_pend.g = s_pend.d = s_pend.gc = -1;
   }
+  constexpr int kDescWords = sizeof(LayerDesc) / 8;
+  static_assert(sizeof(LayerDesc) % 8 == 0 && kDescWords <= 32, "layer descriptor copy");
+  if (warp == 1 && lane < kDescWords)
+    reinterpret_cast<uint64_t*>(&s_ld[0])[lane] = reinterpret_cast<const uint64_t*>(&p.layers[0])[lane];
   __syncthreads();
 
-  auto issue_router = [&](int l) {  // thread 0 only
-    const LayerDesc& Ld = p.layers[l];
+  auto issue_router = [&](int l) {  // thread 0; s_ld[l & 1] holds layer l
+    const LayerDesc& Ld = s_ld[l & 1];
     const int b = l & 1;
+#pragma unroll 1
     for (int m = 0; m < rr_cnt; ++m) {
       const int row = c + m * G;
       const uint16_t* src = (row < E) ? Ld.wr + static_cast<size_t>(row) * H : Ld.wsg;
       copy_tx(rbuf + (static_cast<size_t>(b) * cv.rr_max + m) * H, src, static_cast<uint32_t>(H) * 2, &bar_r[b]);
     }
-    mbar_arrive(&bar_r[b]);
-    s_pend[b] = (l >> 1) & 1;
+    mbar_arrive1(&bar_r[b]);
+    s_pend.r[b] = (l >> 1) & 1;
   };
-  // Waits out every copy this CTA still has in flight (used before leaving early).
-  auto drain = [&]() {
-    __syncthreads();
-    if (tid == 0) {
-      if (s_pend[0] >= 0) mbar_wait(&bar_r[0], s_pend[0], p.hdr, 90);
-      if (s_pend[1] >= 0) mbar_wait(&bar_r[1], s_pend[1], p.hdr, 91);
-      if (s_pend[2] >= 0) mbar_wait(&bar_g, s_pend[2], p.hdr, 92);
-      if (s_pend[3] >= 0) mbar_wait(&bar_d, s_pend[3], p.hdr, 93);
-      if (s_pend[4] >= 0)
-        for (int b = 0; b < 3; ++b) mbar_wait(&bar_gc[b], s_pend[4], p.hdr, 94);
-    }
-    __syncthreads();
-  };
+  auto leave = [&]() { drain(&s_pend, bar_r, &bar_g, &bar_d, bar_gc, nb, p.hdr); };
 
   if (tid == 0) issue_router(0);
 
-  // ---- layer-0 input and residual
-  for (int i = tid; i < H; i += kThreads) {
-    const float v = bf16_to_f32(p.x0[i]);
-    set_x<PS>(xn, xs, xsum, H, i, v);
-    rr[i] = p.r_in ? p.r_in[i] : v;
-    if (c == 0 && p.tr_x) p.tr_x[static_cast<size_t>(p.l0) * H + i] = p.x0[i];
-  }
-  __syncthreads();
-  finish_xsum<PS>(xs, xsum, H);
-  __syncthreads();
+  // lane roles in the dot products: a row of nsg 16-byte code segments is
+  // covered by 32/nsg rows per warp step (nsg < 32) or by CH segments per lane
+  const int nsg = cv.nsg;
+  const int rps = nsg >= 32 ? 1 : 32 / nsg;
+  const int gsub = nsg >= 32 ? 0 : lane / nsg;
+  const int gs0 = nsg >= 32 ? lane : lane % nsg;
+  const int nsgd = cv.nsgd;
+  const int rpsd = 32 / nsgd;
+  const int dsub = lane / nsgd;
+  const int ds = lane % nsgd;
+  // this warp's share of the down work: units (slot, row step), slot-major
+  const int dn_upj = cdiv(nr, rpsd);
+  const int dn_u0 = warp * nslots * dn_upj / kWarps, dn_u1 = (warp + 1) * nslots * dn_upj / kWarps;
+  const int dn_j0 = dn_upj > 0 ? dn_u0 / dn_upj : 0;
+  const int dn_t0 = dn_u0 - dn_j0 * dn_upj;
 
-  unsigned epoch = p.epoch0;
   for (int l = 0; l < p.L; ++l) {
-    const LayerDesc& Ld = p.layers[l];
     const int lg = p.l0 + l;  // layer index within the whole stack (trace rows)
+    const uint32_t tag = static_cast<uint32_t>(l + 1);
+    const uint32_t par = tag & 1u;
     auto stamp = [&](int slot) {
       if (p.tr_t && c == 0 && tid == 0) p.tr_t[static_cast<size_t>(lg) * 8 + slot] = globaltimer_ns();
     };
     stamp(0);
-    if (tid == 0 && l + 1 < p.L) issue_router(l + 1);
+    // next layer's descriptor, then its router rows
+    if (warp == 1 && lane < kDescWords && l + 1 < p.L)
+      reinterpret_cast<uint64_t*>(&s_ld[(l + 1) & 1])[lane] =
+          reinterpret_cast<const uint64_t*>(&p.layers[l + 1])[lane];
 
-    // ---------------- 1. router rows
-    if (!mbar_wait(&bar_r[l & 1], (l >> 1) & 1, p.hdr, 10)) { s_abort = 1; }
-    if (tid == 0) s_pend[l & 1] = -1;
+    // ---------------- 1. this layer's x (and residual)
+    if (l == 0) {
+#pragma unroll 1
+      for (int i = tid; i < H; i += kThreads) {
+        const float v = bf16_to_f32(p.x0[i]);
+        xn[i] = v;
+        rr[i] = p.r_in ? p.r_in[i] : v;
+        if (c == 0 && p.tr_x) p.tr_x[static_cast<size_t>(p.l0) * H + i] = p.x0[i];
+      }
+    } else {
+      // y of the previous layer: 4 rows per thread
+      float ss = 0.f;
+      const int i4 = 4 * tid;
+      if (i4 < H) {
+        const uint32_t ytag = (tag - 1u) & 0xffffu;
+        uint4 w;
+        uint64_t t0 = 0;
+        for (uint32_t it = 0;; ++it) {
+          w = ld_words4(p.ybuf + i4);
+          if ((w.x & 0xffffu) == ytag && (w.y & 0xffffu) == ytag && (w.z & 0xffffu) == ytag &&
+              (w.w & 0xffffu) == ytag)
+            break;
+          MOE_POLL_BACKOFF(it, t0, p.hdr, 20, ab)
+        }
+        const uint32_t wy[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float v = rr[i4 + u] + __uint_as_float(wy[u] & 0xffff0000u);
+          rr[i4 + u] = v;
+          ss = fmaf(v, v, ss);
+        }
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) s_red[warp] = ss;
+      if (__syncthreads_or(ab)) { leave(); return; }
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) tot += s_red[w];
+      const float inv = 1.f / sqrtf(tot / static_cast<float>(H) + p.eps);
+#pragma unroll 1
+      for (int i = tid; i < H; i += kThreads) {
+        const uint16_t xb = f32_to_bf16(rr[i] * inv);
+        xn[i] = bf16_to_f32(xb);
+        if (c == 0 && p.tr_x) p.tr_x[static_cast<size_t>(lg) * H + i] = xb;
+      }
+    }
+    __syncthreads();
+    // x by code segment: xs[(q4 * nsg + s) * 4 + c4] = x[s * PS + q4 * 4 + c4]
+#pragma unroll 1
+    for (int i4 = tid; i4 < H / 4; i4 += kThreads) {
+      const int s = (4 * i4) / PS, q4 = ((4 * i4) % PS) / 4;
+      reinterpret_cast<float4*>(xs)[q4 * nsg + s] = reinterpret_cast<const float4*>(xn)[i4];
+    }
+    if (tid == 0 && l + 1 < p.L) issue_router(l + 1);
+    stamp(1);
+
+    // ---------------- 2. router rows -> logits
     if (warp < rr_cnt) {
+      if (!mbar_ready(&bar_r[l & 1], (l >> 1) & 1, p.hdr, 10)) ab = true;
       const int row = c + warp * G;
       const uint4* wv = reinterpret_cast<const uint4*>(rbuf + (static_cast<size_t>(l & 1) * cv.rr_max + warp) * H);
       float acc = 0.f;
+#pragma unroll 1
       for (int s = lane; s < H / 8; s += 32) {
         const uint4 w8 = wv[s];
         const float4 a = reinterpret_cast<const float4*>(xn)[2 * s];
@@ -350,279 +382,364 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         acc = fmaf(bf16_hi(w8.w), b.w, acc);
       }
       acc = warp_sum(acc);
-      if (lane == 0) p.logits[row] = acc + ((row < E && Ld.rbias) ? Ld.rbias[row] : 0.f);
+      const LayerDesc& Ld = s_ld[l & 1];
+      if (lane == 0) st_word(p.logits + row, tag_f32(acc + ((row < E && Ld.rbias) ? Ld.rbias[row] : 0.f), par));
     }
-    stamp(1);
-    if (!grid_barrier(p, ++epoch, &s_abort)) { drain(); return; }
+    if (tid == 0) s_pend.r[l & 1] = -1;
     stamp(2);
 
-    // ---------------- 2. softmax + top-k (every CTA)
+    // ---------------- 3. softmax + top-k (every CTA, warp 0)
     if (warp == 0) {
-      if (E <= 256) topk_warp<8>(p.logits, E, k, p.renorm, s_idx, s_w);
-      else topk_warp<16>(p.logits, E, k, p.renorm, s_idx, s_w);
-      if (lane == 0) s_sg = (Is > 0) ? 1.f / (1.f + expf(-__ldcg(p.logits + E))) : 0.f;
-      __syncwarp();
-      if (c == 0 && lane < k) {
-        if (p.tr_idx) p.tr_idx[static_cast<size_t>(lg) * k + lane] = s_idx[lane];
-        if (p.tr_w) p.tr_w[static_cast<size_t>(lg) * k + lane] = s_w[lane];
+      uint32_t wl[kTopPer];
+      uint32_t wsg = par;
+      {
+        uint64_t t0 = 0;
+        bool fail = false;
+        for (uint32_t it = 0;; ++it) {
+          bool ok = true;
+#pragma unroll
+          for (int i = 0; i < kTopPer; ++i) {
+            const int e = lane + 32 * i;
+            wl[i] = (e < E) ? ld_word(p.logits + e) : par;
+            ok &= (wl[i] & 1u) == par;
+          }
+          if (Is > 0 && lane == 0) {
+            wsg = ld_word(p.logits + E);
+            ok &= (wsg & 1u) == par;
+          }
+          if (__all_sync(0xffffffffu, ok)) break;
+          // warp-uniform give-up decision (lane 0 checks)
+          if (it == 0) t0 = globaltimer_ns();
+          __nanosleep(128);
+          if ((it & 15u) == 15u && __any_sync(0xffffffffu, lane == 0 && give_up(t0, it, p.hdr, 21))) {
+            fail = true;
+            break;
+          }
+        }
+        ab |= fail;
       }
+      unsigned key[kTopPer];
+      unsigned bk = 0u;
+      int bi = 0;
+#pragma unroll
+      for (int i = 0; i < kTopPer; ++i) {
+        key[i] = (lane + 32 * i < E) ? fkey(__uint_as_float(wl[i])) : 0u;
+        if (key[i] > bk) {
+          bk = key[i];
+          bi = i;
+        }
+      }
+      const float mx = fkey_inv(__reduce_max_sync(0xffffffffu, bk));
+      float z = 0.f;
+      if (!p.renorm) {  // softmax over all E: the words are re-read (complete and tagged by now)
+#pragma unroll 1
+        for (int e = lane; e < E; e += 32) z += expf(__uint_as_float(ld_word(p.logits + e)) - mx);
+        z = warp_sum(z);
+      }
+      unsigned my_k = 0u;
+      int my_e = 0;
+#pragma unroll 1
+      for (int j = 0; j < k; ++j) {
+        // winner: largest key, then lowest expert index
+        const unsigned wk = __reduce_max_sync(0xffffffffu, bk);
+        const unsigned we =
+            __reduce_min_sync(0xffffffffu, bk == wk ? static_cast<unsigned>(lane + 32 * bi) : 0xffffffffu);
+        if (lane == j) {
+          my_k = wk;
+          my_e = static_cast<int>(we);
+        }
+        if (static_cast<int>(we & 31u) == lane) {
+          const int wi = static_cast<int>(we >> 5);
+          bk = 0u;
+          bi = 0;
+#pragma unroll
+          for (int i = 0; i < kTopPer; ++i) {
+            if (i == wi) key[i] = 0u;
+            if (key[i] > bk) {
+              bk = key[i];
+              bi = i;
+            }
+          }
+        }
+      }
+      const float ex = (lane < k) ? expf(fkey_inv(my_k) - mx) : 0.f;
+      const float den = p.renorm ? warp_sum(ex) : z;
+      if (lane < k) {
+        s_idx[lane] = my_e;
+        s_w[lane] = ex / den;
+        if (c == 0) {
+          if (p.tr_idx) p.tr_idx[static_cast<size_t>(lg) * k + lane] = my_e;
+          if (p.tr_w) p.tr_w[static_cast<size_t>(lg) * k + lane] = ex / den;
+        }
+      }
+      if (lane == 0) s_sg = (Is > 0) ? 1.f / (1.f + expf(-__uint_as_float(wsg))) : 0.f;
     }
-    __syncthreads();
+    if (__syncthreads_or(ab)) { leave(); return; }
     stamp(3);
 
-    // ---------------- 3. bulk copies: gate/up scales+biases of this CTA's pairs, down rows
-    // (issued by the 32 lanes of warp 0 in parallel; lane 0 arrives once all are armed)
+    const LayerDesc& Ld = s_ld[l & 1];
+    // ---------------- 4a. bulk copies of this CTA's gate/up rows (warp 0), L2 prefetch of its down rows (warp 1)
     if (warp == 0) {
-      const int ng = cv.ng;
-      // gate/up scale and bias rows: the CTA's pairs fall in at most 3 slots
-      int P = gp0, seg = 0;
-      while (P < gp1) {
-        const bool routed = P < k * I;
-        const int j = routed ? P / I : k;
-        const int sstart = routed ? j * I : k * I;
-        const int send = routed ? (j + 1) * I : k * I + Is;
-        const int n = min(gp1, send) - P;
-        if (lane >= 4 * seg && lane < 4 * seg + 4) {
-          const int which = lane - 4 * seg;  // 0 gate scales, 1 up scales, 2 gate biases, 3 up biases
-          const int i0 = P - sstart;
-          const int q0 = P - gp0;
+      {  // codes: lane = (batch, segment, gate|up)
+        const int b = lane >> 2, sg = (lane >> 1) & 1, gu = lane & 1;
+        const int lo = max(sg == 0 ? 0 : nA, b * kBatch);
+        const int hi = min(sg == 0 ? nA : npc, b * kBatch + kBatch);
+        if (hi > lo) {
+          const int j = jA + sg;
+          const bool routed = j < k;
           const QMat m = routed ? Ld.gu : Ld.sgu;
           const int Ij = routed ? I : Is;
-          const size_t eoff = static_cast<size_t>(routed ? s_idx[j] : 0) * m.sb_stride;
-          const uint16_t* src = ((which & 2) ? m.b : m.s) + eoff + static_cast<size_t>((which & 1) ? Ij + i0 : i0) * ng;
-          copy_tx(gsb + (which * cv.npc_max + q0) * ng, src, static_cast<uint32_t>(n * ng) * 2u, &bar_g);
+          const int row = (sg == 0 ? iA : -nA) + lo;
+          const uint8_t* src = m.q + static_cast<size_t>(routed ? s_idx[j] : 0) * m.q_stride +
+                               static_cast<size_t>(gu * Ij + row) * rowb;
+          copy_tx(dbuf + static_cast<size_t>(gu * cv.npc_max + lo) * rowb, src, static_cast<uint32_t>((hi - lo) * rowb),
+                  &bar_gc[b]);
         }
-        P += n;
-        ++seg;
       }
-      // gate/up code rows of this CTA's pairs, in batches of 16 pairs (one
-      // mbarrier each): per batch and slot segment one copy of gate rows, one of up rows
-      {
-        int c2 = 0;
-        for (int b = 0; b < 3; ++b) {
-          const int q_lo = 16 * b, q_hi = min(npc, 16 * b + 16);
-          int P2 = gp0 + q_lo;
-          while (P2 < gp0 + q_hi) {
-            const bool routed = P2 < k * I;
-            const int j = routed ? P2 / I : k;
-            const int sstart = routed ? j * I : k * I;
-            const int send = routed ? (j + 1) * I : k * I + Is;
-            const int n = min(gp0 + q_hi, send) - P2;
-            const int qq = P2 - gp0;
-            for (int gu = 0; gu < 2; ++gu, ++c2) {
-              if (lane == 16 + (c2 & 15)) {
-                const QMat m = routed ? Ld.gu : Ld.sgu;
-                const int Ij = routed ? I : Is;
-                const uint8_t* src = m.q + static_cast<size_t>(routed ? s_idx[j] : 0) * m.q_stride +
-                                     static_cast<size_t>(gu * Ij + (P2 - sstart)) * rowb;
-                copy_tx(dbuf + (static_cast<size_t>(gu) * cv.npc_max + qq) * rowb, src,
-                        static_cast<uint32_t>(n * rowb), &bar_gc[b]);
-              }
-            }
-            P2 += n;
-          }
+      if (lane < 8) {  // scales and biases: lane = (segment, kind); kind 0/1 gate/up scales, 2/3 gate/up biases
+        const int sg = lane >> 2, kind = lane & 3;
+        const int lo = sg == 0 ? 0 : nA, hi = sg == 0 ? nA : npc;
+        if (hi > lo) {
+          const int j = jA + sg;
+          const bool routed = j < k;
+          const QMat m = routed ? Ld.gu : Ld.sgu;
+          const int Ij = routed ? I : Is;
+          const int row = (sg == 0 ? iA : -nA) + lo;
+          const uint16_t* src = ((kind & 2) ? m.b : m.s) + static_cast<size_t>(routed ? s_idx[j] : 0) * m.sb_stride +
+                                static_cast<size_t>((kind & 1) * Ij + row) * ng;
+          copy_tx(gsb + static_cast<size_t>(kind * cv.npc_max + lo) * ng, src, static_cast<uint32_t>((hi - lo) * ng) * 2u,
+                  &bar_g);
         }
       }
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&bar_g);
-        for (int b = 0; b < 3; ++b) mbar_arrive(&bar_gc[b]);
-        s_pend[2] = l & 1;
-        s_pend[4] = l & 1;
+        mbar_arrive1(&bar_g);
+#pragma unroll 1
+        for (int b = 0; b < nb; ++b) mbar_arrive1(&bar_gc[b]);
+        s_pend.g = l & 1;
+        s_pend.gc = l & 1;
       }
       __syncwarp();
-    }
-
-    // ---------------- 4. gate/up + SwiGLU of this CTA's row pairs
-    {
-      const int ng = cv.ng;
-      bool waited = false;
-      for (int m0 = warp; m0 < npc; m0 += kWarps * RB) {
-        uint4 cg[RB][CH], cu[RB][CH];
-        int qv[RB];
-        if (!waited) {
-          if (!mbar_wait(&bar_g, l & 1, p.hdr, 11)) s_abort = 1;
-          waited = true;
-        }
-#pragma unroll
-        for (int b = 0; b < RB; ++b) {
-          const int q = m0 + b * kWarps;
-          qv[b] = q;
-          if (q < npc) {
-            if (!mbar_wait(&bar_gc[q >> 4], l & 1, p.hdr, 14)) s_abort = 1;
-            const unsigned char* qg = dbuf + static_cast<size_t>(q) * rowb;
-            const unsigned char* qu = dbuf + (static_cast<size_t>(cv.npc_max) + q) * rowb;
-#pragma unroll
-            for (int ch = 0; ch < CH; ++ch) {
-              const int s = lane + 32 * ch;
-              if (s < nseg_x) {
-                cg[b][ch] = *reinterpret_cast<const uint4*>(qg + 16 * s);
-                cu[b][ch] = *reinterpret_cast<const uint4*>(qu + 16 * s);
-              }
-            }
-          }
-        }
-        float ag[RB], au[RB];
-#pragma unroll
-        for (int b = 0; b < RB; ++b) ag[b] = au[b] = 0.f;
-#pragma unroll
-        for (int ch = 0; ch < CH; ++ch) {
-          const int s = lane + 32 * ch;
-          if (s < nseg_x) {
-            float xv[PS];
-#pragma unroll
-            for (int q4 = 0; q4 < PS / 4; ++q4) {
-              const float4 f = reinterpret_cast<const float4*>(xs)[q4 * nseg_x + s];
-              xv[4 * q4] = f.x;
-              xv[4 * q4 + 1] = f.y;
-              xv[4 * q4 + 2] = f.z;
-              xv[4 * q4 + 3] = f.w;
-            }
-            const float xsm = xsum[s];
-            const int g = s * PS / group;
-#pragma unroll
-            for (int b = 0; b < RB; ++b) {
-              if (qv[b] < npc) {
-                const int q = qv[b];
-                const float sg = bf16_to_f32(gsb[(0 * cv.npc_max + q) * ng + g]);
-                const float su = bf16_to_f32(gsb[(1 * cv.npc_max + q) * ng + g]);
-                const float bg = bf16_to_f32(gsb[(2 * cv.npc_max + q) * ng + g]);
-                const float bu = bf16_to_f32(gsb[(3 * cv.npc_max + q) * ng + g]);
-                ag[b] = fmaf(sg, dot_seg<BITS>(cg[b][ch], xv), fmaf(bg, xsm, ag[b]));
-                au[b] = fmaf(su, dot_seg<BITS>(cu[b][ch], xv), fmaf(bu, xsm, au[b]));
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int b = 0; b < RB; ++b) {
-          const float gsum = warp_sum(ag[b]);
-          const float usum = warp_sum(au[b]);
-          if (lane == 0 && qv[b] < npc) {
-            const int P = gp0 + qv[b];
-            const bool routed = P < k * I;
-            const int j = routed ? P / I : k;
-            const int i = routed ? P - j * I : P - k * I;
-            __stcg(p.hbuf + static_cast<size_t>(j) * cv.Imax + i, silu_f(gsum) * usum);
-          }
-        }
-      }
-      if (!waited && npc > 0 && warp == 0) {
-        if (!mbar_wait(&bar_g, l & 1, p.hdr, 12)) s_abort = 1;
-      }
-    }
-    __syncthreads();
-    if (tid == 0) {
-      s_pend[2] = -1;
-      s_pend[4] = -1;
-    }
-    // down rows of every slot into the same buffer (codes, scales, biases: 3 copies
-    // per slot, by warp 0's lanes); they travel while the grid waits on h
-    if (warp == 0) {
-      for (int c3 = lane; c3 < 3 * nslots && nr > 0; c3 += 32) {
-        const int j = c3 / 3, which = c3 % 3;
+    } else if (warp == 1 && nr > 0) {
+#pragma unroll 1
+      for (int t = lane; t < 3 * nslots; t += 32) {
+        const int j = t / 3, which = t % 3;
         const bool routed = j < k;
         const QMat m = routed ? Ld.dn : Ld.sdn;
-        const int Ij = routed ? I : Is;
-        const int ngd = Ij / group;
-        const size_t rowbd = static_cast<size_t>(Ij) * BITS / 8;
-        const int e = routed ? s_idx[j] : 0;
+        const size_t e = routed ? static_cast<size_t>(s_idx[j]) : 0;
+        if (which == 0) {
+          prefetch_l2(m.q + e * m.q_stride + static_cast<size_t>(r0) * rowbd, static_cast<uint32_t>(nr * rowbd));
+        } else {
+          const int el0 = (r0 * ngd) & ~7, el1 = al8(r1 * ngd);
+          prefetch_l2((which == 2 ? m.b : m.s) + e * m.sb_stride + el0, static_cast<uint32_t>(el1 - el0) * 2u);
+        }
+      }
+    }
+
+    // ---------------- 4b. gate/up rows + SwiGLU
+    {
+      float xv[CH][PS];
+      float xsm[CH];
+#pragma unroll
+      for (int ch = 0; ch < CH; ++ch) {
+        const int s = gs0 + 32 * ch;
+        float a = 0.f;
+#pragma unroll
+        for (int q4 = 0; q4 < PS / 4; ++q4) {
+          const float4 f = reinterpret_cast<const float4*>(xs)[q4 * nsg + s];
+          xv[ch][4 * q4] = f.x;
+          xv[ch][4 * q4 + 1] = f.y;
+          xv[ch][4 * q4 + 2] = f.z;
+          xv[ch][4 * q4 + 3] = f.w;
+          a += (f.x + f.y) + (f.z + f.w);
+        }
+        xsm[ch] = a;
+      }
+      bool scales_ready = false;
+#pragma unroll 1
+      for (int b = 0; b < nb; ++b) {
+        const int lo = b * kBatch, n = min(kBatch, npc - lo);
+        if (warp * rps >= 2 * n) continue;  // no row of this batch for this warp
+        if (!scales_ready) {
+          if (!mbar_ready(&bar_g, l & 1, p.hdr, 11)) ab = true;
+          scales_ready = true;
+        }
+        if (!mbar_ready(&bar_gc[b], l & 1, p.hdr, 12)) ab = true;
+        const int rho = warp * rps + gsub;  // [0, n) gate rows, [n, 2n) up rows of the batch
+        const int gu = rho >= n ? 1 : 0;
+        const int q = lo + rho - gu * n;
+        float acc = 0.f;
+        if (rho < 2 * n) {
+          const unsigned char* row = dbuf + static_cast<size_t>(gu * cv.npc_max + q) * rowb;
+          const uint16_t* sc = gsb + static_cast<size_t>(gu * cv.npc_max + q) * ng;
+          const uint16_t* bi = gsb + static_cast<size_t>((2 + gu) * cv.npc_max + q) * ng;
+#pragma unroll
+          for (int ch = 0; ch < CH; ++ch) {
+            const int s = gs0 + 32 * ch;
+            const uint4 cd = *reinterpret_cast<const uint4*>(row + 16 * s);
+            const int g = (s * PS) >> lgG;
+            acc = fmaf(bf16_to_f32(sc[g]), dot_seg<BITS>(cd, xv[ch]), fmaf(bf16_to_f32(bi[g]), xsm[ch], acc));
+          }
+        }
+        if (nsg >= 32) {
+          acc = warp_sum(acc);
+        } else {
+#pragma unroll 1
+          for (int o = nsg >> 1; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        }
+        if (gs0 == 0 && rho < 2 * n) guv[gu * cv.npc_max + q] = acc;
+      }
+    }
+    const bool gu_failed = __syncthreads_or(ab);
+    if (tid == 0) {
+      s_pend.g = -1;
+      s_pend.gc = -1;
+    }
+    if (gu_failed) { leave(); return; }
+    if (tid < npc) {
+      const int P = gp0 + tid;
+      const int j = P < k * I ? (P >> lgI) : k;
+      const int i = P - (j << lgI);
+      const float h = silu_f(guv[tid]) * guv[cv.npc_max + tid];
+      st_word(p.hbuf + static_cast<size_t>(j) * I + i, tag_f32(h, par));
+    }
+    // down rows of every slot into the (now free) same buffer: codes, scales, biases
+    if (warp == 0) {
+#pragma unroll 1
+      for (int t = lane; t < (nr > 0 ? 3 * nslots : 0); t += 32) {
+        const int j = t / 3, which = t % 3;
+        const bool routed = j < k;
+        const QMat m = routed ? Ld.dn : Ld.sdn;
+        const size_t e = routed ? static_cast<size_t>(s_idx[j]) : 0;
         unsigned char* slot = dbuf + static_cast<size_t>(j) * cv.d_slot_bytes;
         if (which == 0) {
-          copy_tx(slot, m.q + static_cast<size_t>(e) * m.q_stride + static_cast<size_t>(r0) * rowbd,
-                  static_cast<uint32_t>(nr * rowbd), &bar_d);
+          copy_tx(slot, m.q + e * m.q_stride + static_cast<size_t>(r0) * rowbd, static_cast<uint32_t>(nr * rowbd), &bar_d);
         } else {
-          const int el0 = (r0 * ngd) & ~7;
-          const int el1 = al8(r1 * ngd);
-          uint16_t* sc = reinterpret_cast<uint16_t*>(slot + static_cast<size_t>(cv.nr_max) * cv.rowb_dmax);
-          const size_t eo = static_cast<size_t>(e) * m.sb_stride + el0;
-          copy_tx(sc + (which == 2 ? cv.d_sc_el : 0), (which == 2 ? m.b : m.s) + eo,
+          const int el0 = (r0 * ngd) & ~7, el1 = al8(r1 * ngd);
+          uint16_t* sc = reinterpret_cast<uint16_t*>(slot + static_cast<size_t>(cv.nr_max) * rowbd);
+          copy_tx(sc + (which == 2 ? cv.d_sc_el : 0), (which == 2 ? m.b : m.s) + e * m.sb_stride + el0,
                   static_cast<uint32_t>(el1 - el0) * 2u, &bar_d);
         }
       }
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&bar_d);
-        s_pend[3] = l & 1;
+        mbar_arrive1(&bar_d);
+        s_pend.d = l & 1;
       }
     }
     stamp(4);
-    if (!grid_barrier(p, ++epoch, &s_abort)) { drain(); return; }
-    stamp(5);
 
-    // ---------------- 5+6. down rows + weighted combine + shared expert
-    // Warp w owns slots w, w+16: its lanes keep one 16-byte code segment's
-    // worth of that slot's h (read once from L2) and walk the CTA's rows; the
-    // per-slot row sums meet in shared memory and are combined in slot order.
-    if (!mbar_wait(&bar_d, l & 1, p.hdr, 13)) s_abort = 1;
-    if (tid == 0) s_pend[3] = -1;
-    const bool last_layer_out = p.layer_mode && (l == p.L - 1);
+    // ---------------- 5a. every slot's h, by down code segment
     {
-      float* dred = reinterpret_cast<float*>(sm + cv.dred);  // [nslots][nr_max]
-      for (int j = warp; j < nslots; j += kWarps) {
-        const bool routed = j < k;
-        const int Ij = routed ? I : Is;
-        const int nsg = Ij / PS;                   // code segments per row (16 or 32 at I = 512)
-        const int rows_per_step = 32 / nsg;        // 2 rows at a time for 16 segments
-        const int s = lane % nsg;
-        const int sub = lane / nsg;                // which of the rows of this step
-        const int ngd = Ij / group;
-        const int rowbd = Ij * BITS / 8;
-        const float* hg = p.hbuf + static_cast<size_t>(j) * cv.Imax + s * PS;
-        float hv[PS];
-        float hsm = 0.f;
+      const int nch = nslots * I / 4;
+      uint4 hv[kHChunks];
+      uint64_t t0 = 0;
+      for (uint32_t it = 0;; ++it) {
+        bool ok = true;
 #pragma unroll
-        for (int q4 = 0; q4 < PS / 4; ++q4) {
-          const float4 f = __ldcg(reinterpret_cast<const float4*>(hg) + q4);
-          hv[4 * q4] = f.x;
-          hv[4 * q4 + 1] = f.y;
-          hv[4 * q4 + 2] = f.z;
-          hv[4 * q4 + 3] = f.w;
-          hsm += (f.x + f.y) + (f.z + f.w);
-        }
-        const unsigned char* slot = dbuf + static_cast<size_t>(j) * cv.d_slot_bytes;
-        const uint16_t* sc = reinterpret_cast<const uint16_t*>(slot + static_cast<size_t>(cv.nr_max) * cv.rowb_dmax);
-        const int off = r0 * ngd - ((r0 * ngd) & ~7);
-        const int g = s * PS / group;
-        for (int rl0 = 0; rl0 < nr; rl0 += rows_per_step) {
-          const int rl = rl0 + sub;
-          float part = 0.f;
-          if (rl < nr) {
-            const uint4 cd = *reinterpret_cast<const uint4*>(slot + static_cast<size_t>(rl) * rowbd + 16 * s);
-            const int ei = off + rl * ngd + g;
-            part = fmaf(bf16_to_f32(sc[ei]), dot_seg<BITS>(cd, hv), bf16_to_f32(sc[cv.d_sc_el + ei]) * hsm);
+        for (int u = 0; u < kHChunks; ++u) {
+          const int ci = tid + u * kThreads;
+          if (ci < nch) {
+            hv[u] = ld_words4(p.hbuf + 4 * ci);
+            ok &= ((hv[u].x & hv[u].y & hv[u].z & hv[u].w & 1u) == par) && (((hv[u].x | hv[u].y | hv[u].z | hv[u].w) & 1u) == par);
           }
-          // sum over the nsg lanes of each row
-          for (int o = nsg >> 1; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-          if (s == 0 && rl < nr) dred[j * cv.nr_max + rl] = part;
         }
+        if (ok) break;
+        MOE_POLL_BACKOFF(it, t0, p.hdr, 22, ab)
       }
-      __syncthreads();
-      if (tid < nr) {
-        const int row = r0 + tid;
-        float acc = 0.f;
-        for (int j = 0; j < k; ++j) acc = fmaf(s_w[j], dred[j * cv.nr_max + tid], acc);
-        if (Is > 0) acc = fmaf(s_sg, dred[k * cv.nr_max + tid], acc);
-        const uint16_t yb = f32_to_bf16(acc);
-        if (last_layer_out) {
-          p.out[row] = yb;
-        } else {
-          p.ybuf[row] = yb;
+#pragma unroll
+      for (int u = 0; u < kHChunks; ++u) {
+        const int ci = tid + u * kThreads;
+        if (ci < nch) {
+          const int j = (4 * ci) >> lgI, i = (4 * ci) & (I - 1);
+          const int s = i / PS, q4 = (i % PS) / 4;
+          reinterpret_cast<uint4*>(hs + static_cast<size_t>(j) * I)[q4 * nsgd + s] = hv[u];
         }
-        if (p.tr_y) p.tr_y[static_cast<size_t>(lg) * H + row] = yb;
       }
     }
-    stamp(6);
-    if (last_layer_out) break;
-    if (!grid_barrier(p, ++epoch, &s_abort)) { drain(); return; }
-    stamp(7);
+    if (__syncthreads_or(ab)) { leave(); return; }
+    stamp(5);
 
-    // ---------------- 7. residual + RMSNorm of the whole vector (every CTA)
+    // ---------------- 5b. down rows of every slot for this CTA's output rows
+    if (!mbar_ready(&bar_d, l & 1, p.hdr, 13)) ab = true;
+    {
+      const int off = r0 * ngd - ((r0 * ngd) & ~7);
+      const int g = (ds * PS) >> lgG;
+      int cur = -1;
+      float hv[PS];
+      float hsm = 0.f;
+      int j = dn_j0, t = dn_t0;
+#pragma unroll 1
+      for (int u = dn_u0; u < dn_u1; ++u, ++t) {
+        if (t == dn_upj) {
+          t = 0;
+          ++j;
+        }
+        if (j != cur) {
+          cur = j;
+          hsm = 0.f;
+          const float4* hj = reinterpret_cast<const float4*>(hs + static_cast<size_t>(j) * I);
+#pragma unroll
+          for (int q4 = 0; q4 < PS / 4; ++q4) {
+            const float4 f = hj[q4 * nsgd + ds];
+            hv[4 * q4] = f.x;
+            hv[4 * q4 + 1] = f.y;
+            hv[4 * q4 + 2] = f.z;
+            hv[4 * q4 + 3] = f.w;
+            hsm += (f.x + f.y) + (f.z + f.w);
+          }
+        }
+        const int rl = t * rpsd + dsub;
+        float part = 0.f;
+        if (rl < nr) {
+          const unsigned char* slot = dbuf + static_cast<size_t>(j) * cv.d_slot_bytes;
+          const uint16_t* sc = reinterpret_cast<const uint16_t*>(slot + static_cast<size_t>(cv.nr_max) * rowbd);
+          const uint4 cd = *reinterpret_cast<const uint4*>(slot + static_cast<size_t>(rl) * rowbd + 16 * ds);
+          const int ei = off + rl * ngd + g;
+          part = fmaf(bf16_to_f32(sc[ei]), dot_seg<BITS>(cd, hv), bf16_to_f32(sc[cv.d_sc_el + ei]) * hsm);
+        }
+#pragma unroll 1
+        for (int o = nsgd >> 1; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (ds == 0 && rl < nr) dred[j * cv.nr_max + rl] = part;
+      }
+    }
+    const bool dn_failed = __syncthreads_or(ab);
+    if (tid == 0) s_pend.d = -1;
+    if (dn_failed) { leave(); return; }
+    if (tid < nr) {
+      const int row = r0 + tid;
+      float acc = 0.f;
+#pragma unroll 1
+      for (int j = 0; j < k; ++j) acc = fmaf(s_w[j], dred[j * cv.nr_max + tid], acc);
+      if (Is > 0) acc = fmaf(s_sg, dred[k * cv.nr_max + tid], acc);
+      const uint16_t yb = f32_to_bf16(acc);
+      st_word(p.ybuf + row, (static_cast<uint32_t>(yb) << 16) | (tag & 0xffffu));
+      if (p.tr_y) p.tr_y[static_cast<size_t>(lg) * H + row] = yb;
+    }
+    stamp(6);
+  }
+
+  // ---------------- the stack's output: residual + RMSNorm after the last layer (CTA 0)
+  if (c == 0) {
+    const uint32_t ytag = static_cast<uint32_t>(p.L) & 0xffffu;
     float ss = 0.f;
-    for (int i = tid; i < H; i += kThreads) {
-      const float v = rr[i] + bf16_to_f32(__ldcg(p.ybuf + i));
-      rr[i] = v;
-      ss = fmaf(v, v, ss);
+    const int i4 = 4 * tid;
+    if (i4 < H) {
+      uint4 w;
+      uint64_t t0 = 0;
+      for (uint32_t it = 0;; ++it) {
+        w = ld_words4(p.ybuf + i4);
+        if ((w.x & 0xffffu) == ytag && (w.y & 0xffffu) == ytag && (w.z & 0xffffu) == ytag && (w.w & 0xffffu) == ytag)
+          break;
+        MOE_POLL_BACKOFF(it, t0, p.hdr, 23, ab)
+      }
+      const uint32_t wy[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float v = rr[i4 + u] + __uint_as_float(wy[u] & 0xffff0000u);
+        rr[i4 + u] = v;
+        ss = fmaf(v, v, ss);
+      }
     }
     ss = warp_sum(ss);
     if (lane == 0) s_red[warp] = ss;
@@ -631,26 +748,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) tot += s_red[w];
     const float inv = 1.f / sqrtf(tot / static_cast<float>(H) + p.eps);
-    const bool final_x = (l == p.L - 1);
+#pragma unroll 1
     for (int i = tid; i < H; i += kThreads) {
-      const uint16_t xb = f32_to_bf16(rr[i] * inv);
-      set_x<PS>(xn, xs, xsum, H, i, bf16_to_f32(xb));
-      if (c == 0) {
-        if (final_x) p.out[i] = xb;
-        else if (p.tr_x) p.tr_x[static_cast<size_t>(lg + 1) * H + i] = xb;
-        if (final_x && p.r_out) p.r_out[i] = rr[i];
-      }
+      p.out[i] = f32_to_bf16(rr[i] * inv);
+      if (p.r_out) p.r_out[i] = rr[i];
     }
-    __syncthreads();
-    finish_xsum<PS>(xs, xsum, H);
-    __syncthreads();
   }
-  drain();
+  leave();
 }
 
-template <int BITS, int CH, int RB>
+template <int BITS, int CH>
 cudaError_t launch_t(const DecodeParams& p, size_t smem, int grid, cudaStream_t stream) {
-  auto kern = decode_stack_kernel<BITS, CH, RB>;
+  auto kern = decode_stack_kernel<BITS, CH>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -662,35 +771,43 @@ cudaError_t launch_t(const DecodeParams& p, size_t smem, int grid, cudaStream_t 
                                      stream);
 }
 
+bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
 }  // namespace
 
 size_t decode_stack_smem(int H, int E, int k, int I, int Is, int group, int bits, int grid) {
-  // the gate/up code rows of a CTA are staged in three batches of 16 pairs
-  if (cdiv(k * I + Is, grid) > 48) return ~size_t(0);
+  const int npc_max = cdiv(k * I + Is, grid) + 1;
+  // at most kMaxBatches batches of pairs, spanning at most two slots
+  if (npc_max > kBatch * kMaxBatches || npc_max > I) return ~size_t(0);
+  if (cdiv(E + (Is > 0 ? 1 : 0), grid) > kWarps) return ~size_t(0);  // one router row per warp
+  if (cdiv(H, grid) > kThreads) return ~size_t(0);
   return carve(H, E, k, I, Is, group, bits, grid).total;
 }
 
 bool decode_stack_supported(int H, int E, int k, int I, int Is, int group, int bits) {
-  const int nseg = H * bits / 128;
-  if (nseg > 128) return false;          // at most 4 code segments per lane per row
-  if ((H / group) % 8 != 0) return false;  // gate/up scale rows are whole 16-byte chunks
-  if (k > 16 || E > 512) return false;
-  (void)I;
-  (void)Is;
+  const int PS = 128 / bits;
+  const int nsg = H / PS, nsgd = I / PS;
+  if (H % PS || I % PS || H > 2048 || H % 4) return false;  // x of a lane's segments stays in registers
+  if (!(pow2(nsg) && nsg <= 32) && !(nsg % 32 == 0 && nsg / 32 <= (bits == 4 ? 2 : 4))) return false;
+  if (!pow2(nsgd) || nsgd > 32) return false;           // a down row is one warp step or less
+  if (Is != 0 && Is != I) return false;                 // every slot has the same down row length
+  if ((H / group) % 8 != 0) return false;               // gate/up scale rows are whole 16-byte chunks
+  if (k > 16 || E > 32 * kTopPer) return false;
+  if ((k + 1) * I > 4 * kHChunks * kThreads) return false;
   return true;
 }
 
 cudaError_t launch_decode_stack(const DecodeParams& p, int bits, int grid, cudaStream_t stream) {
   const size_t smem = decode_stack_smem(p.H, p.E, p.k, p.I, p.Is, p.group, bits, grid);
-  const int nseg = p.H * bits / 128;
+  const int nsg = p.H * bits / 128;
+  const int ch = nsg >= 32 ? nsg / 32 : 1;
   if (bits == 4) {
-    if (nseg <= 32) return launch_t<4, 1, 3>(p, smem, grid, stream);
-    if (nseg <= 64) return launch_t<4, 2, 3>(p, smem, grid, stream);
-    return launch_t<4, 4, 2>(p, smem, grid, stream);
+    if (ch == 1) return launch_t<4, 1>(p, smem, grid, stream);
+    return launch_t<4, 2>(p, smem, grid, stream);
   }
-  if (nseg <= 32) return launch_t<8, 1, 3>(p, smem, grid, stream);
-  if (nseg <= 64) return launch_t<8, 2, 3>(p, smem, grid, stream);
-  return launch_t<8, 4, 2>(p, smem, grid, stream);
+  if (ch == 1) return launch_t<8, 1>(p, smem, grid, stream);
+  if (ch == 2) return launch_t<8, 2>(p, smem, grid, stream);
+  return launch_t<8, 4>(p, smem, grid, stream);
 }
 
 }  // namespace moe
