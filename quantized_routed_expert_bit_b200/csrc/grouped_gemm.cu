@@ -56,7 +56,7 @@ constexpr int kThreads = 512;
 constexpr int kBM = 128;           // tile rows
 constexpr int kBK = 64;            // K per k-block: one quantisation group, one 128-byte swizzle row
 constexpr int kNT = kChunkTokens;  // columns (pairs) per tile
-constexpr int kPBuf = 4;           // TMEM buffers of per-group products in rotation
+constexpr int kPBuf = 8;           // TMEM buffers of per-group products in rotation
 constexpr int kNA = 4;             // unpacked A tiles in flight
 constexpr int kDequantWarp0 = 4;   // warps 4..11
 constexpr int kEpiWarp0 = 12;      // warps 12..15
@@ -167,18 +167,6 @@ __device__ __forceinline__ void unpack32_u8(const uint4 c0, const uint4 c1, uint
     }
     out[i] = make_uint4(r[0], r[1], r[2], r[3]);
   }
-}
-
-// acc[c0 + n] += s * P[n] + b * X[g][c0 + n] for the columns n < cnt - c0 of one 32-column slice.
-template <int C0>
-__device__ __forceinline__ void scale_slice(float* acc, uint32_t ta, float sc, float bi, const float* xs_g, int cnt) {
-  if (cnt <= C0) return;
-  uint32_t v[32];
-  tc::tmem_ld32(ta + C0, v);
-  tc::tmem_wait_ld();
-#pragma unroll
-  for (int n = 0; n < 32; ++n)
-    if (C0 + n < cnt) acc[C0 + n] = fmaf(sc, __uint_as_float(v[n]), fmaf(bi, xs_g[C0 + n], acc[C0 + n]));
 }
 
 // ------------------------------------------------------------------ GEMM kernel
@@ -407,17 +395,37 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       const int start = p.chunks[3 * ci + 1], cnt = p.chunks[3 * ci + 2];
       const int tb = it & 1, tu = it >> 1;
       // group sums of the tile's columns (the down GEMM's come as 4 partial sums, added in order)
+      // (the chunk's sums are contiguous: [cnt][ng] floats, or [cnt][ng][4] partials; 8 vector
+      // loads per lane in flight at a time)
       __syncwarp();
-      for (int i = lane; i < ng * cnt; i += 32) {
-        const int n = i / ng, g = i % ng;
-        float v;
-        if (MODE == 0) {
-          v = __ldg(p.xs_in + static_cast<size_t>(start + n) * ng + g);
-        } else {
-          const float* ps = p.xs_in + (static_cast<size_t>(start + n) * ng + g) * 4;
-          v = (__ldg(ps) + __ldg(ps + 1)) + (__ldg(ps + 2) + __ldg(ps + 3));
+      {
+        const float4* src = reinterpret_cast<const float4*>(p.xs_in + static_cast<size_t>(start) * ng * (MODE == 0 ? 1 : 4));
+        const int nvec = (MODE == 0) ? (cnt * ng) / 4 : cnt * ng;
+#pragma unroll 1
+        for (int v0 = 0; v0 < nvec; v0 += 32 * 8) {
+          float4 f[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int q = v0 + u * 32 + lane;
+            if (q < nvec) f[u] = __ldg(src + q);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int q = v0 + u * 32 + lane;
+            if (q < nvec) {
+              if (MODE == 0) {
+                const int n = (4 * q) / ng, g = (4 * q) % ng;
+                xs[g * kNT + n] = f[u].x;
+                xs[(g + 1) * kNT + n] = f[u].y;
+                xs[(g + 2) * kNT + n] = f[u].z;
+                xs[(g + 3) * kNT + n] = f[u].w;
+              } else {
+                const int n = q / ng, g = q % ng;
+                xs[g * kNT + n] = (f[u].x + f[u].y) + (f[u].z + f[u].w);
+              }
+            }
+          }
         }
-        xs[g * kNT + n] = v;
       }
       __syncwarp();
       if (!warp_wait(&scfull[tb], tu & 1, p.hdr, abort, 60)) break;
@@ -427,17 +435,46 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
 #pragma unroll
       for (int n = 0; n < kNT; ++n) acc[n] = 0.f;
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb, ++kbg) {
-        const int pb = kbg % kPBuf, pu = kbg / kPBuf;
-        if (!warp_wait(&pfull[pb], pu & 1, p.hdr, abort, 61)) { ok = false; break; }
+      // two groups per step: both TMEM loads in flight under one wait
+      for (int kb = 0; kb < nkb; kb += 2, kbg += 2) {
+        const bool two = kb + 1 < nkb;
+        const int pb0 = kbg % kPBuf, pb1 = (kbg + 1) % kPBuf;
+        if (!warp_wait(&pfull[pb0], (kbg / kPBuf) & 1, p.hdr, abort, 61) ||
+            (two && !warp_wait(&pfull[pb1], ((kbg + 1) / kPBuf) & 1, p.hdr, abort, 61))) {
+          ok = false;
+          break;
+        }
         tc::fence_after_sync();
-        const float sc = bf16_to_f32(scs[srow * ng + kb]);
-        const float bi = bf16_to_f32(bis[srow * ng + kb]);
-        const uint32_t ta = tmem + (static_cast<uint32_t>(32 * q) << 16) + pb * kNT;
-        scale_slice<0>(acc, ta, sc, bi, xs + kb * kNT, cnt);
+        const uint32_t tq = tmem + (static_cast<uint32_t>(32 * q) << 16);
+        const float sc0 = bf16_to_f32(scs[srow * ng + kb]);
+        const float bi0 = bf16_to_f32(bis[srow * ng + kb]);
+        const float sc1 = two ? bf16_to_f32(scs[srow * ng + kb + 1]) : 0.f;
+        const float bi1 = two ? bf16_to_f32(bis[srow * ng + kb + 1]) : 0.f;
+        const float* x0 = xs + kb * kNT;
+        // columns in halves of 16 (the upper half only when the chunk has more than 16 pairs)
+#pragma unroll
+        for (int hf = 0; hf < kNT / 16; ++hf) {
+          if (hf * 16 < cnt) {
+            uint32_t v0[16], v1[16];
+            tc::tmem_ld16(tq + pb0 * kNT + hf * 16, v0);
+            if (two) tc::tmem_ld16(tq + pb1 * kNT + hf * 16, v1);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int n = hf * 16 + c;
+              if (n < cnt) {
+                acc[n] = fmaf(sc0, __uint_as_float(v0[c]), fmaf(bi0, x0[n], acc[n]));
+                if (two) acc[n] = fmaf(sc1, __uint_as_float(v1[c]), fmaf(bi1, x0[kNT + n], acc[n]));
+              }
+            }
+          }
+        }
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&pempty[pb]);
+        if (lane == 0) {
+          tc::mbar_arrive(&pempty[pb0]);
+          if (two) tc::mbar_arrive(&pempty[pb1]);
+        }
       }
       if (!ok) break;
       __syncwarp();
@@ -446,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         // rows 2i (gate) and 2i+1 (up) of intermediate index mt*64 + i
         const int i = mt * 64 + (m >> 1);
         const int ip = (BITS == 4) ? ((i & ~7) | perm8_pos(i & 7)) : i;
+        float* hv = acc;  // h replaces the accumulators column by column
 #pragma unroll
         for (int n = 0; n < kNT; ++n) {
           const float u = __shfl_xor_sync(0xffffffffu, acc[n], 1);
@@ -458,10 +496,22 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             p.h_hi[o] = __half_as_ushort(hi);
             p.h_lo[o] = __half_as_ushort(lo);
           }
-          // this warp's share (16 intermediate indices) of the group sum of h
-          const float ws = warp_sum(h);
-          if (lane == 0 && n < cnt) p.hsum_out[(static_cast<size_t>(start + n) * (p.I / 64) + mt) * 4 + q] = ws;
+          hv[n] = h;
         }
+        // this warp's share (16 intermediate indices) of the group sum of h, every column at
+        // once: a butterfly reduce-scatter leaves lane n with the sum of column n
+        static_assert(kNT == 32, "one column per lane");
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+          const bool upper = (lane & o) != 0;
+#pragma unroll
+          for (int i = 0; i < o; ++i) {
+            const float send = upper ? hv[i] : hv[i + o];
+            const float keep = upper ? hv[i + o] : hv[i];
+            hv[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+          }
+        }
+        if (lane < cnt) p.hsum_out[(static_cast<size_t>(start + lane) * (p.I / 64) + mt) * 4 + q] = hv[0];
       } else {
         const int r = mt * kBM + m;
 #pragma unroll

@@ -69,9 +69,11 @@ Layout layout(const moe_config& c, int64_t T) {
   L.y = o;        o += up(static_cast<size_t>(T) * c.hidden * 2);
   L.idx = o;      o += up(static_cast<size_t>(T) * c.top_k * 4);
   L.w = o;        o += up(static_cast<size_t>(T) * c.top_k * 4);
-  L.dlogits = o;  o += up(static_cast<size_t>(c.num_experts + 1) * 4);   // decode exchange words:
-  L.dh = o;       o += up(static_cast<size_t>(c.top_k + 1) * imax * 4);  //   logits, h, y (contiguous,
-  L.dy = o;       o += up(static_cast<size_t>(c.hidden) * 4);             //   zeroed before each launch)
+  // decode exchange words: logits, h, y, each in kDecodeReplicas copies (contiguous, zeroed
+  // before each launch)
+  L.dlogits = o;  o += moe::kDecodeReplicas * up(static_cast<size_t>(c.num_experts + 1) * 4);
+  L.dh = o;       o += moe::kDecodeReplicas * up(static_cast<size_t>(c.top_k + 1) * imax * 4);
+  L.dy = o;       o += moe::kDecodeReplicas * up(static_cast<size_t>(c.hidden) * 4);
   L.dr = o;       o += up(static_cast<size_t>(c.hidden) * 4);
   L.dx = o;       o += up(static_cast<size_t>(c.hidden) * 2);
   L.base_total = o;
@@ -443,6 +445,9 @@ moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, in
   P->logits = reinterpret_cast<uint32_t*>(b + Ly.dlogits);
   P->hbuf = reinterpret_cast<uint32_t*>(b + Ly.dh);
   P->ybuf = reinterpret_cast<uint32_t*>(b + Ly.dy);
+  P->logits_rep = static_cast<int>((Ly.dh - Ly.dlogits) / moe::kDecodeReplicas / 4);
+  P->h_rep = static_cast<int>((Ly.dy - Ly.dh) / moe::kDecodeReplicas / 4);
+  P->y_rep = static_cast<int>((Ly.dr - Ly.dy) / moe::kDecodeReplicas / 4);
   P->hdr = reinterpret_cast<moe::WsHeader*>(b + Ly.hdr);
   uint16_t* xmid = reinterpret_cast<uint16_t*>(b + Ly.dx);
   float* rmid = reinterpret_cast<float*>(b + Ly.dr);

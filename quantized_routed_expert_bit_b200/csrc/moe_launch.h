@@ -62,7 +62,7 @@ struct SortParams {
   WsHeader* hdr;
 };
 
-constexpr int kChunkTokens = 64;  // pairs per GEMM chunk (the MMA N dimension)
+constexpr int kChunkTokens = 32;  // pairs per GEMM chunk (the MMA N dimension)
 
 // Batched path: gather of the sorted pairs' activations and the final combine.
 struct BatchParams {
@@ -106,6 +106,7 @@ struct LayerDesc {
 };
 
 constexpr int kMaxDecodeLayers = 128;  // layers per launch (kernel parameter space)
+constexpr int kDecodeReplicas = 4;     // copies of each exchange word (spreads the readers over more lines)
 
 struct DecodeParams {
   int L, l0;             // layers in this launch; index of its first layer in the stack
@@ -120,10 +121,12 @@ struct DecodeParams {
   float* tr_w;           // [layers][k] or null
   uint16_t* tr_y;        // bf16 [layers][H] or null
   uint64_t* tr_t;        // [layers][8] phase timestamps of CTA 0, or null
-  // exchange words between CTAs (workspace), zero at launch
+  // exchange words between CTAs (workspace), zero at launch; each written to
+  // kDecodeReplicas copies (`*_rep` words apart), CTA c reads copy c % kDecodeReplicas
   uint32_t* logits;      // [E+1] fp32 logits, last mantissa bit = layer parity
   uint32_t* hbuf;        // [k+1][I] fp32 SwiGLU outputs, last mantissa bit = layer parity
   uint32_t* ybuf;        // [H] bf16 layer output << 16 | 16-bit layer tag
+  int logits_rep, h_rep, y_rep;
   WsHeader* hdr;
   LayerDesc layers[kMaxDecodeLayers];
 };

@@ -45,19 +45,18 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBatch = 8;        // gate/up pairs per code batch (one mbarrier each)
-constexpr int kMaxBatches = 8;   // at most 64 pairs per CTA
+constexpr int kBatch = 16;       // gate/up pairs per code batch (one mbarrier each)
+constexpr int kMaxBatches = 4;   // at most 64 pairs per CTA
 constexpr int kHChunks = 4;      // 16-byte chunks of h each thread reads: (k+1)*I <= 4*4*512
 constexpr int kTopPer = 16;      // logits per lane in the top-k warp: E <= 512
 
 __host__ __device__ constexpr uint32_t al128(uint32_t v) { return (v + 127u) & ~127u; }
 __host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
-__host__ __device__ constexpr int al8(int v) { return (v + 7) & ~7; }
 
 // Shared-memory carve-up; identical on host (sizing) and device.
 struct Carve {
-  int PS, nsg, nsgd, nslots, npc_max, ng, nr_max, ngd, rowb, rowbd, d_sc_el, rr_max;
-  uint32_t xs, xn, rr, hs, dred, guv, gsb, dbuf, d_slot_bytes, rbuf, total;
+  int PS, nsg, nsgd, nslots, npc_max, ng, nr_max, ngd, rowb, rowbd, rr_max, nunits, d_sc_el;
+  uint32_t xs, xn, rr, hs, dred, guv, gsb, dbuf, dsc, rbuf, desc, total;
 };
 
 __host__ __device__ inline Carve carve(int H, int E, int k, int I, int Is, int group, int bits, int G) {
@@ -72,8 +71,9 @@ __host__ __device__ inline Carve carve(int H, int E, int k, int I, int Is, int g
   c.ngd = I / group;
   c.rowb = H * bits / 8;
   c.rowbd = I * bits / 8;
-  c.d_sc_el = al8(c.nr_max * c.ngd + 16);
   c.rr_max = cdiv(E + (Is > 0 ? 1 : 0), G);
+  c.nunits = c.nslots * cdiv(c.nr_max, 32 / c.nsgd);  // down work units (slot, row step) of a CTA, at most
+  c.d_sc_el = (c.nr_max * c.ngd + 16 + 7) & ~7;       // a slot's down scales (or biases) of the CTA's rows
   uint32_t o = 0;
   c.xs = o;    o = al128(o + H * 4);
   c.xn = o;    o = al128(o + H * 4);
@@ -82,13 +82,14 @@ __host__ __device__ inline Carve carve(int H, int E, int k, int I, int Is, int g
   c.dred = o;  o = al128(o + c.nslots * c.nr_max * 4);
   c.guv = o;   o = al128(o + 2 * c.npc_max * 4);
   c.gsb = o;   o = al128(o + 4 * c.npc_max * c.ng * 2);
-  c.d_slot_bytes = al128(c.nr_max * c.rowbd + 2 * c.d_sc_el * 2);
-  // one buffer, used first for this CTA's gate/up code rows ([gate rows][up rows]),
-  // then for its down rows of every slot
+  // one buffer: first this CTA's gate/up code rows ([gate rows][up rows]), then its down
+  // code segments by work unit ([unit][lane] x 16 bytes) and down scales and biases by slot
   const uint32_t gu_bytes = 2u * c.npc_max * c.rowb;
-  const uint32_t dn_bytes = c.nslots * c.d_slot_bytes;
+  const uint32_t dn_bytes = c.nunits * 512u + c.nslots * 4u * c.d_sc_el;
   c.dbuf = o;  o = al128(o + (gu_bytes > dn_bytes ? gu_bytes : dn_bytes));
+  c.dsc = c.nunits * 512u;  // offset of the down scales inside dbuf
   c.rbuf = o;  o = al128(o + 2 * c.rr_max * H * 2);
+  c.desc = o;  o = al128(o + kMaxDecodeLayers * sizeof(LayerDesc));  // the launch's layer descriptors
   c.total = o;
   return c;
 }
@@ -102,8 +103,17 @@ __device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+// Per-thread asynchronous 16-byte global -> shared copy (L2 only), and the wait for all of this
+// thread's outstanding ones.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void prefetch_line_l2(const void* a) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
 }
 
 __device__ __forceinline__ void st_word(uint32_t* a, uint32_t v) {
@@ -165,6 +175,45 @@ __device__ __forceinline__ bool mbar_ready(uint64_t* bar, uint32_t parity, WsHea
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.f + expf(-z)); }
 
+// Dot products of one 16-byte code segment with the matching x (or h) values.
+// 8-bit codes: dot_seg<8> (each byte permuted under the exponent of 2^15).
+// 4-bit codes: each 32-bit word is first split into its even and odd nibbles
+// as bytes (two lop3), then every byte goes under the exponent of 2^15 like an
+// 8-bit code: one shared magic constant, so pairs of codes take the packed
+// fp32x2 subtract and fma with no register shuffling. The codes of a word
+// then come out in the order 0,2,4,6,1,3,5,7, and the values they multiply
+// are stored in that order (seg_pos): a dot product does not depend on the
+// order of its terms, and each q*x stays exact.
+template <int BITS>
+__host__ __device__ constexpr int seg_pos(int o) {
+  return BITS == 4 ? ((o & ~7) | (((o & 7) >> 1) + 4 * (o & 1))) : o;
+}
+
+__device__ __forceinline__ float2 dot8_u4_split(uint32_t w, const float* x, float2 acc) {
+  constexpr uint32_t kM = 0x47000000u;  // 2^15
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+  const float2 km = f2(-32768.f, -32768.f);
+  acc = __ffma2_rn(__fadd2_rn(f2(fb(__byte_perm(lo, kM, 0x7504)), fb(__byte_perm(lo, kM, 0x7514))), km), f2(x[0], x[1]), acc);
+  acc = __ffma2_rn(__fadd2_rn(f2(fb(__byte_perm(lo, kM, 0x7524)), fb(__byte_perm(lo, kM, 0x7534))), km), f2(x[2], x[3]), acc);
+  acc = __ffma2_rn(__fadd2_rn(f2(fb(__byte_perm(hi, kM, 0x7504)), fb(__byte_perm(hi, kM, 0x7514))), km), f2(x[4], x[5]), acc);
+  acc = __ffma2_rn(__fadd2_rn(f2(fb(__byte_perm(hi, kM, 0x7524)), fb(__byte_perm(hi, kM, 0x7534))), km), f2(x[6], x[7]), acc);
+  return acc;
+}
+
+template <int BITS>
+__device__ __forceinline__ float dot_seg_dec(const uint4& c, const float* x) {
+  if constexpr (BITS == 4) {
+    float2 acc = f2(0.f, 0.f);
+    acc = dot8_u4_split(c.x, x + 0, acc);
+    acc = dot8_u4_split(c.y, x + 8, acc);
+    acc = dot8_u4_split(c.z, x + 16, acc);
+    acc = dot8_u4_split(c.w, x + 24, acc);
+    return acc.x + acc.y;
+  } else {
+    return dot_seg<8>(c, x);
+  }
+}
+
 // Order-preserving map of a float to an unsigned key (larger float, larger key).
 __device__ __forceinline__ unsigned fkey(float f) {
   const unsigned u = __float_as_uint(f);
@@ -175,20 +224,67 @@ __device__ __forceinline__ float fkey_inv(unsigned k) {
   return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
 }
 
+// Top-k of one token's logits by one warp: lane l holds the logits of experts
+// l, l+32, ... (PER of them, tagged fp32 words). Each lane sorts its keys once
+// (larger logit first, then lower expert index); every round one warp-wide
+// max over the lanes' heads picks the winner (lowest index among equal
+// keys), whose lane pops its head. Lane j < k ends with the j-th pick.
+template <int PER>
+__device__ __forceinline__ void topk_sorted(const uint32_t* wl, int E, int k, int lane, unsigned& my_k, int& my_e,
+                                            unsigned& kmax) {
+  unsigned key[PER];
+  int idx[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    idx[i] = lane + 32 * i;
+    key[i] = (idx[i] < E) ? fkey(__uint_as_float(wl[i])) : 0u;
+  }
+#pragma unroll
+  for (int r = 0; r < PER; ++r) {
+#pragma unroll
+    for (int i = (r & 1); i + 1 < PER; i += 2) {
+      const bool sw = key[i + 1] > key[i] || (key[i + 1] == key[i] && idx[i + 1] < idx[i]);
+      const unsigned k0 = key[i], k1 = key[i + 1];
+      const int i0 = idx[i], i1 = idx[i + 1];
+      key[i] = sw ? k1 : k0;
+      key[i + 1] = sw ? k0 : k1;
+      idx[i] = sw ? i1 : i0;
+      idx[i + 1] = sw ? i0 : i1;
+    }
+  }
+  kmax = __reduce_max_sync(0xffffffffu, key[0]);
+  my_k = 0u;
+  my_e = 0;
+#pragma unroll 1
+  for (int j = 0; j < k; ++j) {
+    const unsigned wk = __reduce_max_sync(0xffffffffu, key[0]);
+    const unsigned we = __reduce_min_sync(0xffffffffu, key[0] == wk ? static_cast<unsigned>(idx[0]) : 0xffffffffu);
+    if (lane == j) {
+      my_k = wk;
+      my_e = static_cast<int>(we);
+    }
+    if (static_cast<unsigned>(idx[0]) == we) {  // expert indices are unique across lanes: the owner pops
+#pragma unroll
+      for (int i = 0; i + 1 < PER; ++i) {
+        key[i] = key[i + 1];
+        idx[i] = idx[i + 1];
+      }
+      key[PER - 1] = 0u;
+    }
+  }
+}
+
 // Copy-phase bookkeeping for leaving early: parities of the phases this CTA
 // still has bulk copies in flight on (-1 = none).
 struct Pending {
-  int r[2], g, d, gc;
+  int r[2], gc;
 };
 
-__device__ __noinline__ void drain(Pending* pend, uint64_t* bar_r, uint64_t* bar_g, uint64_t* bar_d,
-                                   uint64_t* bar_gc, int nb, WsHeader* hdr) {
+__device__ __noinline__ void drain(Pending* pend, uint64_t* bar_r, uint64_t* bar_gc, int nb, WsHeader* hdr) {
   __syncthreads();
   if (threadIdx.x == 0) {
     if (pend->r[0] >= 0) mbar_wait(&bar_r[0], pend->r[0], hdr, 90);
     if (pend->r[1] >= 0) mbar_wait(&bar_r[1], pend->r[1], hdr, 91);
-    if (pend->g >= 0) mbar_wait(bar_g, pend->g, hdr, 92);
-    if (pend->d >= 0) mbar_wait(bar_d, pend->d, hdr, 93);
     if (pend->gc >= 0)
       for (int b = 0; b < nb; ++b) mbar_wait(&bar_gc[b], pend->gc, hdr, 94);
   }
@@ -200,9 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
   constexpr int PS = 128 / BITS;  // codes per 16-byte segment
   extern __shared__ __align__(128) unsigned char sm[];
   __shared__ __align__(8) uint64_t bar_r[2];
-  __shared__ __align__(8) uint64_t bar_g, bar_d;
   __shared__ __align__(8) uint64_t bar_gc[kMaxBatches];
-  __shared__ __align__(16) LayerDesc s_ld[2];
   __shared__ int s_idx[16];
   __shared__ float s_w[16];
   __shared__ float s_sg;
@@ -223,6 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
   uint16_t* gsb = reinterpret_cast<uint16_t*>(sm + cv.gsb);
   unsigned char* dbuf = sm + cv.dbuf;
   uint16_t* rbuf = reinterpret_cast<uint16_t*>(sm + cv.rbuf);
+  const LayerDesc* s_layers = reinterpret_cast<const LayerDesc*>(sm + cv.desc);
 
   // ---- static assignment of this CTA's work
   const int NP = k * I + Is;
@@ -241,6 +336,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
   const int nrows_rt = E + (Is > 0 ? 1 : 0);
   const int rr_cnt = (c < nrows_rt) ? cdiv(nrows_rt - c, G) : 0;
   const int nslots = cv.nslots;
+  // this CTA's copy of the exchange words
+  const uint32_t* lg_in = p.logits + (c % kDecodeReplicas) * p.logits_rep;
+  const uint32_t* h_in = p.hbuf + (c % kDecodeReplicas) * p.h_rep;
+  const uint32_t* y_in = p.ybuf + (c % kDecodeReplicas) * p.y_rep;
   const int rowb = cv.rowb, rowbd = cv.rowbd, ng = cv.ng, ngd = cv.ngd;
   const int lgI = 31 - __clz(I);          // I and group are powers of two
   const int lgG = 31 - __clz(group);
@@ -248,20 +347,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
   if (tid == 0) {
     mbar_init(&bar_r[0], 1);
     mbar_init(&bar_r[1], 1);
-    mbar_init(&bar_g, 1);
-    mbar_init(&bar_d, 1);
     for (int b = 0; b < kMaxBatches; ++b) mbar_init(&bar_gc[b], 1);
     fence_mbar_init();
-    s_pend.r[0] = s_pend.r[1] = s_pend.g = s_pend.d = s_pend.gc = -1;
+    s_pend.r[0] = s_pend.r[1] = s_pend.gc = -1;
   }
-  constexpr int kDescWords = sizeof(LayerDesc) / 8;
-  static_assert(sizeof(LayerDesc) % 8 == 0 && kDescWords <= 32, "layer descriptor copy");
-  if (warp == 1 && lane < kDescWords)
-    reinterpret_cast<uint64_t*>(&s_ld[0])[lane] = reinterpret_cast<const uint64_t*>(&p.layers[0])[lane];
+  // every layer descriptor of the launch into shared memory, once (parameter-space reads
+  // with a runtime index would otherwise miss the constant cache in the middle of a layer)
+  static_assert(sizeof(LayerDesc) % 8 == 0, "layer descriptor copy");
+#pragma unroll 1
+  for (int i = tid; i < p.L * static_cast<int>(sizeof(LayerDesc) / 8); i += kThreads)
+    reinterpret_cast<uint64_t*>(sm + cv.desc)[i] = reinterpret_cast<const uint64_t*>(p.layers)[i];
   __syncthreads();
 
-  auto issue_router = [&](int l) {  // thread 0; s_ld[l & 1] holds layer l
-    const LayerDesc& Ld = s_ld[l & 1];
+  auto issue_router = [&](int l) {  // thread 0
+    const LayerDesc& Ld = s_layers[l];
     const int b = l & 1;
 #pragma unroll 1
     for (int m = 0; m < rr_cnt; ++m) {
@@ -272,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
     mbar_arrive1(&bar_r[b]);
     s_pend.r[b] = (l >> 1) & 1;
   };
-  auto leave = [&]() { drain(&s_pend, bar_r, &bar_g, &bar_d, bar_gc, nb, p.hdr); };
+  auto leave = [&]() { drain(&s_pend, bar_r, bar_gc, nb, p.hdr); };
 
   if (tid == 0) issue_router(0);
 
@@ -289,8 +388,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
   // this warp's share of the down work: units (slot, row step), slot-major
   const int dn_upj = cdiv(nr, rpsd);
   const int dn_u0 = warp * nslots * dn_upj / kWarps, dn_u1 = (warp + 1) * nslots * dn_upj / kWarps;
-  const int dn_j0 = dn_upj > 0 ? dn_u0 / dn_upj : 0;
-  const int dn_t0 = dn_u0 - dn_j0 * dn_upj;
 
   for (int l = 0; l < p.L; ++l) {
     const int lg = p.l0 + l;  // layer index within the whole stack (trace rows)
@@ -300,10 +397,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
       if (p.tr_t && c == 0 && tid == 0) p.tr_t[static_cast<size_t>(lg) * 8 + slot] = globaltimer_ns();
     };
     stamp(0);
-    // next layer's descriptor, then its router rows
-    if (warp == 1 && lane < kDescWords && l + 1 < p.L)
-      reinterpret_cast<uint64_t*>(&s_ld[(l + 1) & 1])[lane] =
-          reinterpret_cast<const uint64_t*>(&p.layers[l + 1])[lane];
 
     // ---------------- 1. this layer's x (and residual)
     if (l == 0) {
@@ -323,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         uint4 w;
         uint64_t t0 = 0;
         for (uint32_t it = 0;; ++it) {
-          w = ld_words4(p.ybuf + i4);
+          w = ld_words4(y_in + i4);
           if ((w.x & 0xffffu) == ytag && (w.y & 0xffffu) == ytag && (w.z & 0xffffu) == ytag &&
               (w.w & 0xffffu) == ytag)
             break;
@@ -352,13 +445,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
       }
     }
     __syncthreads();
-    // x by code segment: xs[(q4 * nsg + s) * 4 + c4] = x[s * PS + q4 * 4 + c4]
+    // x by code segment: xs[(q4 * nsg + s) * 4 + c4] = x[s * PS + o], q4 * 4 + c4 = seg_pos(o)
 #pragma unroll 1
-    for (int i4 = tid; i4 < H / 4; i4 += kThreads) {
-      const int s = (4 * i4) / PS, q4 = ((4 * i4) % PS) / 4;
-      reinterpret_cast<float4*>(xs)[q4 * nsg + s] = reinterpret_cast<const float4*>(xn)[i4];
+    for (int i = tid; i < H; i += kThreads) {
+      const int s = i / PS, op = seg_pos<BITS>(i % PS);
+      xs[((op >> 2) * nsg + s) * 4 + (op & 3)] = xn[i];
     }
-    if (tid == 0 && l + 1 < p.L) issue_router(l + 1);
+    if (tid == kThreads - 32 && l + 1 < p.L) issue_router(l + 1);  // a warp without router rows
     stamp(1);
 
     // ---------------- 2. router rows -> logits
@@ -382,8 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         acc = fmaf(bf16_hi(w8.w), b.w, acc);
       }
       acc = warp_sum(acc);
-      const LayerDesc& Ld = s_ld[l & 1];
-      if (lane == 0) st_word(p.logits + row, tag_f32(acc + ((row < E && Ld.rbias) ? Ld.rbias[row] : 0.f), par));
+      const LayerDesc& Ld = s_layers[l];
+      if (lane < kDecodeReplicas)
+        st_word(p.logits + lane * p.logits_rep + row, tag_f32(acc + ((row < E && Ld.rbias) ? Ld.rbias[row] : 0.f), par));
     }
     if (tid == 0) s_pend.r[l & 1] = -1;
     stamp(2);
@@ -400,11 +494,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
 #pragma unroll
           for (int i = 0; i < kTopPer; ++i) {
             const int e = lane + 32 * i;
-            wl[i] = (e < E) ? ld_word(p.logits + e) : par;
+            wl[i] = (e < E) ? ld_word(lg_in + e) : par;
             ok &= (wl[i] & 1u) == par;
           }
           if (Is > 0 && lane == 0) {
-            wsg = ld_word(p.logits + E);
+            wsg = ld_word(lg_in + E);
             ok &= (wsg & 1u) == par;
           }
           if (__all_sync(0xffffffffu, ok)) break;
@@ -418,49 +512,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         }
         ab |= fail;
       }
-      unsigned key[kTopPer];
-      unsigned bk = 0u;
-      int bi = 0;
-#pragma unroll
-      for (int i = 0; i < kTopPer; ++i) {
-        key[i] = (lane + 32 * i < E) ? fkey(__uint_as_float(wl[i])) : 0u;
-        if (key[i] > bk) {
-          bk = key[i];
-          bi = i;
-        }
-      }
-      const float mx = fkey_inv(__reduce_max_sync(0xffffffffu, bk));
+      unsigned my_k, kmax;
+      int my_e;
+      if (E <= 256) topk_sorted<8>(wl, E, k, lane, my_k, my_e, kmax);
+      else topk_sorted<kTopPer>(wl, E, k, lane, my_k, my_e, kmax);
+      const float mx = fkey_inv(kmax);
       float z = 0.f;
       if (!p.renorm) {  // softmax over all E: the words are re-read (complete and tagged by now)
 #pragma unroll 1
-        for (int e = lane; e < E; e += 32) z += expf(__uint_as_float(ld_word(p.logits + e)) - mx);
+        for (int e = lane; e < E; e += 32) z += expf(__uint_as_float(ld_word(lg_in + e)) - mx);
         z = warp_sum(z);
-      }
-      unsigned my_k = 0u;
-      int my_e = 0;
-#pragma unroll 1
-      for (int j = 0; j < k; ++j) {
-        // winner: largest key, then lowest expert index
-        const unsigned wk = __reduce_max_sync(0xffffffffu, bk);
-        const unsigned we =
-            __reduce_min_sync(0xffffffffu, bk == wk ? static_cast<unsigned>(lane + 32 * bi) : 0xffffffffu);
-        if (lane == j) {
-          my_k = wk;
-          my_e = static_cast<int>(we);
-        }
-        if (static_cast<int>(we & 31u) == lane) {
-          const int wi = static_cast<int>(we >> 5);
-          bk = 0u;
-          bi = 0;
-#pragma unroll
-          for (int i = 0; i < kTopPer; ++i) {
-            if (i == wi) key[i] = 0u;
-            if (key[i] > bk) {
-              bk = key[i];
-              bi = i;
-            }
-          }
-        }
       }
       const float ex = (lane < k) ? expf(fkey_inv(my_k) - mx) : 0.f;
       const float den = p.renorm ? warp_sum(ex) : z;
@@ -477,66 +538,77 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
     if (__syncthreads_or(ab)) { leave(); return; }
     stamp(3);
 
-    const LayerDesc& Ld = s_ld[l & 1];
-    // ---------------- 4a. bulk copies of this CTA's gate/up rows (warp 0), L2 prefetch of its down rows (warp 1)
+    const LayerDesc& Ld = s_layers[l];
+    // ---------------- 4a. this CTA's gate/up code rows: bulk copies by warp 0 (lane = batch,
+    // segment, gate|up); its gate/up scales and biases: one 16-byte load per thread into
+    // shared memory; its down rows: prefetched into L2 for phase 5
     if (warp == 0) {
-      {  // codes: lane = (batch, segment, gate|up)
-        const int b = lane >> 2, sg = (lane >> 1) & 1, gu = lane & 1;
-        const int lo = max(sg == 0 ? 0 : nA, b * kBatch);
-        const int hi = min(sg == 0 ? nA : npc, b * kBatch + kBatch);
-        if (hi > lo) {
-          const int j = jA + sg;
-          const bool routed = j < k;
-          const QMat m = routed ? Ld.gu : Ld.sgu;
-          const int Ij = routed ? I : Is;
-          const int row = (sg == 0 ? iA : -nA) + lo;
-          const uint8_t* src = m.q + static_cast<size_t>(routed ? s_idx[j] : 0) * m.q_stride +
-                               static_cast<size_t>(gu * Ij + row) * rowb;
-          copy_tx(dbuf + static_cast<size_t>(gu * cv.npc_max + lo) * rowb, src, static_cast<uint32_t>((hi - lo) * rowb),
-                  &bar_gc[b]);
-        }
-      }
-      if (lane < 8) {  // scales and biases: lane = (segment, kind); kind 0/1 gate/up scales, 2/3 gate/up biases
-        const int sg = lane >> 2, kind = lane & 3;
-        const int lo = sg == 0 ? 0 : nA, hi = sg == 0 ? nA : npc;
-        if (hi > lo) {
-          const int j = jA + sg;
-          const bool routed = j < k;
-          const QMat m = routed ? Ld.gu : Ld.sgu;
-          const int Ij = routed ? I : Is;
-          const int row = (sg == 0 ? iA : -nA) + lo;
-          const uint16_t* src = ((kind & 2) ? m.b : m.s) + static_cast<size_t>(routed ? s_idx[j] : 0) * m.sb_stride +
-                                static_cast<size_t>((kind & 1) * Ij + row) * ng;
-          copy_tx(gsb + static_cast<size_t>(kind * cv.npc_max + lo) * ng, src, static_cast<uint32_t>((hi - lo) * ng) * 2u,
-                  &bar_g);
-        }
+      // the buffer was last read and written by ordinary loads and per-thread copies
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      const int b = lane >> 2, sg = (lane >> 1) & 1, gu = lane & 1;
+      const int lo = max(sg == 0 ? 0 : nA, b * kBatch);
+      const int hi = min(sg == 0 ? nA : npc, b * kBatch + kBatch);
+      if (b < kMaxBatches && hi > lo) {
+        const int j = jA + sg;
+        const bool routed = j < k;
+        const QMat& m = routed ? Ld.gu : Ld.sgu;
+        const int Ij = routed ? I : Is;
+        const int row = (sg == 0 ? iA : -nA) + lo;
+        const uint8_t* src = m.q + static_cast<size_t>(routed ? s_idx[j] : 0) * m.q_stride +
+                             static_cast<size_t>(gu * Ij + row) * rowb;
+        copy_tx(dbuf + static_cast<size_t>(gu * cv.npc_max + lo) * rowb, src, static_cast<uint32_t>((hi - lo) * rowb),
+                &bar_gc[b]);
       }
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive1(&bar_g);
 #pragma unroll 1
-        for (int b = 0; b < nb; ++b) mbar_arrive1(&bar_gc[b]);
-        s_pend.g = l & 1;
+        for (int bb = 0; bb < nb; ++bb) mbar_arrive1(&bar_gc[bb]);
         s_pend.gc = l & 1;
       }
       __syncwarp();
-    } else if (warp == 1 && nr > 0) {
+    }
+    {
+      // scales and biases, in 16-byte chunks q = (kind * npc + pair) * cpr + part;
+      // kind 0/1 gate/up scales, 2/3 gate/up biases
+      const int cpr = ng >> 3;
+      const int per_kind = npc * cpr;
 #pragma unroll 1
-      for (int t = lane; t < 3 * nslots; t += 32) {
-        const int j = t / 3, which = t % 3;
+      for (int q = tid; q < 4 * per_kind; q += kThreads) {
+        const int kind = q / per_kind, rem = q - kind * per_kind;
+        const int pair = rem / cpr, part = rem - pair * cpr;
+        const int sg = pair < nA ? 0 : 1;
+        const int j = jA + sg;
         const bool routed = j < k;
-        const QMat m = routed ? Ld.dn : Ld.sdn;
+        const QMat& m = routed ? Ld.gu : Ld.sgu;
+        const int Ij = routed ? I : Is;
+        const int row = sg == 0 ? iA + pair : pair - nA;
+        const uint16_t* src = ((kind & 2) ? m.b : m.s) + static_cast<size_t>(routed ? s_idx[j] : 0) * m.sb_stride +
+                              static_cast<size_t>((kind & 1) * Ij + row) * ng + part * 8;
+        *reinterpret_cast<uint4*>(gsb + static_cast<size_t>(kind * cv.npc_max + pair) * ng + part * 8) =
+            __ldg(reinterpret_cast<const uint4*>(src));
+      }
+      // down rows of every slot (codes, scales, biases) into L2: warp w takes slots w, w + 16, ...
+#pragma unroll 1
+      for (int j = warp; j < (nr > 0 ? nslots : 0); j += kWarps) {
+        const bool routed = j < k;
+        const QMat& m = routed ? Ld.dn : Ld.sdn;
         const size_t e = routed ? static_cast<size_t>(s_idx[j]) : 0;
-        if (which == 0) {
-          prefetch_l2(m.q + e * m.q_stride + static_cast<size_t>(r0) * rowbd, static_cast<uint32_t>(nr * rowbd));
-        } else {
-          const int el0 = (r0 * ngd) & ~7, el1 = al8(r1 * ngd);
-          prefetch_l2((which == 2 ? m.b : m.s) + e * m.sb_stride + el0, static_cast<uint32_t>(el1 - el0) * 2u);
+        const uintptr_t a0 = reinterpret_cast<uintptr_t>(m.q + e * m.q_stride + static_cast<size_t>(r0) * rowbd);
+        const int nl = static_cast<int>(((a0 & 127) + static_cast<uintptr_t>(nr) * rowbd + 127) >> 7);
+#pragma unroll 1
+        for (int t = lane; t < nl; t += 32) prefetch_line_l2(reinterpret_cast<const void*>((a0 & ~uintptr_t(127)) + 128u * t));
+        if (lane < 2) {
+          const uintptr_t s0 =
+              reinterpret_cast<uintptr_t>((lane ? m.b : m.s) + e * m.sb_stride + static_cast<size_t>(r0) * ngd);
+          const int ns = static_cast<int>(((s0 & 127) + static_cast<uintptr_t>(nr) * ngd * 2 + 127) >> 7);
+#pragma unroll 1
+          for (int t = 0; t < ns; ++t) prefetch_line_l2(reinterpret_cast<const void*>((s0 & ~uintptr_t(127)) + 128u * t));
         }
       }
     }
+    __syncthreads();  // the scales are in shared memory
 
-    // ---------------- 4b. gate/up rows + SwiGLU
+    // ---------------- 4b. gate/up rows + SwiGLU, batch by batch as the codes land
     {
       float xv[CH][PS];
       float xsm[CH];
@@ -555,81 +627,105 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         }
         xsm[ch] = a;
       }
-      bool scales_ready = false;
 #pragma unroll 1
       for (int b = 0; b < nb; ++b) {
         const int lo = b * kBatch, n = min(kBatch, npc - lo);
         if (warp * rps >= 2 * n) continue;  // no row of this batch for this warp
-        if (!scales_ready) {
-          if (!mbar_ready(&bar_g, l & 1, p.hdr, 11)) ab = true;
-          scales_ready = true;
-        }
         if (!mbar_ready(&bar_gc[b], l & 1, p.hdr, 12)) ab = true;
-        const int rho = warp * rps + gsub;  // [0, n) gate rows, [n, 2n) up rows of the batch
-        const int gu = rho >= n ? 1 : 0;
-        const int q = lo + rho - gu * n;
-        float acc = 0.f;
-        if (rho < 2 * n) {
-          const unsigned char* row = dbuf + static_cast<size_t>(gu * cv.npc_max + q) * rowb;
-          const uint16_t* sc = gsb + static_cast<size_t>(gu * cv.npc_max + q) * ng;
-          const uint16_t* bi = gsb + static_cast<size_t>((2 + gu) * cv.npc_max + q) * ng;
+        // two rows of the batch at a time (rows rw and rw + 16 * rps), for independent work in flight
+#pragma unroll 1
+        for (int rw = warp * rps; rw < 2 * n; rw += 2 * kWarps * rps) {
+          float acc[2];
+          int qv[2], guv_i[2];
 #pragma unroll
-          for (int ch = 0; ch < CH; ++ch) {
-            const int s = gs0 + 32 * ch;
-            const uint4 cd = *reinterpret_cast<const uint4*>(row + 16 * s);
-            const int g = (s * PS) >> lgG;
-            acc = fmaf(bf16_to_f32(sc[g]), dot_seg<BITS>(cd, xv[ch]), fmaf(bf16_to_f32(bi[g]), xsm[ch], acc));
+          for (int r2 = 0; r2 < 2; ++r2) {
+            const int rho = rw + r2 * kWarps * rps + gsub;  // [0, n) gate rows, [n, 2n) up rows of the batch
+            const int gu = rho >= n ? 1 : 0;
+            const int q = lo + rho - gu * n;
+            qv[r2] = rho < 2 * n ? q : -1;
+            guv_i[r2] = gu * cv.npc_max + q;
+            acc[r2] = 0.f;
+            if (rho < 2 * n) {
+              const unsigned char* row = dbuf + static_cast<size_t>(gu * cv.npc_max + q) * rowb;
+              const uint16_t* sc = gsb + static_cast<size_t>(gu * cv.npc_max + q) * ng;
+              const uint16_t* bi = gsb + static_cast<size_t>((2 + gu) * cv.npc_max + q) * ng;
+#pragma unroll
+              for (int ch = 0; ch < CH; ++ch) {
+                const int s = gs0 + 32 * ch;
+                const uint4 cd = *reinterpret_cast<const uint4*>(row + 16 * s);
+                const int g = (s * PS) >> lgG;
+                acc[r2] = fmaf(bf16_to_f32(sc[g]), dot_seg_dec<BITS>(cd, xv[ch]), fmaf(bf16_to_f32(bi[g]), xsm[ch], acc[r2]));
+              }
+            }
+          }
+          if (nsg >= 32) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
+              acc[1] += __shfl_xor_sync(0xffffffffu, acc[1], o);
+            }
+          } else {
+#pragma unroll 1
+            for (int o = nsg >> 1; o > 0; o >>= 1) {
+              acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
+              acc[1] += __shfl_xor_sync(0xffffffffu, acc[1], o);
+            }
+          }
+          if (gs0 == 0) {
+            if (qv[0] >= 0) guv[guv_i[0]] = acc[0];
+            if (qv[1] >= 0) guv[guv_i[1]] = acc[1];
           }
         }
-        if (nsg >= 32) {
-          acc = warp_sum(acc);
-        } else {
-#pragma unroll 1
-          for (int o = nsg >> 1; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        }
-        if (gs0 == 0 && rho < 2 * n) guv[gu * cv.npc_max + q] = acc;
       }
     }
     const bool gu_failed = __syncthreads_or(ab);
-    if (tid == 0) {
-      s_pend.g = -1;
-      s_pend.gc = -1;
-    }
+    if (tid == 0) s_pend.gc = -1;
     if (gu_failed) { leave(); return; }
     if (tid < npc) {
       const int P = gp0 + tid;
       const int j = P < k * I ? (P >> lgI) : k;
       const int i = P - (j << lgI);
       const float h = silu_f(guv[tid]) * guv[cv.npc_max + tid];
-      st_word(p.hbuf + static_cast<size_t>(j) * I + i, tag_f32(h, par));
-    }
-    // down rows of every slot into the (now free) same buffer: codes, scales, biases
-    if (warp == 0) {
-#pragma unroll 1
-      for (int t = lane; t < (nr > 0 ? 3 * nslots : 0); t += 32) {
-        const int j = t / 3, which = t % 3;
-        const bool routed = j < k;
-        const QMat m = routed ? Ld.dn : Ld.sdn;
-        const size_t e = routed ? static_cast<size_t>(s_idx[j]) : 0;
-        unsigned char* slot = dbuf + static_cast<size_t>(j) * cv.d_slot_bytes;
-        if (which == 0) {
-          copy_tx(slot, m.q + e * m.q_stride + static_cast<size_t>(r0) * rowbd, static_cast<uint32_t>(nr * rowbd), &bar_d);
-        } else {
-          const int el0 = (r0 * ngd) & ~7, el1 = al8(r1 * ngd);
-          uint16_t* sc = reinterpret_cast<uint16_t*>(slot + static_cast<size_t>(cv.nr_max) * rowbd);
-          copy_tx(sc + (which == 2 ? cv.d_sc_el : 0), (which == 2 ? m.b : m.s) + e * m.sb_stride + el0,
-                  static_cast<uint32_t>(el1 - el0) * 2u, &bar_d);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive1(&bar_d);
-        s_pend.d = l & 1;
-      }
+#pragma unroll
+      for (int r = 0; r < kDecodeReplicas; ++r)
+        st_word(p.hbuf + r * p.h_rep + static_cast<size_t>(j) * I + i, tag_f32(h, par));
     }
     stamp(4);
 
-    // ---------------- 5a. every slot's h, by down code segment
+    // ---------------- 5a. this CTA's down rows (L2 hits by now) into shared memory by per-thread
+    // asynchronous copies, issued before the wait on h: the code segment of every work unit
+    // u = (slot, row step) of this warp ([u][lane] x 16 bytes), and (warp j % 16) slot j's
+    // scales and biases of the CTA's rows
+    {
+      unsigned char* dcodes = dbuf;
+      uint16_t* dscl = reinterpret_cast<uint16_t*>(dbuf + cv.dsc);
+#pragma unroll 1
+      for (int u = dn_u0; u < dn_u1; ++u) {
+        const int j = u / dn_upj, t = u - j * dn_upj;
+        const int rl = t * rpsd + dsub;
+        if (rl < nr) {
+          const bool routed = j < k;
+          const QMat& m = routed ? Ld.dn : Ld.sdn;
+          const size_t e = routed ? static_cast<size_t>(s_idx[j]) : 0;
+          cp_async16(dcodes + (static_cast<size_t>(u) * 32 + lane) * 16,
+                     m.q + e * m.q_stride + static_cast<size_t>(r0 + rl) * rowbd + 16 * ds);
+        }
+      }
+      const int el0 = (r0 * ngd) & ~7, nel = (((r1 * ngd) + 7) & ~7) - el0;
+#pragma unroll 1
+      for (int j = warp; j < (nr > 0 ? nslots : 0); j += kWarps) {
+        const bool routed = j < k;
+        const QMat& m = routed ? Ld.dn : Ld.sdn;
+        const size_t e = routed ? static_cast<size_t>(s_idx[j]) : 0;
+#pragma unroll 1
+        for (int q = lane; q < 2 * (nel / 8); q += 32) {
+          const int which = q / (nel / 8), part = q - which * (nel / 8);
+          cp_async16(dscl + (2 * j + which) * cv.d_sc_el + 8 * part, (which ? m.b : m.s) + e * m.sb_stride + el0 + 8 * part);
+        }
+      }
+    }
+
+    // ---------------- 5b. every slot's h, by down code segment
     {
       const int nch = nslots * I / 4;
       uint4 hv[kHChunks];
@@ -640,41 +736,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         for (int u = 0; u < kHChunks; ++u) {
           const int ci = tid + u * kThreads;
           if (ci < nch) {
-            hv[u] = ld_words4(p.hbuf + 4 * ci);
+            hv[u] = ld_words4(h_in + 4 * ci);
             ok &= ((hv[u].x & hv[u].y & hv[u].z & hv[u].w & 1u) == par) && (((hv[u].x | hv[u].y | hv[u].z | hv[u].w) & 1u) == par);
           }
         }
         if (ok) break;
         MOE_POLL_BACKOFF(it, t0, p.hdr, 22, ab)
       }
+      cp_async_wait_all();  // this thread's down copies (visible to all after the barrier below)
 #pragma unroll
       for (int u = 0; u < kHChunks; ++u) {
         const int ci = tid + u * kThreads;
         if (ci < nch) {
           const int j = (4 * ci) >> lgI, i = (4 * ci) & (I - 1);
-          const int s = i / PS, q4 = (i % PS) / 4;
-          reinterpret_cast<uint4*>(hs + static_cast<size_t>(j) * I)[q4 * nsgd + s] = hv[u];
+          const int s = i / PS;
+          float* hj = hs + static_cast<size_t>(j) * I;
+          const uint32_t hw[4] = {hv[u].x, hv[u].y, hv[u].z, hv[u].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int op = seg_pos<BITS>((i + e) % PS);
+            hj[((op >> 2) * nsgd + s) * 4 + (op & 3)] = __uint_as_float(hw[e]);
+          }
         }
       }
     }
     if (__syncthreads_or(ab)) { leave(); return; }
     stamp(5);
 
-    // ---------------- 5b. down rows of every slot for this CTA's output rows
-    if (!mbar_ready(&bar_d, l & 1, p.hdr, 13)) ab = true;
+    // ---------------- 5c. down rows of every slot for this CTA's output rows
     {
+      const uint4* dcodes = reinterpret_cast<const uint4*>(dbuf);
+      const uint16_t* dscl = reinterpret_cast<const uint16_t*>(dbuf + cv.dsc);
       const int off = r0 * ngd - ((r0 * ngd) & ~7);
-      const int g = (ds * PS) >> lgG;
+      const int dg = (ds * PS) >> lgG;
       int cur = -1;
       float hv[PS];
       float hsm = 0.f;
-      int j = dn_j0, t = dn_t0;
 #pragma unroll 1
-      for (int u = dn_u0; u < dn_u1; ++u, ++t) {
-        if (t == dn_upj) {
-          t = 0;
-          ++j;
-        }
+      for (int u = dn_u0; u < dn_u1; ++u) {
+        const int j = u / dn_upj, t = u - j * dn_upj;
         if (j != cur) {
           cur = j;
           hsm = 0.f;
@@ -692,20 +792,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         const int rl = t * rpsd + dsub;
         float part = 0.f;
         if (rl < nr) {
-          const unsigned char* slot = dbuf + static_cast<size_t>(j) * cv.d_slot_bytes;
-          const uint16_t* sc = reinterpret_cast<const uint16_t*>(slot + static_cast<size_t>(cv.nr_max) * rowbd);
-          const uint4 cd = *reinterpret_cast<const uint4*>(slot + static_cast<size_t>(rl) * rowbd + 16 * ds);
-          const int ei = off + rl * ngd + g;
-          part = fmaf(bf16_to_f32(sc[ei]), dot_seg<BITS>(cd, hv), bf16_to_f32(sc[cv.d_sc_el + ei]) * hsm);
+          const int ei = off + rl * ngd + dg;
+          part = fmaf(bf16_to_f32(dscl[2 * j * cv.d_sc_el + ei]), dot_seg_dec<BITS>(dcodes[u * 32 + lane], hv),
+                      bf16_to_f32(dscl[(2 * j + 1) * cv.d_sc_el + ei]) * hsm);
         }
 #pragma unroll 1
         for (int o = nsgd >> 1; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
         if (ds == 0 && rl < nr) dred[j * cv.nr_max + rl] = part;
       }
     }
-    const bool dn_failed = __syncthreads_or(ab);
-    if (tid == 0) s_pend.d = -1;
-    if (dn_failed) { leave(); return; }
+    if (__syncthreads_or(ab)) { leave(); return; }
     if (tid < nr) {
       const int row = r0 + tid;
       float acc = 0.f;
@@ -713,7 +809,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
       for (int j = 0; j < k; ++j) acc = fmaf(s_w[j], dred[j * cv.nr_max + tid], acc);
       if (Is > 0) acc = fmaf(s_sg, dred[k * cv.nr_max + tid], acc);
       const uint16_t yb = f32_to_bf16(acc);
-      st_word(p.ybuf + row, (static_cast<uint32_t>(yb) << 16) | (tag & 0xffffu));
+#pragma unroll
+      for (int r = 0; r < kDecodeReplicas; ++r)
+        st_word(p.ybuf + r * p.y_rep + row, (static_cast<uint32_t>(yb) << 16) | (tag & 0xffffu));
       if (p.tr_y) p.tr_y[static_cast<size_t>(lg) * H + row] = yb;
     }
     stamp(6);
@@ -728,7 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
       uint4 w;
       uint64_t t0 = 0;
       for (uint32_t it = 0;; ++it) {
-        w = ld_words4(p.ybuf + i4);
+        w = ld_words4(y_in + i4);
         if ((w.x & 0xffffu) == ytag && (w.y & 0xffffu) == ytag && (w.z & 0xffffu) == ytag && (w.w & 0xffffu) == ytag)
           break;
         MOE_POLL_BACKOFF(it, t0, p.hdr, 23, ab)

@@ -38,6 +38,17 @@ def layer35():
     return lw, DeviceLayer(S35, lw)
 
 
+@pytest.mark.parametrize("key", ["35b", "35b8", "80b"])
+def test_batched_path_is_taken(key):
+    """The workloads' shapes must run on the tensor-core path from 8 tokens up
+    (route, sort, gather, two GEMMs, combine, glue: 7 kernels a layer), not
+    fall back to the token-at-a-time kernels (4 a layer)."""
+    cfg = moe.make_config(synth.SHAPES[key])
+    assert moe.moe_stack_kernel_launches(cfg, 8, 3) == 1 + 7 * 3
+    assert moe.moe_stack_kernel_launches(cfg, 512, 3) == 1 + 7 * 3
+    assert moe.moe_stack_kernel_launches(cfg, 7, 3) == 1 + 4 * 3
+
+
 @pytest.mark.parametrize("T", [7, 8, 16])
 def test_batched_matches_single_token_and_oracle(layer35, T):
     lw, host = layer35
