@@ -21,10 +21,12 @@
 // expert (same article, paragraph 8; Runnel README, "Target").
 //
 // GEMM CTA (one per SM, persistent over tiles), 16 warps:
-//   warp 0      TMA producer: codes (3D map over the expert stack), scales
-//               and biases (per tile), B tiles (128-byte swizzled);
-//   warp 1      TMEM owner; lane 0 issues tcgen05.mma (M=128, N=16..64, K=16);
-//   warps 4-11  unpack codes into exact fp16 integers, swizzled A tiles;
+//   warp 5      TMA producer: codes (3D map over the expert stack);
+//   warp 9      TMA producer: scales and biases (per tile), B tiles (128-byte swizzled);
+//   warps 1,11  MMA issuers: lane 0 issues tcgen05.mma (M=128, N=16/32, K=16) for
+//               even / odd k-blocks (a single issuing thread spends ~0.6 us of
+//               waits, MMAs and commits per k-block; two halve that); warp 1 owns TMEM;
+//   warps 0,2,3,4,6,7,8,10  unpack codes into exact fp16 integers, swizzled A tiles;
 //   warps 12-15 scale and accumulate, then the epilogue.
 // The weight of code q in group g is s*q + b (MLX-style affine groups), so
 // a row's dot product with a column x is  sum_g ( s_g * P_g + b_g * X_g ),
@@ -54,12 +56,26 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kBM = 128;           // tile rows
-constexpr int kBK = 64;            // K per k-block: one quantisation group, one 128-byte swizzle row
+constexpr int kGK = 64;            // K of one quantisation group: one 128-byte swizzle row of fp16
+constexpr int kSG = 2;             // groups per pipeline stage (every wait and arrive covers two)
 constexpr int kNT = kChunkTokens;  // columns (pairs) per tile
-constexpr int kPBuf = 8;           // TMEM buffers of per-group products in rotation
-constexpr int kNA = 4;             // unpacked A tiles in flight
-constexpr int kDequantWarp0 = 4;   // warps 4..11
-constexpr int kEpiWarp0 = 12;      // warps 12..15
+constexpr int kPS = 4;             // stages of per-group products in TMEM (kPS * kSG buffers)
+constexpr int kNA = 2;             // stages of unpacked A tiles in flight
+constexpr int kNB = 4;             // stages of B tiles in flight
+constexpr int kATileBytes = kBM * kGK * 2;          // one group's A tile (16 KiB)
+constexpr int kAStageBytes = kSG * kATileBytes;
+// Warp roles. Warp w runs on sub-partition w % 4; the MMA issuer is a single
+// latency-bound thread, so its sub-partition (1) holds only light roles besides
+// one scaler (the scalers must cover the four TMEM lane quarters, w % 4).
+constexpr int kMmaWarp = 1;        // TMEM owner; issues the MMAs of even k-blocks
+constexpr int kMmaWarp2 = 11;      // issues the MMAs of odd k-blocks (its own commits and drain)
+constexpr int kCodesWarp = 5;      // TMA producer of the codes
+constexpr int kBWarp = 9;          // TMA producer of the B tiles, scales and biases
+constexpr int kEpiWarp0 = 12;      // warps 12..15: scalers + epilogue
+// unpacker index (0..7) of warp w, or -1
+__host__ __device__ constexpr int unpack_index(int w) {
+  return w == 0 ? 0 : w == 2 ? 1 : w == 3 ? 2 : w == 4 ? 3 : w == 6 ? 4 : w == 7 ? 5 : w == 8 ? 6 : w == 10 ? 7 : -1;
+}
 
 __host__ __device__ constexpr uint32_t al1k(uint32_t v) { return (v + 1023u) & ~1023u; }
 
@@ -70,27 +86,25 @@ __host__ __device__ constexpr int perm8_pos(int k) {  // position of element k
 
 struct GemmSmem {
   uint32_t a, b, codes, sc, xs, bar, total;
-  int na, nb, nc, b_stage_bytes, codes_stage_bytes, sc_buf_bytes;
+  int nc, b_stage_bytes, codes_stage_bytes, sc_buf_bytes;
 };
 
-// Rings: codes (nc k-blocks, freed once unpacked), B tiles (nb, freed by the
-// MMAs), unpacked A tiles (na, freed by the MMAs).
-__host__ __device__ inline GemmSmem gemm_smem(int mode, int bits, int K, int group, int na) {
+// Rings, in stages of kSG groups: codes (nc stages, freed once unpacked), B
+// tiles (kNB, freed by the MMAs), unpacked A tiles (kNA, freed by the MMAs).
+__host__ __device__ inline GemmSmem gemm_smem(int mode, int bits, int K) {
   GemmSmem s{};
-  const int ng = K / group;
-  s.na = na;
-  s.nb = 8;
-  s.b_stage_bytes = (mode == 0 ? 1 : 2) * kNT * 128;  // kNT rows x 128 B (x2: h hi and lo)
-  s.codes_stage_bytes = kBM * (kBK * bits / 8);
-  s.nc = (64 * 1024) / s.codes_stage_bytes;           // 64 KiB of codes in flight
-  s.sc_buf_bytes = 2 * kBM * ng * 2;                  // scales and biases of 128 rows
+  const int ng = K / kGK;
+  s.b_stage_bytes = kSG * (mode == 0 ? 1 : 2) * kNT * 128;  // per group kNT rows x 128 B (x2: h hi and lo)
+  s.codes_stage_bytes = kBM * kSG * (kGK * bits / 8);
+  s.nc = (64 * 1024) / s.codes_stage_bytes;                 // 64 KiB of codes in flight
+  s.sc_buf_bytes = 2 * kBM * ng * 2;                        // scales and biases of 128 rows
   uint32_t o = 0;
-  s.a = o;     o = al1k(o + na * kBM * kBK * 2);
-  s.b = o;     o = al1k(o + s.nb * s.b_stage_bytes);
+  s.a = o;     o = al1k(o + kNA * kAStageBytes);
+  s.b = o;     o = al1k(o + kNB * s.b_stage_bytes);
   s.codes = o; o = al1k(o + s.nc * s.codes_stage_bytes);
   s.sc = o;    o = al1k(o + 2 * s.sc_buf_bytes);
   s.xs = o;    o = al1k(o + 4 * ng * kNT * 4);        // group sums of the tile's columns, one copy per scaling warp
-  s.bar = o;   o += 1024;  // up to ~70 mbarriers, the TMEM slot and the abort flag
+  s.bar = o;   o += 1024;  // the mbarriers (~45), the TMEM slot and the abort flag
   s.total = o + 1024;  // slack to align the dynamic base to 1 KiB
   return s;
 }
@@ -171,30 +185,30 @@ __device__ __forceinline__ void unpack32_u8(const uint4 c0, const uint4 c1, uint
 
 // ------------------------------------------------------------------ GEMM kernel
 
-template <int MODE, int BITS, int NA>
+template <int MODE, int BITS>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const GemmSmem L = gemm_smem(MODE, BITS, p.K, kBK, NA);
-  const int NC = L.nc, NB = L.nb;
+  const GemmSmem L = gemm_smem(MODE, BITS, p.K);
+  const int NC = L.nc;
   uint64_t* cfull = reinterpret_cast<uint64_t*>(sm + L.bar);  // [NC] codes landed
   uint64_t* cempty = cfull + NC;                              // [NC] codes unpacked
-  uint64_t* bfull = cempty + NC;                              // [NB] B tile landed
-  uint64_t* bempty = bfull + NB;                              // [NB] MMAs done with the B tile
-  uint64_t* afull = bempty + NB;                              // [NA] A tile written
-  uint64_t* aempty = afull + NA;                              // [NA] MMAs done with the A tile
-  uint64_t* scfull = aempty + NA;                             // [2] scales of a tile landed
+  uint64_t* bfull = cempty + NC;                              // [kNB] B tiles landed
+  uint64_t* bempty = bfull + kNB;                             // [kNB] MMAs done with the B tiles
+  uint64_t* afull = bempty + kNB;                             // [kNA] A tiles written
+  uint64_t* aempty = afull + kNA;                             // [kNA] MMAs done with the A tiles
+  uint64_t* scfull = aempty + kNA;                            // [2] scales of a tile landed
   uint64_t* scempty = scfull + 2;                             // [2] scalers done with them
-  uint64_t* pfull = scempty + 2;                              // [kPBuf] a group's products are in TMEM
-  uint64_t* pempty = pfull + kPBuf;                           // [kPBuf] scalers have read them
-  uint64_t* drain = pempty + kPBuf;                           // MMA issuer: everything issued has finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* pfull = scempty + 2;                              // [kPS] a stage's products are in TMEM
+  uint64_t* pempty = pfull + kPS;                             // [kPS] scalers have read them
+  uint64_t* drain = pempty + kPS;                             // [2] MMA issuers: everything issued has finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int CB = kBK * BITS / 8;          // code bytes per row per k-block
-  const int ng = p.K / kBK;               // groups per row (one per k-block)
-  const int nkb = ng;
+  const int CB = kGK * BITS / 8;          // code bytes per row per group
+  const int ng = p.K / kGK;               // groups per row
+  const int nst = ng / kSG;               // stages per tile (ng is a multiple of 8)
   const int MT = (MODE == 0) ? p.I / 64 : p.H / kBM;
   const int nchunks = *p.nchunks;
   const int ntiles = nchunks * MT;
@@ -204,11 +218,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       mbar_init(&cfull[i], 1);
       mbar_init(&cempty[i], 8);
     }
-    for (int i = 0; i < NB; ++i) {
+    for (int i = 0; i < kNB; ++i) {
       mbar_init(&bfull[i], 1);
       mbar_init(&bempty[i], 1);
     }
-    for (int i = 0; i < NA; ++i) {
+    for (int i = 0; i < kNA; ++i) {
       mbar_init(&afull[i], 8);
       mbar_init(&aempty[i], 1);
     }
@@ -216,16 +230,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       mbar_init(&scfull[i], 1);
       mbar_init(&scempty[i], 4);
     }
-    for (int i = 0; i < kPBuf; ++i) {
+    for (int i = 0; i < kPS; ++i) {
       mbar_init(&pfull[i], 1);
       mbar_init(&pempty[i], 4);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
-    tc::tmem_alloc(tmem_slot, kPBuf * kNT);
+  if (warp == kMmaWarp) {
+    tc::tmem_alloc(tmem_slot, kPS * kSG * kNT);
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
@@ -233,11 +248,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == kCodesWarp) {
     // ------------------------------------------------ codes producer (deep ring, freed by the unpackers)
     if (lane == 0) {
       for (int i = 0; i < 2; ++i) tc::prefetch_tmap(&p.tm_codes[i]);
-      int kbg = 0, last = -1;
+      int sg = 0, last = -1;
       for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
         const int ci = t / MT, mt = t % MT;
         const int e = p.chunks[3 * ci];
@@ -246,29 +261,29 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         const int r0 = (MODE == 0) ? mt * 64 : mt * kBM;
         const int r1 = (MODE == 0) ? p.rows / 2 + mt * 64 : mt * kBM + 64;
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
-          const int s = kbg % NC, u = kbg / NC;
+        for (int st = 0; st < nst; ++st, ++sg) {
+          const int s = sg % NC, u = sg / NC;
           if (u >= 1 && !wait_or_abort(&cempty[s], (u - 1) & 1, p.hdr, abort, 31)) { ok = false; break; }
           unsigned char* cs = sm + L.codes + s * L.codes_stage_bytes;
           tc::mbar_expect_tx(&cfull[s], static_cast<uint32_t>(L.codes_stage_bytes));
-          tc::tma_load_3d(cs, &p.tm_codes[mi], kb * CB, r0, ez, &cfull[s]);
-          tc::tma_load_3d(cs + 64 * CB, &p.tm_codes[mi], kb * CB, r1, ez, &cfull[s]);
+          tc::tma_load_3d(cs, &p.tm_codes[mi], st * kSG * CB, r0, ez, &cfull[s]);
+          tc::tma_load_3d(cs + 64 * kSG * CB, &p.tm_codes[mi], st * kSG * CB, r1, ez, &cfull[s]);
           tc::mbar_arrive(&cfull[s]);
-          last = kbg;
+          last = sg;
         }
         if (!ok) break;
       }
       // leave no copy in flight
       for (int j = (last - NC + 1 > 0 ? last - NC + 1 : 0); j <= last; ++j) mbar_wait(&cfull[j % NC], (j / NC) & 1, p.hdr, 39);
     }
-  } else if (warp == 2) {
+  } else if (warp == kBWarp) {
     // ------------------------------------------------ B tiles and scales producer (freed by MMAs / scalers)
     if (lane == 0) {
       for (int i = 0; i < 2; ++i) {
         tc::prefetch_tmap(&p.tm_scales[i]);
         tc::prefetch_tmap(&p.tm_biases[i]);
       }
-      int kbg = 0, it = 0, last = -1;
+      int sg = 0, it = 0, last = -1;
       int sc_armed[2] = {-1, -1};
       for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++it) {
         const int ci = t / MT, mt = t % MT;
@@ -291,90 +306,106 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         tc::mbar_arrive(&scfull[tb]);
         sc_armed[tb] = tu;
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
-          const int s = kbg % NB, u = kbg / NB;
+        for (int st = 0; st < nst; ++st, ++sg) {
+          const int s = sg % kNB, u = sg / kNB;
           if (u >= 1 && !wait_or_abort(&bempty[s], (u - 1) & 1, p.hdr, abort, 32)) { ok = false; break; }
           unsigned char* bs = sm + L.b + s * L.b_stage_bytes;
-          tc::mbar_expect_tx(&bfull[s], static_cast<uint32_t>(brows) * 128u * (MODE == 0 ? 1u : 2u));
-          tc::tma_load_2d(bs, &p.tm_b[bi], kb * kBK, start, &bfull[s]);
-          if (MODE == 1) tc::tma_load_2d(bs + kNT * 128, &p.tm_b2[bi], kb * kBK, start, &bfull[s]);
+          tc::mbar_expect_tx(&bfull[s], static_cast<uint32_t>(brows) * 128u * kSG * (MODE == 0 ? 1u : 2u));
+#pragma unroll
+          for (int g = 0; g < kSG; ++g) {
+            tc::tma_load_2d(bs + g * kNT * 128, &p.tm_b[bi], (st * kSG + g) * kGK, start, &bfull[s]);
+            if (MODE == 1) tc::tma_load_2d(bs + (kSG + g) * kNT * 128, &p.tm_b2[bi], (st * kSG + g) * kGK, start, &bfull[s]);
+          }
           tc::mbar_arrive(&bfull[s]);
-          last = kbg;
+          last = sg;
         }
         if (!ok) break;
       }
-      for (int j = (last - NB + 1 > 0 ? last - NB + 1 : 0); j <= last; ++j) mbar_wait(&bfull[j % NB], (j / NB) & 1, p.hdr, 37);
+      for (int j = (last - kNB + 1 > 0 ? last - kNB + 1 : 0); j <= last; ++j) mbar_wait(&bfull[j % kNB], (j / kNB) & 1, p.hdr, 37);
       for (int b = 0; b < 2; ++b)
         if (sc_armed[b] >= 0) mbar_wait(&scfull[b], sc_armed[b] & 1, p.hdr, 38);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer: one group per k-block into its own TMEM buffer
+  } else if (warp == kMmaWarp || warp == kMmaWarp2) {
+    // ------------------------------------------------ MMA issuers: each group of a stage into its own TMEM buffer
+    const int par = (warp == kMmaWarp) ? 0 : 1;  // stages of this parity (nst is even)
     if (lane == 0) {
-      int kbg = 0;
+      int sg = 0;
       for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
         const int ci = t / MT;
         const int cnt = p.chunks[3 * ci + 2];
         const int npad = (cnt + 15) & ~15;
         const uint32_t idesc = tc::idesc_f16_f32(kBM, npad);
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
-          const int as = kbg % NA, au = kbg / NA;
-          const int bs = kbg % NB, bu = kbg / NB;
-          const int pb = kbg % kPBuf, pu = kbg / kPBuf;
+        for (int st = 0; st < nst; ++st, ++sg) {
+          if ((sg & 1) != par) continue;
+          const int as = sg % kNA, au = sg / kNA;
+          const int bs = sg % kNB, bu = sg / kNB;
+          const int ps = sg % kPS, pu = sg / kPS;
           if (!wait_or_abort(&afull[as], au & 1, p.hdr, abort, 41) || !wait_or_abort(&bfull[bs], bu & 1, p.hdr, abort, 42) ||
-              (pu >= 1 && !wait_or_abort(&pempty[pb], (pu - 1) & 1, p.hdr, abort, 43))) {
+              (pu >= 1 && !wait_or_abort(&pempty[ps], (pu - 1) & 1, p.hdr, abort, 43))) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
-          const uint32_t a0 = smem_addr(sm + L.a + as * kBM * kBK * 2);
+          const uint32_t a0 = smem_addr(sm + L.a + as * kAStageBytes);
           const uint32_t b0 = smem_addr(sm + L.b + bs * L.b_stage_bytes);
-          const uint32_t dt = tmem + pb * kNT;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = tc::smem_desc_sw128(a0 + kk * 32);
-            tc::mma_f16(dt, ad, tc::smem_desc_sw128(b0 + kk * 32), idesc, kk != 0);
-            if (MODE == 1) tc::mma_f16(dt, ad, tc::smem_desc_sw128(b0 + kNT * 128 + kk * 32), idesc, 1);
+          for (int g = 0; g < kSG; ++g) {
+            const uint32_t dt = tmem + (ps * kSG + g) * kNT;
+            const uint32_t ag = a0 + g * kATileBytes, bg = b0 + g * kNT * 128;
+#pragma unroll
+            for (int kk = 0; kk < kGK / 16; ++kk) {
+              const uint64_t ad = tc::smem_desc_sw128(ag + kk * 32);
+              tc::mma_f16(dt, ad, tc::smem_desc_sw128(bg + kk * 32), idesc, kk != 0);
+              if (MODE == 1) tc::mma_f16(dt, ad, tc::smem_desc_sw128(bg + kSG * kNT * 128 + kk * 32), idesc, 1);
+            }
           }
           tc::commit(&aempty[as]);
           tc::commit(&bempty[bs]);
-          tc::commit(&pfull[pb]);
+          tc::commit(&pfull[ps]);
         }
         if (!ok) break;
       }
       // every MMA issued must be finished before TMEM is released
-      tc::commit(drain);
-      mbar_wait(drain, 0, p.hdr, 49);
+      tc::commit(&drain[par]);
+      mbar_wait(&drain[par], 0, p.hdr, 49);
     }
-  } else if (warp >= kDequantWarp0 && warp < kEpiWarp0) {
-    // ------------------------------------------------ unpackers: 2 threads per row
-    const int d = threadIdx.x - kDequantWarp0 * 32;  // 0..255
-    const int m = d >> 1, half = d & 1;              // A-tile row, which 32 codes of the 64
+  } else if (unpack_index(warp) >= 0) {
+    // ------------------------------------------------ unpackers: 2 threads per row, both groups of a stage
+    const int d = unpack_index(warp) * 32 + lane;  // 0..255
+    const int m = d >> 1, half = d & 1;              // A-tile row, which 32 codes of each group's 64
     // A row m <- staging row: gate/up interleaved for mode 0, identity for mode 1
     const int srow = (MODE == 0) ? ((m & 1) * 64 + (m >> 1)) : m;
-    int kbg = 0;
+    int sg = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       if (warp_aborted(abort)) break;
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb, ++kbg) {
-        const int cs = kbg % NC, cu = kbg / NC;
-        const int as = kbg % NA, au = kbg / NA;
+      for (int st = 0; st < nst; ++st, ++sg) {
+        const int cs = sg % NC, cu = sg / NC;
+        const int as = sg % kNA, au = sg / kNA;
         if (!warp_wait(&cfull[cs], cu & 1, p.hdr, abort, 51)) { ok = false; break; }
         if (au >= 1 && !warp_wait(&aempty[as], (au - 1) & 1, p.hdr, abort, 52)) { ok = false; break; }
-        const unsigned char* crow = sm + L.codes + cs * L.codes_stage_bytes + srow * CB + half * (CB / 2);
-        uint4 outv[4];
-        if (BITS == 4) {
-          unpack32_u4(*reinterpret_cast<const uint4*>(crow), outv);
-        } else {
-          unpack32_u8(*reinterpret_cast<const uint4*>(crow), *reinterpret_cast<const uint4*>(crow + 16), outv);
+        const unsigned char* crow = sm + L.codes + cs * L.codes_stage_bytes + srow * (kSG * CB) + half * (CB / 2);
+        uint4 outv[kSG][4];
+#pragma unroll
+        for (int g = 0; g < kSG; ++g) {
+          if (BITS == 4) {
+            unpack32_u4(*reinterpret_cast<const uint4*>(crow + g * CB), outv[g]);
+          } else {
+            unpack32_u8(*reinterpret_cast<const uint4*>(crow + g * CB), *reinterpret_cast<const uint4*>(crow + g * CB + 16),
+                        outv[g]);
+          }
         }
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&cempty[cs]);  // codes read: the slot can be refilled
-        unsigned char* arow = sm + L.a + as * kBM * kBK * 2 + (m >> 3) * 1024 + (m & 7) * 128;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int chunk = half * 4 + q;
-          *reinterpret_cast<uint4*>(arow + ((chunk ^ (m & 7)) << 4)) = outv[q];
+        for (int g = 0; g < kSG; ++g) {
+          unsigned char* arow = sm + L.a + as * kAStageBytes + g * kATileBytes + (m >> 3) * 1024 + (m & 7) * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = half * 4 + q;
+            *reinterpret_cast<uint4*>(arow + ((chunk ^ (m & 7)) << 4)) = outv[g][q];
+          }
         }
         tc::fence_proxy_async_smem();
         __syncwarp();
@@ -388,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     const int m = 32 * q + lane;    // accumulator row held by this thread
     const int srow = (MODE == 0) ? ((m & 1) * 64 + (m >> 1)) : m;
     float* xs = reinterpret_cast<float*>(sm + L.xs) + q * ng * kNT;  // this warp's [ng][kNT]
-    int kbg = 0, it = 0;
+    int sg = 0, it = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
       if (warp_aborted(abort)) break;
       const int ci = t / MT, mt = t % MT;
@@ -406,21 +437,21 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
           float4 f[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int q = v0 + u * 32 + lane;
-            if (q < nvec) f[u] = __ldg(src + q);
+            const int qq = v0 + u * 32 + lane;
+            if (qq < nvec) f[u] = __ldg(src + qq);
           }
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int q = v0 + u * 32 + lane;
-            if (q < nvec) {
+            const int qq = v0 + u * 32 + lane;
+            if (qq < nvec) {
               if (MODE == 0) {
-                const int n = (4 * q) / ng, g = (4 * q) % ng;
+                const int n = (4 * qq) / ng, g = (4 * qq) % ng;
                 xs[g * kNT + n] = f[u].x;
                 xs[(g + 1) * kNT + n] = f[u].y;
                 xs[(g + 2) * kNT + n] = f[u].z;
                 xs[(g + 3) * kNT + n] = f[u].w;
               } else {
-                const int n = q / ng, g = q % ng;
+                const int n = qq / ng, g = qq % ng;
                 xs[g * kNT + n] = (f[u].x + f[u].y) + (f[u].z + f[u].w);
               }
             }
@@ -435,46 +466,38 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
 #pragma unroll
       for (int n = 0; n < kNT; ++n) acc[n] = 0.f;
       bool ok = true;
-      // two groups per step: both TMEM loads in flight under one wait
-      for (int kb = 0; kb < nkb; kb += 2, kbg += 2) {
-        const bool two = kb + 1 < nkb;
-        const int pb0 = kbg % kPBuf, pb1 = (kbg + 1) % kPBuf;
-        if (!warp_wait(&pfull[pb0], (kbg / kPBuf) & 1, p.hdr, abort, 61) ||
-            (two && !warp_wait(&pfull[pb1], ((kbg + 1) / kPBuf) & 1, p.hdr, abort, 61))) {
-          ok = false;
-          break;
-        }
+      for (int st = 0; st < nst; ++st, ++sg) {
+        const int ps = sg % kPS, pu = sg / kPS;
+        if (!warp_wait(&pfull[ps], pu & 1, p.hdr, abort, 61)) { ok = false; break; }
         tc::fence_after_sync();
-        const uint32_t tq = tmem + (static_cast<uint32_t>(32 * q) << 16);
-        const float sc0 = bf16_to_f32(scs[srow * ng + kb]);
-        const float bi0 = bf16_to_f32(bis[srow * ng + kb]);
-        const float sc1 = two ? bf16_to_f32(scs[srow * ng + kb + 1]) : 0.f;
-        const float bi1 = two ? bf16_to_f32(bis[srow * ng + kb + 1]) : 0.f;
-        const float* x0 = xs + kb * kNT;
+        const uint32_t tq = tmem + (static_cast<uint32_t>(32 * q) << 16) + ps * kSG * kNT;
+        const int g0 = st * kSG;
+        const float sc0 = bf16_to_f32(scs[srow * ng + g0]);
+        const float bi0 = bf16_to_f32(bis[srow * ng + g0]);
+        const float sc1 = bf16_to_f32(scs[srow * ng + g0 + 1]);
+        const float bi1 = bf16_to_f32(bis[srow * ng + g0 + 1]);
+        const float* x0 = xs + g0 * kNT;
         // columns in halves of 16 (the upper half only when the chunk has more than 16 pairs)
 #pragma unroll
         for (int hf = 0; hf < kNT / 16; ++hf) {
           if (hf * 16 < cnt) {
             uint32_t v0[16], v1[16];
-            tc::tmem_ld16(tq + pb0 * kNT + hf * 16, v0);
-            if (two) tc::tmem_ld16(tq + pb1 * kNT + hf * 16, v1);
+            tc::tmem_ld16(tq + hf * 16, v0);
+            tc::tmem_ld16(tq + kNT + hf * 16, v1);
             tc::tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
               const int n = hf * 16 + c;
               if (n < cnt) {
                 acc[n] = fmaf(sc0, __uint_as_float(v0[c]), fmaf(bi0, x0[n], acc[n]));
-                if (two) acc[n] = fmaf(sc1, __uint_as_float(v1[c]), fmaf(bi1, x0[kNT + n], acc[n]));
+                acc[n] = fmaf(sc1, __uint_as_float(v1[c]), fmaf(bi1, x0[kNT + n], acc[n]));
               }
             }
           }
         }
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) {
-          tc::mbar_arrive(&pempty[pb0]);
-          if (two) tc::mbar_arrive(&pempty[pb1]);
-        }
+        if (lane == 0) tc::mbar_arrive(&pempty[ps]);
       }
       if (!ok) break;
       __syncwarp();
@@ -505,10 +528,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         for (int o = 16; o >= 1; o >>= 1) {
           const bool upper = (lane & o) != 0;
 #pragma unroll
-          for (int i = 0; i < o; ++i) {
-            const float send = upper ? hv[i] : hv[i + o];
-            const float keep = upper ? hv[i + o] : hv[i];
-            hv[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+          for (int i2 = 0; i2 < o; ++i2) {
+            const float send = upper ? hv[i2] : hv[i2 + o];
+            const float keep = upper ? hv[i2 + o] : hv[i2];
+            hv[i2] = keep + __shfl_xor_sync(0xffffffffu, send, o);
           }
         }
         if (lane < cnt) p.hsum_out[(static_cast<size_t>(start + lane) * (p.I / 64) + mt) * 4 + q] = hv[0];
@@ -526,9 +549,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, kPBuf * kNT);
+    tc::tmem_dealloc(tmem, kPS * kSG * kNT);
   }
 }
 
@@ -597,10 +620,10 @@ __global__ void __launch_bounds__(256) combine_kernel(BatchParams p) {
   }
 }
 
-template <int MODE, int BITS, int NA>
+template <int MODE, int BITS>
 cudaError_t launch_gemm_t(const GemmParams& g, int grid, cudaStream_t st) {
-  const GemmSmem L = gemm_smem(MODE, BITS, g.K, kBK, NA);
-  auto kern = grouped_gemm_kernel<MODE, BITS, NA>;
+  const GemmSmem L = gemm_smem(MODE, BITS, g.K);
+  auto kern = grouped_gemm_kernel<MODE, BITS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, L.total, st>>>(g);
@@ -611,12 +634,12 @@ cudaError_t launch_gemm_t(const GemmParams& g, int grid, cudaStream_t st) {
 
 size_t grouped_gemm_smem(int mode, int bits, int K, int group) {
   (void)group;
-  return gemm_smem(mode, bits, K, kBK, kNA).total;
+  return gemm_smem(mode, bits, K).total;
 }
 
 cudaError_t launch_grouped_gemm(const GemmParams& g, int mode, int bits, int grid, cudaStream_t st) {
-  if (mode == 0) return bits == 4 ? launch_gemm_t<0, 4, kNA>(g, grid, st) : launch_gemm_t<0, 8, kNA>(g, grid, st);
-  return bits == 4 ? launch_gemm_t<1, 4, kNA>(g, grid, st) : launch_gemm_t<1, 8, kNA>(g, grid, st);
+  if (mode == 0) return bits == 4 ? launch_gemm_t<0, 4>(g, grid, st) : launch_gemm_t<0, 8>(g, grid, st);
+  return bits == 4 ? launch_gemm_t<1, 4>(g, grid, st) : launch_gemm_t<1, 8>(g, grid, st);
 }
 
 cudaError_t launch_gather(const BatchParams& p, int grid, cudaStream_t st) {

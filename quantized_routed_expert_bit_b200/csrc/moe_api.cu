@@ -320,9 +320,9 @@ moe_status batched_ffn(const moe_config& c, const moe_layer_weights& wt, const u
   const moe_qtensor& sdn = shared ? wt.shared_down : wt.down;
   // gate/up: K = H, rows = 2I
   bool ok = map_3d(&gp->tm_codes[0], wt.gate_up.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H * bits / 8, 2 * I, E,
-                   wt.gate_up.q_expert_stride, 64 * bits / 8) &&
+                   wt.gate_up.q_expert_stride, 128 * bits / 8) &&
             map_3d(&gp->tm_codes[1], sgu.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, H * bits / 8, 2 * I, 1,
-                   static_cast<int64_t>(2) * I * H * bits / 8, 64 * bits / 8) &&
+                   static_cast<int64_t>(2) * I * H * bits / 8, 128 * bits / 8) &&
             map_3d(&gp->tm_scales[0], wt.gate_up.scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, H / g, 2 * I, E,
                    wt.gate_up.sb_expert_stride * 2, H / g) &&
             map_3d(&gp->tm_scales[1], sgu.scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, H / g, 2 * I, 1,
@@ -352,9 +352,9 @@ moe_status batched_ffn(const moe_config& c, const moe_layer_weights& wt, const u
   if ((e = moe::launch_grouped_gemm(*gp, 0, bits, sms, st)) != cudaSuccess) return cuda_fail(e, "gate/up GEMM launch");
   // down: K = I, rows = H
   ok = map_3d(&gp->tm_codes[0], wt.down.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, I * bits / 8, H, E,
-              wt.down.q_expert_stride, 64 * bits / 8) &&
+              wt.down.q_expert_stride, 128 * bits / 8) &&
        map_3d(&gp->tm_codes[1], sdn.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, I * bits / 8, H, 1,
-              static_cast<int64_t>(H) * I * bits / 8, 64 * bits / 8) &&
+              static_cast<int64_t>(H) * I * bits / 8, 128 * bits / 8) &&
        map_3d(&gp->tm_scales[0], wt.down.scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, I / g, H, E,
               wt.down.sb_expert_stride * 2, I / g) &&
        map_3d(&gp->tm_scales[1], sdn.scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, I / g, H, 1,
