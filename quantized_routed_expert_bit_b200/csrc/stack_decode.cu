@@ -82,12 +82,14 @@ __host__ __device__ inline Carve carve(int H, int E, int k, int I, int Is, int g
   c.dred = o;  o = al128(o + c.nslots * c.nr_max * 4);
   c.guv = o;   o = al128(o + 2 * c.npc_max * 4);
   c.gsb = o;   o = al128(o + 4 * c.npc_max * c.ng * 2);
-  // one buffer: first this CTA's gate/up code rows ([gate rows][up rows]), then its down
-  // code segments by work unit ([unit][lane] x 16 bytes) and down scales and biases by slot
+  // one buffer: first this CTA's gate/up code rows ([gate rows][up rows]), then (once gate/up
+  // is done) its down code segments by work unit ([unit][lane] x 16 bytes) and its down scales
+  // and biases by slot. (Copying the down rows into a region of their own right after top-k
+  // was measured slower: they compete with the gate/up stream, which is on the critical path.)
   const uint32_t gu_bytes = 2u * c.npc_max * c.rowb;
   const uint32_t dn_bytes = c.nunits * 512u + c.nslots * 4u * c.d_sc_el;
+  c.dsc = c.nunits * 512u;  // offset of the down scales inside the buffer
   c.dbuf = o;  o = al128(o + (gu_bytes > dn_bytes ? gu_bytes : dn_bytes));
-  c.dsc = c.nunits * 512u;  // offset of the down scales inside dbuf
   c.rbuf = o;  o = al128(o + 2 * c.rr_max * H * 2);
   c.desc = o;  o = al128(o + kMaxDecodeLayers * sizeof(LayerDesc));  // the launch's layer descriptors
   c.total = o;
@@ -152,12 +154,11 @@ __device__ __noinline__ bool give_up(uint64_t t0, uint32_t it, WsHeader* hdr, in
   return false;
 }
 
-// Between two polls that found a word not yet written: sleep a little; every
-// 16 polls ask give_up.
+// Between two polls that found a word not yet written (each poll is one L2
+// round trip, no sleep): every 16 polls ask give_up.
 #define MOE_POLL_BACKOFF(it, t0, hdr, where, fail) \
   {                                                \
     if ((it) == 0) (t0) = globaltimer_ns();        \
-    __nanosleep(128);                              \
     if (((it) & 15u) == 15u && give_up((t0), (it), (hdr), (where))) { \
       fail = true;                                 \
       break;                                       \
@@ -388,6 +389,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
   // this warp's share of the down work: units (slot, row step), slot-major
   const int dn_upj = cdiv(nr, rpsd);
   const int dn_u0 = warp * nslots * dn_upj / kWarps, dn_u1 = (warp + 1) * nslots * dn_upj / kWarps;
+  unsigned char* const dnbuf = sm + cv.dbuf;
+  // this CTA's down rows into shared memory by per-thread asynchronous copies: the code
+  // segment of every work unit u = (slot, row step) of this warp ([u][lane] x 16 bytes), and
+  // (warp j % 16) slot j's scales and biases of the CTA's rows
+  auto issue_down = [&](const LayerDesc& Ld) {
+    uint16_t* dscl = reinterpret_cast<uint16_t*>(dnbuf + cv.dsc);
+#pragma unroll 1
+    for (int u = dn_u0; u < dn_u1; ++u) {
+      const int j = u / dn_upj, t = u - j * dn_upj;
+      const int rl = t * rpsd + dsub;
+      if (rl < nr) {
+        const bool routed = j < k;
+        const QMat& m = routed ? Ld.dn : Ld.sdn;
+        const size_t e = routed ? static_cast<size_t>(s_idx[j]) : 0;
+        cp_async16(dnbuf + (static_cast<size_t>(u) * 32 + lane) * 16,
+                   m.q + e * m.q_stride + static_cast<size_t>(r0 + rl) * rowbd + 16 * ds);
+      }
+    }
+    const int el0 = (r0 * ngd) & ~7, nel = (((r1 * ngd) + 7) & ~7) - el0;
+#pragma unroll 1
+    for (int j = warp; j < (nr > 0 ? nslots : 0); j += kWarps) {
+      const bool routed = j < k;
+      const QMat& m = routed ? Ld.dn : Ld.sdn;
+      const size_t e = routed ? static_cast<size_t>(s_idx[j]) : 0;
+#pragma unroll 1
+      for (int q = lane; q < 2 * (nel / 8); q += 32) {
+        const int which = q / (nel / 8), part = q - which * (nel / 8);
+        cp_async16(dscl + (2 * j + which) * cv.d_sc_el + 8 * part, (which ? m.b : m.s) + e * m.sb_stride + el0 + 8 * part);
+      }
+    }
+  };
 
   for (int l = 0; l < p.L; ++l) {
     const int lg = p.l0 + l;  // layer index within the whole stack (trace rows)
@@ -504,7 +536,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
           if (__all_sync(0xffffffffu, ok)) break;
           // warp-uniform give-up decision (lane 0 checks)
           if (it == 0) t0 = globaltimer_ns();
-          __nanosleep(128);
           if ((it & 15u) == 15u && __any_sync(0xffffffffu, lane == 0 && give_up(t0, it, p.hdr, 21))) {
             fail = true;
             break;
@@ -587,6 +618,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         *reinterpret_cast<uint4*>(gsb + static_cast<size_t>(kind * cv.npc_max + pair) * ng + part * 8) =
             __ldg(reinterpret_cast<const uint4*>(src));
       }
+    }
+    {
       // down rows of every slot (codes, scales, biases) into L2: warp w takes slots w, w + 16, ...
 #pragma unroll 1
       for (int j = warp; j < (nr > 0 ? nslots : 0); j += kWarps) {
@@ -692,38 +725,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
     }
     stamp(4);
 
-    // ---------------- 5a. this CTA's down rows (L2 hits by now) into shared memory by per-thread
-    // asynchronous copies, issued before the wait on h: the code segment of every work unit
-    // u = (slot, row step) of this warp ([u][lane] x 16 bytes), and (warp j % 16) slot j's
-    // scales and biases of the CTA's rows
-    {
-      unsigned char* dcodes = dbuf;
-      uint16_t* dscl = reinterpret_cast<uint16_t*>(dbuf + cv.dsc);
-#pragma unroll 1
-      for (int u = dn_u0; u < dn_u1; ++u) {
-        const int j = u / dn_upj, t = u - j * dn_upj;
-        const int rl = t * rpsd + dsub;
-        if (rl < nr) {
-          const bool routed = j < k;
-          const QMat& m = routed ? Ld.dn : Ld.sdn;
-          const size_t e = routed ? static_cast<size_t>(s_idx[j]) : 0;
-          cp_async16(dcodes + (static_cast<size_t>(u) * 32 + lane) * 16,
-                     m.q + e * m.q_stride + static_cast<size_t>(r0 + rl) * rowbd + 16 * ds);
-        }
-      }
-      const int el0 = (r0 * ngd) & ~7, nel = (((r1 * ngd) + 7) & ~7) - el0;
-#pragma unroll 1
-      for (int j = warp; j < (nr > 0 ? nslots : 0); j += kWarps) {
-        const bool routed = j < k;
-        const QMat& m = routed ? Ld.dn : Ld.sdn;
-        const size_t e = routed ? static_cast<size_t>(s_idx[j]) : 0;
-#pragma unroll 1
-        for (int q = lane; q < 2 * (nel / 8); q += 32) {
-          const int which = q / (nel / 8), part = q - which * (nel / 8);
-          cp_async16(dscl + (2 * j + which) * cv.d_sc_el + 8 * part, (which ? m.b : m.s) + e * m.sb_stride + el0 + 8 * part);
-        }
-      }
-    }
+    // ---------------- 5a. this CTA's down rows, L2 hits by now, into the (now free) gate/up
+    // buffer, issued before the wait on h
+    issue_down(Ld);
 
     // ---------------- 5b. every slot's h, by down code segment
     {
@@ -765,15 +769,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
 
     // ---------------- 5c. down rows of every slot for this CTA's output rows
     {
-      const uint4* dcodes = reinterpret_cast<const uint4*>(dbuf);
-      const uint16_t* dscl = reinterpret_cast<const uint16_t*>(dbuf + cv.dsc);
+      const uint4* dcodes = reinterpret_cast<const uint4*>(dnbuf);
+      const uint16_t* dscl = reinterpret_cast<const uint16_t*>(dnbuf + cv.dsc);
       const int off = r0 * ngd - ((r0 * ngd) & ~7);
       const int dg = (ds * PS) >> lgG;
       int cur = -1;
       float hv[PS];
       float hsm = 0.f;
+      // two units of the same slot at a time where possible (independent work in flight)
+      int u = dn_u0;
 #pragma unroll 1
-      for (int u = dn_u0; u < dn_u1; ++u) {
+      while (u < dn_u1) {
         const int j = u / dn_upj, t = u - j * dn_upj;
         if (j != cur) {
           cur = j;
@@ -789,16 +795,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
             hsm += (f.x + f.y) + (f.z + f.w);
           }
         }
-        const int rl = t * rpsd + dsub;
-        float part = 0.f;
-        if (rl < nr) {
-          const int ei = off + rl * ngd + dg;
-          part = fmaf(bf16_to_f32(dscl[2 * j * cv.d_sc_el + ei]), dot_seg_dec<BITS>(dcodes[u * 32 + lane], hv),
-                      bf16_to_f32(dscl[(2 * j + 1) * cv.d_sc_el + ei]) * hsm);
+        const int nu = (u + 1 < dn_u1 && t + 1 < dn_upj) ? 2 : 1;  // warp-uniform
+        float part[2] = {0.f, 0.f};
+        int rlv[2];
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const int rl = (t + v) * rpsd + dsub;
+          rlv[v] = rl;
+          if (v < nu && rl < nr) {
+            const int ei = off + rl * ngd + dg;
+            part[v] = fmaf(bf16_to_f32(dscl[2 * j * cv.d_sc_el + ei]), dot_seg_dec<BITS>(dcodes[(u + v) * 32 + lane], hv),
+                           bf16_to_f32(dscl[(2 * j + 1) * cv.d_sc_el + ei]) * hsm);
+          }
         }
 #pragma unroll 1
-        for (int o = nsgd >> 1; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        if (ds == 0 && rl < nr) dred[j * cv.nr_max + rl] = part;
+        for (int o = nsgd >> 1; o > 0; o >>= 1) {
+          part[0] += __shfl_xor_sync(0xffffffffu, part[0], o);
+          part[1] += __shfl_xor_sync(0xffffffffu, part[1], o);
+        }
+        if (ds == 0) {
+          if (rlv[0] < nr) dred[j * cv.nr_max + rlv[0]] = part[0];
+          if (nu == 2 && rlv[1] < nr) dred[j * cv.nr_max + rlv[1]] = part[1];
+        }
+        u += nu;
       }
     }
     if (__syncthreads_or(ab)) { leave(); return; }
