@@ -7,9 +7,10 @@
 // (or the plain softmax probabilities when renorm = 0).
 //
 // One warp computes one router row (one expert's logit) for a tile of up to
-// 8 tokens. The tile's
-// tokens are staged once in shared memory; router rows stream through with
-// 128-bit loads. The last CTA to finish a token tile (an arrival counter in
+// TT tokens (8 tokens and 4 warps a CTA for small batches; 16 tokens and 32
+// warps from 16 tokens up, so a token tile is read by fewer CTAs). The
+// tile's tokens are staged once in shared memory; router rows stream through
+// with 128-bit loads. The last CTA to finish a token tile (an arrival counter in
 // the workspace, reset by that CTA for the next call) then runs softmax and
 // top-k: one warp per token, each lane holding E/32 logits, k rounds of a
 // shuffle arg-max (larger logit wins, equal logits go to the lower index).
@@ -24,7 +25,6 @@ namespace moe {
 
 namespace {
 
-constexpr int kWarps = 4;
 constexpr int kMaxPerLane = 16;  // E <= 512
 
 __device__ void topk_one_token(const float* lg, int E, int k, int renorm, int32_t* idx_out,
@@ -86,30 +86,31 @@ __device__ void topk_one_token(const float* lg, int E, int k, int renorm, int32_
   }
 }
 
-__global__ void __launch_bounds__(kWarps * 32)
+template <int TT, int WPC>
+__global__ void __launch_bounds__(WPC * 32)
     route_topk_kernel(RouteParams p) {
   extern __shared__ uint4 sx[];  // [tile tokens][H/8] bf16x8
   const int tile = blockIdx.y;
-  const int t0 = tile * kRouteTokTile;
-  const int nt = min(kRouteTokTile, p.T - t0);
+  const int t0 = tile * TT;
+  const int nt = min(TT, p.T - t0);
   const int nseg = p.H / 8;
   const uint4* xg = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t0) * p.H);
   for (int i = threadIdx.x; i < nt * nseg; i += blockDim.x) sx[i] = xg[i];
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * kWarps + warp;
+  const int row = blockIdx.x * WPC + warp;
   if (row < p.E) {
     const uint16_t* wrow = p.wr + static_cast<size_t>(row) * p.H;
-    float acc[kRouteTokTile];
+    float acc[TT];
 #pragma unroll
-    for (int t = 0; t < kRouteTokTile; ++t) acc[t] = 0.f;
+    for (int t = 0; t < TT; ++t) acc[t] = 0.f;
     for (int s = lane; s < nseg; s += 32) {
       const uint4 wv = ldg_stream(wrow + static_cast<size_t>(s) * 8);
       const float w8[8] = {bf16_lo(wv.x), bf16_hi(wv.x), bf16_lo(wv.y), bf16_hi(wv.y),
                            bf16_lo(wv.z), bf16_hi(wv.z), bf16_lo(wv.w), bf16_hi(wv.w)};
 #pragma unroll
-      for (int t = 0; t < kRouteTokTile; ++t) {
+      for (int t = 0; t < TT; ++t) {
         if (t < nt) {
           const uint4 xv = sx[t * nseg + s];
           float a = acc[t];
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
     const float bias = p.rbias ? p.rbias[row] : 0.f;
 #pragma unroll
-    for (int t = 0; t < kRouteTokTile; ++t) {
+    for (int t = 0; t < TT; ++t) {
       const float a = warp_sum(acc[t]);
       if (lane == 0 && t < nt) p.ws.logits[static_cast<size_t>(t0 + t) * p.E + row] = a + bias;
     }
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  for (int t = warp; t < nt; t += kWarps) {
+  for (int t = warp; t < nt; t += WPC) {
     const size_t tok = static_cast<size_t>(t0 + t);
     const float* lg = p.ws.logits + tok * p.E;
     topk_one_token(lg, p.E, p.k, p.renorm, p.idx_out + tok * p.k, p.w_out + tok * p.k);
@@ -153,18 +154,25 @@ __global__ void __launch_bounds__(kWarps * 32)
   if (threadIdx.x == 0) p.ws.counters[tile] = 0u;  // ready for the next call
 }
 
-}  // namespace
-
-cudaError_t launch_route_topk(const RouteParams& p, cudaStream_t stream) {
-  dim3 grid((p.E + kWarps - 1) / kWarps, (p.T + kRouteTokTile - 1) / kRouteTokTile);
-  const size_t smem = static_cast<size_t>(kRouteTokTile) * p.H * 2;
+template <int TT, int WPC>
+cudaError_t launch_t(const RouteParams& p, cudaStream_t stream) {
+  dim3 grid((p.E + WPC - 1) / WPC, (p.T + TT - 1) / TT);
+  const size_t smem = static_cast<size_t>(TT) * p.H * 2;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(route_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(route_topk_kernel<TT, WPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  route_topk_kernel<<<grid, kWarps * 32, smem, stream>>>(p);
+  route_topk_kernel<TT, WPC><<<grid, WPC * 32, smem, stream>>>(p);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route_topk(const RouteParams& p, cudaStream_t stream) {
+  static_assert(kRouteTokTile == 8, "the arrival counters are sized for 8-token tiles (a superset for 16)");
+  if (p.T >= 16) return launch_t<16, 32>(p, stream);
+  return launch_t<8, 4>(p, stream);
 }
 
 }  // namespace moe
