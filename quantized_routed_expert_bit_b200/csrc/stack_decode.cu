@@ -389,23 +389,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
   // this warp's share of the down work: units (slot, row step), slot-major
   const int dn_upj = cdiv(nr, rpsd);
   const int dn_u0 = warp * nslots * dn_upj / kWarps, dn_u1 = (warp + 1) * nslots * dn_upj / kWarps;
+  const int dn_j0 = dn_upj > 0 ? dn_u0 / dn_upj : 0, dn_t0 = dn_u0 - dn_j0 * dn_upj;  // first unit = (slot, step)
   unsigned char* const dnbuf = sm + cv.dbuf;
   // this CTA's down rows into shared memory by per-thread asynchronous copies: the code
   // segment of every work unit u = (slot, row step) of this warp ([u][lane] x 16 bytes), and
   // (warp j % 16) slot j's scales and biases of the CTA's rows
   auto issue_down = [&](const LayerDesc& Ld) {
     uint16_t* dscl = reinterpret_cast<uint16_t*>(dnbuf + cv.dsc);
+    const uint8_t* src = nullptr;  // this lane's code segment of the current slot's first row step
+    int j = dn_j0, t = dn_t0;
 #pragma unroll 1
-    for (int u = dn_u0; u < dn_u1; ++u) {
-      const int j = u / dn_upj, t = u - j * dn_upj;
-      const int rl = t * rpsd + dsub;
-      if (rl < nr) {
+    for (int u = dn_u0; u < dn_u1; ++u, ++t) {
+      if (t == dn_upj) {
+        t = 0;
+        ++j;
+      }
+      if (u == dn_u0 || t == 0) {
         const bool routed = j < k;
         const QMat& m = routed ? Ld.dn : Ld.sdn;
-        const size_t e = routed ? static_cast<size_t>(s_idx[j]) : 0;
-        cp_async16(dnbuf + (static_cast<size_t>(u) * 32 + lane) * 16,
-                   m.q + e * m.q_stride + static_cast<size_t>(r0 + rl) * rowbd + 16 * ds);
+        src = m.q + (routed ? static_cast<size_t>(s_idx[j]) : 0) * m.q_stride + static_cast<size_t>(r0 + dsub) * rowbd +
+              16 * ds;
       }
+      if (t * rpsd + dsub < nr)
+        cp_async16(dnbuf + (static_cast<size_t>(u) * 32 + lane) * 16, src + static_cast<size_t>(t * rpsd) * rowbd);
     }
     const int el0 = (r0 * ngd) & ~7, nel = (((r1 * ngd) + 7) & ~7) - el0;
 #pragma unroll 1
@@ -491,22 +497,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
       if (!mbar_ready(&bar_r[l & 1], (l >> 1) & 1, p.hdr, 10)) ab = true;
       const int row = c + warp * G;
       const uint4* wv = reinterpret_cast<const uint4*>(rbuf + (static_cast<size_t>(l & 1) * cv.rr_max + warp) * H);
-      float acc = 0.f;
-#pragma unroll 1
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;  // four chains
+#pragma unroll 2
       for (int s = lane; s < H / 8; s += 32) {
         const uint4 w8 = wv[s];
         const float4 a = reinterpret_cast<const float4*>(xn)[2 * s];
         const float4 b = reinterpret_cast<const float4*>(xn)[2 * s + 1];
-        acc = fmaf(bf16_lo(w8.x), a.x, acc);
-        acc = fmaf(bf16_hi(w8.x), a.y, acc);
-        acc = fmaf(bf16_lo(w8.y), a.z, acc);
-        acc = fmaf(bf16_hi(w8.y), a.w, acc);
-        acc = fmaf(bf16_lo(w8.z), b.x, acc);
-        acc = fmaf(bf16_hi(w8.z), b.y, acc);
-        acc = fmaf(bf16_lo(w8.w), b.z, acc);
-        acc = fmaf(bf16_hi(w8.w), b.w, acc);
+        a0 = fmaf(bf16_lo(w8.x), a.x, a0);
+        a1 = fmaf(bf16_hi(w8.x), a.y, a1);
+        a2 = fmaf(bf16_lo(w8.y), a.z, a2);
+        a3 = fmaf(bf16_hi(w8.y), a.w, a3);
+        a0 = fmaf(bf16_lo(w8.z), b.x, a0);
+        a1 = fmaf(bf16_hi(w8.z), b.y, a1);
+        a2 = fmaf(bf16_lo(w8.w), b.z, a2);
+        a3 = fmaf(bf16_hi(w8.w), b.w, a3);
       }
-      acc = warp_sum(acc);
+      float acc = warp_sum((a0 + a1) + (a2 + a3));
       const LayerDesc& Ld = s_layers[l];
       if (lane < kDecodeReplicas)
         st_word(p.logits + lane * p.logits_rep + row, tag_f32(acc + ((row < E && Ld.rbias) ? Ld.rbias[row] : 0.f), par));
@@ -569,10 +575,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
     if (__syncthreads_or(ab)) { leave(); return; }
     stamp(3);
 
-    const LayerDesc& Ld = s_layers[l];
     // ---------------- 4a. this CTA's gate/up code rows: bulk copies by warp 0 (lane = batch,
-    // segment, gate|up); its gate/up scales and biases: one 16-byte load per thread into
-    // shared memory; its down rows: prefetched into L2 for phase 5
+    // segment, gate|up), issued after the barrier that publishes the selection (issued by the
+    // top-k warp before it, the early CTAs' copies measurably slowed the logit exchange of the
+    // others); its gate/up scales and biases: one 16-byte load per thread into shared memory;
+    // its down rows: prefetched into L2 for phase 5
+    const LayerDesc& Ld = s_layers[l];
     if (warp == 0) {
       // the buffer was last read and written by ordinary loads and per-thread copies
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -777,10 +785,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
       float hv[PS];
       float hsm = 0.f;
       // two units of the same slot at a time where possible (independent work in flight)
-      int u = dn_u0;
+      int u = dn_u0, j = dn_j0, t = dn_t0;
 #pragma unroll 1
       while (u < dn_u1) {
-        const int j = u / dn_upj, t = u - j * dn_upj;
+        if (t >= dn_upj) {
+          t -= dn_upj;
+          ++j;
+        }
         if (j != cur) {
           cur = j;
           hsm = 0.f;
@@ -818,6 +829,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
           if (nu == 2 && rlv[1] < nr) dred[j * cv.nr_max + rlv[1]] = part[1];
         }
         u += nu;
+        t += nu;
       }
     }
     if (__syncthreads_or(ab)) { leave(); return; }
