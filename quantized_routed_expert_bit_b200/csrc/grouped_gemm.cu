@@ -353,17 +353,19 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             break;
           }
           tc::fence_after_sync();
-          const uint32_t a0 = smem_addr(sm + L.a + as * kAStageBytes);
-          const uint32_t b0 = smem_addr(sm + L.b + bs * L.b_stage_bytes);
+          // descriptors built once per stage; inside the stage they step by their start-address
+          // field (16-byte units): +2 per K step of 16 (32 bytes), +1024 per A tile, +kNT*8 per B tile
+          const uint64_t ad0 = tc::smem_desc_sw128(smem_addr(sm + L.a + as * kAStageBytes));
+          const uint64_t bd0 = tc::smem_desc_sw128(smem_addr(sm + L.b + bs * L.b_stage_bytes));
 #pragma unroll
           for (int g = 0; g < kSG; ++g) {
             const uint32_t dt = tmem + (ps * kSG + g) * kNT;
-            const uint32_t ag = a0 + g * kATileBytes, bg = b0 + g * kNT * 128;
+            const uint64_t ag = ad0 + static_cast<uint64_t>(g * (kATileBytes >> 4));
+            const uint64_t bg = bd0 + static_cast<uint64_t>(g * (kNT * 128 >> 4));
 #pragma unroll
             for (int kk = 0; kk < kGK / 16; ++kk) {
-              const uint64_t ad = tc::smem_desc_sw128(ag + kk * 32);
-              tc::mma_f16(dt, ad, tc::smem_desc_sw128(bg + kk * 32), idesc, kk != 0);
-              if (MODE == 1) tc::mma_f16(dt, ad, tc::smem_desc_sw128(bg + kSG * kNT * 128 + kk * 32), idesc, 1);
+              tc::mma_f16(dt, ag + 2 * kk, bg + 2 * kk, idesc, kk != 0);
+              if (MODE == 1) tc::mma_f16(dt, ag + 2 * kk, bg + (kSG * kNT * 128 >> 4) + 2 * kk, idesc, 1);
             }
           }
           tc::commit(&aempty[as]);
