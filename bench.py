@@ -131,25 +131,42 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.rows)}
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str = "nccl"):
+    """One process per GPU (torchrun sets RANK/LOCAL_RANK/WORLD_SIZE/MASTER_*). The
+    ranks are independent replicas: the process group only carries the barrier
+    and the max-over-ranks of the timed region. `backend="gloo"` (CPU) serves tests."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if world > 1:
+        import datetime
         import torch.distributed as dist
         local = int(os.environ.get("LOCAL_RANK", "0"))
-        torch.cuda.set_device(local)
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
         return dist, dist.get_rank(), world, local
     return None, 0, 1, 0
 
 
-def barrier_max(dist, value: float) -> float:
+def barrier_max(dist, value: float, device: str = "cuda") -> float:
+    """The largest of the ranks' values (the job's time is its slowest rank's)."""
     if dist is None:
         return value
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_token_ids(rank: int, n: int):
+    """Token seeds of one rank: every rank decodes its own tokens (disjoint streams)."""
+    return [rank * 100000 + i for i in range(n)]
+
+
+def job_tokens_per_s(steps: int, world: int, T: int, ms: float) -> float:
+    """Whole-job throughput: the tokens all ranks processed over the slowest rank's time."""
+    return steps * world * T / (ms / 1e3)
 
 
 def host_layers_for(shape, layers_dev, tokens_bits):
@@ -271,11 +288,10 @@ def main():
     nsteps = args.warmup + args.steps
     # each rank its own tokens (independent replicas); a step is one batch of T tokens
     if T == 1:
-        tokens = synth.make_tokens(shape, [rank * 100000 + i for i in range(nsteps)], "cuda",
-                                   seed_id=synth.SHAPE_SEED_ID[key])
+        tokens = synth.make_tokens(shape, rank_token_ids(rank, nsteps), "cuda", seed_id=synth.SHAPE_SEED_ID[key])
     else:
-        tokens = torch.cat([synth.make_batch(shape, T, rank * 100000 + i, "cuda", seed_id=synth.SHAPE_SEED_ID[key])
-                            for i in range(nsteps)])
+        tokens = torch.cat([synth.make_batch(shape, T, i, "cuda", seed_id=synth.SHAPE_SEED_ID[key])
+                            for i in rank_token_ids(rank, nsteps)])
     xout = torch.empty(T, shape.hidden, dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
 
@@ -304,6 +320,16 @@ def main():
     ms = barrier_max(dist, ms)
     status = moe.moe_get_device_status(ws)
 
+    # ---- the same steps again, each bracketed by its own events: the spread of a step
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record(stream)
+    for i in range(args.warmup, nsteps):
+        step(i)
+        evs[i - args.warmup + 1].record(stream)
+    torch.cuda.synchronize()
+    per = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps))
+    pct = {f"p{q}": per[min(len(per) - 1, int(q / 100 * len(per)))] for q in (10, 50, 90)}
+
     # ---- end to end: host tokens in pinned memory, result read back every step
     host_tok = tokens.cpu().pin_memory()
     host_out = torch.empty(T, shape.hidden, dtype=torch.bfloat16).pin_memory()
@@ -328,7 +354,7 @@ def main():
     else:
         bytes_step = touched_bytes_batched(shape, layers, tokens[args.warmup * T:nsteps * T], T, args.steps)
     total_tokens = args.steps * world * T
-    tok_s = total_tokens / (ms / 1e3)
+    tok_s = job_tokens_per_s(args.steps, world, T, ms)
     per_step_s = ms / 1e3 / args.steps
     gbs = bytes_step / per_step_s / 1e9
     peak, peak_src = peaks()
@@ -359,6 +385,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": total_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * shape.hidden * 2, "d2h_bytes_per_step": T * shape.hidden * 2},
+            "step_ms": pct,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "device_status": moe.status_string(status),
