@@ -38,6 +38,11 @@ from quantized_routed_expert_bit_b200 import moe, synth  # noqa: E402
 METRIC = "MoE-layer decode tokens/s and achieved HBM GB/s (% of 8 TB/s) at 1 B200"
 SHAPE_KEY = "35b"
 NOMINAL_HBM_GBS = 8000.0
+# DRAM traffic of decode_stack_kernel per layer (dram__bytes_read.sum + dram__bytes_write.sum from
+# one ncu capture of the first 4 layers of the workload, 68.10 MB read + 4.36 MB written, divided
+# by 4). Each layer reads its own weights once, so the traffic of a launch over L layers is L times
+# this. Only valid for the kernel as captured: set to None when the kernel changes.
+DECODE_TRAFFIC_PER_LAYER = {"35b": (68_101_888 + 4_360_704) / 4}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -367,6 +372,9 @@ def main():
                "sample": f"{evals} (token, layer) evaluations of the bench tokens, {dt:.1f} s of oracle time, "
                          f"scaled to {shape.layers} layers per token; expert copies to the host untimed"}
 
+    traffic = None
+    if persistent and key in DECODE_TRAFFIC_PER_LAYER:
+        traffic = DECODE_TRAFFIC_PER_LAYER[key] * shape.layers
     if rank == 0:
         out = {
             "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -378,7 +386,7 @@ def main():
                          "kernel": ("decode_stack_kernel (the whole stack, one launch per step)" if persistent
                                     else "moe_stack_forward step (router, gate/up, down, glue kernels)"),
                          "achieved": gbs, "peak": peak, "peak_source": peak_src, "unit": "GB/s",
-                         "frac": gbs / peak, "traffic": None,
+                         "frac": gbs / peak, "traffic": traffic,
                          "bytes_per_step": bytes_step,
                          "note": "achieved = algorithmic bytes per step / device time per step (CUDA events "
                                  "on the launch stream around the timed steps)"},

@@ -208,6 +208,22 @@ MOE_API moe_status moe_layer_forward_static(const moe_config* cfg, const moe_lay
                                             int32_t* topk_idx, float* topk_w, int32_t* device_status,
                                             moe_stream_t stream);
 
+/* Self-check of the bounded waits. Every wait inside the kernels of this
+ * library (on an mbarrier, or on a word another CTA writes) gives up after
+ * 2 s or 2^26 polls, records MOE_ERR_TIMEOUT in the workspace status and
+ * returns, so that the context stays usable. This call runs both forms of
+ * wait on events that never happen: it clears the workspace's 64-byte
+ * header (status word included), then one CTA polls a header word that
+ * nothing writes while a second warp waits on an mbarrier that nobody
+ * arrives at. Asynchronous on `stream`; the kernel takes about 2 s. When it
+ * has run, gave_up (device int32, caller-owned) holds bit 0 = the word poll
+ * ended without its word, bit 1 = the mbarrier wait ended without its phase,
+ * and moe_get_device_status returns MOE_ERR_TIMEOUT. Returns
+ * MOE_ERR_WORKSPACE for a NULL, misaligned or smaller-than-64-byte ws,
+ * MOE_ERR_INVALID_ARG for a NULL or misaligned gave_up. Not part of the
+ * method; it exists to test the failure path without faulting the GPU. */
+MOE_API moe_status moe_check_wait_limit(void* ws, size_t ws_bytes, int32_t* gave_up, moe_stream_t stream);
+
 /* Waits for `stream`, then returns and clears the workspace's device status
  * (MOE_OK if no kernel reported an error since the last read). */
 MOE_API moe_status moe_get_device_status(void* ws, moe_stream_t stream);

@@ -623,6 +623,19 @@ moe_status moe_sort_by_expert(const moe_config* cfg, const int32_t* topk_idx, in
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "sort_by_expert launch");
 }
 
+moe_status moe_check_wait_limit(void* ws, size_t ws_bytes, int32_t* gave_up, moe_stream_t stream) {
+  if (!ws || !aligned(ws, kAlign)) return fail(MOE_ERR_WORKSPACE, "workspace NULL or misaligned");
+  if (ws_bytes < sizeof(moe::WsHeader)) return fail(MOE_ERR_WORKSPACE, "workspace too small");
+  moe_status s;
+  if ((s = check_ptr(gave_up, 4, "gave_up"))) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  moe::WsHeader* hdr = static_cast<moe::WsHeader*>(ws);
+  cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(moe::WsHeader), st);
+  if (e == cudaSuccess)
+    e = moe::launch_wait_limit_check(hdr, reinterpret_cast<uint32_t*>(&hdr->pad[0]), gave_up, st);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "wait limit check");
+}
+
 moe_status moe_get_device_status(void* ws, moe_stream_t stream) {
   if (!ws || !aligned(ws, kAlign)) return fail(MOE_ERR_WORKSPACE, "workspace NULL or misaligned");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

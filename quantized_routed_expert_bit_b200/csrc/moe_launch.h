@@ -144,5 +144,6 @@ cudaError_t launch_combine(const BatchParams& p, int grid, cudaStream_t st);
 bool decode_stack_supported(int H, int E, int k, int I, int Is, int group, int bits);
 size_t decode_stack_smem(int H, int E, int k, int I, int Is, int group, int bits, int grid);
 cudaError_t launch_decode_stack(const DecodeParams& p, int bits, int grid, cudaStream_t stream);
+cudaError_t launch_wait_limit_check(WsHeader* hdr, uint32_t* never_set, int32_t* gave_up, cudaStream_t stream);
 
 }  // namespace moe

@@ -900,6 +900,36 @@ cudaError_t launch_t(const DecodeParams& p, size_t smem, int grid, cudaStream_t 
                                      stream);
 }
 
+// Both forms of bounded wait this file uses, run on things that never
+// happen: warp 0 polls a word nothing writes (MOE_POLL_BACKOFF / give_up),
+// warp 1 waits on an mbarrier nobody arrives at (mbar_wait_slow). Each must
+// give up within the library's limits, record MOE_ERR_TIMEOUT and return;
+// bit 0 / bit 1 of *gave_up say which of the two ended without its event.
+__global__ void __launch_bounds__(64) wait_limit_kernel(WsHeader* hdr, uint32_t* never_set, int32_t* gave_up) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_mask;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    s_mask = 0;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    bool fail = false;
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+      if (ld_word(never_set) != 0u) break;
+      MOE_POLL_BACKOFF(it, t0, hdr, 91, fail);
+    }
+    if (fail) atomicOr(&s_mask, 1);
+  } else if (tid == 32) {
+    if (!mbar_wait_slow(&bar, 0, hdr, 92)) atomicOr(&s_mask, 2);
+  }
+  __syncthreads();
+  if (tid == 0) *gave_up = s_mask;
+}
+
 bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
 
 }  // namespace
@@ -937,6 +967,11 @@ cudaError_t launch_decode_stack(const DecodeParams& p, int bits, int grid, cudaS
   if (ch == 1) return launch_t<8, 1>(p, smem, grid, stream);
   if (ch == 2) return launch_t<8, 2>(p, smem, grid, stream);
   return launch_t<8, 4>(p, smem, grid, stream);
+}
+
+cudaError_t launch_wait_limit_check(WsHeader* hdr, uint32_t* never_set, int32_t* gave_up, cudaStream_t stream) {
+  wait_limit_kernel<<<1, 64, 0, stream>>>(hdr, never_set, gave_up);
+  return cudaGetLastError();
 }
 
 }  // namespace moe

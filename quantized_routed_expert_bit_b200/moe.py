@@ -72,13 +72,14 @@ def lib() -> ctypes.CDLL:
         L.moe_stack_kernel_launches.argtypes = [CP, I32, I32]
         L.moe_stack_kernel_launches.restype = I32
         L.moe_get_device_status.argtypes = [P, P]
+        L.moe_check_wait_limit.argtypes = [P, ctypes.c_size_t, P, P]
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_last_error_string.argtypes = []
         L.moe_last_error_string.restype = ctypes.c_char_p
         for f in ("moe_workspace_init", "moe_route_topk", "moe_expert_ffn", "moe_layer_forward",
                   "moe_stack_forward", "moe_sort_by_expert", "moe_get_device_status",
-                  "moe_layer_forward_static"):
+                  "moe_layer_forward_static", "moe_check_wait_limit"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -204,6 +205,11 @@ def moe_sort_by_expert(cfg: Config, topk_idx: torch.Tensor, perm: torch.Tensor, 
 
 def moe_get_device_status(ws: Workspace, stream=None) -> int:
     return int(lib().moe_get_device_status(ws.ptr, _stream(stream)))
+
+
+def moe_check_wait_limit(ws: Workspace, gave_up: torch.Tensor, stream=None):
+    """Runs the bounded-wait self-check (about 2 s on the GPU); gave_up is a device int32 [1]."""
+    _check(lib().moe_check_wait_limit(ws.ptr, ws.nbytes, gave_up.data_ptr(), _stream(stream)))
 
 
 # ---------------------------------------------------------------- launch plan (for reporting)

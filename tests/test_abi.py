@@ -151,3 +151,6 @@ def test_stack_and_sort_validation_errors():
         moe.MOE_ERR_INVALID_ARG
     assert lib.moe_get_device_status(None, None) == moe.MOE_ERR_WORKSPACE
     assert lib.moe_workspace_init(None, 1024, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_check_wait_limit(None, 1024, FAKE, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_check_wait_limit(FAKE, 32, FAKE, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_check_wait_limit(FAKE, 1024, None, None) == moe.MOE_ERR_INVALID_ARG

@@ -7,6 +7,8 @@ empty batches, the largest supported shape, zeroed experts, and the
 device-side bounds check on caller-supplied expert indices.
 """
 
+import re
+
 import numpy as np
 import pytest
 import torch
@@ -105,6 +107,34 @@ def test_bad_expert_index_is_skipped_and_reported(tiny):
     # token 0 is untouched by token 1's bad index
     st = check_tokens(host, bits(x), idx.cpu().numpy(), w.cpu().numpy(), bits(y), [0], "bounds")
     assert st.checked == 1
+
+
+def test_bounded_waits_give_up_and_leave_the_context_usable(tiny):
+    """A word nothing writes and an mbarrier nobody arrives at: both waits end
+    by their limit, the status reads MOE_ERR_TIMEOUT, and a layer run right
+    after on the same stream is still exact."""
+    lw, host, x = tiny
+    cfg = moe.make_config(TINY)
+    ws = moe.Workspace(cfg, 4)
+    gave_up = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    moe.moe_check_wait_limit(ws, gave_up)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    assert moe.moe_get_device_status(ws) == moe.MOE_ERR_TIMEOUT
+    assert re.search(r"detail 9[12]\b", moe.last_error())  # first to give up: 91 word poll, 92 mbarrier
+    assert int(gave_up.item()) == 3
+    assert 1500.0 < ms < 10000.0
+    assert moe.moe_get_device_status(ws) == moe.MOE_OK
+    idx, w, y = _alloc_out(TINY, 4)
+    moe.moe_layer_forward(cfg, moe.make_layer_weights(lw), x[:4], y, idx, w, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == moe.MOE_OK
+    st = check_tokens(host, bits(x), idx.cpu().numpy(), w.cpu().numpy(), bits(y), range(4), "after timeout")
+    assert st.checked == 4
 
 
 def test_zeroed_experts_give_exact_zero():
