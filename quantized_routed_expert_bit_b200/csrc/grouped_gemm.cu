@@ -62,7 +62,6 @@ constexpr int kNT = kChunkTokens;  // columns (pairs) per tile
 constexpr int kPS = 4;             // stages of per-group products in TMEM (kPS * kSG buffers)
 constexpr int kNA = 2;             // stages of unpacked A tiles in flight (a third one, paid for with
                                    // a shallower codes ring, measured slower)
-constexpr uint32_t kSmemLimit = 227u * 1024u;  // opt-in shared memory per block
 constexpr int kNB = 4;             // stages of B tiles in flight
 constexpr int kATileBytes = kBM * kGK * 2;          // one group's A tile (16 KiB)
 constexpr int kAStageBytes = kSG * kATileBytes;
@@ -98,12 +97,8 @@ __host__ __device__ inline GemmSmem gemm_smem(int mode, int bits, int K) {
   const int ng = K / kGK;
   s.b_stage_bytes = kSG * (mode == 0 ? 1 : 2) * kNT * 128;  // per group kNT rows x 128 B (x2: h hi and lo)
   s.codes_stage_bytes = kBM * kSG * (kGK * bits / 8);
+  s.nc = (64 * 1024) / s.codes_stage_bytes;                 // 64 KiB of codes in flight
   s.sc_buf_bytes = 2 * kBM * ng * 2;                        // scales and biases of 128 rows
-  // codes in flight: up to 64 KiB, as much as fits beside everything else
-  const uint32_t rest = al1k(kNA * kAStageBytes) + al1k(kNB * s.b_stage_bytes) + al1k(2 * s.sc_buf_bytes) +
-                        al1k(4 * ng * kNT * 4) + 1024 + 1024;
-  const uint32_t room = rest < kSmemLimit ? kSmemLimit - rest : 0;
-  s.nc = (room < 64u * 1024u ? room : 64u * 1024u) / s.codes_stage_bytes;
   uint32_t o = 0;
   s.a = o;     o = al1k(o + kNA * kAStageBytes);
   s.b = o;     o = al1k(o + kNB * s.b_stage_bytes);

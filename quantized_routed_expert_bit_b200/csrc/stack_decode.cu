@@ -396,22 +396,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
   // (warp j % 16) slot j's scales and biases of the CTA's rows
   auto issue_down = [&](const LayerDesc& Ld) {
     uint16_t* dscl = reinterpret_cast<uint16_t*>(dnbuf + cv.dsc);
-    const uint8_t* src = nullptr;  // this lane's code segment of the current slot's first row step
-    int j = dn_j0, t = dn_t0;
 #pragma unroll 1
-    for (int u = dn_u0; u < dn_u1; ++u, ++t) {
-      if (t == dn_upj) {
-        t = 0;
-        ++j;
-      }
-      if (u == dn_u0 || t == 0) {
+    for (int u = dn_u0; u < dn_u1; ++u) {
+      const int j = u / dn_upj, t = u - j * dn_upj;
+      const int rl = t * rpsd + dsub;
+      if (rl < nr) {
         const bool routed = j < k;
         const QMat& m = routed ? Ld.dn : Ld.sdn;
-        src = m.q + (routed ? static_cast<size_t>(s_idx[j]) : 0) * m.q_stride + static_cast<size_t>(r0 + dsub) * rowbd +
-              16 * ds;
+        const size_t e = routed ? static_cast<size_t>(s_idx[j]) : 0;
+        cp_async16(dnbuf + (static_cast<size_t>(u) * 32 + lane) * 16,
+                   m.q + e * m.q_stride + static_cast<size_t>(r0 + rl) * rowbd + 16 * ds);
       }
-      if (t * rpsd + dsub < nr)
-        cp_async16(dnbuf + (static_cast<size_t>(u) * 32 + lane) * 16, src + static_cast<size_t>(t * rpsd) * rowbd);
     }
     const int el0 = (r0 * ngd) & ~7, nel = (((r1 * ngd) + 7) & ~7) - el0;
 #pragma unroll 1
@@ -497,22 +492,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
       if (!mbar_ready(&bar_r[l & 1], (l >> 1) & 1, p.hdr, 10)) ab = true;
       const int row = c + warp * G;
       const uint4* wv = reinterpret_cast<const uint4*>(rbuf + (static_cast<size_t>(l & 1) * cv.rr_max + warp) * H);
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;  // four chains
-#pragma unroll 2
+      float acc = 0.f;
+#pragma unroll 1
       for (int s = lane; s < H / 8; s += 32) {
         const uint4 w8 = wv[s];
         const float4 a = reinterpret_cast<const float4*>(xn)[2 * s];
         const float4 b = reinterpret_cast<const float4*>(xn)[2 * s + 1];
-        a0 = fmaf(bf16_lo(w8.x), a.x, a0);
-        a1 = fmaf(bf16_hi(w8.x), a.y, a1);
-        a2 = fmaf(bf16_lo(w8.y), a.z, a2);
-        a3 = fmaf(bf16_hi(w8.y), a.w, a3);
-        a0 = fmaf(bf16_lo(w8.z), b.x, a0);
-        a1 = fmaf(bf16_hi(w8.z), b.y, a1);
-        a2 = fmaf(bf16_lo(w8.w), b.z, a2);
-        a3 = fmaf(bf16_hi(w8.w), b.w, a3);
+        acc = fmaf(bf16_lo(w8.x), a.x, acc);
+        acc = fmaf(bf16_hi(w8.x), a.y, acc);
+        acc = fmaf(bf16_lo(w8.y), a.z, acc);
+        acc = fmaf(bf16_hi(w8.y), a.w, acc);
+        acc = fmaf(bf16_lo(w8.z), b.x, acc);
+        acc = fmaf(bf16_hi(w8.z), b.y, acc);
+        acc = fmaf(bf16_lo(w8.w), b.z, acc);
+        acc = fmaf(bf16_hi(w8.w), b.w, acc);
       }
-      float acc = warp_sum((a0 + a1) + (a2 + a3));
+      acc = warp_sum(acc);
       const LayerDesc& Ld = s_layers[l];
       if (lane < kDecodeReplicas)
         st_word(p.logits + lane * p.logits_rep + row, tag_f32(acc + ((row < E && Ld.rbias) ? Ld.rbias[row] : 0.f), par));
@@ -785,13 +780,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
       float hv[PS];
       float hsm = 0.f;
       // two units of the same slot at a time where possible (independent work in flight)
-      int u = dn_u0, j = dn_j0, t = dn_t0;
+      int u = dn_u0;
 #pragma unroll 1
       while (u < dn_u1) {
-        if (t >= dn_upj) {
-          t -= dn_upj;
-          ++j;
-        }
+        const int j = u / dn_upj, t = u - j * dn_upj;
         if (j != cur) {
           cur = j;
           hsm = 0.f;
@@ -829,7 +821,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
           if (nu == 2 && rlv[1] < nr) dred[j * cv.nr_max + rlv[1]] = part[1];
         }
         u += nu;
-        t += nu;
       }
     }
     if (__syncthreads_or(ab)) { leave(); return; }
