@@ -38,11 +38,11 @@ from quantized_routed_expert_bit_b200 import moe, synth  # noqa: E402
 METRIC = "MoE-layer decode tokens/s and achieved HBM GB/s (% of 8 TB/s) at 1 B200"
 SHAPE_KEY = "35b"
 NOMINAL_HBM_GBS = 8000.0
-# DRAM traffic of decode_stack_kernel per layer (dram__bytes_read.sum + dram__bytes_write.sum from
-# one ncu capture of the first 4 layers of the workload, 68.04 MB read + 2.96 MB written, divided
-# by 4). Each layer reads its own weights once, so the traffic of a launch over L layers is L times
-# this. Only valid for the kernel as captured: set to None when the kernel changes.
-DECODE_TRAFFIC_PER_LAYER = {"35b": (68_036_864 + 2_961_152) / 4}
+# DRAM traffic of the persistent decode kernel per layer (dram__bytes_read.sum +
+# dram__bytes_write.sum from one ncu capture of the first 4 layers of the workload, divided by 4).
+# Each layer reads its own weights once, so the traffic of a launch over L layers is L times this.
+# Only valid for the kernel as captured: emptied when the kernel changes.
+DECODE_TRAFFIC_PER_LAYER = {}
 FALLBACK_HBM_GBS = 6650.0
 
 

@@ -193,7 +193,7 @@ MOE_API moe_status moe_sort_by_expert(const moe_config* cfg, const int32_t* topk
  * exists for those callers only.
  * Its scratch is a fixed 2 MiB array inside the library that every GPU that
  * loads the library holds until the process exits; calls whose
- * moe_workspace_size(cfg, T, 1) exceeds 2 MiB (T above about 50 tokens at
+ * moe_workspace_size(cfg, T, 1) exceeds 2 MiB (T above 11 tokens at
  * H=2048, E=256, k=8, I=512) return MOE_ERR_WORKSPACE. The call allocates
  * nothing. The first call on a device looks up the array's device address
  * (with that device current) and keeps it; make that first call before any

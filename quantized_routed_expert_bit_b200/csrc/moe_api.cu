@@ -42,7 +42,7 @@ size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 // Byte offsets of the workspace regions for T tokens.
 struct Layout {
   size_t hdr, counters, logits, sgate, h, r, xa, xb, y, idx, w;
-  size_t dlogits, dh, dy, dr, dx;                         // persistent single-token decode
+  size_t dlogits, dh, dy, dyacc, dcnt, dr, dx;            // persistent single-token decode
   size_t base_total;                                      // end of the regions above
   size_t perm, offs, chunks, nchunks, x16, hhi, hlo, o;   // batched tensor-core path
   size_t xsx, xsh;                                        // group sums of x and of h
@@ -69,11 +69,14 @@ Layout layout(const moe_config& c, int64_t T) {
   L.y = o;        o += up(static_cast<size_t>(T) * c.hidden * 2);
   L.idx = o;      o += up(static_cast<size_t>(T) * c.top_k * 4);
   L.w = o;        o += up(static_cast<size_t>(T) * c.top_k * 4);
-  // decode exchange words: logits, h, y, each in kDecodeReplicas copies (contiguous, zeroed
-  // before each launch)
+  // decode exchange words: logits, h, y, each in kDecodeReplicas copies, then the split
+  // kernel's accumulators and counter (contiguous, zeroed before each launch)
   L.dlogits = o;  o += moe::kDecodeReplicas * up(static_cast<size_t>(c.num_experts + 1) * 4);
   L.dh = o;       o += moe::kDecodeReplicas * up(static_cast<size_t>(c.top_k + 1) * imax * 4);
   L.dy = o;       o += moe::kDecodeReplicas * up(static_cast<size_t>(c.hidden) * 4);
+  // the split decode kernel's y accumulators (kDecodeYBufs x kDecodeReplicas) and arrival counter
+  L.dyacc = o;    o += static_cast<size_t>(moe::kDecodeYBufs) * moe::kDecodeReplicas * up(static_cast<size_t>(c.hidden) * 4);
+  L.dcnt = o;     o += up(4);
   L.dr = o;       o += up(static_cast<size_t>(c.hidden) * 4);
   L.dx = o;       o += up(static_cast<size_t>(c.hidden) * 2);
   L.base_total = o;
@@ -228,12 +231,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 3D map over E matrices [rows][inner] (inner contiguous, `esize` bytes per element),
-// box = (box_inner, 64 rows, 1 expert).
+// box = (box_inner, box_rows, 1 expert).
 bool map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int64_t inner, int64_t rows,
-            int64_t E, int64_t expert_stride_bytes, int box_inner) {
+            int64_t E, int64_t expert_stride_bytes, int box_inner, int box_rows = 64) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(E)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner * esize), static_cast<cuuint64_t>(expert_stride_bytes)};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 64u, 1u};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1u};
   cuuint32_t es[3] = {1u, 1u, 1u};
   return encode_fn()(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -398,17 +401,26 @@ bool dev_info(DevInfo* out) {
   return true;
 }
 
-// Whether one token through a stack runs as the persistent kernel (one
-// launch per up to kMaxDecodeLayers layers) rather than four kernels per layer.
-bool decode_eligible(const moe_config& c, int* grid) {
+// Whether one token through a stack runs as a persistent kernel (one launch
+// per up to kMaxDecodeLayers layers) rather than four kernels per layer, and
+// which: the split kernel where it fits, else the exchange kernel.
+bool decode_eligible(const moe_config& c, int L, int* grid, bool* split = nullptr, size_t* split_smem = nullptr) {
   DevInfo d;
-  if (!dev_info(&d) || !d.coop || d.sms < 1 || d.sms > kMaxGrid) return false;
-  if (!moe::decode_stack_supported(c.hidden, c.num_experts, c.top_k, c.inter, c.shared_inter, c.group, c.bits))
-    return false;
-  const size_t smem =
-      moe::decode_stack_smem(c.hidden, c.num_experts, c.top_k, c.inter, c.shared_inter, c.group, c.bits, d.sms);
-  if (d.smem_optin < 1024 || smem > static_cast<size_t>(d.smem_optin) - 1024) return false;
+  if (!dev_info(&d) || !d.coop || d.sms < 1 || d.sms > kMaxGrid || d.smem_optin < 1024) return false;
+  const size_t limit = static_cast<size_t>(d.smem_optin) - 1024;
+  size_t ss = 0;
+  const bool sp = encode_fn() && moe::decode_split_plan(c.hidden, c.num_experts, c.top_k, c.inter, c.shared_inter,
+                                                        c.group, c.bits, d.sms, L, limit, &ss);
+  if (!sp) {
+    if (!moe::decode_stack_supported(c.hidden, c.num_experts, c.top_k, c.inter, c.shared_inter, c.group, c.bits))
+      return false;
+    const size_t smem =
+        moe::decode_stack_smem(c.hidden, c.num_experts, c.top_k, c.inter, c.shared_inter, c.group, c.bits, d.sms);
+    if (smem > limit) return false;
+  }
   *grid = d.sms;
+  if (split) *split = sp;
+  if (split_smem) *split_smem = ss;
   return true;
 }
 
@@ -425,7 +437,7 @@ moe::LayerDesc layer_desc(const moe_layer_weights& w) {
 }
 
 moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, int L, const uint16_t* x0,
-                        uint16_t* x_out, const moe_trace* trace, void* ws, const Layout& Ly, int grid,
+                        uint16_t* x_out, const moe_trace* trace, void* ws, const Layout& Ly, int grid, bool split,
                         cudaStream_t st) {
   char* b = static_cast<char*>(ws);
   auto P = std::make_unique<moe::DecodeParams>();
@@ -448,6 +460,10 @@ moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, in
   P->logits_rep = static_cast<int>((Ly.dh - Ly.dlogits) / moe::kDecodeReplicas / 4);
   P->h_rep = static_cast<int>((Ly.dy - Ly.dh) / moe::kDecodeReplicas / 4);
   P->y_rep = static_cast<int>((Ly.dr - Ly.dy) / moe::kDecodeReplicas / 4);
+  P->yacc = reinterpret_cast<float*>(b + Ly.dyacc);
+  P->yrep = static_cast<int>(up(static_cast<size_t>(c.hidden) * 4) / 4);
+  P->ybuf_stride = static_cast<int64_t>(moe::kDecodeReplicas) * P->yrep;
+  P->arrive = reinterpret_cast<uint32_t*>(b + Ly.dcnt);
   P->hdr = reinterpret_cast<moe::WsHeader*>(b + Ly.hdr);
   uint16_t* xmid = reinterpret_cast<uint16_t*>(b + Ly.dx);
   float* rmid = reinterpret_cast<float*>(b + Ly.dr);
@@ -461,9 +477,24 @@ moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, in
     P->out = last ? x_out : xmid;
     P->r_out = last ? nullptr : rmid;
     for (int i = 0; i < n; ++i) P->layers[i] = layer_desc(layers[l0 + i]);
+    if (split) {
+      // down codes as (row bytes, H rows, experts), one unit's 32 columns x 256 rows per copy
+      const int64_t rb = static_cast<int64_t>(c.inter) * c.bits / 8;
+      const int ub = 32 * c.bits / 8;
+      for (int i = 0; i < n; ++i) {
+        const moe_layer_weights& w = layers[l0 + i];
+        if (!map_3d(&P->tm_dn[i], w.down.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rb, c.hidden, c.num_experts,
+                    w.down.q_expert_stride, ub, 256))
+          return fail(MOE_ERR_CUDA, "tensor map of layer %d's down codes", l0 + i);
+        if (c.shared_inter > 0 &&
+            !map_3d(&P->tm_sdn[i], w.shared_down.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rb, c.hidden, 1,
+                    rb * c.hidden, ub, 256))
+          return fail(MOE_ERR_CUDA, "tensor map of layer %d's shared down codes", l0 + i);
+      }
+    }
     cudaError_t e = cudaMemsetAsync(b + Ly.dlogits, 0, Ly.dr - Ly.dlogits, st);
     if (e != cudaSuccess) return cuda_fail(e, "exchange word reset");
-    e = moe::launch_decode_stack(*P, c.bits, grid, st);
+    e = split ? moe::launch_decode_split(*P, c.bits, grid, st) : moe::launch_decode_stack(*P, c.bits, grid, st);
     if (e != cudaSuccess) return cuda_fail(e, "decode_stack launch");
   }
   return MOE_OK;
@@ -477,7 +508,7 @@ int32_t moe_stack_kernel_launches(const moe_config* cfg, int32_t T, int32_t L) {
   if (check_cfg(cfg) != MOE_OK || T < 0 || L < 0) return -1;
   if (T == 0 || L == 0) return 0;
   int grid = 0;
-  if (T == 1 && decode_eligible(*cfg, &grid))
+  if (T == 1 && decode_eligible(*cfg, L, &grid))
     return (L + moe::kMaxDecodeLayers - 1) / moe::kMaxDecodeLayers;
   if (batched_eligible(*cfg, T)) return 1 + 7 * L;  // route, sort, gather, 2 GEMMs, combine, glue
   return 1 + 4 * L;
@@ -574,7 +605,9 @@ moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weights* lay
   const moe::WsView v = view(ws, Ly);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int grid = 0;
-  if (T == 1 && decode_eligible(*cfg, &grid)) return stack_decode(*cfg, layers, L, x0, x_out, trace, ws, Ly, grid, st);
+  bool split = false;
+  if (T == 1 && decode_eligible(*cfg, L, &grid, &split))
+    return stack_decode(*cfg, layers, L, x0, x_out, trace, ws, Ly, grid, split, st);
   const bool batched = batched_eligible(*cfg, T);
   const size_t TH = static_cast<size_t>(T) * cfg->hidden;
   const size_t Tk = static_cast<size_t>(T) * cfg->top_k;

@@ -105,9 +105,12 @@ struct LayerDesc {
   QMat gu, dn, sgu, sdn;
 };
 
-constexpr int kMaxDecodeLayers = 128;  // layers per launch (kernel parameter space)
+constexpr int kMaxDecodeLayers = 48;   // layers per launch (kernel parameter space)
 constexpr int kDecodeReplicas = 4;     // copies of each exchange word (spreads the readers over more lines)
+constexpr int kDecodeYBufs = 3;        // y accumulator buffers of the split kernel, used by layers in turn
 
+// Parameters of both persistent decode kernels: decode_stack_kernel (exchanges
+// h between CTAs) and decode_split_kernel (keeps h in the CTA and reduces y).
 struct DecodeParams {
   int L, l0;             // layers in this launch; index of its first layer in the stack
   int H, E, k, I, Is, group, renorm;
@@ -124,11 +127,21 @@ struct DecodeParams {
   // exchange words between CTAs (workspace), zero at launch; each written to
   // kDecodeReplicas copies (`*_rep` words apart), CTA c reads copy c % kDecodeReplicas
   uint32_t* logits;      // [E+1] fp32 logits, last mantissa bit = layer parity
-  uint32_t* hbuf;        // [k+1][I] fp32 SwiGLU outputs, last mantissa bit = layer parity
-  uint32_t* ybuf;        // [H] bf16 layer output << 16 | 16-bit layer tag
+  uint32_t* hbuf;        // [k+1][I] fp32 SwiGLU outputs, last mantissa bit = layer parity (exchange kernel)
+  uint32_t* ybuf;        // [H] bf16 layer output << 16 | 16-bit layer tag (exchange kernel)
   int logits_rep, h_rep, y_rep;
+  // split kernel: y partial sums [kDecodeYBufs][kDecodeReplicas][yrep] fp32 (16-byte aligned;
+  // CTA c adds into copy c % kDecodeReplicas, readers sum the copies) and the arrival counter
+  float* yacc;
+  int yrep;
+  int64_t ybuf_stride;   // floats between buffers (kDecodeReplicas * yrep)
+  uint32_t* arrive;
   WsHeader* hdr;
   LayerDesc layers[kMaxDecodeLayers];
+  // split kernel: 3D maps (row bytes, H rows, experts) over the down codes of the routed and
+  // the shared experts, box (one unit's bytes, 256 rows, 1)
+  CUtensorMap tm_dn[kMaxDecodeLayers];
+  CUtensorMap tm_sdn[kMaxDecodeLayers];
 };
 
 cudaError_t launch_route_topk(const RouteParams& p, cudaStream_t stream);
@@ -143,6 +156,11 @@ cudaError_t launch_combine(const BatchParams& p, int grid, cudaStream_t st);
 
 bool decode_stack_supported(int H, int E, int k, int I, int Is, int group, int bits);
 size_t decode_stack_smem(int H, int E, int k, int I, int Is, int group, int bits, int grid);
+// The split kernel: whether it runs this shape on `grid` CTAs within `smem_limit` bytes of
+// shared memory for launches of up to L layers, and its shared memory.
+bool decode_split_plan(int H, int E, int k, int I, int Is, int group, int bits, int grid, int L, size_t smem_limit,
+                       size_t* smem);
+cudaError_t launch_decode_split(const DecodeParams& p, int bits, int grid, cudaStream_t stream);
 cudaError_t launch_decode_stack(const DecodeParams& p, int bits, int grid, cudaStream_t stream);
 cudaError_t launch_wait_limit_check(WsHeader* hdr, uint32_t* never_set, int32_t* gave_up, cudaStream_t stream);
 

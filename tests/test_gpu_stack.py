@@ -102,19 +102,46 @@ def test_batched_stack_parity(key):
 
 
 def test_decode_stack_longer_than_one_launch():
-    """130 layers: the persistent path splits the stack over two launches and
-    carries the residual stream between them."""
-    shape = synth.MoEShape("chunk-h256-e16", 256, 16, 2, 128, 128, 4, 32, 130, False, 1)
+    """100 layers: the persistent path splits the stack over three launches of
+    at most 48 layers and carries the residual stream between them."""
+    shape = synth.MoEShape("chunk-h256-e16", 256, 16, 2, 128, 128, 4, 32, 100, False, 1)
     cfg = moe.make_config(shape)
-    assert moe.moe_stack_kernel_launches(cfg, 1, shape.layers) == 2
+    assert moe.moe_stack_kernel_launches(cfg, 1, shape.layers) == 3
     layers = [synth.make_layer(shape, l, "cuda", seed_id=400) for l in range(shape.layers)]
     x0 = synth.make_tokens(shape, [3], "cuda", seed_id=400)
     tx, ti, tw, ty, xo = run_stack(shape, layers, x0)
     total = ParityStats()
-    for l in (0, 1, 63, 126, 127, 128, 129):
+    for l in (0, 1, 46, 47, 48, 49, 95, 96, 99):
         total.merge(check_tokens(DeviceLayer(shape, layers[l]), tx[l], ti[l], tw[l], ty[l], [0], f"layer {l}"))
     check_glue(bits(x0), tx, ty, xo)
-    assert total.checked == 7
+    assert total.checked == 9
+
+
+SMALL_STACKS = {
+    # name: (H, E, k, I, Is, bits, group, layers, router bias)
+    "8bit": (256, 16, 2, 128, 128, 8, 32, 6, True),
+    "no-shared": (256, 16, 2, 128, 0, 4, 32, 6, False),
+    "top1-g64": (512, 32, 1, 256, 256, 4, 64, 6, False),
+    "top8-e64": (1024, 64, 8, 128, 128, 4, 32, 6, False),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL_STACKS))
+def test_small_decode_stacks(name):
+    """Format and routing variants of the persistent decode path, every layer
+    teacher-forced against the oracle."""
+    H, E, k, I, Is, b, g, L, rb = SMALL_STACKS[name]
+    shape = synth.MoEShape("stack-" + name, H, E, k, I, Is, b, g, L, rb, 1)
+    assert moe.moe_stack_kernel_launches(moe.make_config(shape), 1, L) == 1
+    layers = [synth.make_layer(shape, l, "cuda", seed_id=500) for l in range(L)]
+    total = ParityStats()
+    for tok in (0, 1, 2):
+        x0 = synth.make_tokens(shape, [tok], "cuda", seed_id=500)
+        tx, ti, tw, ty, xo = run_stack(shape, layers, x0)
+        for l in range(L):
+            total.merge(check_tokens(DeviceLayer(shape, layers[l]), tx[l], ti[l], tw[l], ty[l], [0], f"{name} {l}"))
+        check_glue(bits(x0), tx, ty, xo)
+    assert total.excluded <= 2
 
 
 def test_single_token_path_matches_multi_kernel_path():
