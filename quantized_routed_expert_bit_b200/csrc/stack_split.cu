@@ -18,7 +18,7 @@
 //      layer over the experts' down codes) and the expert's whole down scale
 //      and bias matrices by two bulk copies. Each thread takes four output
 //      rows and forms the unit's routing-weighted partial of y for them, then
-//      adds it to a replicated fp32 accumulator with one vector reduction.
+//      adds it to a replicated fp32 accumulator (reductions in L2).
 // The y of a layer is then the sum of the k*I/32 + Is/32 partials: no h
 // exchange between CTAs, and no CTA reads more than its own unit of any
 // expert. Routing fan-out and shared experts: Swiftlet article (xix.ai),
@@ -101,11 +101,9 @@ __host__ __device__ inline Carve carve(int H, int E, int I, int Is, int group, i
   return c;
 }
 
-// Four consecutive fp32 accumulators += v, in L2 (one vector reduction).
-__device__ __forceinline__ void red_add_v4(float* a, const float (&v)[4]) {
-  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(a), "f"(v[0]), "f"(v[1]),
-               "f"(v[2]), "f"(v[3])
-               : "memory");
+// An fp32 accumulator += v, in L2 (a reduction: no value comes back).
+__device__ __forceinline__ void red_add(float* a, float v) {
+  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(a), "f"(v) : "memory");
 }
 
 // 3D tiled tensor copy (x innermost) into this CTA's shared memory, completing on `bar`.
@@ -542,9 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
     if (tid == 0) s_pend.dn = -1;
     stamp(4);
 
-    // ---------------- 5. the unit's partial of y for rows 4t .. 4t+3:
+    // ---------------- 5. the unit's partial of y for rows t, t + 512, t + 1024, t + 1536 (a warp
+    // reads 32 consecutive rows of codes, and reduces into 32 consecutive words of y):
     // routing weight x (scale x codes . h + bias x sum h)
-    if (npc > 0 && tid < HT) {
+    if (npc > 0) {
       float hv[kUnit];
       float hsum = 0.f;
 #pragma unroll
@@ -559,22 +558,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
       const float wgt = u_routed ? s_w[jA] : s_sg;
       const uint16_t* dsc = reinterpret_cast<const uint16_t*>(dss);
       const uint16_t* dbi = dsc + static_cast<size_t>(H) * ngd;
-      float yp[4];
+      float* yrow = p.yacc + static_cast<size_t>(l % kDecodeYBufs) * p.ybuf_stride +
+                    static_cast<size_t>(c % kDecodeReplicas) * p.yrep;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int r = 4 * tid + q;
-        float d;
-        if constexpr (BITS == 4) {
-          d = dot_seg_dec<4>(*reinterpret_cast<const uint4*>(dcd + r * cv.UB), hv);
-        } else {
-          d = dot_seg<8>(*reinterpret_cast<const uint4*>(dcd + r * cv.UB), hv) +
-              dot_seg<8>(*reinterpret_cast<const uint4*>(dcd + r * cv.UB + 16), hv + 16);
+        const int r = tid + q * kThreads;
+        if (r < H) {
+          float d;
+          if constexpr (BITS == 4) {
+            d = dot_seg_dec<4>(*reinterpret_cast<const uint4*>(dcd + r * cv.UB), hv);
+          } else {
+            d = dot_seg<8>(*reinterpret_cast<const uint4*>(dcd + r * cv.UB), hv) +
+                dot_seg<8>(*reinterpret_cast<const uint4*>(dcd + r * cv.UB + 16), hv + 16);
+          }
+          red_add(yrow + r, wgt * fmaf(bf16_to_f32(dsc[r * ngd + u_g]), d, bf16_to_f32(dbi[r * ngd + u_g]) * hsum));
         }
-        yp[q] = wgt * fmaf(bf16_to_f32(dsc[r * ngd + u_g]), d, bf16_to_f32(dbi[r * ngd + u_g]) * hsum);
       }
-      red_add_v4(p.yacc + static_cast<size_t>(l % kDecodeYBufs) * p.ybuf_stride +
-                     static_cast<size_t>(c % kDecodeReplicas) * p.yrep + 4 * tid,
-                 yp);
     }
     if (__syncthreads_or(ab)) { leave(); return; }
     if (tid == 0) {
