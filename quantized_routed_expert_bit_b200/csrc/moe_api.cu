@@ -404,13 +404,14 @@ bool dev_info(DevInfo* out) {
 // Whether one token through a stack runs as a persistent kernel (one launch
 // per up to kMaxDecodeLayers layers) rather than four kernels per layer, and
 // which: the split kernel where it fits, else the exchange kernel.
-bool decode_eligible(const moe_config& c, int L, int* grid, bool* split = nullptr, size_t* split_smem = nullptr) {
+bool decode_eligible(const moe_config& c, int L, int* grid, bool* split = nullptr, int* split_late = nullptr) {
   DevInfo d;
   if (!dev_info(&d) || !d.coop || d.sms < 1 || d.sms > kMaxGrid || d.smem_optin < 1024) return false;
   const size_t limit = static_cast<size_t>(d.smem_optin) - 1024;
   size_t ss = 0;
+  int late = 0;
   const bool sp = encode_fn() && moe::decode_split_plan(c.hidden, c.num_experts, c.top_k, c.inter, c.shared_inter,
-                                                        c.group, c.bits, d.sms, L, limit, &ss);
+                                                        c.group, c.bits, d.sms, L, limit, &ss, &late);
   if (!sp) {
     if (!moe::decode_stack_supported(c.hidden, c.num_experts, c.top_k, c.inter, c.shared_inter, c.group, c.bits))
       return false;
@@ -420,7 +421,7 @@ bool decode_eligible(const moe_config& c, int L, int* grid, bool* split = nullpt
   }
   *grid = d.sms;
   if (split) *split = sp;
-  if (split_smem) *split_smem = ss;
+  if (split_late) *split_late = late;
   return true;
 }
 
@@ -438,7 +439,7 @@ moe::LayerDesc layer_desc(const moe_layer_weights& w) {
 
 moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, int L, const uint16_t* x0,
                         uint16_t* x_out, const moe_trace* trace, void* ws, const Layout& Ly, int grid, bool split,
-                        cudaStream_t st) {
+                        int split_late, cudaStream_t st) {
   char* b = static_cast<char*>(ws);
   auto P = std::make_unique<moe::DecodeParams>();
   P->H = c.hidden;
@@ -464,6 +465,7 @@ moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, in
   P->yrep = static_cast<int>(up(static_cast<size_t>(c.hidden) * 4) / 4);
   P->ybuf_stride = static_cast<int64_t>(moe::kDecodeReplicas) * P->yrep;
   P->arrive = reinterpret_cast<uint32_t*>(b + Ly.dcnt);
+  P->split_late = split_late;
   P->hdr = reinterpret_cast<moe::WsHeader*>(b + Ly.hdr);
   uint16_t* xmid = reinterpret_cast<uint16_t*>(b + Ly.dx);
   float* rmid = reinterpret_cast<float*>(b + Ly.dr);
@@ -606,8 +608,9 @@ moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weights* lay
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int grid = 0;
   bool split = false;
-  if (T == 1 && decode_eligible(*cfg, L, &grid, &split))
-    return stack_decode(*cfg, layers, L, x0, x_out, trace, ws, Ly, grid, split, st);
+  int split_late = 0;
+  if (T == 1 && decode_eligible(*cfg, L, &grid, &split, &split_late))
+    return stack_decode(*cfg, layers, L, x0, x_out, trace, ws, Ly, grid, split, split_late, st);
   const bool batched = batched_eligible(*cfg, T);
   const size_t TH = static_cast<size_t>(T) * cfg->hidden;
   const size_t Tk = static_cast<size_t>(T) * cfg->top_k;

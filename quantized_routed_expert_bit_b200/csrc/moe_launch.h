@@ -134,6 +134,7 @@ struct DecodeParams {
   // CTA c adds into copy c % kDecodeReplicas, readers sum the copies) and the arrival counter
   float* yacc;
   int yrep;
+  int split_late;        // split kernel: down data copied into the gate/up buffer once gate/up is done
   int64_t ybuf_stride;   // floats between buffers (kDecodeReplicas * yrep)
   uint32_t* arrive;
   WsHeader* hdr;
@@ -159,7 +160,7 @@ size_t decode_stack_smem(int H, int E, int k, int I, int Is, int group, int bits
 // The split kernel: whether it runs this shape on `grid` CTAs within `smem_limit` bytes of
 // shared memory for launches of up to L layers, and its shared memory.
 bool decode_split_plan(int H, int E, int k, int I, int Is, int group, int bits, int grid, int L, size_t smem_limit,
-                       size_t* smem);
+                       size_t* smem, int* late);
 cudaError_t launch_decode_split(const DecodeParams& p, int bits, int grid, cudaStream_t stream);
 cudaError_t launch_decode_stack(const DecodeParams& p, int bits, int grid, cudaStream_t stream);
 cudaError_t launch_wait_limit_check(WsHeader* hdr, uint32_t* never_set, int32_t* gave_up, cudaStream_t stream);

@@ -74,7 +74,7 @@ struct Carve {
   uint32_t xs, xn, rr, hl, guv, gsb, dbuf, dcd, dss, rbuf, desc, total;
 };
 
-__host__ __device__ inline Carve carve(int H, int E, int I, int Is, int group, int bits, int G, int L) {
+__host__ __device__ inline Carve carve(int H, int E, int I, int Is, int group, int bits, int G, int L, int late) {
   Carve c{};
   c.PS = 128 / bits;
   c.nsg = H / c.PS;
@@ -92,9 +92,18 @@ __host__ __device__ inline Carve carve(int H, int E, int I, int Is, int group, i
   c.hl = o;    o = al128(o + kUnit * 4);
   c.guv = o;   o = al128(o + 2 * kUnit * 4);
   c.gsb = o;   o = al128(o + 4 * kUnit * c.ng * 2);
-  c.dbuf = o;  o = al128(o + 2 * kUnit * c.rowb);                // gate/up code rows
-  c.dcd = o;   o = al128(o + H * c.UB);                          // the unit's down codes [row][UB]
-  c.dss = o;   o = al128(o + 2 * H * c.ngd * 2);                 // the expert's down scales, then biases
+  const uint32_t gu_bytes = 2 * kUnit * c.rowb;                 // gate/up code rows
+  const uint32_t dn_bytes = al128(H * c.UB) + 2 * H * c.ngd * 2;  // the unit's down codes [row][UB], then
+                                                                  // the expert's down scales and biases
+  if (late) {  // the down data reuses the gate/up buffer once gate/up is done
+    c.dbuf = o;  o = al128(o + (gu_bytes > dn_bytes ? gu_bytes : dn_bytes));
+    c.dcd = c.dbuf;
+    c.dss = c.dbuf + al128(H * c.UB);
+  } else {
+    c.dbuf = o;  o = al128(o + gu_bytes);
+    c.dcd = o;   o = al128(o + H * c.UB);
+    c.dss = o;   o = al128(o + 2 * H * c.ngd * 2);
+  }
   c.rbuf = o;  o = al128(o + 2 * c.rr_max * H * 2);
   c.desc = o;  o = al128(o + L * sizeof(LayerDesc));             // the launch's layer descriptors
   c.total = o;
@@ -151,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
   const int G = gridDim.x, c = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   bool ab = false;  // a wait of this thread gave up; combined over the CTA at each phase end
-  const Carve cv = carve(H, E, I, Is, group, BITS, G, p.L);
+  const Carve cv = carve(H, E, I, Is, group, BITS, G, p.L, p.split_late);
   float* xs = reinterpret_cast<float*>(sm + cv.xs);  // x by 16-byte code segment (conflict-free float4 reads)
   float* xn = reinterpret_cast<float*>(sm + cv.xn);  // x in natural order
   float* rr = reinterpret_cast<float*>(sm + cv.rr);  // residual stream, fp32
@@ -245,6 +254,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
       MOE_POLL_BACKOFF(it, t0, p.hdr, where, ab)
     }
     __threadfence();
+  };
+
+  // the unit's down data (thread 32): 256-row tiles of its 32 columns of the down codes, and
+  // the expert's whole down scale and bias matrices
+  auto issue_down = [&](const LayerDesc& Ld, int l) {
+    const QMat& m = u_routed ? Ld.dn : Ld.sdn;
+    const CUtensorMap* tm = u_routed ? &p.tm_dn[l] : &p.tm_sdn[l];
+    const int e = u_routed ? s_idx[jA] : 0;
+    const uint32_t sbytes = static_cast<uint32_t>(H) * ngd * 2;
+    // the buffer may last have been read by ordinary loads (gate/up or the previous layer's down)
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive_expect_tx(&bar_dn, static_cast<uint32_t>(H) * cv.UB + 2 * sbytes);
+#pragma unroll 1
+    for (int r0 = 0; r0 < H; r0 += kBoxRows) tma_3d(dcd + r0 * cv.UB, tm, iA * BITS / 8, r0, e, &bar_dn);
+    bulk_g2s(dss, m.s + static_cast<size_t>(e) * m.sb_stride, sbytes, &bar_dn);
+    bulk_g2s(dss + sbytes, m.b + static_cast<size_t>(e) * m.sb_stride, sbytes, &bar_dn);
+    s_pend.dn = l & 1;
   };
 
   for (int l = 0; l < p.L; ++l) {
@@ -439,18 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
             __ldg(reinterpret_cast<const uint4*>(src));
       }
     }
-    if (tid == 32 && npc > 0) {
-      const QMat& m = u_routed ? Ld.dn : Ld.sdn;
-      const CUtensorMap* tm = u_routed ? &p.tm_dn[l] : &p.tm_sdn[l];
-      const int e = u_routed ? s_idx[jA] : 0;
-      const uint32_t sbytes = static_cast<uint32_t>(H) * ngd * 2;
-      mbar_arrive_expect_tx(&bar_dn, static_cast<uint32_t>(H) * cv.UB + 2 * sbytes);
-#pragma unroll 1
-      for (int r0 = 0; r0 < H; r0 += kBoxRows) tma_3d(dcd + r0 * cv.UB, tm, iA * BITS / 8, r0, e, &bar_dn);
-      bulk_g2s(dss, m.s + static_cast<size_t>(e) * m.sb_stride, sbytes, &bar_dn);
-      bulk_g2s(dss + sbytes, m.b + static_cast<size_t>(e) * m.sb_stride, sbytes, &bar_dn);
-      s_pend.dn = l & 1;
-    }
+    if (!p.split_late && tid == 32 && npc > 0) issue_down(Ld, l);
     {
       // this CTA's slice of the accumulators of layer l + 1
       const int nz = kDecodeReplicas * p.yrep;
@@ -535,6 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
     if (tid == 0) s_pend.gc = -1;
     if (gu_failed) { leave(); return; }
     if (tid < npc) hl[(tid & ~15) | seg_pos<BITS>(tid & 15)] = silu_f(guv[tid]) * guv[cv.npc_max + tid];
+    if (p.split_late && tid == 32 && npc > 0) issue_down(s_layers[l], l);  // into the freed gate/up buffer
     if (npc > 0 && tid < HT && !mbar_ready(&bar_dn, l & 1, p.hdr, 13)) ab = true;
     if (__syncthreads_or(ab)) { leave(); return; }
     if (tid == 0) s_pend.dn = -1;
@@ -635,7 +651,7 @@ bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
 }  // namespace
 
 bool decode_split_plan(int H, int E, int k, int I, int Is, int group, int bits, int grid, int L, size_t smem_limit,
-                       size_t* smem) {
+                       size_t* smem, int* late) {
   if (grid < 1 || L < 1) return false;
   if (L > kMaxDecodeLayers) L = kMaxDecodeLayers;
   const int PS = 128 / bits;
@@ -648,14 +664,19 @@ bool decode_split_plan(int H, int E, int k, int I, int Is, int group, int bits, 
   if (k > 16 || E > 32 * kTopPer) return false;
   if ((k * I + Is) / kUnit > grid) return false;  // at most one unit per CTA
   if (cdiv(E + (Is > 0 ? 1 : 0), grid) > kWarps) return false;  // one router row per warp
-  const size_t need = carve(H, E, I, Is, group, bits, grid, L).total;
-  if (need > smem_limit) return false;
-  *smem = need;
-  return true;
+  for (int lt = 0; lt < 2; ++lt) {  // down data in a region of its own if it fits, else after gate/up
+    const size_t need = carve(H, E, I, Is, group, bits, grid, L, lt).total;
+    if (need <= smem_limit) {
+      *smem = need;
+      *late = lt;
+      return true;
+    }
+  }
+  return false;
 }
 
 cudaError_t launch_decode_split(const DecodeParams& p, int bits, int grid, cudaStream_t stream) {
-  const size_t smem = carve(p.H, p.E, p.I, p.Is, p.group, bits, grid, p.L).total;
+  const size_t smem = carve(p.H, p.E, p.I, p.Is, p.group, bits, grid, p.L, p.split_late).total;
   const int nsg = p.H * bits / 128;
   const int ch = nsg >= 32 ? nsg / 32 : 1;
   if (bits == 4) {
