@@ -42,7 +42,7 @@ NOMINAL_HBM_GBS = 8000.0
 # dram__bytes_write.sum from one ncu capture of the first 4 layers of the workload, divided by 4).
 # Each layer reads its own weights once, so the traffic of a launch over L layers is L times this.
 # Only valid for the kernel as captured: emptied when the kernel changes.
-DECODE_TRAFFIC_PER_LAYER = {"35b": (68_036_352 + 1_571_328) / 4}  # decode_split_kernel, 69.61 MB / 4 layers
+DECODE_TRAFFIC_PER_LAYER = {"35b": (68_037_888 + 1_585_408) / 4}  # decode_split_kernel, 69.62 MB / 4 layers
 FALLBACK_HBM_GBS = 6650.0
 
 
