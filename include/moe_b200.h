@@ -170,8 +170,9 @@ MOE_API moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weig
 
 /* Number of kernel launches moe_stack_forward makes for T tokens and L
  * layers on the current device: a single token runs the whole stack as one
- * persistent kernel (one launch per 128 layers) when the shape fits it;
- * otherwise 1 + 4*L. -1 on a bad configuration. */
+ * persistent kernel (one launch per 48 layers) when the shape fits it; 8 or
+ * more tokens run the batched path (1 + 7*L) where it applies; otherwise
+ * 1 + 4*L. -1 on a bad configuration. */
 MOE_API int32_t moe_stack_kernel_launches(const moe_config* cfg, int32_t T, int32_t L);
 
 /* The batched path's grouping step on its own: the T*k (token, slot) pairs
