@@ -353,6 +353,7 @@ def main():
     e2e_ms = barrier_max(dist, e0.elapsed_time(e1))
 
     launches_per_step = moe.moe_stack_kernel_launches(cfg, T, shape.layers)
+    path = moe.moe_stack_path_name(cfg, T, shape.layers)
     persistent = launches_per_step < shape.layers
     if T == 1:
         bytes_step = touched_bytes_per_token(shape)
@@ -383,8 +384,8 @@ def main():
             "data": "synthetic", "config": workload_config(shape),
             "hbm_gbs": gbs, "hbm_frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm",
-                         "kernel": ("decode_stack_kernel (the whole stack, one launch per step)" if persistent
-                                    else "moe_stack_forward step (router, gate/up, down, glue kernels)"),
+                         "kernel": (f"{path} (the whole stack, one launch per step)" if persistent
+                                    else f"moe_stack_forward step on the {path} path (all its kernels)"),
                          "achieved": gbs, "peak": peak, "peak_source": peak_src, "unit": "GB/s",
                          "frac": gbs / peak, "traffic": traffic,
                          "bytes_per_step": bytes_step,

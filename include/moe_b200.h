@@ -175,6 +175,13 @@ MOE_API moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weig
  * 1 + 4*L. -1 on a bad configuration. */
 MOE_API int32_t moe_stack_kernel_launches(const moe_config* cfg, int32_t T, int32_t L);
 
+/* Name of the path moe_stack_forward takes for T tokens and L layers on the
+ * current device (a static string): "decode_split_kernel" or
+ * "decode_stack_kernel" (one token, the persistent kernels), "batched" (the
+ * grouped tensor-core path), "per_layer" (four kernels per layer), "none"
+ * (T or L is 0); NULL on a bad configuration. */
+MOE_API const char* moe_stack_path_name(const moe_config* cfg, int32_t T, int32_t L);
+
 /* The batched path's grouping step on its own: the T*k (token, slot) pairs
  * of topk_idx [T][k] grouped by expert, stable in (token, slot) order, with
  * the shared expert (if cfg->shared_inter > 0) as expert E taken by every

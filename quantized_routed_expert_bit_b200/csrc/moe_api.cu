@@ -516,6 +516,16 @@ int32_t moe_stack_kernel_launches(const moe_config* cfg, int32_t T, int32_t L) {
   return 1 + 4 * L;
 }
 
+const char* moe_stack_path_name(const moe_config* cfg, int32_t T, int32_t L) {
+  if (check_cfg(cfg) != MOE_OK || T < 0 || L < 0) return nullptr;
+  if (T == 0 || L == 0) return "none";
+  int grid = 0;
+  bool split = false;
+  if (T == 1 && decode_eligible(*cfg, L, &grid, &split)) return split ? "decode_split_kernel" : "decode_stack_kernel";
+  if (batched_eligible(*cfg, T)) return "batched";
+  return "per_layer";
+}
+
 size_t moe_workspace_size(const moe_config* cfg, int32_t T, int32_t L) {
   (void)L;
   if (check_cfg(cfg) != MOE_OK || T < 0) return 0;

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.moe_layer_forward_static.argtypes = [CP, LP, P, I32, P, P, P, P, P]
         L.moe_stack_kernel_launches.argtypes = [CP, I32, I32]
         L.moe_stack_kernel_launches.restype = I32
+        L.moe_stack_path_name.argtypes = [CP, I32, I32]
+        L.moe_stack_path_name.restype = ctypes.c_char_p
         L.moe_get_device_status.argtypes = [P, P]
         L.moe_check_wait_limit.argtypes = [P, ctypes.c_size_t, P, P]
         L.moe_status_string.argtypes = [ctypes.c_int]
@@ -218,3 +220,9 @@ def moe_check_wait_limit(ws: Workspace, gave_up: torch.Tensor, stream=None):
 def moe_stack_kernel_launches(cfg: Config, T: int, L: int) -> int:
     """Kernels one moe_stack_forward call launches on the current device."""
     return int(lib().moe_stack_kernel_launches(ctypes.byref(cfg), int(T), int(L)))
+
+
+def moe_stack_path_name(cfg: Config, T: int, L: int) -> Optional[str]:
+    """The path one moe_stack_forward call takes on the current device (None on a bad configuration)."""
+    name = lib().moe_stack_path_name(ctypes.byref(cfg), int(T), int(L))
+    return None if name is None else name.decode()

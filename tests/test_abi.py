@@ -154,3 +154,7 @@ def test_stack_and_sort_validation_errors():
     assert lib.moe_check_wait_limit(None, 1024, FAKE, None) == moe.MOE_ERR_WORKSPACE
     assert lib.moe_check_wait_limit(FAKE, 32, FAKE, None) == moe.MOE_ERR_WORKSPACE
     assert lib.moe_check_wait_limit(FAKE, 1024, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_stack_path_name(None, 1, 1) is None
+    assert lib.moe_stack_path_name(ctypes.byref(c), 0, 4) == b"none"
+    assert lib.moe_stack_path_name(ctypes.byref(c), 1, 4) in (b"decode_split_kernel", b"decode_stack_kernel",
+                                                               b"per_layer")

@@ -47,6 +47,8 @@ def test_batched_path_is_taken(key):
     assert moe.moe_stack_kernel_launches(cfg, 8, 3) == 1 + 7 * 3
     assert moe.moe_stack_kernel_launches(cfg, 512, 3) == 1 + 7 * 3
     assert moe.moe_stack_kernel_launches(cfg, 7, 3) == 1 + 4 * 3
+    assert moe.moe_stack_path_name(cfg, 8, 3) == moe.moe_stack_path_name(cfg, 512, 3) == "batched"
+    assert moe.moe_stack_path_name(cfg, 7, 3) == "per_layer"
 
 
 @pytest.mark.parametrize("T", [7, 8, 16])

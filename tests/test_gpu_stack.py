@@ -59,6 +59,9 @@ def check_glue(x0_bits, tx, ty, xo):
 @pytest.mark.parametrize("key", ["35b", "80b", "35b8"])
 def test_decode_stack_parity(key):
     shape = synth.SHAPES[key]
+    # which persistent kernel runs each stack on a 148-SM B200 (a silent fallback would fail here)
+    want = {"35b": "decode_split_kernel", "35b8": "decode_split_kernel", "80b": "decode_stack_kernel"}[key]
+    assert moe.moe_stack_path_name(moe.make_config(shape), 1, shape.layers) == want
     layers = [synth.make_layer(shape, l, "cuda") for l in range(shape.layers)]
     total = ParityStats()
     for tok in (0, 1):
