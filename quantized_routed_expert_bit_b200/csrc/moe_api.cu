@@ -460,7 +460,7 @@ moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, in
   P->ybuf = reinterpret_cast<uint32_t*>(b + Ly.dy);
   P->logits_rep = static_cast<int>((Ly.dh - Ly.dlogits) / moe::kDecodeReplicas / 4);
   P->h_rep = static_cast<int>((Ly.dy - Ly.dh) / moe::kDecodeReplicas / 4);
-  P->y_rep = static_cast<int>((Ly.dr - Ly.dy) / moe::kDecodeReplicas / 4);
+  P->y_rep = static_cast<int>((Ly.dyacc - Ly.dy) / moe::kDecodeReplicas / 4);
   P->yacc = reinterpret_cast<float*>(b + Ly.dyacc);
   P->yrep = static_cast<int>(up(static_cast<size_t>(c.hidden) * 4) / 4);
   P->ybuf_stride = static_cast<int64_t>(moe::kDecodeReplicas) * P->yrep;
