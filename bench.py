@@ -51,7 +51,7 @@ def touched_bytes_per_token(shape: synth.MoEShape) -> int:
     selected experts and the shared expert (packed codes + bf16 scales and
     biases), the router E*H*2, the shared gate H*2 and the router bias E*4."""
     per_layer = shape.top_k * shape.expert_bytes() + shape.expert_bytes(shape.shared_inter)
-    per_layer += shape.num_experts * shape.hidden * 2 + shape.hidden * 2
+    per_layer += shape.num_experts * shape.hidden * 2 + (shape.hidden * 2 if shape.shared_inter > 0 else 0)
     if shape.router_bias:
         per_layer += shape.num_experts * 4
     return per_layer * shape.layers
@@ -74,7 +74,8 @@ def touched_bytes_batched(shape, layers_dev, tokens, T, steps):
         torch.cuda.synchronize()
         for l in range(shape.layers):
             distinct += int(torch.unique(ti[l]).numel())
-    per_layer_fixed = shape.expert_bytes(shape.shared_inter) + shape.num_experts * shape.hidden * 2 + shape.hidden * 2
+    per_layer_fixed = (shape.expert_bytes(shape.shared_inter) + shape.num_experts * shape.hidden * 2 +
+                       (shape.hidden * 2 if shape.shared_inter > 0 else 0))
     return (distinct / steps) * shape.expert_bytes() + shape.layers * per_layer_fixed
 
 
