@@ -16,8 +16,10 @@
 //   5. the unit's 32 columns of all H down rows arrive alongside the gate/up
 //      rows: 256-row tiles by the tensor memory accelerator (one 3D map per
 //      layer over the experts' down codes) and the expert's whole down scale
-//      and bias matrices by two bulk copies. Each thread takes four output
-//      rows and forms the unit's routing-weighted partial of y for them, then
+//      and bias matrices by two bulk copies (where they do not fit beside
+//      the gate/up rows, into the gate/up buffer once gate/up is done: the
+//      late-copy mode). Thread t takes output rows t, t + 512, t + 1024,
+//      t + 1536, forms the unit's routing-weighted partial of y for them, and
 //      adds it to a replicated fp32 accumulator (reductions in L2).
 // The y of a layer is then the sum of the k*I/32 + Is/32 partials: no h
 // exchange between CTAs, and no CTA reads more than its own unit of any
