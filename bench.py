@@ -41,8 +41,19 @@ NOMINAL_HBM_GBS = 8000.0
 # DRAM traffic of the persistent decode kernel per layer (dram__bytes_read.sum +
 # dram__bytes_write.sum from one ncu capture of the first 4 layers of the workload, divided by 4).
 # Each layer reads its own weights once, so the traffic of a launch over L layers is L times this.
-# Only valid for the kernel as captured: emptied when the kernel changes.
-DECODE_TRAFFIC_PER_LAYER = {"35b": (68_037_888 + 1_585_408) / 4}  # decode_split_kernel, 69.62 MB / 4 layers
+# Keyed by the workload and a hash of the kernel's source files: a capture of another revision of
+# the kernel is not reported (traffic null).
+KERNEL_SOURCES = ("stack_split.cu", "decode_common.cuh", "moe_common.cuh", "moe_launch.h")
+DECODE_TRAFFIC_PER_LAYER = {}
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "quantized_routed_expert_bit_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -64,7 +75,7 @@ def touched_bytes_batched(shape, layers_dev, tokens, T, steps):
     own routing of the stack (trace), averaged over the timed steps."""
     cfg = moe.make_config(shape)
     ws = moe.Workspace(cfg, T, L=shape.layers)
-    arr = moe.make_layer_array([moe.make_layer_weights(lw) for lw in layers_dev])
+    arr = moe.make_layer_array([moe.make_layer_weights(lw, cfg) for lw in layers_dev])
     ti = torch.empty(shape.layers, T, shape.top_k, dtype=torch.int32, device="cuda")
     xo = torch.empty(T, shape.hidden, dtype=torch.bfloat16, device="cuda")
     distinct = 0
@@ -288,7 +299,7 @@ def main():
     cfg = moe.make_config(shape)
     layers = [synth.make_layer(shape, l, "cuda", seed_id=synth.SHAPE_SEED_ID[key])
               for l in range(shape.layers)]
-    arr = moe.make_layer_array([moe.make_layer_weights(lw) for lw in layers])
+    arr = moe.make_layer_array([moe.make_layer_weights(lw, cfg) for lw in layers])
     T = shape.tokens
     ws = moe.Workspace(cfg, T, L=shape.layers)
     nsteps = args.warmup + args.steps
@@ -375,8 +386,9 @@ def main():
                          f"scaled to {shape.layers} layers per token; expert copies to the host untimed"}
 
     traffic = None
-    if persistent and key in DECODE_TRAFFIC_PER_LAYER:
-        traffic = DECODE_TRAFFIC_PER_LAYER[key] * shape.layers
+    src_hash = kernel_source_hash()
+    if persistent and (key, src_hash) in DECODE_TRAFFIC_PER_LAYER:
+        traffic = DECODE_TRAFFIC_PER_LAYER[(key, src_hash)] * shape.layers
     if rank == 0:
         out = {
             "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,

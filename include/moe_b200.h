@@ -112,6 +112,21 @@ typedef struct {
   moe_qtensor shared_gate_up;    /* 1 matrix [2Is][H] (ignored when shared_inter == 0) */
   moe_qtensor shared_down;       /* 1 matrix [H][Is] */
   const uint16_t* shared_gate_w; /* bf16 [H], the shared expert's sigmoid gate */
+  /* Optional decode-ready copies of the down projections, written once at
+   * load time (16-byte aligned). The single-token decode splits the
+   * intermediate into units of 32 columns and reads, per unit, those 32
+   * columns of all H down rows and their quantisation group's scale and
+   * bias; in these layouts both are contiguous blocks:
+   *   down_units     codes [E][I/32][H][32*bits/8]   (moe_prepare_down_units)
+   *   down_sb        bf16 (scale, bias) [E][I/group][H][2] (moe_prepare_down_sb)
+   * and shared_down_units / shared_down_sb the same for the shared expert
+   * (E = 1, Is in place of I). NULL: the decode reads `down` / `shared_down`
+   * in their canonical layout instead (same results, slower). The other
+   * paths never read them. */
+  const uint16_t* down_sb;
+  const uint16_t* shared_down_sb;
+  const uint8_t* down_units;
+  const uint8_t* shared_down_units;
 } moe_layer_weights;
 
 /* Per-layer record of a stack run; any member may be NULL (not recorded). */
@@ -120,9 +135,12 @@ typedef struct {
   int32_t* idx;  /* [L][T][k] selected experts */
   float* w;      /* [L][T][k] routing weights */
   uint16_t* y;   /* bf16 [L][T][H] output of each layer */
-  uint64_t* t;   /* [L][8] device clock (ns) at the phase boundaries of each layer, single-token
-                    persistent path only: 0 layer start, 1 router done, 2 routing barrier passed,
-                    3 top-k done, 4 gate/up done, 5 h barrier passed, 6 down done, 7 y barrier passed */
+  uint64_t* t;   /* [L][8] device clock (ns) at the phase boundaries of each layer as CTA 0 sees
+                    them, single-token persistent path only. decode_split_kernel: 0 layer start,
+                    1 x ready, 2 router rows done, 3 top-k done, 4 first gate/up batch landed,
+                    5 down data landed, 6 down done, 7 arrival counted. decode_stack_kernel:
+                    0 layer start, 1 router done, 2 routing barrier passed, 3 top-k done,
+                    4 gate/up done, 5 h barrier passed, 6 down done, 7 y barrier passed */
 } moe_trace;
 
 /* Bytes of workspace the calls below need for T tokens (L is unused and
@@ -192,6 +210,39 @@ MOE_API moe_status moe_sort_by_expert(const moe_config* cfg, const int32_t* topk
                               int32_t* perm, int32_t* offsets,
                               void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Bytes of the group-major copy of the scales and biases of n_experts down
+ * matrices [H][K] (K = inter for the routed experts, shared_inter for the
+ * shared one): n_experts * (K/group) * H * 4. 0 on a bad configuration or K
+ * that is not a positive multiple of the group. */
+MOE_API size_t moe_down_sb_size(const moe_config* cfg, int32_t n_experts, int32_t K);
+
+/* Writes the group-major copy of `down`'s scales and biases into `out`
+ * (caller-owned device memory of moe_down_sb_size bytes, 16-byte aligned):
+ * out[((e*(K/group) + g)*H + r)*2 + 0] = scale of row r, group g of expert e,
+ * and + 1 the bias. A pure re-layout (no arithmetic), meant to run once when
+ * the weights are loaded; the result goes into moe_layer_weights.down_sb
+ * (or .shared_down_sb with n_experts = 1 and K = shared_inter). Asynchronous
+ * on `stream`. Not on the pages: a layout of this library's decode kernel. */
+MOE_API moe_status moe_prepare_down_sb(const moe_config* cfg, const moe_qtensor* down, int32_t n_experts,
+                                       int32_t K, uint16_t* out, moe_stream_t stream);
+
+/* Bytes of the unit-major copy of the codes of n_experts down matrices
+ * [H][K]: n_experts * K * H * bits / 8 (the size of the codes themselves).
+ * 0 on a bad configuration or K that is not a positive multiple of 32 and
+ * of the group. */
+MOE_API size_t moe_down_units_size(const moe_config* cfg, int32_t n_experts, int32_t K);
+
+/* Writes the unit-major copy of `down`'s codes into `out` (caller-owned
+ * device memory of moe_down_units_size bytes, 16-byte aligned): the codes of
+ * columns [32u, 32u+32) of row r of expert e go to
+ * out + ((e*(K/32) + u)*H + r) * (32*bits/8). A pure re-layout, meant to run
+ * once when the weights are loaded; the result goes into
+ * moe_layer_weights.down_units (or .shared_down_units with n_experts = 1
+ * and K = shared_inter). Asynchronous on `stream`. Not on the pages: a
+ * layout of this library's decode kernel. */
+MOE_API moe_status moe_prepare_down_units(const moe_config* cfg, const moe_qtensor* down, int32_t n_experts,
+                                          int32_t K, uint8_t* out, moe_stream_t stream);
+
 /* moe_layer_forward without a workspace, for callers that cannot allocate
  * device memory or pass a scratch buffer of their own: code inside a host
  * framework that owns all device memory and forbids allocation after
@@ -199,16 +250,25 @@ MOE_API moe_status moe_sort_by_expert(const moe_config* cfg, const int32_t* topk
  * latency-critical paths where an allocation (which may synchronise the
  * device) is not allowed. The pages have no counterpart of this call; it
  * exists for those callers only.
- * Its scratch is a fixed 2 MiB array inside the library that every GPU that
- * loads the library holds until the process exits; calls whose
- * moe_workspace_size(cfg, T, 1) exceeds 2 MiB (T above 11 tokens at
- * H=2048, E=256, k=8, I=512) return MOE_ERR_WORKSPACE. The call allocates
- * nothing. The first call on a device looks up the array's device address
- * (with that device current) and keeps it; make that first call before any
- * stream capture. Every call shares the one array: calls that overlap on the
- * GPU (other streams, other threads) race and must be serialised by the
- * caller. Each call clears the status word and counters it needs. Arguments
- * as moe_layer_forward; device_status (optional, device int32) receives the
+ * It runs the per-token kernels of moe_layer_forward (router + top-k,
+ * gate/up + SwiGLU, down + combine) for every T; it never takes the batched
+ * tensor-core path that moe_layer_forward uses from 8 tokens up. Its scratch
+ * is a fixed 2 MiB array inside the library that every GPU that loads the
+ * library holds until the process exits. The scratch a call needs is the
+ * per-token part of the workspace layout (status word, routing counters,
+ * logits, gate values, h, and the buffers of the single-token decode), which
+ * grows with T; a call whose part exceeds 2 MiB returns MOE_ERR_WORKSPACE
+ * before anything is enqueued. At H=2048, E=256, k=8, I=Is=512 that admits
+ * T <= 46 tokens; at H=2048, E=512, k=10, I=Is=512, T <= 41. The call
+ * allocates nothing. The first call on a device looks up the array's device
+ * address (with that device current) and keeps it; make that first call
+ * before any stream capture. The kept address is that of the device's
+ * current context: after cudaDeviceReset (or any teardown of the primary
+ * context) it is stale, so do not call this entry point again in that
+ * process. Every call shares the one array: calls that overlap on the GPU
+ * (other streams, other threads) race and must be serialised by the caller.
+ * Each call clears the status word and counters it needs. Arguments as
+ * moe_layer_forward; device_status (optional, device int32) receives the
  * call's device status (0 = MOE_OK, else a moe_status) when the stream gets
  * there. */
 MOE_API moe_status moe_layer_forward_static(const moe_config* cfg, const moe_layer_weights* w,

@@ -422,4 +422,66 @@ cudaError_t launch_glue(const GlueParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- group-major down scales
+
+namespace {
+
+// out[((e * ng + g) * rows + r) * 2 + {0, 1}] = (scale, bias) of row r, group g of expert e:
+// one thread per (e, g, r), 4 bytes out.
+__global__ void prepare_down_sb_kernel(const uint16_t* __restrict__ s, const uint16_t* __restrict__ b, int64_t stride,
+                                       int n, int rows, int ng, uint32_t* __restrict__ out) {
+  const int64_t total = static_cast<int64_t>(n) * ng * rows;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(i % rows);
+    const int64_t eg = i / rows;
+    const int g = static_cast<int>(eg % ng);
+    const int64_t e = eg / ng;
+    const int64_t src = e * stride + static_cast<int64_t>(r) * ng + g;
+    out[i] = static_cast<uint32_t>(s[src]) | (static_cast<uint32_t>(b[src]) << 16);
+  }
+}
+
+}  // namespace
+
+namespace {
+
+// One thread per 16 bytes of the output: out[((e * nu + u) * rows + r) * ub + b] = q[e][r][u * ub + b].
+__global__ void prepare_down_units_kernel(const uint8_t* __restrict__ q, int64_t q_stride, int n, int rows, int rowb,
+                                          int ub, uint8_t* __restrict__ out) {
+  const int nu = rowb / ub, per = ub / 16;
+  const int64_t total = static_cast<int64_t>(n) * nu * rows * per;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int part = static_cast<int>(i % per);
+    const int64_t eur = i / per;
+    const int r = static_cast<int>(eur % rows);
+    const int64_t eu = eur / rows;
+    const int u = static_cast<int>(eu % nu);
+    const int64_t e = eu / nu;
+    const uint4 v = *reinterpret_cast<const uint4*>(q + e * q_stride + static_cast<int64_t>(r) * rowb + u * ub + 16 * part);
+    *reinterpret_cast<uint4*>(out + 16 * i) = v;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prepare_down_units(const uint8_t* q, int64_t q_stride, int n, int rows, int rowb, int ub,
+                                      uint8_t* out, cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>(n) * rows * (rowb / 16);
+  const int64_t blocks = (total + 255) / 256;
+  prepare_down_units_kernel<<<static_cast<int>(blocks < 65535 ? blocks : 65535), 256, 0, stream>>>(
+      q, q_stride, n, rows, rowb, ub, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prepare_down_sb(const uint16_t* scales, const uint16_t* biases, int64_t stride, int n, int rows,
+                                   int ngroups, uint16_t* out, cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>(n) * ngroups * rows;
+  const int64_t blocks = (total + 255) / 256;
+  prepare_down_sb_kernel<<<static_cast<int>(blocks < 65535 ? blocks : 65535), 256, 0, stream>>>(
+      scales, biases, stride, n, rows, ngroups, reinterpret_cast<uint32_t*>(out));
+  return cudaGetLastError();
+}
+
 }  // namespace moe

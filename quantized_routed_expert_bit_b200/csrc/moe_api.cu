@@ -163,7 +163,14 @@ moe_status check_weights(const moe_config& c, const moe_layer_weights* w, bool n
       return s;
     if ((s = check_qt(w->shared_down, c.hidden, c.shared_inter, c.bits, c.group, 1, "shared_down"))) return s;
     if ((s = check_ptr(w->shared_gate_w, 16, "shared_gate_w"))) return s;
+    if (w->shared_down_sb && !aligned(w->shared_down_sb, 16))
+      return fail(MOE_ERR_INVALID_ARG, "shared_down_sb is not 16-byte aligned");
+    if (w->shared_down_units && !aligned(w->shared_down_units, 16))
+      return fail(MOE_ERR_INVALID_ARG, "shared_down_units is not 16-byte aligned");
   }
+  if (w->down_sb && !aligned(w->down_sb, 16)) return fail(MOE_ERR_INVALID_ARG, "down_sb is not 16-byte aligned");
+  if (w->down_units && !aligned(w->down_units, 16))
+    return fail(MOE_ERR_INVALID_ARG, "down_units is not 16-byte aligned");
   return MOE_OK;
 }
 
@@ -434,6 +441,10 @@ moe::LayerDesc layer_desc(const moe_layer_weights& w) {
   d.dn = qmat(w.down);
   d.sgu = qmat(w.shared_gate_up);
   d.sdn = qmat(w.shared_down);
+  d.dsb = w.down_sb;
+  d.sdsb = w.shared_down_sb;
+  d.dcu = w.down_units;
+  d.sdcu = w.shared_down_units;
   return d;
 }
 
@@ -669,6 +680,49 @@ moe_status moe_sort_by_expert(const moe_config* cfg, const int32_t* topk_idx, in
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "sort_by_expert launch");
 }
 
+size_t moe_down_sb_size(const moe_config* cfg, int32_t n_experts, int32_t K) {
+  if (check_cfg(cfg) != MOE_OK || n_experts < 1 || K < cfg->group || K % cfg->group) return 0;
+  return static_cast<size_t>(n_experts) * (K / cfg->group) * cfg->hidden * 4;
+}
+
+moe_status moe_prepare_down_sb(const moe_config* cfg, const moe_qtensor* down, int32_t n_experts, int32_t K,
+                               uint16_t* out, moe_stream_t stream) {
+  moe_status s;
+  if ((s = check_cfg(cfg))) return s;
+  if (!down) return fail(MOE_ERR_INVALID_ARG, "down is NULL");
+  if (n_experts < 1 || K < cfg->group || K % cfg->group)
+    return fail(MOE_ERR_INVALID_ARG, "n_experts=%d K=%d (K a positive multiple of group %d)", n_experts, K,
+                cfg->group);
+  if ((s = check_qt(*down, cfg->hidden, K, cfg->bits, cfg->group, n_experts, "down"))) return s;
+  if ((s = check_ptr(out, 16, "out"))) return s;
+  const int64_t stride = n_experts > 1 ? down->sb_expert_stride : static_cast<int64_t>(cfg->hidden) * (K / cfg->group);
+  cudaError_t e = moe::launch_prepare_down_sb(down->scales, down->biases, stride, n_experts, cfg->hidden,
+                                              K / cfg->group, out, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "prepare_down_sb launch");
+}
+
+size_t moe_down_units_size(const moe_config* cfg, int32_t n_experts, int32_t K) {
+  if (check_cfg(cfg) != MOE_OK || n_experts < 1 || K < cfg->group || K % cfg->group || K % 32) return 0;
+  return static_cast<size_t>(n_experts) * K * cfg->hidden * cfg->bits / 8;
+}
+
+moe_status moe_prepare_down_units(const moe_config* cfg, const moe_qtensor* down, int32_t n_experts, int32_t K,
+                                  uint8_t* out, moe_stream_t stream) {
+  moe_status s;
+  if ((s = check_cfg(cfg))) return s;
+  if (!down) return fail(MOE_ERR_INVALID_ARG, "down is NULL");
+  if (n_experts < 1 || K < cfg->group || K % cfg->group || K % 32)
+    return fail(MOE_ERR_INVALID_ARG, "n_experts=%d K=%d (K a positive multiple of 32 and of group %d)", n_experts, K,
+                cfg->group);
+  if ((s = check_qt(*down, cfg->hidden, K, cfg->bits, cfg->group, n_experts, "down"))) return s;
+  if ((s = check_ptr(out, 16, "out"))) return s;
+  const int rowb = K * cfg->bits / 8;
+  const int64_t stride = n_experts > 1 ? down->q_expert_stride : static_cast<int64_t>(cfg->hidden) * rowb;
+  cudaError_t e = moe::launch_prepare_down_units(down->q, stride, n_experts, cfg->hidden, rowb, 32 * cfg->bits / 8,
+                                                 out, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "prepare_down_units launch");
+}
+
 moe_status moe_check_wait_limit(void* ws, size_t ws_bytes, int32_t* gave_up, moe_stream_t stream) {
   if (!ws || !aligned(ws, kAlign)) return fail(MOE_ERR_WORKSPACE, "workspace NULL or misaligned");
   if (ws_bytes < sizeof(moe::WsHeader)) return fail(MOE_ERR_WORKSPACE, "workspace too small");
@@ -719,10 +773,11 @@ const char* moe_last_error_string(void) { return g_last_error.c_str(); }
 
 // ---------------------------------------------------------------- allocation-free layer call
 //
-// moe_layer_forward_static runs the same kernels as moe_layer_forward but
-// takes no workspace: its scratch (status word, routing counters, logits,
-// gate activations) lives in the fixed array below, which every GPU that
-// loads this library holds until the process exits. It serves callers that
+// moe_layer_forward_static runs the per-token kernels of moe_layer_forward
+// (never the batched tensor-core path) and takes no workspace: its scratch
+// (status word, routing counters, logits, gate activations: the regions of
+// the workspace layout below `base_total`) lives in the fixed array below,
+// which every GPU that loads this library holds until the process exits. It serves callers that
 // cannot call cudaMalloc or hand the library a buffer of their own: code
 // running inside a host framework that owns all device memory and forbids
 // allocation after start-up, plugins that are handed only their inputs and
@@ -741,7 +796,9 @@ void* g_static_ptr[kMaxDevices] = {};
 
 // Device address of g_static_scratch on the current device. In host code the
 // symbol's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and kept.
+// once per device (with that device current) and kept. The kept address
+// belongs to the device's primary context as it was at that first call; it
+// is stale after cudaDeviceReset, which the header tells callers.
 moe_status static_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

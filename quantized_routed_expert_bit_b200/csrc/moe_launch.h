@@ -103,6 +103,10 @@ struct LayerDesc {
   const float* rbias;    // fp32 [E] or null
   const uint16_t* wsg;   // bf16 [H] shared-expert gate vector (when Is > 0)
   QMat gu, dn, sgu, sdn;
+  const uint16_t* dsb;   // split kernel: group-major down (scale, bias) [E][I/group][H][2] (moe_prepare_down_sb)
+  const uint16_t* sdsb;  // the same for the shared expert [1][Is/group][H][2]
+  const uint8_t* dcu;    // split kernel: unit-major down codes [E][I/32][H][32*bits/8] (moe_prepare_down_units)
+  const uint8_t* sdcu;   // the same for the shared expert
 };
 
 constexpr int kMaxDecodeLayers = 48;   // layers per launch (kernel parameter space)
@@ -134,7 +138,7 @@ struct DecodeParams {
   // CTA c adds into copy c % kDecodeReplicas, readers sum the copies) and the arrival counter
   float* yacc;
   int yrep;
-  int split_late;        // split kernel: down data copied into the gate/up buffer once gate/up is done
+  int split_late;        // split kernel: down codes copied into the first gate/up batch's space once it is read
   int64_t ybuf_stride;   // floats between buffers (kDecodeReplicas * yrep)
   uint32_t* arrive;
   WsHeader* hdr;
@@ -164,5 +168,13 @@ bool decode_split_plan(int H, int E, int k, int I, int Is, int group, int bits, 
 cudaError_t launch_decode_split(const DecodeParams& p, int bits, int grid, cudaStream_t stream);
 cudaError_t launch_decode_stack(const DecodeParams& p, int bits, int grid, cudaStream_t stream);
 cudaError_t launch_wait_limit_check(WsHeader* hdr, uint32_t* never_set, int32_t* gave_up, cudaStream_t stream);
+// Group-major copy of one down tensor's scales and biases: out[e][g][r][0..1] = (scale, bias) of row r,
+// group g of expert e (n experts of `rows` rows and ngroups groups, expert stride `stride` elements).
+// Unit-major copy of one down tensor's codes: out[e][u][r][0..ub) = codes of columns [32u, 32u+32) of row r
+// (ub = 32*bits/8 bytes; n experts of `rows` rows of rowb bytes, expert stride q_stride bytes).
+cudaError_t launch_prepare_down_units(const uint8_t* q, int64_t q_stride, int n, int rows, int rowb, int ub,
+                                      uint8_t* out, cudaStream_t stream);
+cudaError_t launch_prepare_down_sb(const uint16_t* scales, const uint16_t* biases, int64_t stride, int n, int rows,
+                                   int ngroups, uint16_t* out, cudaStream_t stream);
 
 }  // namespace moe

@@ -3,29 +3,47 @@
 //
 // One CTA per SM, all co-resident (cooperative launch), walks every layer:
 //   1. residual + parameter-free RMSNorm of the previous layer's output
-//      (every CTA redundantly, identical arithmetic), giving this layer's x;
+//      (every CTA redundantly, identical arithmetic), giving this layer's x,
+//      kept as fp32 for the router and as a fixed-point integer vector for
+//      the expert dot products (below);
 //   2. router rows: each CTA owns E/G rows of the router (plus the shared
 //      expert's gate vector as row E), prefetched into shared memory by bulk
 //      copies one layer ahead, and publishes their logits;
-//   3. softmax + top-k in every CTA from all published logits (one warp);
+//   3. softmax + top-k in every CTA from all published logits (one warp),
+//      which at once issues the bulk copies of its CTA's unit (4.);
 //   4. the CTA's unit: 32 consecutive columns of one selected expert's
 //      intermediate (the k*I + Is columns of the selected experts, one unit
 //      per CTA, the remaining CTAs idle here). Its 32 packed gate/up row pairs
-//      land in shared memory by bulk copies, the dot products dequantize in
-//      registers, and SwiGLU gives the unit's 32 values of h;
-//   5. the unit's 32 columns of all H down rows arrive alongside the gate/up
-//      rows: 256-row tiles by the tensor memory accelerator (one 3D map per
-//      layer over the experts' down codes) and the expert's whole down scale
-//      and bias matrices by two bulk copies (where they do not fit beside
-//      the gate/up rows, into the gate/up buffer once gate/up is done: the
-//      late-copy mode). Thread t takes output rows t, t + 512, t + 1024,
-//      t + 1536, forms the unit's routing-weighted partial of y for them, and
-//      adds it to a replicated fp32 accumulator (reductions in L2).
+//      with their scales and biases land in shared memory in two batches of
+//      16 pairs, the dot products run on integer dot-product instructions,
+//      and SwiGLU gives the unit's 32 values of h;
+//   5. the unit's 32 columns of all H down rows and their scales and biases
+//      (bulk copies of the contiguous blocks that moe_prepare_down_units and
+//      moe_prepare_down_sb lay out; without those copies, 256-row tiles of the
+//      canonical codes by the tensor memory accelerator) are requested right
+//      behind the gate/up batches, or, where they do not fit beside the
+//      gate/up rows, into the first batch's space as soon as every warp is
+//      done with it (the mid-copy mode). Thread t takes output rows t,
+//      t + 512, ..., forms the unit's routing-weighted partial of y for them,
+//      and adds it to a replicated fp32 accumulator (reductions in L2).
 // The y of a layer is then the sum of the k*I/32 + Is/32 partials: no h
 // exchange between CTAs, and no CTA reads more than its own unit of any
 // expert. Routing fan-out and shared experts: Swiftlet article (xix.ai),
 // paragraphs 4 and 8; Runnel README, "Target". Low-bit groups: same article,
 // paragraph 8. Packed gate/up: Runnel README, introduction and "Streaming CLI".
+//
+// Integer dot products. A group's share of a row's dot product is
+// s_g * sum(q x) + b_g * sum(x). The activations (x, and the unit's h) are
+// turned into one fixed-point vector per layer: X_i = rint(x_i * 2^S) with S
+// chosen from max|x| so that |X_i| < 2^22, which is exact for every x_i
+// within 14 binades of the largest (bf16 x has 8 significant bits; h is
+// rounded to 22 bits below its largest element, finer than an fp32 sum of
+// the products). X is split into three bytes, X = 65536*X2 + 256*X1 + X0
+// (X2 signed, X1 and X0 unsigned), and sum(q X) is three exact integer sums
+// of byte products (dp4a: four byte products and an add per instruction),
+// recombined in fp32 once per 16-byte segment of codes and scaled back by
+// 2^-S. 4-bit codes are split into even and odd nibbles as bytes first (two
+// masks), so x is laid out in the same even/odd order.
 //
 // Two exchanges between CTAs per layer, neither a grid barrier:
 //  - logits are fp32 words whose least significant mantissa bit is replaced
@@ -63,24 +81,26 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBatch = 16;                    // gate/up pairs per code batch (one mbarrier each)
 constexpr int kUnit = 32;                     // columns of the intermediate per CTA
-constexpr int kMaxBatches = kUnit / kBatch;
+constexpr int kNB = kUnit / kBatch;           // batches per unit
 constexpr int kTopPer = 16;                   // logits per lane in the top-k warp: E <= 512
 constexpr int kBoxRows = 256;                 // down rows per tensor copy
+constexpr int kQ = 24;                        // u32 words of fixed-point quads per 32 codes (8 quads x 3 bytes)
 
 __host__ __device__ constexpr uint32_t al128(uint32_t v) { return (v + 127u) & ~127u; }
 __host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 // Shared-memory carve-up; identical on host (sizing) and device.
 struct Carve {
-  int PS, nsg, npc_max, ng, ngd, rowb, rr_max, HT, UB;
-  uint32_t xs, xn, rr, hl, guv, gsb, dbuf, dcd, dss, rbuf, desc, total;
+  int PS, nsg, QS, QSP, ng, ngd, rowb, rr_max, HT, UB;
+  uint32_t xn, xq, hq, guv, gsb, gcd, dcd, dhi, dsb, rbuf, desc, total;
 };
 
 __host__ __device__ inline Carve carve(int H, int E, int I, int Is, int group, int bits, int G, int L, int late) {
   Carve c{};
-  c.PS = 128 / bits;
-  c.nsg = H / c.PS;
-  c.npc_max = kUnit;
+  c.PS = 128 / bits;          // codes per 16-byte segment
+  c.nsg = H / c.PS;           // segments per gate/up row
+  c.QS = 3 * (c.PS / 4);      // quad words of x per segment (3 bytes x PS/4 quads)
+  c.QSP = c.QS + 1;           // + the segment's sum of X (odd stride: conflict-free by segment)
   c.ng = H / group;
   c.ngd = I / group;
   c.rowb = H * bits / 8;
@@ -88,26 +108,25 @@ __host__ __device__ inline Carve carve(int H, int E, int I, int Is, int group, i
   c.HT = H / 4;
   c.UB = kUnit * bits / 8;  // bytes of one down row inside the unit
   uint32_t o = 0;
-  c.xs = o;    o = al128(o + H * 4);
-  c.xn = o;    o = al128(o + H * 4);
-  c.rr = o;    o = al128(o + H * 4);
-  c.hl = o;    o = al128(o + kUnit * 4);
+  c.xn = o;    o = al128(o + H * 4);                       // x, fp32, natural order (router)
+  c.xq = o;    o = al128(o + c.QSP * c.nsg * 4);           // x quads [nsg][QS] + sum of X, per segment
+  c.hq = o;    o = al128(o + kQ * 4);                      // the unit's h quads
   c.guv = o;   o = al128(o + 2 * kUnit * 4);
-  c.gsb = o;   o = al128(o + 4 * kUnit * c.ng * 2);
-  const uint32_t gu_bytes = 2 * kUnit * c.rowb;                 // gate/up code rows
-  const uint32_t dn_bytes = al128(H * c.UB) + 2 * H * c.ngd * 2;  // the unit's down codes [row][UB], then
-                                                                  // the expert's down scales and biases
-  if (late) {  // the down data reuses the gate/up buffer once gate/up is done
-    c.dbuf = o;  o = al128(o + (gu_bytes > dn_bytes ? gu_bytes : dn_bytes));
-    c.dcd = c.dbuf;
-    c.dss = c.dbuf + al128(H * c.UB);
+  c.gsb = o;   o = al128(o + 4 * kUnit * c.ng * 2);        // [gate sc, up sc, gate bi, up bi][pair][ng]
+  const uint32_t gu_bytes = 2 * kUnit * c.rowb;             // [gate|up][pair][rowb]
+  c.gcd = o;   o = al128(o + gu_bytes);
+  if (late) {
+    // mid-copy mode: down rows [0, H/2) take the first batch's gate rows, [H/2, H) its up rows
+    // (H/2 rows of 32 codes are exactly 16 rows of H codes)
+    c.dcd = c.gcd;
+    c.dhi = c.gcd + kUnit * c.rowb;
   } else {
-    c.dbuf = o;  o = al128(o + gu_bytes);
-    c.dcd = o;   o = al128(o + H * c.UB);
-    c.dss = o;   o = al128(o + 2 * H * c.ngd * 2);
+    c.dcd = o;  o = al128(o + H * c.UB);
+    c.dhi = c.dcd + (H / 2) * c.UB;
   }
+  c.dsb = o;   o = al128(o + H * 4);                       // down (scale, bias) of the unit's group, [H][2]
   c.rbuf = o;  o = al128(o + 2 * c.rr_max * H * 2);
-  c.desc = o;  o = al128(o + L * sizeof(LayerDesc));             // the launch's layer descriptors
+  c.desc = o;  o = al128(o + L * sizeof(LayerDesc));       // the launch's layer descriptors
   c.total = o;
   return c;
 }
@@ -125,6 +144,64 @@ __device__ __forceinline__ void tma_3d(void* dst, const CUtensorMap* m, int x, i
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
+
+// Byte dot products: 4 unsigned code bytes times 4 signed (.s32) or unsigned (.u32) bytes, plus c.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// sum over one 16-byte segment of codes of q * X (X given as its quads: q3[j][.] byte j of X; for
+// 4-bit codes quads (2w, 2w+1) hold the even and odd elements of word w), as an fp32 number.
+template <int BITS>
+__device__ __forceinline__ float seg_dot(const uint4& c, const uint32_t* q2, const uint32_t* q1, const uint32_t* q0) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  int a2 = 0;
+  uint32_t a1 = 0u, a0 = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if constexpr (BITS == 4) {
+      const uint32_t lo = w[i] & 0x0F0F0F0Fu, hi = (w[i] >> 4) & 0x0F0F0F0Fu;
+      a2 = dp4a_us(lo, q2[2 * i], a2);
+      a2 = dp4a_us(hi, q2[2 * i + 1], a2);
+      a1 = dp4a_uu(lo, q1[2 * i], a1);
+      a1 = dp4a_uu(hi, q1[2 * i + 1], a1);
+      a0 = dp4a_uu(lo, q0[2 * i], a0);
+      a0 = dp4a_uu(hi, q0[2 * i + 1], a0);
+    } else {
+      a2 = dp4a_us(w[i], q2[i], a2);
+      a1 = dp4a_uu(w[i], q1[i], a1);
+      a0 = dp4a_uu(w[i], q0[i], a0);
+    }
+  }
+  // |a2| < 2^20, a1 * 256 + a0 < 2^29: both exact in int, one fp32 rounding each
+  return fmaf(static_cast<float>(a2), 65536.f, static_cast<float>(a1 * 256u + a0));
+}
+
+// Byte j (0, 1, 2) of the fixed-point value X (|X| < 2^23; byte 2 is the signed top byte).
+__device__ __forceinline__ uint32_t xbyte(int X, int j) { return static_cast<uint32_t>(X >> (8 * j)) & 0xFFu; }
+
+// Where code position o (0..PS-1) of a segment sits among the segment's quad bytes:
+// quad index (word*2 + odd for 4-bit, word for 8-bit) * 4 + byte.
+template <int BITS>
+__host__ __device__ constexpr int quad_pos(int o) {
+  return BITS == 4 ? ((o >> 3) * 2 + (o & 1)) * 4 + ((o & 7) >> 1) : o;
+}
+
+// 2^S with S chosen so that |x| < 2^22 * 2^-S for |x| <= m (a power of two, clamped to fp32 range).
+__device__ __forceinline__ int fix_exp(float m) {
+  if (!(m > 0.f)) return 0;
+  int e = ((__float_as_uint(m) >> 23) & 0xFF) - 127;  // floor(log2 m) for normal m
+  if (e < -100) e = -100;
+  return 21 - e;
+}
+__device__ __forceinline__ float pow2f(int s) { return __uint_as_float(static_cast<uint32_t>(s + 127) << 23); }
 
 // Copy-phase bookkeeping for leaving early: parities of the phases this CTA
 // still has bulk copies in flight on (-1 = none).
@@ -148,14 +225,17 @@ __device__ __noinline__ void drain(Pending* pend, uint64_t* bar_r, uint64_t* bar
 template <int BITS, int CH>
 __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int PS = 128 / BITS;  // codes per 16-byte segment
+  constexpr int QW = PS / 4;      // quads per segment per byte plane
   extern __shared__ __align__(128) unsigned char sm[];
   __shared__ __align__(8) uint64_t bar_r[2];
-  __shared__ __align__(8) uint64_t bar_gc[kMaxBatches];
+  __shared__ __align__(8) uint64_t bar_gc[kNB];
   __shared__ __align__(8) uint64_t bar_dn;
   __shared__ int s_idx[16];
   __shared__ float s_w[16];
   __shared__ float s_sg;
-  __shared__ float s_red[kWarps];
+  __shared__ float s_red[2][kWarps];
+  __shared__ float s_hx[2];  // the unit's sum of X_h, and 2^-S_h
+  __shared__ int s_b0;       // mid-copy mode: warps done with the first gate/up batch
   __shared__ Pending s_pend;
 
   const int H = p.H, E = p.E, k = p.k, I = p.I, Is = p.Is, group = p.group;
@@ -163,45 +243,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   bool ab = false;  // a wait of this thread gave up; combined over the CTA at each phase end
   const Carve cv = carve(H, E, I, Is, group, BITS, G, p.L, p.split_late);
-  float* xs = reinterpret_cast<float*>(sm + cv.xs);  // x by 16-byte code segment (conflict-free float4 reads)
-  float* xn = reinterpret_cast<float*>(sm + cv.xn);  // x in natural order
-  float* rr = reinterpret_cast<float*>(sm + cv.rr);  // residual stream, fp32
-  float* hl = reinterpret_cast<float*>(sm + cv.hl);  // the unit's h, in code order
+  float* xn = reinterpret_cast<float*>(sm + cv.xn);
+  uint32_t* xq = reinterpret_cast<uint32_t*>(sm + cv.xq);
+  uint32_t* hq = reinterpret_cast<uint32_t*>(sm + cv.hq);
   float* guv = reinterpret_cast<float*>(sm + cv.guv);
   uint16_t* gsb = reinterpret_cast<uint16_t*>(sm + cv.gsb);
-  unsigned char* dbuf = sm + cv.dbuf;
-  unsigned char* dcd = sm + cv.dcd;
-  unsigned char* dss = sm + cv.dss;
+  unsigned char* gcd = sm + cv.gcd;
+  unsigned char* dcd = sm + cv.dcd;    // down rows [0, H/2)
+  unsigned char* dhi = sm + cv.dhi;    // down rows [H/2, H)
+  const int H2 = H / 2;
+  const uint32_t* dsb = reinterpret_cast<const uint32_t*>(sm + cv.dsb);
   uint16_t* rbuf = reinterpret_cast<uint16_t*>(sm + cv.rbuf);
   const LayerDesc* s_layers = reinterpret_cast<const LayerDesc*>(sm + cv.desc);
 
   // ---- static assignment of this CTA's work: unit c (if any) = columns [32c, 32c + 32) of the
   // flattened (slot, column) space, slot j at [j * I, (j + 1) * I), the shared expert last
   const int NP = k * I + Is;
-  const int gp0 = c < NP / kUnit ? c * kUnit : 0;
-  const int npc = c < NP / kUnit ? kUnit : 0;
-  const int gp1 = gp0 + npc;
-  const int nb = cdiv(npc, kBatch);
-  // gate/up code of the batches below handles a pair range over up to two slots; a unit is in one
-  const int jA = gp0 < k * I ? gp0 / I : k;
-  const int nA = npc;
-  const int iA = gp0 - (jA < k ? jA * I : k * I);
+  const bool has_unit = c < NP / kUnit;
+  const int gp0 = has_unit ? c * kUnit : 0;
+  const int jA = gp0 < k * I ? gp0 / I : k;                // the unit's slot (k = shared expert)
+  const int iA = gp0 - (jA < k ? jA * I : k * I);          // first column inside the slot
   const bool u_routed = jA < k;
-  const int u_g = iA / group;  // the unit's quantisation group along the down rows
+  const int u_g = iA / group;                              // the unit's quantisation group along the down rows
   const int nrows_rt = E + (Is > 0 ? 1 : 0);
   const int rr_cnt = (c < nrows_rt) ? cdiv(nrows_rt - c, G) : 0;
   const uint32_t* lg_in = p.logits + (c % kDecodeReplicas) * p.logits_rep;  // this CTA's copy of the logits
-  const int rowb = cv.rowb, ng = cv.ng, ngd = cv.ngd, HT = cv.HT;
+  const int rowb = cv.rowb, ng = cv.ng, HT = cv.HT, nsg = cv.nsg;
   const int lgG = 31 - __clz(group);  // group is a power of two
-  (void)gp1;
+  const int nb = has_unit ? kNB : 0;
 
   if (tid == 0) {
     mbar_init(&bar_r[0], 1);
     mbar_init(&bar_r[1], 1);
-    for (int b = 0; b < kMaxBatches; ++b) mbar_init(&bar_gc[b], 1);
+    for (int b = 0; b < kNB; ++b) mbar_init(&bar_gc[b], 1);
     mbar_init(&bar_dn, 1);
     fence_mbar_init();
     s_pend.r[0] = s_pend.r[1] = s_pend.gc = s_pend.dn = -1;
+    s_b0 = 0;
   }
   // every layer descriptor of the launch into shared memory, once (parameter-space reads
   // with a runtime index would otherwise miss the constant cache in the middle of a layer)
@@ -229,7 +307,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
 
   // lane roles in the gate/up dot products: a row of nsg 16-byte code segments is
   // covered by 32/nsg rows per warp step (nsg < 32) or by CH segments per lane
-  const int nsg = cv.nsg;
   const int rps = nsg >= 32 ? 1 : 32 / nsg;
   const int gsub = nsg >= 32 ? 0 : lane / nsg;
   const int gs0 = nsg >= 32 ? lane : lane % nsg;
@@ -247,33 +324,95 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
       y[3] += __uint_as_float(w.w);
     }
   };
-  // thread 0: wait until `target` arrivals are in, then an acquire fence
+  // thread 0: wait until `target` arrivals are in (acquire loads: what the arriving CTAs wrote
+  // before their release arrivals is visible after)
   auto wait_arrivals = [&](uint32_t target, int where) {
     if (tid != 0) return;
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
-      if (ld_word(p.arrive) >= target) break;
+      uint32_t v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.arrive) : "memory");
+      if (v >= target) break;
       MOE_POLL_BACKOFF(it, t0, p.hdr, where, ab)
     }
-    __threadfence();
+  };
+  // block-wide sum of a and max of b (all threads call; every thread gets both)
+  auto block_sum_max = [&](float a, float b, float& sa, float& mb) {
+    a = warp_sum(a);
+    b = warp_max(b);
+    if (lane == 0) {
+      s_red[0][warp] = a;
+      s_red[1][warp] = b;
+    }
+    __syncthreads();
+    sa = 0.f;
+    mb = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      sa += s_red[0][w];
+      mb = fmaxf(mb, s_red[1][w]);
+    }
   };
 
-  // the unit's down data (thread 32): 256-row tiles of its 32 columns of the down codes, and
-  // the expert's whole down scale and bias matrices
-  auto issue_down = [&](const LayerDesc& Ld, int l) {
-    const QMat& m = u_routed ? Ld.dn : Ld.sdn;
-    const CUtensorMap* tm = u_routed ? &p.tm_dn[l] : &p.tm_sdn[l];
-    const int e = u_routed ? s_idx[jA] : 0;
-    const uint32_t sbytes = static_cast<uint32_t>(H) * ngd * 2;
-    // the buffer may last have been read by ordinary loads (gate/up or the previous layer's down)
+  // the unit's down data (one thread): 256-row tiles of its 32 columns of the down codes, and
+  // the (scale, bias) pairs of its group for all H rows from the group-major copy (when the
+  // layer has one; else the down phase reads them from the canonical layout)
+  auto issue_down = [&](const LayerDesc& Ld, int l, int e) {
+    const uint16_t* sbm = u_routed ? Ld.dsb : Ld.sdsb;
+    const uint8_t* cdm = u_routed ? Ld.dcu : Ld.sdcu;
+    const size_t eu = u_routed ? e : 0;
+    // the buffers may last have been read by ordinary loads (gate/up or the previous layer's down)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_arrive_expect_tx(&bar_dn, static_cast<uint32_t>(H) * cv.UB + 2 * sbytes);
+    mbar_arrive_expect_tx(&bar_dn, static_cast<uint32_t>(H) * (cv.UB + (sbm ? 4 : 0)));
+    if (cdm) {  // the unit's 32 columns of all rows: one contiguous block, in two halves
+      const uint8_t* src = cdm + ((eu * (u_routed ? I : Is) / kUnit) + iA / kUnit) * H * cv.UB;
+      bulk_g2s(dcd, src, static_cast<uint32_t>(H2) * cv.UB, &bar_dn);
+      bulk_g2s(dhi, src + static_cast<size_t>(H2) * cv.UB, static_cast<uint32_t>(H2) * cv.UB, &bar_dn);
+    } else {
+      const CUtensorMap* tm = u_routed ? &p.tm_dn[l] : &p.tm_sdn[l];
 #pragma unroll 1
-    for (int r0 = 0; r0 < H; r0 += kBoxRows) tma_3d(dcd + r0 * cv.UB, tm, iA * BITS / 8, r0, e, &bar_dn);
-    bulk_g2s(dss, m.s + static_cast<size_t>(e) * m.sb_stride, sbytes, &bar_dn);
-    bulk_g2s(dss + sbytes, m.b + static_cast<size_t>(e) * m.sb_stride, sbytes, &bar_dn);
+      for (int r0 = 0; r0 < H; r0 += kBoxRows)
+        tma_3d(r0 < H2 ? dcd + r0 * cv.UB : dhi + (r0 - H2) * cv.UB, tm, iA * BITS / 8, r0, static_cast<int>(eu),
+               &bar_dn);
+    }
+    if (sbm)
+      bulk_g2s(sm + cv.dsb, sbm + (eu * cv.ngd + u_g) * H * 2, static_cast<uint32_t>(H) * 4, &bar_dn);
     s_pend.dn = l & 1;
   };
+
+  // the unit's gate/up data (one whole warp, converged): batch 0's code rows with the scales and
+  // biases of the whole unit, then batch 1's code rows; then (unless in mid-copy mode) the down data
+  auto issue_unit = [&](const LayerDesc& Ld, int l, int e) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    const QMat& mq = u_routed ? Ld.gu : Ld.sgu;
+    const int Ij = u_routed ? I : Is;
+    const uint8_t* qb = mq.q + static_cast<size_t>(e) * mq.q_stride;
+    const uint16_t* sb = mq.s + static_cast<size_t>(e) * mq.sb_stride;
+    const uint16_t* bb = mq.b + static_cast<size_t>(e) * mq.sb_stride;
+    const uint32_t cb = static_cast<uint32_t>(kBatch) * rowb, sbb = static_cast<uint32_t>(kUnit) * ng * 2;
+#pragma unroll 1
+    for (int b = 0; b < kNB; ++b) {
+      const int r0 = iA + b * kBatch;  // first gate row of the batch; its up row is Ij + r0
+      if (lane == 0) mbar_arrive_expect_tx(&bar_gc[b], 2 * cb + (b == 0 ? 4 * sbb : 0u));
+      __syncwarp();
+      if (lane < (b == 0 ? 6 : 2)) {
+        const int gu = lane & 1, kind = lane >> 1;  // kind 0 codes, 1 scales, 2 biases
+        if (kind == 0)
+          bulk_g2s(gcd + static_cast<size_t>(gu * kUnit + b * kBatch) * rowb,
+                   qb + static_cast<size_t>(gu * Ij + r0) * rowb, cb, &bar_gc[b]);
+        else
+          bulk_g2s(gsb + static_cast<size_t>(((kind - 1) * 2 + gu) * kUnit) * ng,
+                   (kind == 1 ? sb : bb) + static_cast<size_t>(gu * Ij + iA) * ng, sbb, &bar_gc[b]);
+      }
+    }
+    if (lane == 0) {
+      s_pend.gc = l & 1;
+      if (!p.split_late) issue_down(Ld, l, e);
+    }
+    __syncwarp();
+  };
+
+  float rr4[4] = {0.f, 0.f, 0.f, 0.f};  // residual stream, rows 4t .. 4t+3 (t < H/4)
 
   for (int l = 0; l < p.L; ++l) {
     const int lg = p.l0 + l;  // layer index within the whole stack (trace rows)
@@ -284,52 +423,103 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
     };
     stamp(0);
 
-    // ---------------- 1. this layer's x (and residual)
+    // ---------------- 1. this layer's x (and residual), fp32 and fixed point
+    float xv[4] = {0.f, 0.f, 0.f, 0.f};
+    float m;
     if (l == 0) {
-#pragma unroll 1
-      for (int i = tid; i < H; i += kThreads) {
-        const float v = bf16_to_f32(p.x0[i]);
-        xn[i] = v;
-        rr[i] = p.r_in ? p.r_in[i] : v;
-        if (c == 0 && p.tr_x) p.tr_x[static_cast<size_t>(p.l0) * H + i] = p.x0[i];
+      float mx = 0.f;
+      if (tid < HT) {
+        const uint2 w = *reinterpret_cast<const uint2*>(p.x0 + 4 * tid);
+        xv[0] = bf16_lo(w.x);
+        xv[1] = bf16_hi(w.x);
+        xv[2] = bf16_lo(w.y);
+        xv[3] = bf16_hi(w.y);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          rr4[u] = p.r_in ? p.r_in[4 * tid + u] : xv[u];
+          mx = fmaxf(mx, fabsf(xv[u]));
+        }
+        if (c == 0 && p.tr_x) *reinterpret_cast<uint2*>(p.tr_x + static_cast<size_t>(p.l0) * H + 4 * tid) = w;
       }
+      float unused;
+      block_sum_max(0.f, mx, unused, m);
     } else {
       wait_arrivals(static_cast<uint32_t>(G) * static_cast<uint32_t>(l), 20);
       if (__syncthreads_or(ab)) { leave(); return; }
-      float ss = 0.f;
+      float ss = 0.f, mx = 0.f;
       if (tid < HT) {
         float y[4];
         read_y(l - 1, y);
+        uint16_t yb[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const uint16_t yb = f32_to_bf16(y[u]);
-          const float v = rr[4 * tid + u] + bf16_to_f32(yb);
-          rr[4 * tid + u] = v;
-          ss = fmaf(v, v, ss);
-          if (c == 0 && p.tr_y) p.tr_y[static_cast<size_t>(lg - 1) * H + 4 * tid + u] = yb;
+          yb[u] = f32_to_bf16(y[u]);
+          rr4[u] += bf16_to_f32(yb[u]);
+          ss = fmaf(rr4[u], rr4[u], ss);
+          mx = fmaxf(mx, fabsf(rr4[u]));
         }
+        if (c == 0 && p.tr_y)
+          *reinterpret_cast<uint2*>(p.tr_y + static_cast<size_t>(lg - 1) * H + 4 * tid) =
+              make_uint2(yb[0] | (static_cast<uint32_t>(yb[1]) << 16), yb[2] | (static_cast<uint32_t>(yb[3]) << 16));
       }
-      ss = warp_sum(ss);
-      if (lane == 0) s_red[warp] = ss;
-      __syncthreads();
-      float tot = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) tot += s_red[w];
+      float tot;
+      block_sum_max(ss, mx, tot, m);
       const float inv = 1.f / sqrtf(tot / static_cast<float>(H) + p.eps);
-#pragma unroll 1
-      for (int i = tid; i < H; i += kThreads) {
-        const uint16_t xb = f32_to_bf16(rr[i] * inv);
-        xn[i] = bf16_to_f32(xb);
-        if (c == 0 && p.tr_x) p.tr_x[static_cast<size_t>(lg) * H + i] = xb;
+      m *= inv;
+      // bf16 rounding of the largest |r * inv| can reach the next power of two: fix_exp leaves one bit for it
+      if (tid < HT) {
+        uint16_t xb[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          xb[u] = f32_to_bf16(rr4[u] * inv);
+          xv[u] = bf16_to_f32(xb[u]);
+        }
+        if (c == 0 && p.tr_x)
+          *reinterpret_cast<uint2*>(p.tr_x + static_cast<size_t>(lg) * H + 4 * tid) =
+              make_uint2(xb[0] | (static_cast<uint32_t>(xb[1]) << 16), xb[2] | (static_cast<uint32_t>(xb[3]) << 16));
       }
+    }
+    const int S = fix_exp(m);
+    const float sx = pow2f(S), isx = pow2f(-S);
+    if (tid < HT) {
+      *reinterpret_cast<float4*>(xn + 4 * tid) = make_float4(xv[0], xv[1], xv[2], xv[3]);
+      // fixed point; this thread's rows 4t..4t+3 give one quad of every byte plane
+      int X[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) X[u] = __float2int_rn(xv[u] * sx);
+      int xs = (X[0] + X[1]) + (X[2] + X[3]);
+      int e[4], qi, sg;
+      if constexpr (BITS == 4) {
+        // rows 4t..4t+3 are positions 4h..4h+3 of word w (h = t & 1) of segment t / 8: thread h = 0
+        // builds the word's even quad (its positions 0, 2 and the partner's 4, 6), h = 1 the odd
+        // quad (the partner's positions 1, 3 and its own 5, 7)
+        const int h = tid & 1;
+        const int r0 = __shfl_xor_sync(0xffffffffu, h ? X[0] : X[1], 1);
+        const int r1 = __shfl_xor_sync(0xffffffffu, h ? X[2] : X[3], 1);
+        e[0] = h ? r0 : X[0];
+        e[1] = h ? r1 : X[2];
+        e[2] = h ? X[1] : r0;
+        e[3] = h ? X[3] : r1;
+        qi = ((tid >> 1) & 3) * 2 + h;
+        sg = tid >> 3;
+      } else {
+        e[0] = X[0];
+        e[1] = X[1];
+        e[2] = X[2];
+        e[3] = X[3];
+        qi = tid & 3;
+        sg = tid >> 2;
+      }
+#pragma unroll
+      for (int j = 0; j < 3; ++j)
+        xq[sg * cv.QSP + j * QW + qi] =
+            xbyte(e[0], j) | (xbyte(e[1], j) << 8) | (xbyte(e[2], j) << 16) | (xbyte(e[3], j) << 24);
+      // PS / 4 threads per segment
+#pragma unroll
+      for (int o = 1; o < PS / 4; o <<= 1) xs += __shfl_xor_sync(0xffffffffu, xs, o);
+      if ((tid & (PS / 4 - 1)) == 0) xq[sg * cv.QSP + cv.QS] = __float_as_uint(static_cast<float>(xs));
     }
     __syncthreads();
-    // x by code segment: xs[(q4 * nsg + s) * 4 + c4] = x[s * PS + o], q4 * 4 + c4 = seg_pos(o)
-#pragma unroll 1
-    for (int i = tid; i < H; i += kThreads) {
-      const int s = i / PS, op = seg_pos<BITS>(i % PS);
-      xs[((op >> 2) * nsg + s) * 4 + (op & 3)] = xn[i];
-    }
     if (tid == kThreads - 32 && l + 1 < p.L) issue_router(l + 1);  // a warp without router rows
     stamp(1);
 
@@ -338,22 +528,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
       if (!mbar_ready(&bar_r[l & 1], (l >> 1) & 1, p.hdr, 10)) ab = true;
       const int row = c + warp * G;
       const uint4* wv = reinterpret_cast<const uint4*>(rbuf + (static_cast<size_t>(l & 1) * cv.rr_max + warp) * H);
-      float acc = 0.f;
-#pragma unroll 1
+      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll 4
       for (int s = lane; s < H / 8; s += 32) {
         const uint4 w8 = wv[s];
         const float4 a = reinterpret_cast<const float4*>(xn)[2 * s];
         const float4 b = reinterpret_cast<const float4*>(xn)[2 * s + 1];
-        acc = fmaf(bf16_lo(w8.x), a.x, acc);
-        acc = fmaf(bf16_hi(w8.x), a.y, acc);
-        acc = fmaf(bf16_lo(w8.y), a.z, acc);
-        acc = fmaf(bf16_hi(w8.y), a.w, acc);
-        acc = fmaf(bf16_lo(w8.z), b.x, acc);
-        acc = fmaf(bf16_hi(w8.z), b.y, acc);
-        acc = fmaf(bf16_lo(w8.w), b.z, acc);
-        acc = fmaf(bf16_hi(w8.w), b.w, acc);
+        acc0 = fmaf(bf16_lo(w8.x), a.x, acc0);
+        acc1 = fmaf(bf16_hi(w8.x), a.y, acc1);
+        acc2 = fmaf(bf16_lo(w8.y), a.z, acc2);
+        acc3 = fmaf(bf16_hi(w8.y), a.w, acc3);
+        acc0 = fmaf(bf16_lo(w8.z), b.x, acc0);
+        acc1 = fmaf(bf16_hi(w8.z), b.y, acc1);
+        acc2 = fmaf(bf16_lo(w8.w), b.z, acc2);
+        acc3 = fmaf(bf16_hi(w8.w), b.w, acc3);
       }
-      acc = warp_sum(acc);
+      const float acc = warp_sum((acc0 + acc1) + (acc2 + acc3));
       const LayerDesc& Ld = s_layers[l];
       if (lane < kDecodeReplicas)
         st_word(p.logits + lane * p.logits_rep + row, tag_f32(acc + ((row < E && Ld.rbias) ? Ld.rbias[row] : 0.f), par));
@@ -361,7 +551,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
     if (tid == 0) s_pend.r[l & 1] = -1;
     stamp(2);
 
-    // ---------------- 3. softmax + top-k (every CTA, warp 0)
+    // ---------------- 3. softmax + top-k (every CTA, warp 0), then the unit's copies
+    const LayerDesc& Ld = s_layers[l];
     if (warp == 0) {
       uint32_t wl[kTopPer];
       uint32_t wsg = par;
@@ -394,6 +585,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
       int my_e;
       if (E <= 256) topk_sorted<8>(wl, E, k, lane, my_k, my_e, kmax);
       else topk_sorted<kTopPer>(wl, E, k, lane, my_k, my_e, kmax);
+      // the unit's copies, at once (lane jA holds slot jA's pick). Issuing a routed unit's copies in
+      // the round that picks its expert, or the shared expert's one layer ahead, measured slower:
+      // their traffic delays the other CTAs' polls of the logits
+      if (has_unit && !__any_sync(0xffffffffu, ab))  // warp-uniform: issue_unit has __syncwarp
+        issue_unit(Ld, l, u_routed ? __shfl_sync(0xffffffffu, my_e, jA) : 0);
       const float mx = fkey_inv(kmax);
       float z = 0.f;
       if (!p.renorm) {  // softmax over all E: the words are re-read (complete and tagged by now)
@@ -415,116 +611,55 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
     }
     if (__syncthreads_or(ab)) { leave(); return; }
     stamp(3);
-
-    // ---------------- 4a. the unit's gate/up code rows: bulk copies by warp 0 (lane = batch,
-    // segment, gate|up), issued after the barrier that publishes the selection; its gate/up
-    // scales and biases: one 16-byte load per thread into shared memory; its down codes (tensor
-    // tiles) and the expert's down scales and biases (bulk copies): thread 32
-    const LayerDesc& Ld = s_layers[l];
-    if (warp == 0) {
-      // the buffer was last read and written by ordinary loads and per-thread copies
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      const int b = lane >> 2, sg = (lane >> 1) & 1, gu = lane & 1;
-      const int lo = max(sg == 0 ? 0 : nA, b * kBatch);
-      const int hi = min(sg == 0 ? nA : npc, b * kBatch + kBatch);
-      if (b < kMaxBatches && hi > lo) {
-        const int j = jA + sg;
-        const bool routed = j < k;
-        const QMat& m = routed ? Ld.gu : Ld.sgu;
-        const int Ij = routed ? I : Is;
-        const int row = (sg == 0 ? iA : -nA) + lo;
-        const uint8_t* src = m.q + static_cast<size_t>(routed ? s_idx[j] : 0) * m.q_stride +
-                             static_cast<size_t>(gu * Ij + row) * rowb;
-        copy_tx(dbuf + static_cast<size_t>(gu * cv.npc_max + lo) * rowb, src, static_cast<uint32_t>((hi - lo) * rowb),
-                &bar_gc[b]);
-      }
-      __syncwarp();
-      if (lane == 0) {
-#pragma unroll 1
-        for (int bb = 0; bb < nb; ++bb) mbar_arrive1(&bar_gc[bb]);
-        s_pend.gc = l & 1;
-      }
-      __syncwarp();
-    }
-    {
-      // scales and biases, in 16-byte chunks q = (kind * npc + pair) * cpr + part;
-      // kind 0/1 gate/up scales, 2/3 gate/up biases
-      const int cpr = ng >> 3;
-      const int per_kind = npc * cpr;
-#pragma unroll 1
-      for (int q = tid; q < 4 * per_kind; q += kThreads) {
-        const int kind = q / per_kind, rem = q - kind * per_kind;
-        const int pair = rem / cpr, part = rem - pair * cpr;
-        const int sg = pair < nA ? 0 : 1;
-        const int j = jA + sg;
-        const bool routed = j < k;
-        const QMat& m = routed ? Ld.gu : Ld.sgu;
-        const int Ij = routed ? I : Is;
-        const int row = sg == 0 ? iA + pair : pair - nA;
-        const uint16_t* src = ((kind & 2) ? m.b : m.s) + static_cast<size_t>(routed ? s_idx[j] : 0) * m.sb_stride +
-                              static_cast<size_t>((kind & 1) * Ij + row) * ng + part * 8;
-        *reinterpret_cast<uint4*>(gsb + static_cast<size_t>(kind * cv.npc_max + pair) * ng + part * 8) =
-            __ldg(reinterpret_cast<const uint4*>(src));
-      }
-    }
-    if (!p.split_late && tid == 32 && npc > 0) issue_down(Ld, l);
-    {
+    if (tid >= 32) {
       // this CTA's slice of the accumulators of layer l + 1
       const int nz = kDecodeReplicas * p.yrep;
       uint32_t* zb = reinterpret_cast<uint32_t*>(p.yacc + static_cast<size_t>((l + 1) % kDecodeYBufs) * p.ybuf_stride);
       const int z1 = static_cast<int>(static_cast<int64_t>(c + 1) * nz / G);
 #pragma unroll 1
-      for (int i = static_cast<int>(static_cast<int64_t>(c) * nz / G) + tid; i < z1; i += kThreads) st_word(zb + i, 0u);
+      for (int i = static_cast<int>(static_cast<int64_t>(c) * nz / G) + tid - 32; i < z1; i += kThreads - 32)
+        st_word(zb + i, 0u);
     }
-    __syncthreads();  // the gate/up scales are in shared memory
 
-    // ---------------- 4b. gate/up rows + SwiGLU, batch by batch as the codes land
-    {
-      float xv[CH][PS];
+    // ---------------- 4. gate/up rows + SwiGLU, batch by batch as the codes land
+    if (has_unit) {
+      uint32_t xr[CH][3 * QW];  // this lane's segments of X, by byte plane
       float xsm[CH];
 #pragma unroll
       for (int ch = 0; ch < CH; ++ch) {
         const int s = gs0 + 32 * ch;
-        float a = 0.f;
 #pragma unroll
-        for (int q4 = 0; q4 < PS / 4; ++q4) {
-          const float4 f = reinterpret_cast<const float4*>(xs)[q4 * nsg + s];
-          xv[ch][4 * q4] = f.x;
-          xv[ch][4 * q4 + 1] = f.y;
-          xv[ch][4 * q4 + 2] = f.z;
-          xv[ch][4 * q4 + 3] = f.w;
-          a += (f.x + f.y) + (f.z + f.w);
-        }
-        xsm[ch] = a;
+        for (int q = 0; q < 3 * QW; ++q) xr[ch][q] = xq[s * cv.QSP + q];
+        xsm[ch] = __uint_as_float(xq[s * cv.QSP + cv.QS]);
       }
 #pragma unroll 1
-      for (int b = 0; b < nb; ++b) {
-        const int lo = b * kBatch, n = min(kBatch, npc - lo);
-        if (warp * rps >= 2 * n) continue;  // no row of this batch for this warp
+      for (int b = 0; b < kNB; ++b) {
+        if (warp * rps >= 2 * kBatch) continue;  // no row of this batch for this warp
         if (!mbar_ready(&bar_gc[b], l & 1, p.hdr, 12)) ab = true;
+        if (b == 0) stamp(4);
         // two rows of the batch at a time (rows rw and rw + 16 * rps), for independent work in flight
 #pragma unroll 1
-        for (int rw = warp * rps; rw < 2 * n; rw += 2 * kWarps * rps) {
+        for (int rw = warp * rps; rw < 2 * kBatch; rw += 2 * kWarps * rps) {
           float acc[2];
-          int qv[2], guv_i[2];
+          int gi[2];
 #pragma unroll
           for (int r2 = 0; r2 < 2; ++r2) {
-            const int rho = rw + r2 * kWarps * rps + gsub;  // [0, n) gate rows, [n, 2n) up rows of the batch
-            const int gu = rho >= n ? 1 : 0;
-            const int q = lo + rho - gu * n;
-            qv[r2] = rho < 2 * n ? q : -1;
-            guv_i[r2] = gu * cv.npc_max + q;
+            const int rho = rw + r2 * kWarps * rps + gsub;  // [0, 16) gate rows, [16, 32) up rows of the batch
+            const int gu = rho >= kBatch ? 1 : 0;
+            const int q = b * kBatch + rho - gu * kBatch;  // pair within the unit
+            gi[r2] = rho < 2 * kBatch ? gu * kUnit + q : -1;
             acc[r2] = 0.f;
-            if (rho < 2 * n) {
-              const unsigned char* row = dbuf + static_cast<size_t>(gu * cv.npc_max + q) * rowb;
-              const uint16_t* sc = gsb + static_cast<size_t>(gu * cv.npc_max + q) * ng;
-              const uint16_t* bi = gsb + static_cast<size_t>((2 + gu) * cv.npc_max + q) * ng;
+            if (rho < 2 * kBatch) {
+              const unsigned char* row = gcd + static_cast<size_t>(gu * kUnit + q) * rowb;
+              const uint16_t* sc = gsb + static_cast<size_t>(gu * kUnit + q) * ng;
+              const uint16_t* bi = gsb + static_cast<size_t>((2 + gu) * kUnit + q) * ng;
 #pragma unroll
               for (int ch = 0; ch < CH; ++ch) {
                 const int s = gs0 + 32 * ch;
                 const uint4 cd = *reinterpret_cast<const uint4*>(row + 16 * s);
                 const int g = (s * PS) >> lgG;
-                acc[r2] = fmaf(bf16_to_f32(sc[g]), dot_seg_dec<BITS>(cd, xv[ch]), fmaf(bf16_to_f32(bi[g]), xsm[ch], acc[r2]));
+                const float d = seg_dot<BITS>(cd, xr[ch] + 2 * QW, xr[ch] + QW, xr[ch]);
+                acc[r2] = fmaf(bf16_to_f32(sc[g]), d, fmaf(bf16_to_f32(bi[g]), xsm[ch], acc[r2]));
               }
             }
           }
@@ -542,8 +677,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
             }
           }
           if (gs0 == 0) {
-            if (qv[0] >= 0) guv[guv_i[0]] = acc[0];
-            if (qv[1] >= 0) guv[guv_i[1]] = acc[1];
+            if (gi[0] >= 0) guv[gi[0]] = acc[0] * isx;
+            if (gi[1] >= 0) guv[gi[1]] = acc[1] * isx;
+          }
+        }
+        if (p.split_late && b == 0) {
+          // mid-copy mode: the last warp done with the first batch's rows issues the down copies
+          // into their space (the other warps go on with the second batch)
+          __syncwarp();
+          if (lane == 0) {
+            __threadfence_block();
+            const int nw0 = min(kWarps, cdiv(2 * kBatch, rps));
+            if (atomicAdd(&s_b0, 1) == nw0 - 1) {
+              __threadfence_block();
+              s_b0 = 0;
+              issue_down(s_layers[l], l, u_routed ? s_idx[jA] : 0);
+            }
           }
         }
       }
@@ -551,31 +700,42 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
     const bool gu_failed = __syncthreads_or(ab);
     if (tid == 0) s_pend.gc = -1;
     if (gu_failed) { leave(); return; }
-    if (tid < npc) hl[(tid & ~15) | seg_pos<BITS>(tid & 15)] = silu_f(guv[tid]) * guv[cv.npc_max + tid];
-    if (p.split_late && tid == 32 && npc > 0) issue_down(s_layers[l], l);  // into the freed gate/up buffer
-    if (npc > 0 && tid < HT && !mbar_ready(&bar_dn, l & 1, p.hdr, 13)) ab = true;
+    if (has_unit && warp == 0) {
+      // SwiGLU, then the unit's h in fixed point (its own exponent) as quads for the down rows
+      const float h = silu_f(guv[lane]) * guv[kUnit + lane];
+      const int Sh = fix_exp(warp_max(fabsf(h)));
+      const int X = __float2int_rn(h * pow2f(Sh));
+      int hs = X;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) hs += __shfl_xor_sync(0xffffffffu, hs, o);
+      // one down row of the unit = 32 codes: 4-bit, one segment of 8 quads; 8-bit, two segments of 4
+      const int qp = (BITS == 4) ? quad_pos<4>(lane) : lane;
+      unsigned char* hqb = reinterpret_cast<unsigned char*>(hq);
+#pragma unroll
+      for (int j = 0; j < 3; ++j) hqb[(j * 8 + (qp >> 2)) * 4 + (qp & 3)] = static_cast<unsigned char>(xbyte(X, j));
+      if (lane == 0) {
+        s_hx[0] = static_cast<float>(hs);
+        s_hx[1] = pow2f(-Sh);
+      }
+    }
+    if (has_unit && tid < HT && !mbar_ready(&bar_dn, l & 1, p.hdr, 13)) ab = true;
     if (__syncthreads_or(ab)) { leave(); return; }
     if (tid == 0) s_pend.dn = -1;
-    stamp(4);
+    stamp(5);
 
-    // ---------------- 5. the unit's partial of y for rows t, t + 512, t + 1024, t + 1536 (a warp
-    // reads 32 consecutive rows of codes, and reduces into 32 consecutive words of y):
-    // routing weight x (scale x codes . h + bias x sum h)
-    if (npc > 0) {
-      float hv[kUnit];
-      float hsum = 0.f;
+    // ---------------- 5. the unit's partial of y for rows t, t + 512, ... (a warp reads 32
+    // consecutive rows of codes, and reduces into 32 consecutive words of y):
+    // routing weight x 2^-S_h x (scale x codes . X_h + bias x sum X_h)
+    if (has_unit) {
+      uint32_t hr[kQ];
 #pragma unroll
-      for (int q4 = 0; q4 < kUnit / 4; ++q4) {
-        const float4 f = reinterpret_cast<const float4*>(hl)[q4];
-        hv[4 * q4] = f.x;
-        hv[4 * q4 + 1] = f.y;
-        hv[4 * q4 + 2] = f.z;
-        hv[4 * q4 + 3] = f.w;
-        hsum += (f.x + f.y) + (f.z + f.w);
-      }
-      const float wgt = u_routed ? s_w[jA] : s_sg;
-      const uint16_t* dsc = reinterpret_cast<const uint16_t*>(dss);
-      const uint16_t* dbi = dsc + static_cast<size_t>(H) * ngd;
+      for (int q = 0; q < kQ; ++q) hr[q] = hq[q];
+      const float hsX = s_hx[0];
+      const float wgt = (u_routed ? s_w[jA] : s_sg) * s_hx[1];
+      const LayerDesc& Ld5 = s_layers[l];
+      const bool gm = (u_routed ? Ld5.dsb : Ld5.sdsb) != nullptr;
+      const QMat& dm = u_routed ? Ld5.dn : Ld5.sdn;
+      const size_t sb0 = static_cast<size_t>(u_routed ? s_idx[jA] : 0) * dm.sb_stride + u_g;
       float* yrow = p.yacc + static_cast<size_t>(l % kDecodeYBufs) * p.ybuf_stride +
                     static_cast<size_t>(c % kDecodeReplicas) * p.yrep;
 #pragma unroll
@@ -583,22 +743,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
         const int r = tid + q * kThreads;
         if (r < H) {
           float d;
+          const unsigned char* drow = r < H2 ? dcd + r * cv.UB : dhi + (r - H2) * cv.UB;
           if constexpr (BITS == 4) {
-            d = dot_seg_dec<4>(*reinterpret_cast<const uint4*>(dcd + r * cv.UB), hv);
+            d = seg_dot<4>(*reinterpret_cast<const uint4*>(drow), hr + 16, hr + 8, hr);
           } else {
-            d = dot_seg<8>(*reinterpret_cast<const uint4*>(dcd + r * cv.UB), hv) +
-                dot_seg<8>(*reinterpret_cast<const uint4*>(dcd + r * cv.UB + 16), hv + 16);
+            d = seg_dot<8>(*reinterpret_cast<const uint4*>(drow), hr + 16, hr + 8, hr) +
+                seg_dot<8>(*reinterpret_cast<const uint4*>(drow + 16), hr + 20, hr + 12, hr + 4);
           }
-          red_add(yrow + r, wgt * fmaf(bf16_to_f32(dsc[r * ngd + u_g]), d, bf16_to_f32(dbi[r * ngd + u_g]) * hsum));
+          float sc, bi;
+          if (gm) {
+            const uint32_t sbw = dsb[r];
+            sc = bf16_lo(sbw);
+            bi = bf16_hi(sbw);
+          } else {
+            sc = bf16_to_f32(__ldg(dm.s + sb0 + static_cast<size_t>(r) * cv.ngd));
+            bi = bf16_to_f32(__ldg(dm.b + sb0 + static_cast<size_t>(r) * cv.ngd));
+          }
+          red_add(yrow + r, wgt * fmaf(sc, d, bi * hsX));
         }
       }
     }
     if (__syncthreads_or(ab)) { leave(); return; }
-    if (tid == 0) {
-      __threadfence();  // this CTA's reductions and zeroes, ordered by the barrier, before its arrival
-      atomicAdd(p.arrive, 1u);
-    }
+
     stamp(6);
+    // the arrival: a release reduction (this CTA's reductions and zeroes, ordered before it by
+    // the barrier, are visible to whoever acquires the count)
+    if (tid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.arrive) : "memory");
+    stamp(7);
   }
 
   // ---------------- the stack's output: residual + RMSNorm after the last layer (CTA 0)
@@ -612,23 +783,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const uint16_t yb = f32_to_bf16(y[u]);
-        const float v = rr[4 * tid + u] + bf16_to_f32(yb);
-        rr[4 * tid + u] = v;
-        ss = fmaf(v, v, ss);
+        rr4[u] += bf16_to_f32(yb);
+        ss = fmaf(rr4[u], rr4[u], ss);
         if (p.tr_y) p.tr_y[static_cast<size_t>(p.l0 + p.L - 1) * H + 4 * tid + u] = yb;
       }
     }
-    ss = warp_sum(ss);
-    if (lane == 0) s_red[warp] = ss;
-    __syncthreads();
-    float tot = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) tot += s_red[w];
+    float tot, unused;
+    block_sum_max(ss, 0.f, tot, unused);
     const float inv = 1.f / sqrtf(tot / static_cast<float>(H) + p.eps);
-#pragma unroll 1
-    for (int i = tid; i < H; i += kThreads) {
-      p.out[i] = f32_to_bf16(rr[i] * inv);
-      if (p.r_out) p.r_out[i] = rr[i];
+    if (tid < HT) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        p.out[4 * tid + u] = f32_to_bf16(rr4[u] * inv);
+        if (p.r_out) p.r_out[4 * tid + u] = rr4[u];
+      }
     }
   }
   leave();
@@ -658,15 +826,15 @@ bool decode_split_plan(int H, int E, int k, int I, int Is, int group, int bits, 
   if (L > kMaxDecodeLayers) L = kMaxDecodeLayers;
   const int PS = 128 / bits;
   const int nsg = H / PS;
-  if (H % PS || H > 2048 || H % kBoxRows) return false;  // x of a lane's segments in registers; whole tiles
+  if (H % PS || H > 4 * kThreads || H % kBoxRows) return false;  // rows 4t..4t+3 per thread; whole tiles
   if (!(pow2(nsg) && nsg <= 32) && !(nsg % 32 == 0 && nsg / 32 <= (bits == 4 ? 2 : 4))) return false;
   if (Is != 0 && Is != I) return false;          // one down row length (and scale row) for every slot
   if (I % kUnit || !pow2(group) || group % kUnit || I % group) return false;  // a unit lies in one group
-  if ((H / group) % 8 != 0) return false;        // gate/up scale rows are whole 16-byte chunks
   if (k > 16 || E > 32 * kTopPer) return false;
   if ((k * I + Is) / kUnit > grid) return false;  // at most one unit per CTA
   if (cdiv(E + (Is > 0 ? 1 : 0), grid) > kWarps) return false;  // one router row per warp
-  for (int lt = 0; lt < 2; ++lt) {  // down data in a region of its own if it fits, else after gate/up
+  for (int lt = 0; lt < 2; ++lt) {  // down codes in a region of their own if they fit, else mid-copy mode
+    if (lt == 1 && H % (2 * kBoxRows)) break;  // the halves hold whole 256-row tiles
     const size_t need = carve(H, E, I, Is, group, bits, grid, L, lt).total;
     if (need <= smem_limit) {
       *smem = need;

@@ -44,7 +44,8 @@ class QTensor(ctypes.Structure):
 
 class LayerWeights(ctypes.Structure):
     _fields_ = [("router_w", P), ("router_bias", P), ("gate_up", QTensor), ("down", QTensor),
-                ("shared_gate_up", QTensor), ("shared_down", QTensor), ("shared_gate_w", P)]
+                ("shared_gate_up", QTensor), ("shared_down", QTensor), ("shared_gate_w", P),
+                ("down_sb", P), ("shared_down_sb", P), ("down_units", P), ("shared_down_units", P)]
 
 
 class Trace(ctypes.Structure):
@@ -69,6 +70,12 @@ def lib() -> ctypes.CDLL:
         L.moe_stack_forward.argtypes = [CP, LP, I32, P, I32, P, ctypes.POINTER(Trace), P, ctypes.c_size_t, P]
         L.moe_sort_by_expert.argtypes = [CP, P, I32, P, P, P, ctypes.c_size_t, P]
         L.moe_layer_forward_static.argtypes = [CP, LP, P, I32, P, P, P, P, P]
+        L.moe_down_sb_size.argtypes = [CP, I32, I32]
+        L.moe_down_sb_size.restype = ctypes.c_size_t
+        L.moe_prepare_down_sb.argtypes = [CP, ctypes.POINTER(QTensor), I32, I32, P, P]
+        L.moe_down_units_size.argtypes = [CP, I32, I32]
+        L.moe_down_units_size.restype = ctypes.c_size_t
+        L.moe_prepare_down_units.argtypes = [CP, ctypes.POINTER(QTensor), I32, I32, P, P]
         L.moe_stack_kernel_launches.argtypes = [CP, I32, I32]
         L.moe_stack_kernel_launches.restype = I32
         L.moe_stack_path_name.argtypes = [CP, I32, I32]
@@ -125,10 +132,67 @@ def _qtensor(qt) -> QTensor:
                    qt.q.stride(0) * qt.q.element_size(), qt.scales.stride(0))
 
 
-def make_layer_weights(lw) -> LayerWeights:
-    """LayerWeights struct over a synth.LayerWeights (the caller keeps lw alive)."""
+def moe_down_sb_size(cfg: Config, n_experts: int, K: int) -> int:
+    return int(lib().moe_down_sb_size(ctypes.byref(cfg), int(n_experts), int(K)))
+
+
+def moe_prepare_down_sb(cfg: Config, qt, out: torch.Tensor, stream=None):
+    """Group-major (scale, bias) copy of a down tensor (synth.QTensor [n][H][K]) into out
+    (uint8 device tensor of moe_down_sb_size bytes)."""
+    n, K = qt.q.shape[0], qt.K
+    if out.numel() * out.element_size() < moe_down_sb_size(cfg, n, K):
+        raise MoEError(MOE_ERR_INVALID_ARG, "out is smaller than moe_down_sb_size")
+    q = _qtensor(qt)
+    _check(lib().moe_prepare_down_sb(ctypes.byref(cfg), ctypes.byref(q), n, K, out.data_ptr(), _stream(stream)))
+
+
+def moe_down_units_size(cfg: Config, n_experts: int, K: int) -> int:
+    return int(lib().moe_down_units_size(ctypes.byref(cfg), int(n_experts), int(K)))
+
+
+def moe_prepare_down_units(cfg: Config, qt, out: torch.Tensor, stream=None):
+    """Unit-major copy of a down tensor's codes (synth.QTensor [n][H][K]) into out
+    (uint8 device tensor of moe_down_units_size bytes)."""
+    n, K = qt.q.shape[0], qt.K
+    if out.numel() * out.element_size() < moe_down_units_size(cfg, n, K):
+        raise MoEError(MOE_ERR_INVALID_ARG, "out is smaller than moe_down_units_size")
+    q = _qtensor(qt)
+    _check(lib().moe_prepare_down_units(ctypes.byref(cfg), ctypes.byref(q), n, K, out.data_ptr(), _stream(stream)))
+
+
+def prepare_layer(cfg: Config, lw):
+    """The decode-ready down copies of a layer on the GPU (made once, kept on lw):
+    (down_sb, shared_down_sb, down_units, shared_down_units) as uint8 device tensors
+    (the shared ones None without a shared expert)."""
+    got = lw.__dict__.get("_decode_copies")
+    if got is None:
+        dev = lw.down.q.device
+        n, K = lw.down.q.shape[0], lw.down.K
+        dsb = torch.empty(moe_down_sb_size(cfg, n, K), dtype=torch.uint8, device=dev)
+        moe_prepare_down_sb(cfg, lw.down, dsb)
+        dcu = torch.empty(moe_down_units_size(cfg, n, K), dtype=torch.uint8, device=dev)
+        moe_prepare_down_units(cfg, lw.down, dcu)
+        sdsb = sdcu = None
+        if lw.shared_down is not None and cfg.shared_inter > 0:
+            sdsb = torch.empty(moe_down_sb_size(cfg, 1, lw.shared_down.K), dtype=torch.uint8, device=dev)
+            moe_prepare_down_sb(cfg, lw.shared_down, sdsb)
+            sdcu = torch.empty(moe_down_units_size(cfg, 1, lw.shared_down.K), dtype=torch.uint8, device=dev)
+            moe_prepare_down_units(cfg, lw.shared_down, sdcu)
+        got = (dsb, sdsb, dcu, sdcu)
+        lw.__dict__["_decode_copies"] = got
+    return got
+
+
+def make_layer_weights(lw, cfg: Optional[Config] = None) -> LayerWeights:
+    """LayerWeights struct over a synth.LayerWeights (the caller keeps lw alive). With cfg
+    given and the weights on the GPU, the group-major down scale/bias copies the single-token
+    decode reads are made once (prepare_layer) and referenced too."""
+    dsb = sdsb = dcu = sdcu = None
+    if cfg is not None and lw.down.q.is_cuda:
+        dsb, sdsb, dcu, sdcu = prepare_layer(cfg, lw)
     return LayerWeights(lw.router_w.data_ptr(), _p(lw.router_bias), _qtensor(lw.gate_up), _qtensor(lw.down),
-                        _qtensor(lw.shared_gate_up), _qtensor(lw.shared_down), _p(lw.shared_gate_w))
+                        _qtensor(lw.shared_gate_up), _qtensor(lw.shared_down), _p(lw.shared_gate_w),
+                        _p(dsb), _p(sdsb), _p(dcu), _p(sdcu))
 
 
 class Workspace:

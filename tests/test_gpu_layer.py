@@ -190,7 +190,7 @@ def test_largest_supported_shape():
     host = DeviceLayer(shape, lw)
     ids, x = gap_filtered_tokens(shape, host, 3, "cuda")
     idx, w, y = _run_layer(shape, lw, x)
-    st = check_tokens(host, bits(x), idx, w, y, range(3), "max", threads=8, ulp_floor=True)
+    st = check_tokens(host, bits(x), idx, w, y, range(3), "max", threads=8)
     print(f"max shape: max-abs {st.max_abs:.2e} rel-L2 {st.max_rel_l2:.2e}")
     del lw
     torch.cuda.empty_cache()

@@ -32,7 +32,13 @@ def _with_workspace(cfg, W, x, shape):
     return idx.cpu().numpy(), w.cpu().numpy(), bits(y)
 
 
-@pytest.mark.parametrize("key,T", [("tiny", 16), ("35b", 8)])
+# The largest token count the 2 MiB static scratch admits at the 35b shape
+# (H=2048, E=256, k=8, I=Is=512): the per-token regions of the workspace
+# layout for 46 tokens take 2,063,360 bytes, for 47 tokens 2,103,296.
+T_MAX_35B = 46
+
+
+@pytest.mark.parametrize("key,T", [("tiny", 16), ("35b", 8), ("35b", T_MAX_35B)])
 def test_static_scratch_call_matches_workspace_call(key, T):
     shape = synth.SHAPES[key]
     lw = synth.make_layer(shape, 0, "cuda")
@@ -58,14 +64,17 @@ def test_static_scratch_call_matches_workspace_call(key, T):
             assert max_abs <= Y_MAX_ABS and rel <= Y_REL_L2, f"call {call} token {t}"
 
 
-def test_static_scratch_rejects_too_many_tokens():
-    shape = synth.SHAPES["tiny"]
+@pytest.mark.parametrize("key,T", [("35b", T_MAX_35B + 1), ("tiny", 4096)])
+def test_static_scratch_rejects_too_many_tokens(key, T):
+    """One token past the limit is refused before anything is enqueued (the
+    35b case is the boundary itself; T_MAX_35B passes above)."""
+    shape = synth.SHAPES[key]
     lw = synth.make_layer(shape, 0, "cuda")
     cfg = moe.make_config(shape)
-    T = 4096
-    assert moe.moe_workspace_size(cfg, T) > (2 << 20)
     x = torch.zeros(T, shape.hidden, dtype=torch.bfloat16, device="cuda")
-    y = torch.empty_like(x)
+    y = torch.full_like(x, 7.0)
     with pytest.raises(moe.MoEError) as ei:
         moe.moe_layer_forward_static(cfg, moe.make_layer_weights(lw), x, y, None, None)
     assert ei.value.status == moe.MOE_ERR_WORKSPACE and "static scratch" in str(ei.value)
+    torch.cuda.synchronize()
+    assert bool((y == 7.0).all()), "a refused call must not write its output"
