@@ -202,39 +202,83 @@ def host_layers_for(shape, layers_dev, tokens_bits):
     return hosts
 
 
-def cpu_oracle_tokens_per_s(shape, layers_dev, x_tokens, threads: int, budget_s: float = 12.0):
-    """The oracle (as it stands) on a bounded sample of the workload: tokens
-    through all layers, one layer at a time, until `budget_s` of CPU time is
-    spent. Only the oracle calls are timed. Returns (tokens/s, evaluations, seconds)."""
+def traced_stack(shape, cfg, arr, ws, x0):
+    """One token through the stack with a trace: the GPU's own input, selection and output of
+    every layer (outside any timing)."""
+    L, H, k = shape.layers, shape.hidden, shape.top_k
+    tx = torch.empty(L, 1, H, dtype=torch.bfloat16, device="cuda")
+    ti = torch.empty(L, 1, k, dtype=torch.int32, device="cuda")
+    tw = torch.empty(L, 1, k, dtype=torch.float32, device="cuda")
+    ty = torch.empty(L, 1, H, dtype=torch.bfloat16, device="cuda")
+    xo = torch.empty(1, H, dtype=torch.bfloat16, device="cuda")
+    moe.moe_stack_forward(cfg, arr, x0, xo, ws, trace=moe.Trace(tx.data_ptr(), ti.data_ptr(), tw.data_ptr(),
+                                                               ty.data_ptr()))
+    torch.cuda.synchronize()
+    return synth.bf16_bits(tx), ti.cpu().numpy(), tw.cpu().numpy(), synth.bf16_bits(ty)
+
+
+def cpu_oracle_leg(shape, cfg, arr, ws, layers_dev, x_tokens, threads: int, budget_s: float = 12.0):
+    """The oracle (as it stands) on a bounded sample of the workload, timed on the host cores:
+    (token, layer) evaluations on the GPU's own input of that layer (from a traced run of the
+    same token), until `budget_s` of oracle time is spent. Only the oracle calls are timed.
+    Each evaluation is also compared with the GPU's output of that layer: the same three checks
+    the GPU tests apply (expert set where the k-th/(k+1)-th logit gap exceeds 1e-4, weights within
+    1e-5, bf16 output within max-abs 2e-2 and rel-L2 1e-3 of the oracle's rounded output).
+    Returns (tokens/s, evaluations, seconds, parity summary)."""
+    import numpy as np
     import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from parity import GAP_MIN, W_TOL, Y_MAX_ABS, Y_REL_L2, y_errors
     spent, evals = 0.0, 0
+    par = {"pairs": 0, "gap_excluded": 0, "index_mismatch": 0, "max_w_err": 0.0, "max_abs": 0.0,
+           "max_rel_l2": 0.0}
     for i in range(x_tokens.shape[0]):
-        x = synth.bf16_bits(x_tokens[i:i + 1])
+        tx, ti, tw, ty = traced_stack(shape, cfg, arr, ws, x_tokens[i:i + 1])
         for l0 in range(0, shape.layers, 8):
-            hosts = host_layers_for(shape, layers_dev[l0:l0 + 8], [x])
-            for h in hosts:
+            hosts = host_layers_for(shape, layers_dev[l0:l0 + 8], [tx[l] for l in range(l0, min(l0 + 8, shape.layers))])
+            for dl, h in enumerate(hosts):
+                l = l0 + dl
                 t0 = time.perf_counter()
-                oracle.layer_forward(h, x, threads=threads)
+                ref = oracle.layer_forward(h, tx[l], threads=threads)
                 spent += time.perf_counter() - t0
                 evals += 1
+                par["pairs"] += 1
+                gi = ti[l][0].astype(np.int64)
+                if ref["gap"][0] > GAP_MIN:
+                    if set(gi.tolist()) != set(ref["idx"][0].tolist()):
+                        par["index_mismatch"] += 1
+                    else:
+                        rw = dict(zip(ref["idx"][0].tolist(), ref["w"][0].tolist()))
+                        par["max_w_err"] = max(par["max_w_err"], max(abs(float(tw[l][0][j]) - rw[int(gi[j])])
+                                                                     for j in range(len(gi))))
+                else:
+                    par["gap_excluded"] += 1
+                    ref = oracle.layer_forward(h, tx[l], force_idx=ti[l], threads=threads)
+                ma, rel, _ = y_errors(ty[l][0], ref)
+                par["max_abs"] = max(par["max_abs"], ma)
+                par["max_rel_l2"] = max(par["max_rel_l2"], rel)
             if spent >= budget_s:
                 break
         if spent >= budget_s:
             break
+    par["pass"] = bool(par["index_mismatch"] == 0 and par["max_w_err"] <= W_TOL and par["max_abs"] <= Y_MAX_ABS
+                       and par["max_rel_l2"] <= Y_REL_L2)
     per_token = spent / evals * shape.layers
-    return 1.0 / per_token, evals, spent
+    return 1.0 / per_token, evals, spent, par
 
 
 def run_reference(args):
-    """Reference arm: the CPU oracle timed on this host (rank 0 only)."""
+    """Reference arm: the CPU oracle timed on this host (rank 0 only). Each step is a bounded
+    sample of the workload (one token through `n_layers` of its layers); `ms_per_step` is the
+    measured time of that sample and `value` scales it to the whole stack."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import oracle
     shape = synth.SHAPES[SHAPE_KEY]
-    threads = os.cpu_count() or 1
+    cores = os.cpu_count() or 1
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    threads = min(threads, shape.top_k + 1)  # the oracle runs one expert per thread
+    threads = min(cores, shape.top_k + 1)  # the oracle runs one expert per thread
     n_layers = 2
     layers = [synth.make_layer(shape, l, dev) for l in range(n_layers)]
     tokens = synth.make_tokens(shape, list(range(args.warmup + args.steps)), dev)
@@ -243,21 +287,30 @@ def run_reference(args):
     for i in range(args.warmup):
         for h in hosts:
             oracle.layer_forward(h, xs[i], threads=threads)
-    t0 = time.perf_counter()
+    per = []
     for i in range(args.warmup, args.warmup + args.steps):
+        t0 = time.perf_counter()
         for h in hosts:
             oracle.layer_forward(h, xs[i], threads=threads)
-    dt = time.perf_counter() - t0
-    sec_per_token = dt / args.steps * (shape.layers / n_layers)
-    value = 1.0 / sec_per_token
-    sample = f"1 token x {n_layers} of {shape.layers} layers per step, scaled to {shape.layers}"
+        per.append(time.perf_counter() - t0)
+    dt = sum(per)
+    sample_ms = dt / args.steps * 1e3
+    scale = shape.layers / n_layers
+    value = 1.0 / (dt / args.steps * scale)
+    sample = (f"1 token x {n_layers} of {shape.layers} layers per step (measured {sample_ms:.1f} ms per step); "
+              f"value scaled by {scale:.0f} to the whole stack")
     out = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec_per_token * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sample_ms,
+        "ms_per_step_note": f"measured time of one sampled step ({n_layers} of {shape.layers} layers); "
+                            f"the whole-stack time per token is {sample_ms * scale:.1f} ms",
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(shape),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "threads": threads, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "step_ms_raw": [round(x * 1e3, 3) for x in per],
+        "seeds": seeds_desc(SHAPE_KEY, list(range(args.warmup, args.warmup + args.steps))),
     }
     print(json.dumps(out), flush=True)
 
@@ -271,6 +324,117 @@ def workload_config(shape):
                   "resident expert stack, a new token (new experts) every step"}
 
 
+def seeds_desc(key, token_ids):
+    cid = synth.SHAPE_SEED_ID[key]
+    return {"weights": f"tensor t of layer l: {cid}*1000003 + l*1009 + t (synth.layer_seed)",
+            "tokens": f"token i: {cid}*1000003 + 999983 + i (synth.token_seed), batch b: token_seed(1000000 + b)",
+            "token_ids": [token_ids[0], token_ids[-1]] if token_ids else []}
+
+
+# The GPU tests that check each workload's path element by element against the oracle.
+PARITY_TESTS = {
+    "35b": "tests/test_gpu_stack.py::test_decode_stack_parity[35b]",
+    "80b": "tests/test_gpu_stack.py::test_decode_stack_parity[80b]",
+    "35b8": "tests/test_gpu_stack.py::test_decode_stack_parity[35b8]",
+    "35b_t64": "tests/test_gpu_stack.py::test_batched_stack_parity[35b_t64]",
+    "35b_t512": "tests/test_gpu_stack.py::test_batched_stack_parity[35b_t512]",
+}
+
+
+class Workload:
+    """One workload's stack on the device, ready to step: weights (with their decode-ready
+    copies), a workspace and the tokens of `nsteps` steps."""
+
+    def __init__(self, key, nsteps, rank=0, layers=0):
+        self.key = key
+        shape = synth.SHAPES[key]
+        if layers:
+            import dataclasses
+            shape = dataclasses.replace(shape, layers=layers, name=shape.name + f"-first{layers}")
+        self.shape = shape
+        self.cfg = moe.make_config(shape)
+        sid = synth.SHAPE_SEED_ID[key]
+        self.layers = [synth.make_layer(shape, l, "cuda", seed_id=sid) for l in range(shape.layers)]
+        self.arr = moe.make_layer_array([moe.make_layer_weights(lw, self.cfg) for lw in self.layers])
+        self.T = shape.tokens
+        self.ws = moe.Workspace(self.cfg, self.T, L=shape.layers)
+        self.token_ids = rank_token_ids(rank, nsteps)
+        if self.T == 1:
+            self.tokens = synth.make_tokens(shape, self.token_ids, "cuda", seed_id=sid)
+        else:
+            self.tokens = torch.cat([synth.make_batch(shape, self.T, i, "cuda", seed_id=sid) for i in self.token_ids])
+        self.xout = torch.empty(self.T, shape.hidden, dtype=torch.bfloat16, device="cuda")
+
+    def step(self, i, stream):
+        T = self.T
+        moe.moe_stack_forward(self.cfg, self.arr, self.tokens[i * T:(i + 1) * T], self.xout, self.ws, stream=stream)
+
+    def path(self):
+        return moe.moe_stack_path_name(self.cfg, self.T, self.shape.layers)
+
+    def launches(self):
+        return moe.moe_stack_kernel_launches(self.cfg, self.T, self.shape.layers)
+
+    def bytes_per_step(self, warmup, steps):
+        if self.T == 1:
+            return touched_bytes_per_token(self.shape)
+        T = self.T
+        return touched_bytes_batched(self.shape, self.layers, self.tokens[warmup * T:(warmup + steps) * T], T, steps)
+
+
+def per_step_ms(wl, first, steps, stream):
+    """Each step between its own events (device time): the raw per-step list."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    evs[0].record(stream)
+    for i in range(first, first + steps):
+        wl.step(i, stream)
+        evs[i - first + 1].record(stream)
+    torch.cuda.synchronize()
+    return [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+
+
+def pct(v):
+    v = sorted(v)
+    return {f"p{q}": v[min(len(v) - 1, int(q / 100 * len(v)))] for q in (10, 50, 90)}
+
+
+def secondary(keys, steps, warmup, peak, budget_s=150.0):
+    """The other workloads, each timed like the headline on its own stack (made, timed and
+    freed in turn), within about budget_s of wall time: tokens/s, algorithmic GB/s and the
+    fraction of the measured copy peak, the per-step spread, the path and its launches."""
+    out = {}
+    t_start = time.time()
+    stream = torch.cuda.current_stream()
+    for key in keys:
+        if time.time() - t_start > budget_s:
+            out[key] = {"skipped": "time budget of the secondary block spent"}
+            continue
+        wl = Workload(key, warmup + steps)
+        for i in range(warmup):
+            wl.step(i, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(warmup, warmup + steps):
+            wl.step(i, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        status = moe.moe_get_device_status(wl.ws)
+        raw = per_step_ms(wl, warmup, steps, stream)
+        b = wl.bytes_per_step(warmup, steps)
+        gbs = b / (ms / 1e3 / steps) / 1e9
+        out[key] = {"workload": workload_config(wl.shape)["workload"], "tokens_per_s": steps * wl.T / (ms / 1e3),
+                    "ms_per_step": ms / steps, "bytes_per_step": b, "hbm_gbs": gbs, "frac_of_measured_peak": gbs / peak,
+                    "frac_of_8tbs": gbs / NOMINAL_HBM_GBS, "step_ms": pct(raw),
+                    "step_ms_raw": [round(x, 4) for x in raw], "path": wl.path(), "launches_per_step": wl.launches(),
+                    "steps": steps, "warmup": warmup, "device_status": moe.status_string(status),
+                    "parity_test": PARITY_TESTS.get(key), "seeds": seeds_desc(key, wl.token_ids)}
+        del wl
+        torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -278,6 +442,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the other workloads' block")
     ap.add_argument("--layers", type=int, default=0,
                     help="profile a shorter stack (small ncu case); the default is the full stack")
     ap.add_argument("--workload", default=SHAPE_KEY, choices=sorted(synth.SHAPES),
@@ -292,33 +457,16 @@ def main():
     dist, rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
     key = args.workload
-    shape = synth.SHAPES[key]
-    if args.layers:
-        import dataclasses
-        shape = dataclasses.replace(shape, layers=args.layers, name=shape.name + f"-first{args.layers}")
-    cfg = moe.make_config(shape)
-    layers = [synth.make_layer(shape, l, "cuda", seed_id=synth.SHAPE_SEED_ID[key])
-              for l in range(shape.layers)]
-    arr = moe.make_layer_array([moe.make_layer_weights(lw, cfg) for lw in layers])
-    T = shape.tokens
-    ws = moe.Workspace(cfg, T, L=shape.layers)
     nsteps = args.warmup + args.steps
     # each rank its own tokens (independent replicas); a step is one batch of T tokens
-    if T == 1:
-        tokens = synth.make_tokens(shape, rank_token_ids(rank, nsteps), "cuda", seed_id=synth.SHAPE_SEED_ID[key])
-    else:
-        tokens = torch.cat([synth.make_batch(shape, T, i, "cuda", seed_id=synth.SHAPE_SEED_ID[key])
-                            for i in rank_token_ids(rank, nsteps)])
-    xout = torch.empty(T, shape.hidden, dtype=torch.bfloat16, device="cuda")
+    wl = Workload(key, nsteps, rank, args.layers)
+    shape, T = wl.shape, wl.T
     stream = torch.cuda.current_stream()
 
-    def step(i):
-        moe.moe_stack_forward(cfg, arr, tokens[i * T:(i + 1) * T], xout, ws, stream=stream)
-
     for i in range(args.warmup):
-        step(i)
+        wl.step(i, stream)
     torch.cuda.synchronize()
-    assert moe.moe_get_device_status(ws) == moe.MOE_OK
+    assert moe.moe_get_device_status(wl.ws) == moe.MOE_OK
 
     # ---- device-timed region: inputs resident in HBM
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -328,27 +476,20 @@ def main():
         torch.cuda.synchronize()
         ev0.record(stream)
         for i in range(args.warmup, nsteps):
-            step(i)
+            wl.step(i, stream)
         ev1.record(stream)
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
     ms = ev0.elapsed_time(ev1)
     ms = barrier_max(dist, ms)
-    status = moe.moe_get_device_status(ws)
+    status = moe.moe_get_device_status(wl.ws)
 
     # ---- the same steps again, each bracketed by its own events: the spread of a step
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    evs[0].record(stream)
-    for i in range(args.warmup, nsteps):
-        step(i)
-        evs[i - args.warmup + 1].record(stream)
-    torch.cuda.synchronize()
-    per = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps))
-    pct = {f"p{q}": per[min(len(per) - 1, int(q / 100 * len(per)))] for q in (10, 50, 90)}
+    raw = per_step_ms(wl, args.warmup, args.steps, stream)
 
     # ---- end to end: host tokens in pinned memory, result read back every step
-    host_tok = tokens.cpu().pin_memory()
+    host_tok = wl.tokens.cpu().pin_memory()
     host_out = torch.empty(T, shape.hidden, dtype=torch.bfloat16).pin_memory()
     xin = torch.empty(T, shape.hidden, dtype=torch.bfloat16, device="cuda")
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -358,19 +499,16 @@ def main():
     e0.record(stream)
     for i in range(args.warmup, nsteps):
         xin.copy_(host_tok[i * T:(i + 1) * T], non_blocking=True)
-        moe.moe_stack_forward(cfg, arr, xin, xout, ws, stream=stream)
-        host_out.copy_(xout, non_blocking=True)
+        moe.moe_stack_forward(wl.cfg, wl.arr, xin, wl.xout, wl.ws, stream=stream)
+        host_out.copy_(wl.xout, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = barrier_max(dist, e0.elapsed_time(e1))
 
-    launches_per_step = moe.moe_stack_kernel_launches(cfg, T, shape.layers)
-    path = moe.moe_stack_path_name(cfg, T, shape.layers)
+    launches_per_step = wl.launches()
+    path = wl.path()
     persistent = launches_per_step < shape.layers
-    if T == 1:
-        bytes_step = touched_bytes_per_token(shape)
-    else:
-        bytes_step = touched_bytes_batched(shape, layers, tokens[args.warmup * T:nsteps * T], T, args.steps)
+    bytes_step = wl.bytes_per_step(args.warmup, args.steps)
     total_tokens = args.steps * world * T
     tok_s = job_tokens_per_s(args.steps, world, T, ms)
     per_step_s = ms / 1e3 / args.steps
@@ -379,21 +517,31 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and T == 1:
-        threads = min(os.cpu_count() or 1, shape.top_k + 1)  # one expert per thread
-        v, evals, dt = cpu_oracle_tokens_per_s(shape, layers, tokens, threads)
-        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"{evals} (token, layer) evaluations of the bench tokens, {dt:.1f} s of oracle time, "
-                         f"scaled to {shape.layers} layers per token; expert copies to the host untimed"}
+        cores = os.cpu_count() or 1
+        threads = min(cores, shape.top_k + 1)  # one expert per thread
+        v, evals, dt, par = cpu_oracle_leg(shape, wl.cfg, wl.arr, wl.ws, wl.layers, wl.tokens[:4], threads)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "threads": threads, "kind": "oracle",
+               "sample": f"{evals} (token, layer) evaluations of the first bench tokens on the GPU's own per-layer "
+                         f"inputs, {dt:.1f} s of oracle time, scaled to {shape.layers} layers per token; expert "
+                         "copies to the host untimed",
+               "parity": par}
 
     traffic = None
     src_hash = kernel_source_hash()
     if persistent and (key, src_hash) in DECODE_TRAFFIC_PER_LAYER:
         traffic = DECODE_TRAFFIC_PER_LAYER[(key, src_hash)] * shape.layers
+    sec = None
+    if world == 1 and not args.no_secondary and not args.layers and key == SHAPE_KEY:
+        del wl
+        torch.cuda.empty_cache()
+        sec = secondary([k for k in ("80b", "35b8", "35b_t64", "35b_t512") if k != key], 32, args.warmup, peak)
     if rank == 0:
         out = {
             "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "weights": f"u{shape.bits} affine g{shape.group}, bf16 scale/bias",
+            "arithmetic": "exact integer byte dot products (dp4a) of the codes with a 22-bit fixed-point copy of the "
+                          "activations, fp32 scale/bias and sums" if path == "decode_split_kernel" else "fp32",
             "data": "synthetic", "config": workload_config(shape),
             "hbm_gbs": gbs, "hbm_frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm",
@@ -401,16 +549,22 @@ def main():
                                     else f"moe_stack_forward step on the {path} path (all its kernels)"),
                          "achieved": gbs, "peak": peak, "peak_source": peak_src, "unit": "GB/s",
                          "frac": gbs / peak, "traffic": traffic,
+                         "traffic_note": None if traffic is not None else
+                         f"no ncu capture of this kernel revision (source hash {src_hash})",
                          "bytes_per_step": bytes_step,
                          "note": "achieved = algorithmic bytes per step / device time per step (CUDA events "
                                  "on the launch stream around the timed steps)"},
             "cpu_baseline": cpu,
             "e2e": {"value": total_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * shape.hidden * 2, "d2h_bytes_per_step": T * shape.hidden * 2},
-            "step_ms": pct,
+            "step_ms": pct(raw),
+            "step_ms_raw": [round(x, 4) for x in raw],
+            "seeds": seeds_desc(key, wl.token_ids if sec is None else rank_token_ids(rank, nsteps)),
+            "parity_test": PARITY_TESTS.get(key),
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "device_status": moe.status_string(status),
+            "secondary": sec,
         }
         print(json.dumps(out), flush=True)
     if dist is not None:

@@ -483,6 +483,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
     const float sx = pow2f(S), isx = pow2f(-S);
     if (tid < HT) {
       *reinterpret_cast<float4*>(xn + 4 * tid) = make_float4(xv[0], xv[1], xv[2], xv[3]);
+    }
+    __syncthreads();
+    if (tid == kThreads - 32 && l + 1 < p.L) issue_router(l + 1);  // a warp without router rows
+    stamp(1);
+
+    // ---------------- 2. router rows -> logits
+    if (warp < rr_cnt) {
+      if (!mbar_ready(&bar_r[l & 1], (l >> 1) & 1, p.hdr, 10)) ab = true;
+      const int row = c + warp * G;
+      const uint4* wv = reinterpret_cast<const uint4*>(rbuf + (static_cast<size_t>(l & 1) * cv.rr_max + warp) * H);
+      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll 4
+      for (int s = lane; s < H / 8; s += 32) {
+        const uint4 w8 = wv[s];
+        const float4 a = reinterpret_cast<const float4*>(xn)[2 * s];
+        const float4 b = reinterpret_cast<const float4*>(xn)[2 * s + 1];
+        acc0 = fmaf(bf16_lo(w8.x), a.x, acc0);
+        acc1 = fmaf(bf16_hi(w8.x), a.y, acc1);
+        acc2 = fmaf(bf16_lo(w8.y), a.z, acc2);
+        acc3 = fmaf(bf16_hi(w8.y), a.w, acc3);
+        acc0 = fmaf(bf16_lo(w8.z), b.x, acc0);
+        acc1 = fmaf(bf16_hi(w8.z), b.y, acc1);
+        acc2 = fmaf(bf16_lo(w8.w), b.z, acc2);
+        acc3 = fmaf(bf16_hi(w8.w), b.w, acc3);
+      }
+      const float acc = warp_sum((acc0 + acc1) + (acc2 + acc3));
+      const LayerDesc& Ld = s_layers[l];
+      if (lane < kDecodeReplicas)
+        st_word(p.logits + lane * p.logits_rep + row, tag_f32(acc + ((row < E && Ld.rbias) ? Ld.rbias[row] : 0.f), par));
+    }
+    if (tid == 0) s_pend.r[l & 1] = -1;
+    stamp(2);
+    // this layer's x in fixed point (needed from the gate/up phase on, after the top-k barrier)
+    if (tid < HT) {
       // fixed point; this thread's rows 4t..4t+3 give one quad of every byte plane
       int X[4];
 #pragma unroll
@@ -519,37 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
       for (int o = 1; o < PS / 4; o <<= 1) xs += __shfl_xor_sync(0xffffffffu, xs, o);
       if ((tid & (PS / 4 - 1)) == 0) xq[sg * cv.QSP + cv.QS] = __float_as_uint(static_cast<float>(xs));
     }
-    __syncthreads();
-    if (tid == kThreads - 32 && l + 1 < p.L) issue_router(l + 1);  // a warp without router rows
-    stamp(1);
 
-    // ---------------- 2. router rows -> logits
-    if (warp < rr_cnt) {
-      if (!mbar_ready(&bar_r[l & 1], (l >> 1) & 1, p.hdr, 10)) ab = true;
-      const int row = c + warp * G;
-      const uint4* wv = reinterpret_cast<const uint4*>(rbuf + (static_cast<size_t>(l & 1) * cv.rr_max + warp) * H);
-      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll 4
-      for (int s = lane; s < H / 8; s += 32) {
-        const uint4 w8 = wv[s];
-        const float4 a = reinterpret_cast<const float4*>(xn)[2 * s];
-        const float4 b = reinterpret_cast<const float4*>(xn)[2 * s + 1];
-        acc0 = fmaf(bf16_lo(w8.x), a.x, acc0);
-        acc1 = fmaf(bf16_hi(w8.x), a.y, acc1);
-        acc2 = fmaf(bf16_lo(w8.y), a.z, acc2);
-        acc3 = fmaf(bf16_hi(w8.y), a.w, acc3);
-        acc0 = fmaf(bf16_lo(w8.z), b.x, acc0);
-        acc1 = fmaf(bf16_hi(w8.z), b.y, acc1);
-        acc2 = fmaf(bf16_lo(w8.w), b.z, acc2);
-        acc3 = fmaf(bf16_hi(w8.w), b.w, acc3);
-      }
-      const float acc = warp_sum((acc0 + acc1) + (acc2 + acc3));
-      const LayerDesc& Ld = s_layers[l];
-      if (lane < kDecodeReplicas)
-        st_word(p.logits + lane * p.logits_rep + row, tag_f32(acc + ((row < E && Ld.rbias) ? Ld.rbias[row] : 0.f), par));
-    }
-    if (tid == 0) s_pend.r[l & 1] = -1;
-    stamp(2);
 
     // ---------------- 3. softmax + top-k (every CTA, warp 0), then the unit's copies
     const LayerDesc& Ld = s_layers[l];
