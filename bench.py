@@ -435,6 +435,53 @@ def secondary(keys, steps, warmup, peak, budget_s=150.0):
     return out
 
 
+def dispatch_sweep(steps=8, warmup=3, Ts=(1, 2, 4, 8, 16, 24, 32, 48, 64)):
+    """The per-token kernels against the batched tensor-core path for T tokens through the 35b
+    stack (moe_set_batched_min_tokens picks the path; one token through a stack always runs the
+    persistent decode kernel): one JSON line per (T, path) with its device time per step, then
+    the faster path per T."""
+    shape = synth.SHAPES[SHAPE_KEY]
+    cfg = moe.make_config(shape)
+    sid = synth.SHAPE_SEED_ID[SHAPE_KEY]
+    layers = [synth.make_layer(shape, l, "cuda", seed_id=sid) for l in range(shape.layers)]
+    arr = moe.make_layer_array([moe.make_layer_weights(lw, cfg) for lw in layers])
+    stream = torch.cuda.current_stream()
+    best = {}
+    for T in Ts:
+        x = [synth.make_tokens(shape, [i], "cuda", seed_id=sid) if T == 1 else
+             synth.make_batch(shape, T, i, "cuda", seed_id=sid) for i in range(warmup + steps)]
+        xo = torch.empty(T, shape.hidden, dtype=torch.bfloat16, device="cuda")
+        ws = moe.Workspace(cfg, T, L=shape.layers)
+        for path, thr in (("per_layer", 1 << 30), ("batched", 1)):
+            prev = moe.moe_set_batched_min_tokens(thr)
+            name = moe.moe_stack_path_name(cfg, T, shape.layers)
+            if T > 1 and name != path:
+                moe.moe_set_batched_min_tokens(prev)
+                continue
+            for i in range(warmup):
+                moe.moe_stack_forward(cfg, arr, x[i], xo, ws, stream=stream)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(warmup, warmup + steps):
+                moe.moe_stack_forward(cfg, arr, x[i], xo, ws, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            launches = moe.moe_stack_kernel_launches(cfg, T, shape.layers)
+            moe.moe_set_batched_min_tokens(prev)
+            assert moe.moe_get_device_status(ws) == moe.MOE_OK
+            ms = e0.elapsed_time(e1) / steps
+            rec = {"sweep": "dispatch", "workload": shape.name, "T": T, "path": name, "ms_per_step": ms,
+                   "tokens_per_s": T / (ms / 1e3), "launches_per_step": launches}
+            print(json.dumps(rec), flush=True)
+            if T not in best or ms < best[T][1]:
+                best[T] = (name, ms)
+            if T == 1:
+                break  # one token: the persistent kernel whatever the threshold
+        del ws
+    print(json.dumps({"sweep": "dispatch", "faster_path": {str(T): b[0] for T, b in best.items()}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -443,6 +490,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true", help="skip the other workloads' block")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the per-token path against the batched path for T = 1..64 tokens and exit")
     ap.add_argument("--layers", type=int, default=0,
                     help="profile a shorter stack (small ncu case); the default is the full stack")
     ap.add_argument("--workload", default=SHAPE_KEY, choices=sorted(synth.SHAPES),
@@ -454,6 +503,9 @@ def main():
         run_reference(args)
         return
 
+    if args.sweep:
+        dispatch_sweep()
+        return
     dist, rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
     key = args.workload

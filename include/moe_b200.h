@@ -200,6 +200,15 @@ MOE_API int32_t moe_stack_kernel_launches(const moe_config* cfg, int32_t T, int3
  * (T or L is 0); NULL on a bad configuration. */
 MOE_API const char* moe_stack_path_name(const moe_config* cfg, int32_t T, int32_t L);
 
+/* Sets the token count from which moe_layer_forward, moe_expert_ffn and
+ * moe_stack_forward take the batched tensor-core path (where the shape
+ * supports it) instead of the per-token kernels, for the whole process and
+ * every device; T < 1 restores the default (8). Returns the previous value.
+ * A single token through a stack keeps its persistent kernel whatever the
+ * value. Meant for measuring the two paths against each other (bench.py
+ * --sweep); calls already enqueued are not affected. Not on the pages. */
+MOE_API int32_t moe_set_batched_min_tokens(int32_t T);
+
 /* The batched path's grouping step on its own: the T*k (token, slot) pairs
  * of topk_idx [T][k] grouped by expert, stable in (token, slot) order, with
  * the shared expert (if cfg->shared_inter > 0) as expert E taken by every

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <memory>
 #include <mutex>
@@ -49,7 +50,8 @@ struct Layout {
   size_t total;
 };
 
-constexpr int kBatchMinTokens = 8;  // from this many tokens the grouped tensor-core path runs
+constexpr int kBatchMinTokens = 8;  // from this many tokens the grouped tensor-core path runs (default)
+std::atomic<int> g_batch_min{kBatchMinTokens};  // moe_set_batched_min_tokens
 
 constexpr int kMaxGrid = 1024;  // largest persistent decode grid
 
@@ -269,7 +271,7 @@ int device_sms() {
 }
 
 bool batched_eligible(const moe_config& c, int T) {
-  if (T < kBatchMinTokens) return false;
+  if (T < g_batch_min.load(std::memory_order_relaxed)) return false;
   if (c.group != 64) return false;  // one quantisation group per GEMM k-block
   if (c.shared_inter != 0 && c.shared_inter != c.inter) return false;
   if ((c.hidden / c.group) % 8 || (c.inter / c.group) % 8 || c.hidden % 256 || c.inter % 64) return false;
@@ -411,14 +413,15 @@ bool dev_info(DevInfo* out) {
 // Whether one token through a stack runs as a persistent kernel (one launch
 // per up to kMaxDecodeLayers layers) rather than four kernels per layer, and
 // which: the split kernel where it fits, else the exchange kernel.
-bool decode_eligible(const moe_config& c, int L, int* grid, bool* split = nullptr, int* split_late = nullptr) {
+bool decode_eligible(const moe_config& c, int L, int* grid, bool* split = nullptr, int* split_late = nullptr,
+                     int* split_two = nullptr) {
   DevInfo d;
   if (!dev_info(&d) || !d.coop || d.sms < 1 || d.sms > kMaxGrid || d.smem_optin < 1024) return false;
   const size_t limit = static_cast<size_t>(d.smem_optin) - 1024;
   size_t ss = 0;
-  int late = 0;
+  int late = 0, two = 0;
   const bool sp = encode_fn() && moe::decode_split_plan(c.hidden, c.num_experts, c.top_k, c.inter, c.shared_inter,
-                                                        c.group, c.bits, d.sms, L, limit, &ss, &late);
+                                                        c.group, c.bits, d.sms, L, limit, &ss, &late, &two);
   if (!sp) {
     if (!moe::decode_stack_supported(c.hidden, c.num_experts, c.top_k, c.inter, c.shared_inter, c.group, c.bits))
       return false;
@@ -429,6 +432,7 @@ bool decode_eligible(const moe_config& c, int L, int* grid, bool* split = nullpt
   *grid = d.sms;
   if (split) *split = sp;
   if (split_late) *split_late = late;
+  if (split_two) *split_two = two;
   return true;
 }
 
@@ -450,7 +454,7 @@ moe::LayerDesc layer_desc(const moe_layer_weights& w) {
 
 moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, int L, const uint16_t* x0,
                         uint16_t* x_out, const moe_trace* trace, void* ws, const Layout& Ly, int grid, bool split,
-                        int split_late, cudaStream_t st) {
+                        int split_late, int split_two, cudaStream_t st) {
   char* b = static_cast<char*>(ws);
   auto P = std::make_unique<moe::DecodeParams>();
   P->H = c.hidden;
@@ -477,6 +481,7 @@ moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, in
   P->ybuf_stride = static_cast<int64_t>(moe::kDecodeReplicas) * P->yrep;
   P->arrive = reinterpret_cast<uint32_t*>(b + Ly.dcnt);
   P->split_late = split_late;
+  P->split_two = split_two;
   P->hdr = reinterpret_cast<moe::WsHeader*>(b + Ly.hdr);
   uint16_t* xmid = reinterpret_cast<uint16_t*>(b + Ly.dx);
   float* rmid = reinterpret_cast<float*>(b + Ly.dr);
@@ -629,9 +634,9 @@ moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weights* lay
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int grid = 0;
   bool split = false;
-  int split_late = 0;
-  if (T == 1 && decode_eligible(*cfg, L, &grid, &split, &split_late))
-    return stack_decode(*cfg, layers, L, x0, x_out, trace, ws, Ly, grid, split, split_late, st);
+  int split_late = 0, split_two = 0;
+  if (T == 1 && decode_eligible(*cfg, L, &grid, &split, &split_late, &split_two))
+    return stack_decode(*cfg, layers, L, x0, x_out, trace, ws, Ly, grid, split, split_late, split_two, st);
   const bool batched = batched_eligible(*cfg, T);
   const size_t TH = static_cast<size_t>(T) * cfg->hidden;
   const size_t Tk = static_cast<size_t>(T) * cfg->top_k;
@@ -721,6 +726,10 @@ moe_status moe_prepare_down_units(const moe_config* cfg, const moe_qtensor* down
   cudaError_t e = moe::launch_prepare_down_units(down->q, stride, n_experts, cfg->hidden, rowb, 32 * cfg->bits / 8,
                                                  out, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "prepare_down_units launch");
+}
+
+int32_t moe_set_batched_min_tokens(int32_t T) {
+  return g_batch_min.exchange(T < 1 ? kBatchMinTokens : T);
 }
 
 moe_status moe_check_wait_limit(void* ws, size_t ws_bytes, int32_t* gave_up, moe_stream_t stream) {

@@ -139,6 +139,7 @@ struct DecodeParams {
   float* yacc;
   int yrep;
   int split_late;        // split kernel: down codes copied into the first gate/up batch's space once it is read
+  int split_two;         // split kernel: more units than CTAs (some CTAs take two: a second down buffer)
   int64_t ybuf_stride;   // floats between buffers (kDecodeReplicas * yrep)
   uint32_t* arrive;
   WsHeader* hdr;
@@ -164,7 +165,7 @@ size_t decode_stack_smem(int H, int E, int k, int I, int Is, int group, int bits
 // The split kernel: whether it runs this shape on `grid` CTAs within `smem_limit` bytes of
 // shared memory for launches of up to L layers, and its shared memory.
 bool decode_split_plan(int H, int E, int k, int I, int Is, int group, int bits, int grid, int L, size_t smem_limit,
-                       size_t* smem, int* late);
+                       size_t* smem, int* late, int* two = nullptr);
 cudaError_t launch_decode_split(const DecodeParams& p, int bits, int grid, cudaStream_t stream);
 cudaError_t launch_decode_stack(const DecodeParams& p, int bits, int grid, cudaStream_t stream);
 cudaError_t launch_wait_limit_check(WsHeader* hdr, uint32_t* never_set, int32_t* gave_up, cudaStream_t stream);

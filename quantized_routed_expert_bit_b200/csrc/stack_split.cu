@@ -92,10 +92,11 @@ __host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
 // Shared-memory carve-up; identical on host (sizing) and device.
 struct Carve {
   int PS, nsg, QS, QSP, ng, ngd, rowb, rr_max, HT, UB;
-  uint32_t xn, xq, hq, guv, gsb, gcd, dcd, dhi, dsb, rbuf, desc, total;
+  uint32_t xn, xq, hq, guv, gsb, gcd, dcd, dhi, dsb, dcd2, dsb2, rbuf, desc, total;
 };
 
-__host__ __device__ inline Carve carve(int H, int E, int I, int Is, int group, int bits, int G, int L, int late) {
+__host__ __device__ inline Carve carve(int H, int E, int I, int Is, int group, int bits, int G, int L, int late,
+                                       int two) {
   Carve c{};
   c.PS = 128 / bits;          // codes per 16-byte segment
   c.nsg = H / c.PS;           // segments per gate/up row
@@ -125,6 +126,10 @@ __host__ __device__ inline Carve carve(int H, int E, int I, int Is, int group, i
     c.dhi = c.dcd + (H / 2) * c.UB;
   }
   c.dsb = o;   o = al128(o + H * 4);                       // down (scale, bias) of the unit's group, [H][2]
+  if (two) {  // a CTA with a second unit: its down data has a buffer of its own
+    c.dcd2 = o;  o = al128(o + H * c.UB);
+    c.dsb2 = o;  o = al128(o + H * 4);
+  }
   c.rbuf = o;  o = al128(o + 2 * c.rr_max * H * 2);
   c.desc = o;  o = al128(o + L * sizeof(LayerDesc));       // the launch's layer descriptors
   c.total = o;
@@ -203,10 +208,96 @@ __device__ __forceinline__ int fix_exp(float m) {
 }
 __device__ __forceinline__ float pow2f(int s) { return __uint_as_float(static_cast<uint32_t>(s + 127) << 23); }
 
+// Top-k of one token's logits by one warp for 16 logits per lane (E <= 512): the lane's logits of
+// experts lane + 32i, i < 8 and i >= 8, are sorted as two lists of 8 (larger logit first, then
+// lower expert index); each round the lane offers the better of its two heads, one warp-wide max
+// picks the winner (lowest index among equal keys) and its lane pops that head. Lane j < k ends
+// with the j-th pick. The same result as topk_sorted<16>, with two 8-sorts instead of a 16-sort.
+__device__ __forceinline__ void topk_halves(const uint32_t* wl, int E, int k, int lane, unsigned& my_k, int& my_e,
+                                            unsigned& kmax) {
+  unsigned ka[8], kb[8];
+  int ia[8], ib[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    ia[i] = lane + 32 * i;
+    ib[i] = lane + 32 * (i + 8);
+    ka[i] = (ia[i] < E) ? fkey(__uint_as_float(wl[i])) : 0u;
+    kb[i] = (ib[i] < E) ? fkey(__uint_as_float(wl[i + 8])) : 0u;
+  }
+  auto sort8 = [](unsigned (&key)[8], int (&idx)[8]) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+#pragma unroll
+      for (int i = (r & 1); i + 1 < 8; i += 2) {
+        const bool sw = key[i + 1] > key[i] || (key[i + 1] == key[i] && idx[i + 1] < idx[i]);
+        const unsigned k0 = key[i], k1 = key[i + 1];
+        const int i0 = idx[i], i1 = idx[i + 1];
+        key[i] = sw ? k1 : k0;
+        key[i + 1] = sw ? k0 : k1;
+        idx[i] = sw ? i1 : i0;
+        idx[i + 1] = sw ? i0 : i1;
+      }
+    }
+  };
+  sort8(ka, ia);
+  sort8(kb, ib);
+  my_k = 0u;
+  my_e = 0;
+  kmax = 0u;
+#pragma unroll 1
+  for (int j = 0; j < k; ++j) {
+    const bool fb = kb[0] > ka[0] || (kb[0] == ka[0] && ib[0] < ia[0]);  // the lane's better head
+    const unsigned hk = fb ? kb[0] : ka[0];
+    const int hi = fb ? ib[0] : ia[0];
+    const unsigned wk = __reduce_max_sync(0xffffffffu, hk);
+    const unsigned we = __reduce_min_sync(0xffffffffu, hk == wk ? static_cast<unsigned>(hi) : 0xffffffffu);
+    if (j == 0) kmax = wk;
+    if (lane == j) {
+      my_k = wk;
+      my_e = static_cast<int>(we);
+    }
+    if (static_cast<unsigned>(hi) == we) {  // the owner pops the head it offered
+      if (fb) {
+#pragma unroll
+        for (int i = 0; i + 1 < 8; ++i) {
+          kb[i] = kb[i + 1];
+          ib[i] = ib[i + 1];
+        }
+        kb[7] = 0u;
+      } else {
+#pragma unroll
+        for (int i = 0; i + 1 < 8; ++i) {
+          ka[i] = ka[i + 1];
+          ia[i] = ia[i + 1];
+        }
+        ka[7] = 0u;
+      }
+    }
+  }
+}
+
+// One unit of work: 32 consecutive columns of one slot's intermediate.
+struct Unit {
+  int j;       // slot: 0..k-1 the selected experts in rank order, k the shared expert
+  int i0;      // first column inside the slot
+  int g;       // its quantisation group along the down rows
+  bool routed;
+};
+
+__device__ __forceinline__ Unit unit_of(int u, int k, int I, int group) {
+  const int gp0 = u * 32;
+  Unit U;
+  U.j = gp0 < k * I ? gp0 / I : k;
+  U.i0 = gp0 - (U.j < k ? U.j * I : k * I);
+  U.g = U.i0 / group;
+  U.routed = U.j < k;
+  return U;
+}
+
 // Copy-phase bookkeeping for leaving early: parities of the phases this CTA
 // still has bulk copies in flight on (-1 = none).
 struct Pending {
-  int r[2], gc, dn;
+  int r[2], gc, dn[2];
 };
 
 __device__ __noinline__ void drain(Pending* pend, uint64_t* bar_r, uint64_t* bar_gc, uint64_t* bar_dn, int nb,
@@ -217,19 +308,20 @@ __device__ __noinline__ void drain(Pending* pend, uint64_t* bar_r, uint64_t* bar
     if (pend->r[1] >= 0) mbar_wait(&bar_r[1], pend->r[1], hdr, 91);
     if (pend->gc >= 0)
       for (int b = 0; b < nb; ++b) mbar_wait(&bar_gc[b], pend->gc, hdr, 94);
-    if (pend->dn >= 0) mbar_wait(bar_dn, pend->dn, hdr, 95);
+    if (pend->dn[0] >= 0) mbar_wait(&bar_dn[0], pend->dn[0], hdr, 95);
+    if (pend->dn[1] >= 0) mbar_wait(&bar_dn[1], pend->dn[1], hdr, 96);
   }
   __syncthreads();
 }
 
-template <int BITS, int CH>
+template <int BITS, int CH, bool TWO>
 __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int PS = 128 / BITS;  // codes per 16-byte segment
   constexpr int QW = PS / 4;      // quads per segment per byte plane
   extern __shared__ __align__(128) unsigned char sm[];
   __shared__ __align__(8) uint64_t bar_r[2];
   __shared__ __align__(8) uint64_t bar_gc[kNB];
-  __shared__ __align__(8) uint64_t bar_dn;
+  __shared__ __align__(8) uint64_t bar_dn[2];  // down data of the CTA's first and second unit
   __shared__ int s_idx[16];
   __shared__ float s_w[16];
   __shared__ float s_sg;
@@ -242,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
   const int G = gridDim.x, c = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   bool ab = false;  // a wait of this thread gave up; combined over the CTA at each phase end
-  const Carve cv = carve(H, E, I, Is, group, BITS, G, p.L, p.split_late);
+  const Carve cv = carve(H, E, I, Is, group, BITS, G, p.L, p.split_late, p.split_two);
   float* xn = reinterpret_cast<float*>(sm + cv.xn);
   uint32_t* xq = reinterpret_cast<uint32_t*>(sm + cv.xq);
   uint32_t* hq = reinterpret_cast<uint32_t*>(sm + cv.hq);
@@ -256,15 +348,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
   uint16_t* rbuf = reinterpret_cast<uint16_t*>(sm + cv.rbuf);
   const LayerDesc* s_layers = reinterpret_cast<const LayerDesc*>(sm + cv.desc);
 
-  // ---- static assignment of this CTA's work: unit c (if any) = columns [32c, 32c + 32) of the
-  // flattened (slot, column) space, slot j at [j * I, (j + 1) * I), the shared expert last
-  const int NP = k * I + Is;
-  const bool has_unit = c < NP / kUnit;
-  const int gp0 = has_unit ? c * kUnit : 0;
-  const int jA = gp0 < k * I ? gp0 / I : k;                // the unit's slot (k = shared expert)
-  const int iA = gp0 - (jA < k ? jA * I : k * I);          // first column inside the slot
-  const bool u_routed = jA < k;
-  const int u_g = iA / group;                              // the unit's quantisation group along the down rows
+  // ---- static assignment of this CTA's work: units c and c + G (where they exist) of the
+  // flattened (slot, column) space cut into 32-column units, slot j at [j * I, (j + 1) * I), the
+  // shared expert last. A CTA with two units does them one after the other.
+  const int NU = (k * I + Is) / kUnit;
+  const int nu = (c < NU ? 1 : 0) + (TWO && c + G < NU ? 1 : 0);
+  const bool has_unit = nu > 0;
+  const Unit U0 = unit_of(c, k, I, group);
+  const Unit U1 = unit_of(c + G, k, I, group);
   const int nrows_rt = E + (Is > 0 ? 1 : 0);
   const int rr_cnt = (c < nrows_rt) ? cdiv(nrows_rt - c, G) : 0;
   const uint32_t* lg_in = p.logits + (c % kDecodeReplicas) * p.logits_rep;  // this CTA's copy of the logits
@@ -276,9 +367,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
     mbar_init(&bar_r[0], 1);
     mbar_init(&bar_r[1], 1);
     for (int b = 0; b < kNB; ++b) mbar_init(&bar_gc[b], 1);
-    mbar_init(&bar_dn, 1);
+    mbar_init(&bar_dn[0], 1);
+    mbar_init(&bar_dn[1], 1);
     fence_mbar_init();
-    s_pend.r[0] = s_pend.r[1] = s_pend.gc = s_pend.dn = -1;
+    s_pend.r[0] = s_pend.r[1] = s_pend.gc = s_pend.dn[0] = s_pend.dn[1] = -1;
     s_b0 = 0;
   }
   // every layer descriptor of the launch into shared memory, once (parameter-space reads
@@ -301,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
     mbar_arrive1(&bar_r[b]);
     s_pend.r[b] = (l >> 1) & 1;
   };
-  auto leave = [&]() { drain(&s_pend, bar_r, bar_gc, &bar_dn, nb, p.hdr); };
+  auto leave = [&]() { drain(&s_pend, bar_r, bar_gc, bar_dn, nb, p.hdr); };
 
   if (tid == 0) issue_router(0);
 
@@ -354,38 +446,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
     }
   };
 
-  // the unit's down data (one thread): 256-row tiles of its 32 columns of the down codes, and
-  // the (scale, bias) pairs of its group for all H rows from the group-major copy (when the
-  // layer has one; else the down phase reads them from the canonical layout)
-  auto issue_down = [&](const LayerDesc& Ld, int l, int e) {
-    const uint16_t* sbm = u_routed ? Ld.dsb : Ld.sdsb;
-    const uint8_t* cdm = u_routed ? Ld.dcu : Ld.sdcu;
-    const size_t eu = u_routed ? e : 0;
+  // a unit's down data (one thread) into down buffer `db` (0, or 1 for a CTA's second unit): its
+  // 32 columns of all H down rows (one contiguous block of the unit-major copy, else 256-row tiles
+  // of the canonical codes) and the (scale, bias) pairs of its group for all H rows from the
+  // group-major copy (when the layer has one; else the down phase reads the canonical layout)
+  auto issue_down = [&](const LayerDesc& Ld, int l, const Unit& U, int e, int db) {
+    const uint16_t* sbm = U.routed ? Ld.dsb : Ld.sdsb;
+    const uint8_t* cdm = U.routed ? Ld.dcu : Ld.sdcu;
+    const size_t eu = U.routed ? e : 0;
+    unsigned char* lo = db ? sm + cv.dcd2 : dcd;
+    unsigned char* hi = db ? sm + cv.dcd2 + H2 * cv.UB : dhi;
+    uint64_t* bar = &bar_dn[db];
     // the buffers may last have been read by ordinary loads (gate/up or the previous layer's down)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_arrive_expect_tx(&bar_dn, static_cast<uint32_t>(H) * (cv.UB + (sbm ? 4 : 0)));
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(H) * (cv.UB + (sbm ? 4 : 0)));
     if (cdm) {  // the unit's 32 columns of all rows: one contiguous block, in two halves
-      const uint8_t* src = cdm + ((eu * (u_routed ? I : Is) / kUnit) + iA / kUnit) * H * cv.UB;
-      bulk_g2s(dcd, src, static_cast<uint32_t>(H2) * cv.UB, &bar_dn);
-      bulk_g2s(dhi, src + static_cast<size_t>(H2) * cv.UB, static_cast<uint32_t>(H2) * cv.UB, &bar_dn);
+      const uint8_t* src = cdm + ((eu * (U.routed ? I : Is) / kUnit) + U.i0 / kUnit) * H * cv.UB;
+      bulk_g2s(lo, src, static_cast<uint32_t>(H2) * cv.UB, bar);
+      bulk_g2s(hi, src + static_cast<size_t>(H2) * cv.UB, static_cast<uint32_t>(H2) * cv.UB, bar);
     } else {
-      const CUtensorMap* tm = u_routed ? &p.tm_dn[l] : &p.tm_sdn[l];
+      const CUtensorMap* tm = U.routed ? &p.tm_dn[l] : &p.tm_sdn[l];
 #pragma unroll 1
       for (int r0 = 0; r0 < H; r0 += kBoxRows)
-        tma_3d(r0 < H2 ? dcd + r0 * cv.UB : dhi + (r0 - H2) * cv.UB, tm, iA * BITS / 8, r0, static_cast<int>(eu),
-               &bar_dn);
+        tma_3d(r0 < H2 ? lo + r0 * cv.UB : hi + (r0 - H2) * cv.UB, tm, U.i0 * BITS / 8, r0, static_cast<int>(eu), bar);
     }
     if (sbm)
-      bulk_g2s(sm + cv.dsb, sbm + (eu * cv.ngd + u_g) * H * 2, static_cast<uint32_t>(H) * 4, &bar_dn);
-    s_pend.dn = l & 1;
+      bulk_g2s(sm + (db ? cv.dsb2 : cv.dsb), sbm + (eu * cv.ngd + U.g) * H * 2, static_cast<uint32_t>(H) * 4, bar);
+    s_pend.dn[db] = l & 1;
   };
 
-  // the unit's gate/up data (one whole warp, converged): batch 0's code rows with the scales and
-  // biases of the whole unit, then batch 1's code rows; then (unless in mid-copy mode) the down data
-  auto issue_unit = [&](const LayerDesc& Ld, int l, int e) {
+  // a unit's gate/up data (one whole warp, converged): batch 0's code rows with the scales and
+  // biases of the whole unit, then batch 1's code rows, completing phase `gpar` of the batch
+  // barriers; then (unless in mid-copy mode) its down data into down buffer db
+  auto issue_unit = [&](const LayerDesc& Ld, int l, const Unit& U, int e, int gpar, int db) {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    const QMat& mq = u_routed ? Ld.gu : Ld.sgu;
-    const int Ij = u_routed ? I : Is;
+    const QMat& mq = U.routed ? Ld.gu : Ld.sgu;
+    const int Ij = U.routed ? I : Is;
+    const int iA = U.i0;
     const uint8_t* qb = mq.q + static_cast<size_t>(e) * mq.q_stride;
     const uint16_t* sb = mq.s + static_cast<size_t>(e) * mq.sb_stride;
     const uint16_t* bb = mq.b + static_cast<size_t>(e) * mq.sb_stride;
@@ -406,13 +503,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
       }
     }
     if (lane == 0) {
-      s_pend.gc = l & 1;
-      if (!p.split_late) issue_down(Ld, l, e);
+      s_pend.gc = gpar;
+      if (!p.split_late) issue_down(Ld, l, U, e, db);
     }
     __syncwarp();
   };
 
   float rr4[4] = {0.f, 0.f, 0.f, 0.f};  // residual stream, rows 4t .. 4t+3 (t < H/4)
+  uint32_t gph = 0;  // completed phases of the gate/up batch barriers (one per unit processed)
 
   for (int l = 0; l < p.L; ++l) {
     const int lg = p.l0 + l;  // layer index within the whole stack (trace rows)
@@ -588,12 +686,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
       unsigned my_k, kmax;
       int my_e;
       if (E <= 256) topk_sorted<8>(wl, E, k, lane, my_k, my_e, kmax);
-      else topk_sorted<kTopPer>(wl, E, k, lane, my_k, my_e, kmax);
+      else topk_halves(wl, E, k, lane, my_k, my_e, kmax);
       // the unit's copies, at once (lane jA holds slot jA's pick). Issuing a routed unit's copies in
       // the round that picks its expert, or the shared expert's one layer ahead, measured slower:
       // their traffic delays the other CTAs' polls of the logits
       if (has_unit && !__any_sync(0xffffffffu, ab))  // warp-uniform: issue_unit has __syncwarp
-        issue_unit(Ld, l, u_routed ? __shfl_sync(0xffffffffu, my_e, jA) : 0);
+        issue_unit(Ld, l, U0, U0.routed ? __shfl_sync(0xffffffffu, my_e, U0.j) : 0, gph & 1, 0);
       const float mx = fkey_inv(kmax);
       float z = 0.f;
       if (!p.renorm) {  // softmax over all E: the words are re-read (complete and tagged by now)
@@ -625,149 +723,167 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
         st_word(zb + i, 0u);
     }
 
-    // ---------------- 4. gate/up rows + SwiGLU, batch by batch as the codes land
-    if (has_unit) {
-      uint32_t xr[CH][3 * QW];  // this lane's segments of X, by byte plane
-      float xsm[CH];
+    // ---------------- 4./5. the CTA's units in turn (a lambda: without TWO it is called once, with
+    // ui = 0, so that the single-unit kernel is straight-line code); false = leave the kernel
+    auto unit_body = [&](const int ui, const Unit& U) -> bool {
+      // ---------------- 4. gate/up rows + SwiGLU, batch by batch as the codes land
+      {
+        uint32_t xr[CH][3 * QW];  // this lane's segments of X, by byte plane
+        float xsm[CH];
 #pragma unroll
-      for (int ch = 0; ch < CH; ++ch) {
-        const int s = gs0 + 32 * ch;
+        for (int ch = 0; ch < CH; ++ch) {
+          const int s = gs0 + 32 * ch;
 #pragma unroll
-        for (int q = 0; q < 3 * QW; ++q) xr[ch][q] = xq[s * cv.QSP + q];
-        xsm[ch] = __uint_as_float(xq[s * cv.QSP + cv.QS]);
-      }
+          for (int q = 0; q < 3 * QW; ++q) xr[ch][q] = xq[s * cv.QSP + q];
+          xsm[ch] = __uint_as_float(xq[s * cv.QSP + cv.QS]);
+        }
 #pragma unroll 1
-      for (int b = 0; b < kNB; ++b) {
-        if (warp * rps >= 2 * kBatch) continue;  // no row of this batch for this warp
-        if (!mbar_ready(&bar_gc[b], l & 1, p.hdr, 12)) ab = true;
-        if (b == 0) stamp(4);
-        // two rows of the batch at a time (rows rw and rw + 16 * rps), for independent work in flight
+        for (int b = 0; b < kNB; ++b) {
+          if (warp * rps >= 2 * kBatch) continue;  // no row of this batch for this warp
+          if (!mbar_ready(&bar_gc[b], gph & 1, p.hdr, 12)) ab = true;
+          if (b == 0) stamp(4);
+          // two rows of the batch at a time (rows rw and rw + 16 * rps), for independent work in flight
 #pragma unroll 1
-        for (int rw = warp * rps; rw < 2 * kBatch; rw += 2 * kWarps * rps) {
-          float acc[2];
-          int gi[2];
+          for (int rw = warp * rps; rw < 2 * kBatch; rw += 2 * kWarps * rps) {
+            float acc[2];
+            int gi[2];
 #pragma unroll
-          for (int r2 = 0; r2 < 2; ++r2) {
-            const int rho = rw + r2 * kWarps * rps + gsub;  // [0, 16) gate rows, [16, 32) up rows of the batch
-            const int gu = rho >= kBatch ? 1 : 0;
-            const int q = b * kBatch + rho - gu * kBatch;  // pair within the unit
-            gi[r2] = rho < 2 * kBatch ? gu * kUnit + q : -1;
-            acc[r2] = 0.f;
-            if (rho < 2 * kBatch) {
-              const unsigned char* row = gcd + static_cast<size_t>(gu * kUnit + q) * rowb;
-              const uint16_t* sc = gsb + static_cast<size_t>(gu * kUnit + q) * ng;
-              const uint16_t* bi = gsb + static_cast<size_t>((2 + gu) * kUnit + q) * ng;
+            for (int r2 = 0; r2 < 2; ++r2) {
+              const int rho = rw + r2 * kWarps * rps + gsub;  // [0, 16) gate rows, [16, 32) up rows of the batch
+              const int gu = rho >= kBatch ? 1 : 0;
+              const int q = b * kBatch + rho - gu * kBatch;  // pair within the unit
+              gi[r2] = rho < 2 * kBatch ? gu * kUnit + q : -1;
+              acc[r2] = 0.f;
+              if (rho < 2 * kBatch) {
+                const unsigned char* row = gcd + static_cast<size_t>(gu * kUnit + q) * rowb;
+                const uint16_t* sc = gsb + static_cast<size_t>(gu * kUnit + q) * ng;
+                const uint16_t* bi = gsb + static_cast<size_t>((2 + gu) * kUnit + q) * ng;
 #pragma unroll
-              for (int ch = 0; ch < CH; ++ch) {
-                const int s = gs0 + 32 * ch;
-                const uint4 cd = *reinterpret_cast<const uint4*>(row + 16 * s);
-                const int g = (s * PS) >> lgG;
-                const float d = seg_dot<BITS>(cd, xr[ch] + 2 * QW, xr[ch] + QW, xr[ch]);
-                acc[r2] = fmaf(bf16_to_f32(sc[g]), d, fmaf(bf16_to_f32(bi[g]), xsm[ch], acc[r2]));
+                for (int ch = 0; ch < CH; ++ch) {
+                  const int s = gs0 + 32 * ch;
+                  const uint4 cd = *reinterpret_cast<const uint4*>(row + 16 * s);
+                  const int g = (s * PS) >> lgG;
+                  const float d = seg_dot<BITS>(cd, xr[ch] + 2 * QW, xr[ch] + QW, xr[ch]);
+                  acc[r2] = fmaf(bf16_to_f32(sc[g]), d, fmaf(bf16_to_f32(bi[g]), xsm[ch], acc[r2]));
+                }
+              }
+            }
+            if (nsg >= 32) {
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) {
+                acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
+                acc[1] += __shfl_xor_sync(0xffffffffu, acc[1], o);
+              }
+            } else {
+#pragma unroll 1
+              for (int o = nsg >> 1; o > 0; o >>= 1) {
+                acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
+                acc[1] += __shfl_xor_sync(0xffffffffu, acc[1], o);
+              }
+            }
+            if (gs0 == 0) {
+              if (gi[0] >= 0) guv[gi[0]] = acc[0] * isx;
+              if (gi[1] >= 0) guv[gi[1]] = acc[1] * isx;
+            }
+          }
+          if (p.split_late && b == 0) {
+            // mid-copy mode: the last warp done with the first batch's rows issues the down copies
+            // into their space (the other warps go on with the second batch)
+            __syncwarp();
+            if (lane == 0) {
+              __threadfence_block();
+              const int nw0 = min(kWarps, cdiv(2 * kBatch, rps));
+              if (atomicAdd(&s_b0, 1) == nw0 - 1) {
+                __threadfence_block();
+                s_b0 = 0;
+                issue_down(s_layers[l], l, U, U.routed ? s_idx[U.j] : 0, 0);
               }
             }
           }
-          if (nsg >= 32) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-              acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
-              acc[1] += __shfl_xor_sync(0xffffffffu, acc[1], o);
-            }
-          } else {
-#pragma unroll 1
-            for (int o = nsg >> 1; o > 0; o >>= 1) {
-              acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
-              acc[1] += __shfl_xor_sync(0xffffffffu, acc[1], o);
-            }
-          }
-          if (gs0 == 0) {
-            if (gi[0] >= 0) guv[gi[0]] = acc[0] * isx;
-            if (gi[1] >= 0) guv[gi[1]] = acc[1] * isx;
-          }
-        }
-        if (p.split_late && b == 0) {
-          // mid-copy mode: the last warp done with the first batch's rows issues the down copies
-          // into their space (the other warps go on with the second batch)
-          __syncwarp();
-          if (lane == 0) {
-            __threadfence_block();
-            const int nw0 = min(kWarps, cdiv(2 * kBatch, rps));
-            if (atomicAdd(&s_b0, 1) == nw0 - 1) {
-              __threadfence_block();
-              s_b0 = 0;
-              issue_down(s_layers[l], l, u_routed ? s_idx[jA] : 0);
-            }
-          }
         }
       }
-    }
-    const bool gu_failed = __syncthreads_or(ab);
-    if (tid == 0) s_pend.gc = -1;
-    if (gu_failed) { leave(); return; }
-    if (has_unit && warp == 0) {
-      // SwiGLU, then the unit's h in fixed point (its own exponent) as quads for the down rows
-      const float h = silu_f(guv[lane]) * guv[kUnit + lane];
-      const int Sh = fix_exp(warp_max(fabsf(h)));
-      const int X = __float2int_rn(h * pow2f(Sh));
-      int hs = X;
+      const bool gu_failed = __syncthreads_or(ab);
+      if (tid == 0) s_pend.gc = -1;
+      ++gph;
+      if (gu_failed) { leave(); return false; }
+      // the second unit's copies go out as soon as the first's gate/up rows are read
+      if (TWO && ui + 1 < nu && warp == 0) issue_unit(s_layers[l], l, U1, U1.routed ? s_idx[U1.j] : 0, gph & 1, 1);
+      if (warp == 0) {
+        // SwiGLU, then the unit's h in fixed point (its own exponent) as quads for the down rows
+        const float h = silu_f(guv[lane]) * guv[kUnit + lane];
+        const int Sh = fix_exp(warp_max(fabsf(h)));
+        const int X = __float2int_rn(h * pow2f(Sh));
+        int hs = X;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) hs += __shfl_xor_sync(0xffffffffu, hs, o);
-      // one down row of the unit = 32 codes: 4-bit, one segment of 8 quads; 8-bit, two segments of 4
-      const int qp = (BITS == 4) ? quad_pos<4>(lane) : lane;
-      unsigned char* hqb = reinterpret_cast<unsigned char*>(hq);
+        for (int o = 16; o > 0; o >>= 1) hs += __shfl_xor_sync(0xffffffffu, hs, o);
+        // one down row of the unit = 32 codes: 4-bit, one segment of 8 quads; 8-bit, two segments of 4
+        const int qp = (BITS == 4) ? quad_pos<4>(lane) : lane;
+        unsigned char* hqb = reinterpret_cast<unsigned char*>(hq);
 #pragma unroll
-      for (int j = 0; j < 3; ++j) hqb[(j * 8 + (qp >> 2)) * 4 + (qp & 3)] = static_cast<unsigned char>(xbyte(X, j));
-      if (lane == 0) {
-        s_hx[0] = static_cast<float>(hs);
-        s_hx[1] = pow2f(-Sh);
+        for (int j = 0; j < 3; ++j) hqb[(j * 8 + (qp >> 2)) * 4 + (qp & 3)] = static_cast<unsigned char>(xbyte(X, j));
+        if (lane == 0) {
+          s_hx[0] = static_cast<float>(hs);
+          s_hx[1] = pow2f(-Sh);
+        }
       }
-    }
-    if (has_unit && tid < HT && !mbar_ready(&bar_dn, l & 1, p.hdr, 13)) ab = true;
-    if (__syncthreads_or(ab)) { leave(); return; }
-    if (tid == 0) s_pend.dn = -1;
-    stamp(5);
+      if (tid < HT && !mbar_ready(&bar_dn[ui], l & 1, p.hdr, 13)) ab = true;
+      if (__syncthreads_or(ab)) { leave(); return false; }
+      if (tid == 0) s_pend.dn[ui] = -1;
+      stamp(5);
 
-    // ---------------- 5. the unit's partial of y for rows t, t + 512, ... (a warp reads 32
-    // consecutive rows of codes, and reduces into 32 consecutive words of y):
-    // routing weight x 2^-S_h x (scale x codes . X_h + bias x sum X_h)
-    if (has_unit) {
-      uint32_t hr[kQ];
+      // ---------------- 5. the unit's partial of y for rows t, t + 512, ... (a warp reads 32
+      // consecutive rows of codes, and reduces into 32 consecutive words of y):
+      // routing weight x 2^-S_h x (scale x codes . X_h + bias x sum X_h)
+      {
+        uint32_t hr[kQ];
 #pragma unroll
-      for (int q = 0; q < kQ; ++q) hr[q] = hq[q];
-      const float hsX = s_hx[0];
-      const float wgt = (u_routed ? s_w[jA] : s_sg) * s_hx[1];
-      const LayerDesc& Ld5 = s_layers[l];
-      const bool gm = (u_routed ? Ld5.dsb : Ld5.sdsb) != nullptr;
-      const QMat& dm = u_routed ? Ld5.dn : Ld5.sdn;
-      const size_t sb0 = static_cast<size_t>(u_routed ? s_idx[jA] : 0) * dm.sb_stride + u_g;
-      float* yrow = p.yacc + static_cast<size_t>(l % kDecodeYBufs) * p.ybuf_stride +
-                    static_cast<size_t>(c % kDecodeReplicas) * p.yrep;
+        for (int q = 0; q < kQ; ++q) hr[q] = hq[q];
+        const float hsX = s_hx[0];
+        const float wgt = (U.routed ? s_w[U.j] : s_sg) * s_hx[1];
+        const LayerDesc& Ld5 = s_layers[l];
+        const bool gm = (U.routed ? Ld5.dsb : Ld5.sdsb) != nullptr;
+        const QMat& dm = U.routed ? Ld5.dn : Ld5.sdn;
+        const size_t sb0 = static_cast<size_t>(U.routed ? s_idx[U.j] : 0) * dm.sb_stride + U.g;
+        const unsigned char* dlo = ui ? sm + cv.dcd2 : dcd;
+        const unsigned char* dhh = ui ? sm + cv.dcd2 + H2 * cv.UB : dhi;
+        const uint32_t* dsbu = ui ? reinterpret_cast<const uint32_t*>(sm + cv.dsb2) : dsb;
+        float* yrow = p.yacc + static_cast<size_t>(l % kDecodeYBufs) * p.ybuf_stride +
+                      static_cast<size_t>(c % kDecodeReplicas) * p.yrep;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int r = tid + q * kThreads;
-        if (r < H) {
-          float d;
-          const unsigned char* drow = r < H2 ? dcd + r * cv.UB : dhi + (r - H2) * cv.UB;
-          if constexpr (BITS == 4) {
-            d = seg_dot<4>(*reinterpret_cast<const uint4*>(drow), hr + 16, hr + 8, hr);
-          } else {
-            d = seg_dot<8>(*reinterpret_cast<const uint4*>(drow), hr + 16, hr + 8, hr) +
-                seg_dot<8>(*reinterpret_cast<const uint4*>(drow + 16), hr + 20, hr + 12, hr + 4);
+        for (int q = 0; q < 4; ++q) {
+          const int r = tid + q * kThreads;
+          if (r < H) {
+            float d;
+            const unsigned char* drow = r < H2 ? dlo + r * cv.UB : dhh + (r - H2) * cv.UB;
+            if constexpr (BITS == 4) {
+              d = seg_dot<4>(*reinterpret_cast<const uint4*>(drow), hr + 16, hr + 8, hr);
+            } else {
+              d = seg_dot<8>(*reinterpret_cast<const uint4*>(drow), hr + 16, hr + 8, hr) +
+                  seg_dot<8>(*reinterpret_cast<const uint4*>(drow + 16), hr + 20, hr + 12, hr + 4);
+            }
+            float sc, bi;
+            if (gm) {
+              const uint32_t sbw = dsbu[r];
+              sc = bf16_lo(sbw);
+              bi = bf16_hi(sbw);
+            } else {
+              sc = bf16_to_f32(__ldg(dm.s + sb0 + static_cast<size_t>(r) * cv.ngd));
+              bi = bf16_to_f32(__ldg(dm.b + sb0 + static_cast<size_t>(r) * cv.ngd));
+            }
+            red_add(yrow + r, wgt * fmaf(sc, d, bi * hsX));
           }
-          float sc, bi;
-          if (gm) {
-            const uint32_t sbw = dsb[r];
-            sc = bf16_lo(sbw);
-            bi = bf16_hi(sbw);
-          } else {
-            sc = bf16_to_f32(__ldg(dm.s + sb0 + static_cast<size_t>(r) * cv.ngd));
-            bi = bf16_to_f32(__ldg(dm.b + sb0 + static_cast<size_t>(r) * cv.ngd));
-          }
-          red_add(yrow + r, wgt * fmaf(sc, d, bi * hsX));
         }
       }
+      if (__syncthreads_or(ab)) { leave(); return false; }
+      return true;
+    };
+    if constexpr (TWO) {
+#pragma unroll 1
+      for (int ui = 0; ui < nu; ++ui)
+        if (!unit_body(ui, ui == 0 ? U0 : U1)) return;
+    } else {
+      if (has_unit && !unit_body(0, U0)) return;
     }
-    if (__syncthreads_or(ab)) { leave(); return; }
 
     stamp(6);
     // the arrival: a release reduction (this CTA's reductions and zeroes, ordered before it by
@@ -806,9 +922,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
   leave();
 }
 
-template <int BITS, int CH>
+template <int BITS, int CH, bool TWO>
 cudaError_t launch_t(const DecodeParams& p, size_t smem, int grid, cudaStream_t stream) {
-  auto kern = decode_split_kernel<BITS, CH>;
+  auto kern = decode_split_kernel<BITS, CH, TWO>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -825,7 +941,7 @@ bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
 }  // namespace
 
 bool decode_split_plan(int H, int E, int k, int I, int Is, int group, int bits, int grid, int L, size_t smem_limit,
-                       size_t* smem, int* late) {
+                       size_t* smem, int* late, int* two_out) {
   if (grid < 1 || L < 1) return false;
   if (L > kMaxDecodeLayers) L = kMaxDecodeLayers;
   const int PS = 128 / bits;
@@ -835,14 +951,17 @@ bool decode_split_plan(int H, int E, int k, int I, int Is, int group, int bits, 
   if (Is != 0 && Is != I) return false;          // one down row length (and scale row) for every slot
   if (I % kUnit || !pow2(group) || group % kUnit || I % group) return false;  // a unit lies in one group
   if (k > 16 || E > 32 * kTopPer) return false;
-  if ((k * I + Is) / kUnit > grid) return false;  // at most one unit per CTA
+  const int nunits = (k * I + Is) / kUnit;
+  if (nunits > 2 * grid) return false;  // at most two units per CTA
   if (cdiv(E + (Is > 0 ? 1 : 0), grid) > kWarps) return false;  // one router row per warp
+  const int two = nunits > grid ? 1 : 0;
   for (int lt = 0; lt < 2; ++lt) {  // down codes in a region of their own if they fit, else mid-copy mode
-    if (lt == 1 && H % (2 * kBoxRows)) break;  // the halves hold whole 256-row tiles
-    const size_t need = carve(H, E, I, Is, group, bits, grid, L, lt).total;
+    if (lt == 1 && (two || H % (2 * kBoxRows))) break;  // the halves hold whole 256-row tiles; one unit
+    const size_t need = carve(H, E, I, Is, group, bits, grid, L, lt, two).total;
     if (need <= smem_limit) {
       *smem = need;
       *late = lt;
+      if (two_out) *two_out = two;
       return true;
     }
   }
@@ -850,16 +969,25 @@ bool decode_split_plan(int H, int E, int k, int I, int Is, int group, int bits, 
 }
 
 cudaError_t launch_decode_split(const DecodeParams& p, int bits, int grid, cudaStream_t stream) {
-  const size_t smem = carve(p.H, p.E, p.I, p.Is, p.group, bits, grid, p.L, p.split_late).total;
+  const size_t smem = carve(p.H, p.E, p.I, p.Is, p.group, bits, grid, p.L, p.split_late, p.split_two).total;
   const int nsg = p.H * bits / 128;
   const int ch = nsg >= 32 ? nsg / 32 : 1;
-  if (bits == 4) {
-    if (ch == 1) return launch_t<4, 1>(p, smem, grid, stream);
-    return launch_t<4, 2>(p, smem, grid, stream);
+  if (p.split_two) {  // more units than CTAs: the loop over a CTA's two units
+    if (bits == 4) {
+      if (ch == 1) return launch_t<4, 1, true>(p, smem, grid, stream);
+      return launch_t<4, 2, true>(p, smem, grid, stream);
+    }
+    if (ch == 1) return launch_t<8, 1, true>(p, smem, grid, stream);
+    if (ch == 2) return launch_t<8, 2, true>(p, smem, grid, stream);
+    return launch_t<8, 4, true>(p, smem, grid, stream);
   }
-  if (ch == 1) return launch_t<8, 1>(p, smem, grid, stream);
-  if (ch == 2) return launch_t<8, 2>(p, smem, grid, stream);
-  return launch_t<8, 4>(p, smem, grid, stream);
+  if (bits == 4) {
+    if (ch == 1) return launch_t<4, 1, false>(p, smem, grid, stream);
+    return launch_t<4, 2, false>(p, smem, grid, stream);
+  }
+  if (ch == 1) return launch_t<8, 1, false>(p, smem, grid, stream);
+  if (ch == 2) return launch_t<8, 2, false>(p, smem, grid, stream);
+  return launch_t<8, 4, false>(p, smem, grid, stream);
 }
 
 }  // namespace moe

@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.moe_down_units_size.argtypes = [CP, I32, I32]
         L.moe_down_units_size.restype = ctypes.c_size_t
         L.moe_prepare_down_units.argtypes = [CP, ctypes.POINTER(QTensor), I32, I32, P, P]
+        L.moe_set_batched_min_tokens.argtypes = [I32]
+        L.moe_set_batched_min_tokens.restype = I32
         L.moe_stack_kernel_launches.argtypes = [CP, I32, I32]
         L.moe_stack_kernel_launches.restype = I32
         L.moe_stack_path_name.argtypes = [CP, I32, I32]
@@ -185,14 +187,21 @@ def prepare_layer(cfg: Config, lw):
 
 def make_layer_weights(lw, cfg: Optional[Config] = None) -> LayerWeights:
     """LayerWeights struct over a synth.LayerWeights (the caller keeps lw alive). With cfg
-    given and the weights on the GPU, the group-major down scale/bias copies the single-token
-    decode reads are made once (prepare_layer) and referenced too."""
+    given, the weights on the GPU and a shape that decode_split_kernel runs, the decode-ready
+    down copies that kernel reads (unit-major codes, group-major scales and biases) are made
+    once (prepare_layer) and referenced too."""
     dsb = sdsb = dcu = sdcu = None
-    if cfg is not None and lw.down.q.is_cuda:
+    if cfg is not None and lw.down.q.is_cuda and split_decode(cfg):
         dsb, sdsb, dcu, sdcu = prepare_layer(cfg, lw)
     return LayerWeights(lw.router_w.data_ptr(), _p(lw.router_bias), _qtensor(lw.gate_up), _qtensor(lw.down),
                         _qtensor(lw.shared_gate_up), _qtensor(lw.shared_down), _p(lw.shared_gate_w),
                         _p(dsb), _p(sdsb), _p(dcu), _p(sdcu))
+
+
+def split_decode(cfg: Config) -> bool:
+    """Whether one token through a stack of this shape runs decode_split_kernel on the current
+    device: the only reader of the decode-ready copies, made only then."""
+    return moe_stack_path_name(cfg, 1, 1) == "decode_split_kernel"
 
 
 class Workspace:
@@ -284,6 +293,12 @@ def moe_check_wait_limit(ws: Workspace, gave_up: torch.Tensor, stream=None):
 def moe_stack_kernel_launches(cfg: Config, T: int, L: int) -> int:
     """Kernels one moe_stack_forward call launches on the current device."""
     return int(lib().moe_stack_kernel_launches(ctypes.byref(cfg), int(T), int(L)))
+
+
+def moe_set_batched_min_tokens(T: int) -> int:
+    """Token count from which the batched tensor-core path runs (process-wide); T < 1 restores
+    the default. Returns the previous value."""
+    return int(lib().moe_set_batched_min_tokens(int(T)))
 
 
 def moe_stack_path_name(cfg: Config, T: int, L: int) -> Optional[str]:

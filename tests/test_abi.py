@@ -158,3 +158,32 @@ def test_stack_and_sort_validation_errors():
     assert lib.moe_stack_path_name(ctypes.byref(c), 0, 4) == b"none"
     assert lib.moe_stack_path_name(ctypes.byref(c), 1, 4) in (b"decode_split_kernel", b"decode_stack_kernel",
                                                                b"per_layer")
+
+
+def test_batched_threshold_knob():
+    """moe_set_batched_min_tokens returns the previous threshold; T < 1 restores the default 8."""
+    lib = moe.lib()
+    assert lib.moe_set_batched_min_tokens(3) == 8
+    assert lib.moe_set_batched_min_tokens(100) == 3
+    assert lib.moe_set_batched_min_tokens(0) == 100
+    assert lib.moe_set_batched_min_tokens(-5) == 8
+    assert lib.moe_set_batched_min_tokens(0) == 8
+
+
+def test_prepare_calls_validate_before_the_device():
+    """The load-time re-layouts refuse bad arguments without touching the device."""
+    c = cfg35()
+    lib = moe.lib()
+    qt = moe.QTensor(FAKE, FAKE, FAKE, 2048 * 256, 2048 * 8)
+    assert lib.moe_down_sb_size(ctypes.byref(c), 256, 512) == 256 * 8 * 2048 * 4
+    assert lib.moe_down_units_size(ctypes.byref(c), 256, 512) == 256 * 512 * 2048 // 2
+    assert lib.moe_down_sb_size(ctypes.byref(c), 256, 500) == 0        # K not a multiple of the group
+    assert lib.moe_down_units_size(ctypes.byref(c), 0, 512) == 0
+    assert lib.moe_prepare_down_sb(ctypes.byref(c), None, 256, 512, FAKE, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_prepare_down_sb(ctypes.byref(c), ctypes.byref(qt), 256, 512, FAKE + 2, None) == \
+        moe.MOE_ERR_INVALID_ARG                                        # misaligned output
+    assert lib.moe_prepare_down_units(ctypes.byref(c), ctypes.byref(qt), 256, 96, FAKE, None) == \
+        moe.MOE_ERR_INVALID_ARG                                        # K not a multiple of the group
+    short = moe.QTensor(FAKE, FAKE, FAKE, 100, 2048 * 8)
+    assert lib.moe_prepare_down_units(ctypes.byref(c), ctypes.byref(short), 256, 512, FAKE, None) == \
+        moe.MOE_ERR_INVALID_ARG                                        # expert stride below one expert

@@ -63,7 +63,7 @@ def check_glue(x0_bits, tx, ty, xo):
 def test_decode_stack_parity(key):
     shape = synth.SHAPES[key]
     # which persistent kernel runs each stack on a 148-SM B200 (a silent fallback would fail here)
-    want = {"35b": "decode_split_kernel", "35b8": "decode_split_kernel", "80b": "decode_stack_kernel"}[key]
+    want = "decode_split_kernel"
     assert moe.moe_stack_path_name(moe.make_config(shape), 1, shape.layers) == want
     layers = [synth.make_layer(shape, l, "cuda") for l in range(shape.layers)]
     total = ParityStats()
@@ -137,6 +137,8 @@ SMALL_STACKS = {
     "no-shared": (256, 16, 2, 128, 0, 4, 32, 6, False),
     "top1-g64": (512, 32, 1, 256, 256, 4, 64, 6, False),
     "top8-e64": (1024, 64, 8, 128, 128, 4, 32, 6, False),
+    # (5 * 1024 + 1024) / 32 = 192 units: more than one per SM, some CTAs take two
+    "two-units": (256, 16, 5, 1024, 1024, 4, 32, 4, False),
 }
 
 
