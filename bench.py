@@ -435,40 +435,44 @@ def secondary(keys, steps, warmup, peak, budget_s=150.0):
     return out
 
 
-def dispatch_sweep(steps=8, warmup=3, Ts=(1, 2, 4, 8, 16, 24, 32, 48, 64)):
-    """The per-token kernels against the batched tensor-core path for T tokens through the 35b
-    stack (moe_set_batched_min_tokens picks the path; one token through a stack always runs the
-    persistent decode kernel): one JSON line per (T, path) with its device time per step, then
-    the faster path per T."""
-    shape = synth.SHAPES[SHAPE_KEY]
+def dispatch_sweep(steps=8, warmup=3, Ts=(1, 2, 3, 4, 6, 8, 12, 16, 24, 32, 48, 64), key=None):
+    """The three multi-token paths for T tokens through a stack (the per-token kernels, the grouped
+    GEMV, the batched tensor-core path; moe_set_gemv_min_tokens / moe_set_batched_min_tokens pick
+    one; one token through a stack always runs the persistent decode kernel): one JSON line per
+    (T, path) with its device time per step, then the fastest path per T."""
+    key = key or SHAPE_KEY
+    shape = synth.SHAPES[key]
     cfg = moe.make_config(shape)
-    sid = synth.SHAPE_SEED_ID[SHAPE_KEY]
+    sid = synth.SHAPE_SEED_ID[key]
     layers = [synth.make_layer(shape, l, "cuda", seed_id=sid) for l in range(shape.layers)]
     arr = moe.make_layer_array([moe.make_layer_weights(lw, cfg) for lw in layers])
     stream = torch.cuda.current_stream()
     best = {}
+    paths = (("per_layer", 1 << 30, 1 << 30), ("grouped_gemv", 1, 1 << 30), ("batched", 1 << 30, 1))
     for T in Ts:
         x = [synth.make_tokens(shape, [i], "cuda", seed_id=sid) if T == 1 else
              synth.make_batch(shape, T, i, "cuda", seed_id=sid) for i in range(warmup + steps)]
         xo = torch.empty(T, shape.hidden, dtype=torch.bfloat16, device="cuda")
         ws = moe.Workspace(cfg, T, L=shape.layers)
-        for path, thr in (("per_layer", 1 << 30), ("batched", 1)):
-            prev = moe.moe_set_batched_min_tokens(thr)
-            name = moe.moe_stack_path_name(cfg, T, shape.layers)
-            if T > 1 and name != path:
-                moe.moe_set_batched_min_tokens(prev)
-                continue
-            for i in range(warmup):
-                moe.moe_stack_forward(cfg, arr, x[i], xo, ws, stream=stream)
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for i in range(warmup, warmup + steps):
-                moe.moe_stack_forward(cfg, arr, x[i], xo, ws, stream=stream)
-            e1.record(stream)
-            torch.cuda.synchronize()
-            launches = moe.moe_stack_kernel_launches(cfg, T, shape.layers)
-            moe.moe_set_batched_min_tokens(prev)
+        for path, gthr, bthr in paths:
+            pg, pb = moe.moe_set_gemv_min_tokens(gthr), moe.moe_set_batched_min_tokens(bthr)
+            try:
+                name = moe.moe_stack_path_name(cfg, T, shape.layers)
+                launches = moe.moe_stack_kernel_launches(cfg, T, shape.layers)
+                if T > 1 and name != path:
+                    continue
+                for i in range(warmup):
+                    moe.moe_stack_forward(cfg, arr, x[i], xo, ws, stream=stream)
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for i in range(warmup, warmup + steps):
+                    moe.moe_stack_forward(cfg, arr, x[i], xo, ws, stream=stream)
+                e1.record(stream)
+                torch.cuda.synchronize()
+            finally:
+                moe.moe_set_gemv_min_tokens(pg)
+                moe.moe_set_batched_min_tokens(pb)
             assert moe.moe_get_device_status(ws) == moe.MOE_OK
             ms = e0.elapsed_time(e1) / steps
             rec = {"sweep": "dispatch", "workload": shape.name, "T": T, "path": name, "ms_per_step": ms,
@@ -477,9 +481,10 @@ def dispatch_sweep(steps=8, warmup=3, Ts=(1, 2, 4, 8, 16, 24, 32, 48, 64)):
             if T not in best or ms < best[T][1]:
                 best[T] = (name, ms)
             if T == 1:
-                break  # one token: the persistent kernel whatever the threshold
+                break  # one token: the persistent kernel whatever the thresholds
         del ws
-    print(json.dumps({"sweep": "dispatch", "faster_path": {str(T): b[0] for T, b in best.items()}}), flush=True)
+    print(json.dumps({"sweep": "dispatch", "workload": shape.name,
+                      "fastest_path": {str(T): b[0] for T, b in best.items()}}), flush=True)
 
 
 def main():
@@ -504,7 +509,7 @@ def main():
         return
 
     if args.sweep:
-        dispatch_sweep()
+        dispatch_sweep(key=args.workload)
         return
     dist, rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)

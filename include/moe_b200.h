@@ -188,15 +188,18 @@ MOE_API moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weig
 
 /* Number of kernel launches moe_stack_forward makes for T tokens and L
  * layers on the current device: a single token runs the whole stack as one
- * persistent kernel (one launch per 48 layers) when the shape fits it; 8 or
- * more tokens run the batched path (1 + 7*L) where it applies; otherwise
- * 1 + 4*L. -1 on a bad configuration. */
+ * persistent kernel (one launch per 48 layers) when the shape fits it; from
+ * the batched threshold up (moe_set_batched_min_tokens) the batched path
+ * (1 + 7*L) where it applies; from the GEMV threshold up
+ * (moe_set_gemv_min_tokens) the grouped GEMV (1 + 6*L) where it applies;
+ * otherwise 1 + 4*L. -1 on a bad configuration. */
 MOE_API int32_t moe_stack_kernel_launches(const moe_config* cfg, int32_t T, int32_t L);
 
 /* Name of the path moe_stack_forward takes for T tokens and L layers on the
  * current device (a static string): "decode_split_kernel" or
  * "decode_stack_kernel" (one token, the persistent kernels), "batched" (the
- * grouped tensor-core path), "per_layer" (four kernels per layer), "none"
+ * grouped tensor-core path), "grouped_gemv" (a few tokens per expert, CUDA
+ * cores), "per_layer" (four kernels per layer), "none"
  * (T or L is 0); NULL on a bad configuration. */
 MOE_API const char* moe_stack_path_name(const moe_config* cfg, int32_t T, int32_t L);
 
@@ -208,6 +211,14 @@ MOE_API const char* moe_stack_path_name(const moe_config* cfg, int32_t T, int32_
  * value. Meant for measuring the two paths against each other (bench.py
  * --sweep); calls already enqueued are not affected. Not on the pages. */
 MOE_API int32_t moe_set_batched_min_tokens(int32_t T);
+
+/* Sets the token count from which those calls take the grouped GEMV path
+ * (a few tokens per expert: each selected expert's weights read once for
+ * all of its tokens, dot products on the CUDA cores) instead of the
+ * per-token kernels, below the batched threshold; T < 1 restores the
+ * default (2). Returns the previous value. Process-wide, as above. Not on
+ * the pages. */
+MOE_API int32_t moe_set_gemv_min_tokens(int32_t T);
 
 /* The batched path's grouping step on its own: the T*k (token, slot) pairs
  * of topk_idx [T][k] grouped by expert, stable in (token, slot) order, with

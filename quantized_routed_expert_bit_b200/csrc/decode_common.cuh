@@ -189,5 +189,72 @@ __device__ __forceinline__ void topk_sorted(const uint32_t* wl, int E, int k, in
   }
 }
 
+// ---------------------------------------------------------------- fixed-point dot products
+//
+// A group's share of a row's dot product is s_g * sum(q x) + b_g * sum(x). The activations are
+// turned into integers X_i = rint(x_i * 2^S), S chosen from max|x| (fix_exp) so that |X| <= 2^22,
+// split into three bytes X = 65536*X2 + 256*X1 + X0 (X2 signed), and sum(q X) is three exact
+// integer sums of byte products (dp4a), recombined in fp32 once per 16-byte segment of codes.
+// 4-bit codes are split into even and odd nibbles as bytes (two masks), so the activations are laid
+// out in the same order: quad_pos gives where code position o of a segment sits among its quad bytes.
+
+// Byte dot products: 4 unsigned code bytes times 4 signed (.s32) or unsigned (.u32) bytes, plus c.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// sum over one 16-byte segment of codes of q * X (X given as its quads: q3[j][.] byte j of X; for
+// 4-bit codes quads (2w, 2w+1) hold the even and odd elements of word w), as an fp32 number.
+template <int BITS>
+__device__ __forceinline__ float seg_dot(const uint4& c, const uint32_t* q2, const uint32_t* q1, const uint32_t* q0) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  int a2 = 0;
+  uint32_t a1 = 0u, a0 = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if constexpr (BITS == 4) {
+      const uint32_t lo = w[i] & 0x0F0F0F0Fu, hi = (w[i] >> 4) & 0x0F0F0F0Fu;
+      a2 = dp4a_us(lo, q2[2 * i], a2);
+      a2 = dp4a_us(hi, q2[2 * i + 1], a2);
+      a1 = dp4a_uu(lo, q1[2 * i], a1);
+      a1 = dp4a_uu(hi, q1[2 * i + 1], a1);
+      a0 = dp4a_uu(lo, q0[2 * i], a0);
+      a0 = dp4a_uu(hi, q0[2 * i + 1], a0);
+    } else {
+      a2 = dp4a_us(w[i], q2[i], a2);
+      a1 = dp4a_uu(w[i], q1[i], a1);
+      a0 = dp4a_uu(w[i], q0[i], a0);
+    }
+  }
+  // |a2| < 2^20, a1 * 256 + a0 < 2^29: both exact in int, one fp32 rounding each
+  return fmaf(static_cast<float>(a2), 65536.f, static_cast<float>(a1 * 256u + a0));
+}
+
+// Byte j (0, 1, 2) of the fixed-point value X (|X| < 2^23; byte 2 is the signed top byte).
+__device__ __forceinline__ uint32_t xbyte(int X, int j) { return static_cast<uint32_t>(X >> (8 * j)) & 0xFFu; }
+
+// Where code position o (0..PS-1) of a segment sits among the segment's quad bytes:
+// quad index (word*2 + odd for 4-bit, word for 8-bit) * 4 + byte.
+template <int BITS>
+__host__ __device__ constexpr int quad_pos(int o) {
+  return BITS == 4 ? ((o >> 3) * 2 + (o & 1)) * 4 + ((o & 7) >> 1) : o;
+}
+
+// 2^S with S chosen so that |x| < 2^22 * 2^-S for |x| <= m (a power of two, clamped to fp32 range).
+__device__ __forceinline__ int fix_exp(float m) {
+  if (!(m > 0.f)) return 0;
+  int e = ((__float_as_uint(m) >> 23) & 0xFF) - 127;  // floor(log2 m) for normal m
+  if (e < -100) e = -100;
+  return 21 - e;
+}
+__device__ __forceinline__ float pow2f(int s) { return __uint_as_float(static_cast<uint32_t>(s + 127) << 23); }
+
 }  // namespace
 }  // namespace moe

@@ -45,13 +45,17 @@ struct Layout {
   size_t hdr, counters, logits, sgate, h, r, xa, xb, y, idx, w;
   size_t dlogits, dh, dy, dyacc, dcnt, dr, dx;            // persistent single-token decode
   size_t base_total;                                      // end of the regions above
-  size_t perm, offs, chunks, nchunks, x16, hhi, hlo, o;   // batched tensor-core path
+  size_t perm, offs, chunks, nchunks, x16, hhi, hlo, o;   // batched paths (o: one plane per unit group for
+                                                          // the grouped GEMV, the first for the GEMM)
   size_t xsx, xsh;                                        // group sums of x and of h
+  size_t gxq, gxsc;                                       // grouped GEMV: fixed-point x, 2^-S per token
   size_t total;
 };
 
 constexpr int kBatchMinTokens = 8;  // from this many tokens the grouped tensor-core path runs (default)
 std::atomic<int> g_batch_min{kBatchMinTokens};  // moe_set_batched_min_tokens
+constexpr int kGemvMinTokens = 2;  // from this many tokens the grouped GEMV runs (default)
+std::atomic<int> g_gemv_min{kGemvMinTokens};  // moe_set_gemv_min_tokens
 
 constexpr int kMaxGrid = 1024;  // largest persistent decode grid
 
@@ -85,14 +89,20 @@ Layout layout(const moe_config& c, int64_t T) {
   const size_t np = static_cast<size_t>(T) * (c.top_k + 1);
   L.perm = o;     o += up(np * 4);
   L.offs = o;     o += up(static_cast<size_t>(c.num_experts + 2) * 4);
-  L.chunks = o;   o += up((static_cast<size_t>(c.num_experts) + 2 + np / moe::kChunkTokens + 1) * 12);
+  L.chunks = o;   o += up((static_cast<size_t>(c.num_experts) + 2 + np / moe::kGvTPI + 1) * 12);
   L.nchunks = o;  o += up(4);
   L.x16 = o;      o += up(np * c.hidden * 2);
   L.hhi = o;      o += up(np * imax * 2);
   L.hlo = o;      o += up(np * imax * 2);
-  L.o = o;        o += up(np * c.hidden * 4);
+  const size_t nq = c.inter / (32 * moe::kGvUPI) > 0 ? c.inter / (32 * moe::kGvUPI) : 1;
+  L.o = o;        o += up(nq * np * c.hidden * 4);
   L.xsx = o;      o += up(np * (c.hidden / 64 + 1) * 4);
   L.xsh = o;      o += up(np * (imax / 64 + 1) * 4 * 4);
+  {
+    const size_t ps = 128 / c.bits, nsg = c.hidden / ps, qsp = 3 * (ps / 4) + 1;
+    L.gxq = o;    o += up(static_cast<size_t>(T) * nsg * qsp * 4);
+    L.gxsc = o;   o += up(static_cast<size_t>(T) * 4);
+  }
   L.total = o;
   return L;
 }
@@ -385,6 +395,89 @@ moe_status batched_ffn(const moe_config& c, const moe_layer_weights& wt, const u
   return MOE_OK;
 }
 
+// ---------------------------------------------------------------- grouped GEMV path
+
+int device_smem_optin() {
+  int dev = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return 0;
+  return optin;
+}
+
+// Whether T tokens take the grouped GEMV (a few tokens per expert, CUDA cores): from
+// moe_set_gemv_min_tokens tokens up, below the batched tensor-core path's threshold (or where that
+// path does not apply), for shapes whose units of 32 columns come in whole groups of kGvUPI.
+bool gemv_eligible(const moe_config& c, int T) {
+  if (T < g_gemv_min.load(std::memory_order_relaxed)) return false;
+  if (batched_eligible(c, T)) return false;
+  if (!encode_fn()) return false;
+  const int optin = device_smem_optin();
+  if (optin < 1024) return false;
+  return moe::grouped_gemv_supported(c.hidden, c.inter, c.shared_inter, c.group, c.bits,
+                                     static_cast<size_t>(optin) - 1024);
+}
+
+// Experts' gate/up and down for T tokens given their selection, as grouped matrix-vector products.
+moe_status gemv_ffn(const moe_config& c, const moe_layer_weights& wt, const uint16_t* x, int T, const int32_t* idx,
+                    const float* w, uint16_t* y, void* ws, const Layout& Ly, cudaStream_t st) {
+  char* b = static_cast<char*>(ws);
+  const moe::WsView v = view(ws, Ly);
+  const int H = c.hidden, I = c.inter, k = c.top_k, E = c.num_experts;
+  const bool shared = c.shared_inter > 0;
+  const int np = T * k + (shared ? T : 0);
+  int32_t* perm = reinterpret_cast<int32_t*>(b + Ly.perm);
+  int32_t* chunks = reinterpret_cast<int32_t*>(b + Ly.chunks);
+  int32_t* nchunks = reinterpret_cast<int32_t*>(b + Ly.nchunks);
+  uint32_t* xq = reinterpret_cast<uint32_t*>(b + Ly.gxq);
+  float* xsc = reinterpret_cast<float*>(b + Ly.gxsc);
+  float* o = reinterpret_cast<float*>(b + Ly.o);
+  const int sms = device_sms();
+  if (sms < 1) return fail(MOE_ERR_CUDA, "no device");
+  moe::SortParams sp{idx, T, k, E, shared ? 1 : 0, perm, reinterpret_cast<int32_t*>(b + Ly.offs), chunks, nchunks,
+                     moe::kGvTPI, v.hdr};
+  cudaError_t e = moe::launch_sort_by_expert(sp, st);
+  if (e != cudaSuccess) return cuda_fail(e, "sort launch");
+  if ((e = moe::launch_xquant(x, wt.shared_gate_w, T, H, c.shared_inter, c.bits, xq, xsc, v.sgate, st)) != cudaSuccess)
+    return cuda_fail(e, "xquant launch");
+  auto gp = std::make_unique<moe::GemvParams>();
+  gp->chunks = chunks;
+  gp->nchunks = nchunks;
+  gp->perm = perm;
+  gp->xq = xq;
+  gp->xsc = xsc;
+  gp->gu = qmat(wt.gate_up);
+  gp->dn = qmat(wt.down);
+  gp->sgu = qmat(shared ? wt.shared_gate_up : wt.gate_up);
+  gp->sdn = qmat(shared ? wt.shared_down : wt.down);
+  gp->dcu = wt.down_units;
+  gp->dsb = wt.down_sb;
+  gp->sdcu = shared ? wt.shared_down_units : nullptr;
+  gp->sdsb = shared ? wt.shared_down_sb : nullptr;
+  const int64_t rb = static_cast<int64_t>(I) * c.bits / 8;
+  const int ub = 32 * c.bits / 8;
+  if (!wt.down_units &&
+      !map_3d(&gp->tm_dn, wt.down.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rb, H, E, wt.down.q_expert_stride, ub, 256))
+    return fail(MOE_ERR_CUDA, "tensor map of the down codes");
+  if (shared && !wt.shared_down_units &&
+      !map_3d(&gp->tm_sdn, wt.shared_down.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rb, H, 1, rb * H, ub, 256))
+    return fail(MOE_ERR_CUDA, "tensor map of the shared down codes");
+  gp->o = o;
+  gp->T = T;
+  gp->k = k;
+  gp->H = H;
+  gp->E = E;
+  gp->I = I;
+  gp->group = c.group;
+  gp->npairs = np;
+  gp->hdr = v.hdr;
+  if ((e = moe::launch_grouped_gemv(*gp, c.bits, sms, st)) != cudaSuccess) return cuda_fail(e, "grouped GEMV launch");
+  const int nq = I / (32 * moe::kGvUPI);
+  if ((e = moe::launch_gv_combine(o, w, v.sgate, T, k, H, c.shared_inter, nq, np, y, sms * 4, st)) != cudaSuccess)
+    return cuda_fail(e, "combine launch");
+  return MOE_OK;
+}
+
 // Device facts the persistent decode needs, looked up once per device.
 struct DevInfo {
   bool ok = false;
@@ -529,6 +622,7 @@ int32_t moe_stack_kernel_launches(const moe_config* cfg, int32_t T, int32_t L) {
   if (T == 1 && decode_eligible(*cfg, L, &grid))
     return (L + moe::kMaxDecodeLayers - 1) / moe::kMaxDecodeLayers;
   if (batched_eligible(*cfg, T)) return 1 + 7 * L;  // route, sort, gather, 2 GEMMs, combine, glue
+  if (gemv_eligible(*cfg, T)) return 1 + 6 * L;     // route, sort, xquant, GEMV, combine, glue
   return 1 + 4 * L;
 }
 
@@ -539,6 +633,7 @@ const char* moe_stack_path_name(const moe_config* cfg, int32_t T, int32_t L) {
   bool split = false;
   if (T == 1 && decode_eligible(*cfg, L, &grid, &split)) return split ? "decode_split_kernel" : "decode_stack_kernel";
   if (batched_eligible(*cfg, T)) return "batched";
+  if (gemv_eligible(*cfg, T)) return "grouped_gemv";
   return "per_layer";
 }
 
@@ -587,6 +682,8 @@ moe_status moe_expert_ffn(const moe_config* cfg, const moe_layer_weights* w, con
   if ((s = check_ws(*cfg, ws, ws_bytes, T, &L))) return s;
   if (batched_eligible(*cfg, T))
     return batched_ffn(*cfg, *w, x, T, topk_idx, topk_w, y, ws, L, reinterpret_cast<cudaStream_t>(stream));
+  if (gemv_eligible(*cfg, T))
+    return gemv_ffn(*cfg, *w, x, T, topk_idx, topk_w, y, ws, L, reinterpret_cast<cudaStream_t>(stream));
   return ffn(*cfg, *w, x, T, topk_idx, topk_w, y, view(ws, L), reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -610,6 +707,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if ((s = route(*cfg, x, T, w->router_w, w->router_bias, idx, wt, v, st))) return s;
   if (batched_eligible(*cfg, T)) return batched_ffn(*cfg, *w, x, T, idx, wt, y, ws, L, st);
+  if (gemv_eligible(*cfg, T)) return gemv_ffn(*cfg, *w, x, T, idx, wt, y, ws, L, st);
   return ffn(*cfg, *w, x, T, idx, wt, y, v, st);
 }
 
@@ -638,6 +736,7 @@ moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weights* lay
   if (T == 1 && decode_eligible(*cfg, L, &grid, &split, &split_late, &split_two))
     return stack_decode(*cfg, layers, L, x0, x_out, trace, ws, Ly, grid, split, split_late, split_two, st);
   const bool batched = batched_eligible(*cfg, T);
+  const bool gemv = !batched && gemv_eligible(*cfg, T);
   const size_t TH = static_cast<size_t>(T) * cfg->hidden;
   const size_t Tk = static_cast<size_t>(T) * cfg->top_k;
   float* r = reinterpret_cast<float*>(b + Ly.r);
@@ -657,6 +756,7 @@ moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weights* lay
     uint16_t* y = (trace && trace->y) ? trace->y + l * TH : reinterpret_cast<uint16_t*>(b + Ly.y);
     if ((s = route(*cfg, xcur, T, layers[l].router_w, layers[l].router_bias, idx, wt, v, st))) return s;
     if (batched) s = batched_ffn(*cfg, layers[l], xcur, T, idx, wt, y, ws, Ly, st);
+    else if (gemv) s = gemv_ffn(*cfg, layers[l], xcur, T, idx, wt, y, ws, Ly, st);
     else s = ffn(*cfg, layers[l], xcur, T, idx, wt, y, v, st);
     if (s) return s;
     uint16_t* xnext;
@@ -730,6 +830,10 @@ moe_status moe_prepare_down_units(const moe_config* cfg, const moe_qtensor* down
 
 int32_t moe_set_batched_min_tokens(int32_t T) {
   return g_batch_min.exchange(T < 1 ? kBatchMinTokens : T);
+}
+
+int32_t moe_set_gemv_min_tokens(int32_t T) {
+  return g_gemv_min.exchange(T < 1 ? kGemvMinTokens : T);
 }
 
 moe_status moe_check_wait_limit(void* ws, size_t ws_bytes, int32_t* gave_up, moe_stream_t stream) {

@@ -150,6 +150,34 @@ struct DecodeParams {
   CUtensorMap tm_sdn[kMaxDecodeLayers];
 };
 
+// Grouped GEMV (csrc/grouped_gemv.cu): the batched path on the CUDA cores for a few tokens per
+// expert. A work item is (chunk of <= kGvTPI pairs of one expert, group of kGvUPI 32-column units).
+constexpr int kGvTPI = 4;  // pairs per chunk
+constexpr int kGvUPI = 4;  // units per item
+struct GemvParams {
+  const int32_t* chunks;   // [nchunks][3]: expert (E = shared), first sorted position, pair count
+  const int32_t* nchunks;
+  const int32_t* perm;     // sorted position -> pair id
+  const uint32_t* xq;      // [T][H / codes-per-16-bytes][quad words + 1] fixed-point x of every token
+  const float* xsc;        // [T] 2^-S of every token's x
+  QMat gu, dn, sgu, sdn;
+  const uint8_t* dcu;      // unit-major down codes (moe_prepare_down_units) or null
+  const uint8_t* sdcu;
+  const uint16_t* dsb;     // group-major down scales and biases (moe_prepare_down_sb) or null
+  const uint16_t* sdsb;
+  CUtensorMap tm_dn, tm_sdn;  // canonical down codes (when dcu / sdcu are null)
+  float* o;                // [I / (32 kGvUPI)][npairs][H] partial expert outputs by pair id
+  int T, k, H, E, I, group, npairs;
+  WsHeader* hdr;
+};
+bool grouped_gemv_supported(int H, int I, int Is, int group, int bits, size_t smem_limit);
+size_t grouped_gemv_smem(int H, int I, int group, int bits);
+cudaError_t launch_xquant(const uint16_t* x, const uint16_t* wsg, int T, int H, int Is, int bits, uint32_t* xq,
+                          float* xsc, float* sgate, cudaStream_t st);
+cudaError_t launch_grouped_gemv(const GemvParams& p, int bits, int grid, cudaStream_t st);
+cudaError_t launch_gv_combine(const float* o, const float* w, const float* sgate, int T, int k, int H, int Is, int nq,
+                              int npairs, uint16_t* y, int grid, cudaStream_t st);
+
 cudaError_t launch_route_topk(const RouteParams& p, cudaStream_t stream);
 cudaError_t launch_expert_ffn(const FfnParams& p, int bits, cudaStream_t stream);
 cudaError_t launch_glue(const GlueParams& p, cudaStream_t stream);

@@ -40,15 +40,29 @@ def layer35():
 
 @pytest.mark.parametrize("key", ["35b", "35b8", "80b"])
 def test_batched_path_is_taken(key):
-    """The workloads' shapes must run on the tensor-core path from 8 tokens up
-    (route, sort, gather, two GEMMs, combine, glue: 7 kernels a layer), not
-    fall back to the token-at-a-time kernels (4 a layer)."""
+    """With the thresholds at 8 (batched) and 2 (grouped GEMV), the workloads'
+    shapes run on the tensor-core path from 8 tokens up (route, sort, gather,
+    two GEMMs, combine, glue: 7 kernels a layer), on the grouped GEMV from 2
+    to 7 tokens (route, quantise x, sort, GEMV, combine, glue: 6 a layer; 4-bit
+    shapes only), and on the token-at-a-time kernels (4 a layer) when the GEMV
+    is switched off."""
     cfg = moe.make_config(synth.SHAPES[key])
-    assert moe.moe_stack_kernel_launches(cfg, 8, 3) == 1 + 7 * 3
-    assert moe.moe_stack_kernel_launches(cfg, 512, 3) == 1 + 7 * 3
-    assert moe.moe_stack_kernel_launches(cfg, 7, 3) == 1 + 4 * 3
-    assert moe.moe_stack_path_name(cfg, 8, 3) == moe.moe_stack_path_name(cfg, 512, 3) == "batched"
-    assert moe.moe_stack_path_name(cfg, 7, 3) == "per_layer"
+    pb, pg = moe.moe_set_batched_min_tokens(8), moe.moe_set_gemv_min_tokens(2)
+    try:
+        assert moe.moe_stack_kernel_launches(cfg, 8, 3) == 1 + 7 * 3
+        assert moe.moe_stack_kernel_launches(cfg, 512, 3) == 1 + 7 * 3
+        assert moe.moe_stack_path_name(cfg, 8, 3) == moe.moe_stack_path_name(cfg, 512, 3) == "batched"
+        if synth.SHAPES[key].bits == 4:
+            assert moe.moe_stack_kernel_launches(cfg, 7, 3) == 1 + 6 * 3
+            assert moe.moe_stack_path_name(cfg, 7, 3) == moe.moe_stack_path_name(cfg, 2, 3) == "grouped_gemv"
+        else:  # 8-bit: two buffers of 32 gate/up row pairs (2 x 136 KB) exceed shared memory
+            assert moe.moe_stack_path_name(cfg, 7, 3) == "per_layer"
+        moe.moe_set_gemv_min_tokens(1 << 30)
+        assert moe.moe_stack_kernel_launches(cfg, 7, 3) == 1 + 4 * 3
+        assert moe.moe_stack_path_name(cfg, 7, 3) == "per_layer"
+    finally:
+        moe.moe_set_batched_min_tokens(pb)
+        moe.moe_set_gemv_min_tokens(pg)
 
 
 @pytest.mark.parametrize("T", [7, 8, 16])

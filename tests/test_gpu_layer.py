@@ -76,11 +76,35 @@ def test_tiny_route_and_ffn_calls_match_layer(tiny):
 
 
 def test_batch_equals_single_token_calls(tiny):
+    """The per-token kernels give a token the same bits alone as in a batch of 13."""
     lw, host, x = tiny
-    idx, w, y = _run_layer(TINY, lw, x[:13])
-    for t in range(13):
-        i1, w1, y1 = _run_layer(TINY, lw, x[t:t + 1])
-        assert np.array_equal(i1[0], idx[t]) and np.array_equal(w1[0], w[t]) and np.array_equal(y1[0], y[t])
+    pg = moe.moe_set_gemv_min_tokens(1 << 30)  # keep 13 tokens on the per-token kernels
+    try:
+        assert moe.moe_stack_path_name(moe.make_config(TINY), 13, 1) == "per_layer"
+        idx, w, y = _run_layer(TINY, lw, x[:13])
+        for t in range(13):
+            i1, w1, y1 = _run_layer(TINY, lw, x[t:t + 1])
+            assert np.array_equal(i1[0], idx[t]) and np.array_equal(w1[0], w[t]) and np.array_equal(y1[0], y[t])
+    finally:
+        moe.moe_set_gemv_min_tokens(pg)
+
+
+def test_grouped_gemv_is_batch_invariant(tiny):
+    """On the grouped GEMV a token's output depends on its own x alone (its own fixed-point scale,
+    partial sums combined in a fixed order): the same bits in a batch of 13 as in a batch of two
+    copies of it."""
+    lw, host, x = tiny
+    pg, pb = moe.moe_set_gemv_min_tokens(2), moe.moe_set_batched_min_tokens(1 << 30)
+    try:
+        assert moe.moe_stack_path_name(moe.make_config(TINY), 13, 1) == "grouped_gemv"
+        idx, w, y = _run_layer(TINY, lw, x[:13])
+        for t in range(13):
+            i2, w2, y2 = _run_layer(TINY, lw, x[t:t + 1].repeat(2, 1))
+            for r in range(2):
+                assert np.array_equal(i2[r], idx[t]) and np.array_equal(w2[r], w[t]) and np.array_equal(y2[r], y[t])
+    finally:
+        moe.moe_set_gemv_min_tokens(pg)
+        moe.moe_set_batched_min_tokens(pb)
 
 
 def test_empty_batch_is_noop(tiny):

@@ -176,10 +176,18 @@ def test_single_token_path_matches_multi_kernel_path():
     layers = [synth.make_layer(shape, l, "cuda", seed_id=2) for l in range(shape.layers)]
     cfg = moe.make_config(shape)
     assert moe.moe_stack_kernel_launches(cfg, 1, 4) == 1
-    assert moe.moe_stack_kernel_launches(cfg, 2, 4) == 17
     x1 = synth.make_tokens(shape, [7], "cuda", seed_id=2)
     tx, ti, tw, ty, _ = run_stack(shape, layers, x1)
     ws = moe.Workspace(cfg, 2)
+    pg = moe.moe_set_gemv_min_tokens(1 << 30)  # the four-kernel per-token path for T=2
+    try:
+        assert moe.moe_stack_kernel_launches(cfg, 2, 4) == 17
+        _compare_with_per_layer(shape, cfg, layers, tx, ti, tw, ty, ws)
+    finally:
+        moe.moe_set_gemv_min_tokens(pg)
+
+
+def _compare_with_per_layer(shape, cfg, layers, tx, ti, tw, ty, ws):
     for l in range(shape.layers):
         xl = torch.from_numpy(tx[l].astype(np.int16)).view(torch.bfloat16).cuda().repeat(2, 1)
         y = torch.empty(2, shape.hidden, dtype=torch.bfloat16, device="cuda")
