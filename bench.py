@@ -336,8 +336,8 @@ PARITY_TESTS = {
     "35b": "tests/test_gpu_stack.py::test_decode_stack_parity[35b]",
     "80b": "tests/test_gpu_stack.py::test_decode_stack_parity[80b]",
     "35b8": "tests/test_gpu_stack.py::test_decode_stack_parity[35b8]",
-    "35b_t64": "tests/test_gpu_stack.py::test_batched_stack_parity[35b_t64]",
-    "35b_t512": "tests/test_gpu_stack.py::test_batched_stack_parity[35b_t512]",
+    "35b_t64": "tests/test_gpu_stack.py::test_batched_stack_parity[35b_t64-grouped_gemv]",
+    "35b_t512": "tests/test_gpu_stack.py::test_batched_stack_parity[35b_t512-batched]",
 }
 
 
@@ -435,7 +435,7 @@ def secondary(keys, steps, warmup, peak, budget_s=150.0):
     return out
 
 
-def dispatch_sweep(steps=8, warmup=3, Ts=(1, 2, 3, 4, 6, 8, 12, 16, 24, 32, 48, 64), key=None):
+def dispatch_sweep(steps=8, warmup=3, Ts=(1, 2, 3, 4, 6, 8, 12, 16, 24, 32, 48, 64, 96, 128, 192, 256, 512), key=None):
     """The three multi-token paths for T tokens through a stack (the per-token kernels, the grouped
     GEMV, the batched tensor-core path; moe_set_gemv_min_tokens / moe_set_batched_min_tokens pick
     one; one token through a stack always runs the persistent decode kernel): one JSON line per

@@ -206,7 +206,7 @@ MOE_API const char* moe_stack_path_name(const moe_config* cfg, int32_t T, int32_
 /* Sets the token count from which moe_layer_forward, moe_expert_ffn and
  * moe_stack_forward take the batched tensor-core path (where the shape
  * supports it) instead of the per-token kernels, for the whole process and
- * every device; T < 1 restores the default (8). Returns the previous value.
+ * every device; T < 1 restores the default (128). Returns the previous value.
  * A single token through a stack keeps its persistent kernel whatever the
  * value. Meant for measuring the two paths against each other (bench.py
  * --sweep); calls already enqueued are not affected. Not on the pages. */
@@ -216,7 +216,7 @@ MOE_API int32_t moe_set_batched_min_tokens(int32_t T);
  * (a few tokens per expert: each selected expert's weights read once for
  * all of its tokens, dot products on the CUDA cores) instead of the
  * per-token kernels, below the batched threshold; T < 1 restores the
- * default (2). Returns the previous value. Process-wide, as above. Not on
+ * default (8). Returns the previous value. Process-wide, as above. Not on
  * the pages. */
 MOE_API int32_t moe_set_gemv_min_tokens(int32_t T);
 

@@ -357,30 +357,76 @@ __global__ void __launch_bounds__(kWarps * 32)
 
 // ------------------------------------------------------------------ stack glue
 
+// One CTA per token, 256 threads, each thread runs of 8 elements (H <= 8192): every load of the
+// token is issued before the first add, then r += y (or r = x), the sum of squares, and x_out.
+constexpr int kGlueRuns = 4;  // runs of 8 per thread: 4 * 256 * 8 = 8192 elements
 __global__ void __launch_bounds__(256) glue_kernel(GlueParams p) {
   const int t = blockIdx.x;
   float* r = p.r + static_cast<size_t>(t) * p.H;
+  const size_t row = static_cast<size_t>(t) * p.H;
+  const int n8 = p.H / 8;
+  float4 ra[kGlueRuns][2];
+  uint4 ya[kGlueRuns];
+#pragma unroll
+  for (int c = 0; c < kGlueRuns; ++c) {
+    const int i8 = threadIdx.x + 256 * c;
+    if (i8 < n8) {
+      if (p.y) {
+        ra[c][0] = *reinterpret_cast<const float4*>(r + 8 * i8);
+        ra[c][1] = *reinterpret_cast<const float4*>(r + 8 * i8 + 4);
+        ya[c] = *reinterpret_cast<const uint4*>(p.y + row + 8 * i8);
+      } else {
+        ya[c] = *reinterpret_cast<const uint4*>(p.x_in + row + 8 * i8);
+      }
+    }
+  }
   float ss = 0.f;
-  for (int i = threadIdx.x; i < p.H; i += blockDim.x) {
-    const size_t o = static_cast<size_t>(t) * p.H + i;
-    const float v = p.y ? r[i] + bf16_to_f32(p.y[o]) : bf16_to_f32(p.x_in[o]);
-    r[i] = v;
-    ss = fmaf(v, v, ss);
+#pragma unroll
+  for (int c = 0; c < kGlueRuns; ++c) {
+    const int i8 = threadIdx.x + 256 * c;
+    if (i8 < n8) {
+      const uint4 v = ya[c];
+      float a[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                    bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+      if (p.y) {
+        a[0] += ra[c][0].x;
+        a[1] += ra[c][0].y;
+        a[2] += ra[c][0].z;
+        a[3] += ra[c][0].w;
+        a[4] += ra[c][1].x;
+        a[5] += ra[c][1].y;
+        a[6] += ra[c][1].z;
+        a[7] += ra[c][1].w;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ss = fmaf(a[u], a[u], ss);
+      ra[c][0] = make_float4(a[0], a[1], a[2], a[3]);
+      ra[c][1] = make_float4(a[4], a[5], a[6], a[7]);
+      *reinterpret_cast<float4*>(r + 8 * i8) = ra[c][0];
+      *reinterpret_cast<float4*>(r + 8 * i8 + 4) = ra[c][1];
+    }
   }
   if (!p.x_out) return;
-  __shared__ float red[32];
+  __shared__ float red[8];
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
-  if (threadIdx.x < 32) {
-    float v = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.f;
-    v = warp_sum(v);
-    if (threadIdx.x == 0) red[0] = v;
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += red[w];
+  const float inv = 1.f / sqrtf(tot / static_cast<float>(p.H) + p.eps);
+#pragma unroll
+  for (int c = 0; c < kGlueRuns; ++c) {
+    const int i8 = threadIdx.x + 256 * c;
+    if (i8 < n8) {
+      uint4 o;
+      o.x = static_cast<uint32_t>(f32_to_bf16(ra[c][0].x * inv)) | (static_cast<uint32_t>(f32_to_bf16(ra[c][0].y * inv)) << 16);
+      o.y = static_cast<uint32_t>(f32_to_bf16(ra[c][0].z * inv)) | (static_cast<uint32_t>(f32_to_bf16(ra[c][0].w * inv)) << 16);
+      o.z = static_cast<uint32_t>(f32_to_bf16(ra[c][1].x * inv)) | (static_cast<uint32_t>(f32_to_bf16(ra[c][1].y * inv)) << 16);
+      o.w = static_cast<uint32_t>(f32_to_bf16(ra[c][1].z * inv)) | (static_cast<uint32_t>(f32_to_bf16(ra[c][1].w * inv)) << 16);
+      *reinterpret_cast<uint4*>(p.x_out + row + 8 * i8) = o;
+    }
   }
-  __syncthreads();
-  const float inv = 1.f / sqrtf(red[0] / static_cast<float>(p.H) + p.eps);
-  for (int i = threadIdx.x; i < p.H; i += blockDim.x)
-    p.x_out[static_cast<size_t>(t) * p.H + i] = f32_to_bf16(r[i] * inv);
 }
 
 template <typename K>

@@ -1,30 +1,34 @@
 // The batched path for a few tokens per expert: a grouped matrix-vector
 // product on the CUDA cores. Tokens are grouped by expert (counting sort,
-// sort_by_expert.cu, in chunks of at most kTPI pairs), and each chunk's
+// sort_by_expert.cu, in chunks of at most kGvTPI pairs), and each chunk's
 // expert weights are read once for all of the chunk's tokens, 32 columns of
 // the intermediate (a unit) at a time:
 //
 //   xquant   every token's x as the fixed-point quads of the integer dot
 //            products (decode_common.cuh: X = rint(x * 2^S), three bytes),
 //            per token its own S; also the shared expert's sigmoid gate;
-//   gemv     per work item (chunk, group of kUPI units): for each unit, the
-//            32 gate/up row pairs and their scales and biases (bulk copies,
-//            two buffers so that the next unit's rows stream in while this
-//            one is computed), h = silu(gate) * up for each of the chunk's
-//            tokens, then the unit's 32 columns of all H down rows (one
-//            contiguous block of the unit-major down copy) against each
-//            token's h; each thread keeps its rows' sums for every token of
-//            the chunk in registers over the item's units and stores them
-//            once, as the item's partial of each pair's expert output;
+//   gemv     per work item (chunk, group of upi units, upi = 1, 2 or 4 as
+//            gemv_units_per_item picks for the batch size): the item's
+//            tokens' quads (bulk copies, issued while the previous item's
+//            down rows are computed); for each unit, the 32 gate/up row pairs
+//            and their scales and biases (bulk copies, two buffers so that
+//            the next unit's rows stream in while this one is computed),
+//            h = silu(gate) * up for each of the chunk's tokens, then the
+//            unit's 32 columns of all H down rows (one contiguous block of
+//            the unit-major down copy) against each token's h; each thread
+//            keeps its rows' sums for every token of the chunk in registers
+//            over the item's units and stores them once, as the item's
+//            partial of each pair's expert output;
 //   combine  y = sum_j w_j (sum over items of o_j) + gate * o_shared, rank
 //            order, one bf16 rounding.
-// With 1-4 tokens per expert (batches of up to a few dozen tokens over 256
-// experts) the tensor cores would multiply mostly padding, and the path is
-// bound by reading every selected expert once; the dot products run as in
-// the single-token decode kernel (stack_split.cu). MLX-style affine groups
-// (Swiftlet article on xix.ai, paragraph 8), packed routed gate/up (Runnel
-// README, introduction and "Streaming CLI"), shared expert (same article,
-// paragraph 8; Runnel README, "Target").
+// With 1-4 tokens per expert (batches of up to about a hundred tokens over
+// 256 experts) the tensor cores would multiply mostly padding; the dot
+// products run as in the single-token decode kernel (stack_split.cu), so
+// with more than a token or two per chunk the kernel is bound by its integer
+// instruction issue rather than by reading every selected expert once.
+// MLX-style affine groups (Swiftlet article on xix.ai, paragraph 8), packed
+// routed gate/up (Runnel README, introduction and "Streaming CLI"), shared
+// expert (same article, paragraph 8; Runnel README, "Target").
 
 #include "decode_common.cuh"
 #include "moe_common.cuh"
@@ -56,7 +60,7 @@ __host__ __device__ inline GvCarve gv_carve(int H, int I, int group, int bits) {
   c.PS = 128 / bits;
   c.nsg = H / c.PS;
   c.QS = 3 * (c.PS / 4);
-  c.QSP = c.QS + 1;
+  c.QSP = bits == 4 ? xq_stride<4>() : xq_stride<8>();  // quads + sum, padded for 16-byte loads
   c.ng = H / group;
   c.ngd = I / group;
   c.rowb = H * bits / 8;
@@ -99,15 +103,18 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
   extern __shared__ __align__(128) unsigned char sm[];
   __shared__ __align__(8) uint64_t bar_gc[2][kNB];  // gate/up batches of buffer 0 / 1
   __shared__ __align__(8) uint64_t bar_dn;
-  __shared__ int s_pend_gc[2], s_pend_dn;           // copies in flight (phase parity, -1 = none)
+  __shared__ __align__(8) uint64_t bar_x;           // the item's tokens' quads
+  __shared__ int s_pend_gc[2], s_pend_dn, s_pend_x; // copies in flight (phase parity, -1 = none)
   __shared__ float s_xsc[kGvTPI];                   // 2^-S of the item's tokens' x
+  __shared__ int s_first, s_cnt;                    // the item's pairs: first sorted position, count
 
   const int H = p.H, I = p.I, group = p.group;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const GvCarve cv = gv_carve(H, I, group, BITS);
   const int rowb = cv.rowb, ng = cv.ng, nsg = cv.nsg;
   const int lgG = 31 - __clz(group);
-  const int NQ = I / (kUnit * kGvUPI);       // unit groups per expert
+  const int upi = p.upi;                     // units per item
+  const int NQ = I / (kUnit * upi);          // unit groups per expert
   const int nitems = *p.nchunks * NQ;
   bool ab = false;
 
@@ -115,22 +122,23 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
     for (int b = 0; b < 2; ++b)
       for (int i = 0; i < kNB; ++i) mbar_init(&bar_gc[b][i], 1);
     mbar_init(&bar_dn, 1);
+    mbar_init(&bar_x, 1);
     fence_mbar_init();
-    s_pend_gc[0] = s_pend_gc[1] = s_pend_dn = -1;
+    s_pend_gc[0] = s_pend_gc[1] = s_pend_dn = s_pend_x = -1;
   }
   __syncthreads();
 
-  // the CTA's stream of units: unit m belongs to item blockIdx.x + (m / kGvUPI) * gridDim.x
+  // the CTA's stream of units: unit m belongs to item blockIdx.x + (m / upi) * gridDim.x
   auto unit_of = [&](int m, GvUnit& u) -> bool {
-    const int it = blockIdx.x + (m / kGvUPI) * gridDim.x;
+    const int it = blockIdx.x + (m / upi) * gridDim.x;
     if (it >= nitems) return false;
     u.ci = it / NQ;
     u.q = it - u.ci * NQ;
-    u.uu = m % kGvUPI;
+    u.uu = m % upi;
     const int e = p.chunks[3 * u.ci];
     u.routed = e < p.E;
     u.e = u.routed ? e : 0;
-    u.i0 = (u.q * kGvUPI + u.uu) * kUnit;
+    u.i0 = (u.q * upi + u.uu) * kUnit;
     return true;
   };
   // gate/up rows of unit u into buffer b (one thread): batch 0 (16 gate + 16 up rows, every
@@ -175,6 +183,31 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
                static_cast<uint32_t>(H) * 4, &bar_dn);
     s_pend_dn = par;
   };
+  // the item of unit u: its pairs (one thread) and its tokens' quads (one bulk copy per token, rows of
+  // the per-token table xquant_kernel wrote) with their 2^-S; phase `par` of bar_x
+  const int xwords = nsg * cv.QSP;
+  auto issue_x = [&](const GvUnit& u, int par) {
+    const int first = p.chunks[3 * u.ci + 1], cnt_u = p.chunks[3 * u.ci + 2];
+    int tok[kGvTPI];
+#pragma unroll
+    for (int t = 0; t < kGvTPI; ++t) {
+      const int pid = t < cnt_u ? p.perm[first + t] : 0;
+      tok[t] = pid < p.T * p.k ? pid / p.k : pid - p.T * p.k;
+    }
+    s_first = first;
+    s_cnt = cnt_u;
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the buffer was read by ordinary loads
+    mbar_arrive_expect_tx(&bar_x, static_cast<uint32_t>(cnt_u * xwords * 4));
+#pragma unroll
+    for (int t = 0; t < kGvTPI; ++t)
+      if (t < cnt_u) {
+        bulk_g2s(sm + cv.xqs + t * xwords * 4, p.xq + static_cast<size_t>(tok[t]) * xwords,
+                 static_cast<uint32_t>(xwords * 4), &bar_x);
+        s_xsc[t] = p.xsc[tok[t]];
+      }
+    s_pend_x = par;
+  };
+  constexpr int kXThread = kThreads - 32;  // lane 0 of the last warp (idle in SwiGLU for <= kGvTPI tokens)
   auto drain = [&]() {
     __syncthreads();
     if (tid == 0) {
@@ -182,11 +215,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
         if (s_pend_gc[b] >= 0)
           for (int i = 0; i < kNB; ++i) mbar_wait(&bar_gc[b][i], s_pend_gc[b], p.hdr, 70);
       if (s_pend_dn >= 0) mbar_wait(&bar_dn, s_pend_dn, p.hdr, 71);
+      if (s_pend_x >= 0) mbar_wait(&bar_x, s_pend_x, p.hdr, 74);
     }
     __syncthreads();
   };
 
-  // prologue: the first two units' gate/up rows, the first unit's down data
+  // prologue: the first two units' gate/up rows, the first unit's down data, the first item's x
   GvUnit u0;
   if (!unit_of(0, u0)) return;
   if (tid == 0) {
@@ -195,6 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
     if (unit_of(1, u1)) issue_gu(u1, 1, 0);
     issue_dn(u0, 0);
   }
+  if (tid == kXThread) issue_x(u0, 0);
+  __syncthreads();
 
   // lane roles in the gate/up dot products (as in the decode kernel)
   const int rps = nsg >= 32 ? 1 : 32 / nsg;
@@ -212,22 +248,15 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
     if (!unit_of(m, u)) break;
     const int b = m & 1;  // gate/up buffer; its phase parity (m / 2) & 1; the down phase m & 1
     if (u.uu == 0) {
-      // ---- a new item: its tokens' quads into shared memory, the accumulators cleared
-      first = p.chunks[3 * u.ci + 1];
-      cnt = p.chunks[3 * u.ci + 2];
-      const int words = nsg * cv.QSP;
-      for (int t = 0; t < cnt; ++t) {
-        const int pid = p.perm[first + t];
-        const int tok = pid < p.T * p.k ? pid / p.k : pid - p.T * p.k;
-        const uint32_t* src = p.xq + static_cast<size_t>(tok) * words;
-        for (int i = tid; i < words; i += kThreads) xqs[t * words + i] = __ldg(src + i);
-        if (tid == 0) s_xsc[t] = p.xsc[tok];
-      }
+      // ---- a new item (its pairs and x issued during the previous item): the accumulators cleared,
+      // the x quads awaited
+      first = s_first;
+      cnt = s_cnt;
 #pragma unroll
       for (int t = 0; t < kGvTPI; ++t)
 #pragma unroll
         for (int r = 0; r < 4; ++r) acc[t][r] = 0.f;
-      __syncthreads();
+      if (!mbar_wait(&bar_x, (m / upi) & 1, p.hdr, 75)) ab = true;
     }
     // ---- gate/up + SwiGLU of unit u for every token of the item
     {
@@ -269,7 +298,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
               const int s = gs0 + 32 * ch;
               uint32_t xr[3 * QW];
 #pragma unroll
-              for (int w = 0; w < 3 * QW; ++w) xr[w] = xt[s * cv.QSP + w];
+              for (int w = 0; w < 3 * QW; w += 4) {
+                const uint4 v4 = *reinterpret_cast<const uint4*>(xt + s * cv.QSP + w);
+                xr[w] = v4.x;
+                xr[w + 1] = v4.y;
+                xr[w + 2] = v4.z;
+                xr[w + 3] = v4.w;
+              }
               const float xsm = __uint_as_float(xt[s * cv.QSP + cv.QS]);
 #pragma unroll
               for (int r2 = 0; r2 < 2; ++r2) {
@@ -305,6 +340,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
     if (tid == 0) {
       GvUnit un;
       if (unit_of(m + 2, un)) issue_gu(un, b, ((m + 2) >> 1) & 1);
+    }
+    // after the item's last gate/up the x buffer is free: the next item's pairs and x
+    if (tid == kXThread && u.uu == upi - 1) {
+      s_pend_x = -1;
+      GvUnit un;
+      if (unit_of(m + 1, un)) issue_x(un, ((m + 1) / upi) & 1);
     }
     // SwiGLU; each token's h as fixed point (its own exponent), quads for the down rows
     if (warp < cnt) {
@@ -373,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
       if (unit_of(m + 1, un)) issue_dn(un, (m + 1) & 1);
     }
     // ---- the item's last unit: its partial of each pair's expert output
-    if (u.uu == kGvUPI - 1) {
+    if (u.uu == upi - 1) {
       float* ob = p.o + static_cast<size_t>(u.q) * p.npairs * H;
 #pragma unroll
       for (int t = 0; t < kGvTPI; ++t) {
@@ -391,16 +432,19 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
   drain();
 }
 
-// Every token's x as the fixed-point quads the gate/up dot products read ([T][nsg][QSP] words:
-// per segment the three byte planes' quads and the segment's sum of X), its 2^-S, and the shared
-// expert's sigmoid gate. One CTA per token, H/4 threads, each thread 4 consecutive elements.
+// Every token's x as the fixed-point quads the gate/up dot products read ([T][nsg][QSP] words,
+// QSP = xq_stride: per segment the three byte planes' quads, the segment's sum of X, padding), its
+// 2^-S, and the shared expert's sigmoid gate. One CTA per token, H/4 threads, each thread 4
+// consecutive elements (element group g = thread g: its partner group g ^ 1 is the neighbouring
+// lane, the PS / 4 groups of a segment are consecutive lanes).
 template <int BITS>
 __global__ void xquant_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wsg, int H, int Is,
                               uint32_t* __restrict__ xq, float* __restrict__ xsc, float* __restrict__ sgate) {
   constexpr int PS = 128 / BITS;
   constexpr int QW = PS / 4;
   const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nsg = H / PS, QSP = 3 * QW + 1;
+  constexpr int QSP = xq_stride<BITS>();
+  const int nsg = H / PS;
   __shared__ float s_red[2][16];
   const uint2 wv = *reinterpret_cast<const uint2*>(x + static_cast<size_t>(t) * H + 4 * tid);
   const float xv[4] = {bf16_lo(wv.x), bf16_hi(wv.x), bf16_lo(wv.y), bf16_hi(wv.y)};
@@ -462,29 +506,65 @@ __global__ void xquant_kernel(const uint16_t* __restrict__ x, const uint16_t* __
 }
 
 // y[t][r] = bf16( sum_j w[t][j] * sum_q O[q][t*k+j][r] + gate[t] * sum_q O[q][T*k+t][r] ), rank order,
-// the partials of each pair summed in order, the shared expert last.
+// the partials of each pair summed in order, the shared expert last. Each thread four consecutive rows
+// (16-byte loads); the (pair, partial) terms are walked in that order 16 loads at a time, across pair
+// boundaries, so a thread waits for ceil((k + 1) * nq / 16) round trips.
 __global__ void __launch_bounds__(256) gv_combine_kernel(const float* __restrict__ o, const float* __restrict__ w,
                                                          const float* __restrict__ sgate, int T, int k, int H, int Is,
                                                          int nq, int npairs, uint16_t* __restrict__ y) {
-  const size_t n = static_cast<size_t>(T) * H;
+  constexpr int kBatchLoads = 16;
+  const size_t n4 = static_cast<size_t>(T) * H / 4;
   const size_t plane = static_cast<size_t>(npairs) * H;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+  const int nslot = k + (Is > 0 ? 1 : 0);
+  const int nterm = nslot * nq;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const int t = static_cast<int>(i / H), r = static_cast<int>(i % H);
-    float acc = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const size_t base = (static_cast<size_t>(t) * k + j) * H + r;
-      float v = 0.f;
-      for (int q = 0; q < nq; ++q) v += o[q * plane + base];
-      acc = fmaf(w[static_cast<size_t>(t) * k + j], v, acc);
+    const int t = static_cast<int>((4 * i) / H), r = static_cast<int>((4 * i) % H);
+    auto term_addr = [&](int j, int q) -> const float4* {  // slot j, partial q
+      const size_t pid = j < k ? static_cast<size_t>(t) * k + j : static_cast<size_t>(T) * k + t;
+      return reinterpret_cast<const float4*>(o + q * plane + pid * H + r);
+    };
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f), s = acc;
+    int jl = 0, ql = 0;  // next term to load
+    int jc = 0, qc = 0;  // next term to add
+#pragma unroll 1
+    for (int f0 = 0; f0 < nterm; f0 += kBatchLoads) {
+      float4 v[kBatchLoads];
+#pragma unroll
+      for (int b = 0; b < kBatchLoads; ++b)
+        if (f0 + b < nterm) {
+          v[b] = __ldg(term_addr(jl, ql));
+          if (++ql == nq) {
+            ql = 0;
+            ++jl;
+          }
+        }
+#pragma unroll
+      for (int b = 0; b < kBatchLoads; ++b)
+        if (f0 + b < nterm) {
+          if (qc == 0) {
+            s = v[b];
+          } else {
+            s.x += v[b].x;
+            s.y += v[b].y;
+            s.z += v[b].z;
+            s.w += v[b].w;
+          }
+          if (++qc == nq) {  // the pair's sum is complete
+            const float c = jc < k ? w[static_cast<size_t>(t) * k + jc] : sgate[t];
+            acc.x = fmaf(c, s.x, acc.x);
+            acc.y = fmaf(c, s.y, acc.y);
+            acc.z = fmaf(c, s.z, acc.z);
+            acc.w = fmaf(c, s.w, acc.w);
+            qc = 0;
+            ++jc;
+          }
+        }
     }
-    if (Is > 0) {
-      const size_t base = (static_cast<size_t>(T) * k + t) * H + r;
-      float v = 0.f;
-      for (int q = 0; q < nq; ++q) v += o[q * plane + base];
-      acc = fmaf(sgate[t], v, acc);
-    }
-    y[i] = f32_to_bf16(acc);
+    uint2 packed;
+    packed.x = static_cast<uint32_t>(f32_to_bf16(acc.x)) | (static_cast<uint32_t>(f32_to_bf16(acc.y)) << 16);
+    packed.y = static_cast<uint32_t>(f32_to_bf16(acc.z)) | (static_cast<uint32_t>(f32_to_bf16(acc.w)) << 16);
+    *reinterpret_cast<uint2*>(y + 4 * i) = packed;
   }
 }
 

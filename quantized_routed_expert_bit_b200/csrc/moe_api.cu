@@ -52,9 +52,9 @@ struct Layout {
   size_t total;
 };
 
-constexpr int kBatchMinTokens = 8;  // from this many tokens the grouped tensor-core path runs (default)
+constexpr int kBatchMinTokens = 128;  // from this many tokens the grouped tensor-core path runs (default)
 std::atomic<int> g_batch_min{kBatchMinTokens};  // moe_set_batched_min_tokens
-constexpr int kGemvMinTokens = 2;  // from this many tokens the grouped GEMV runs (default)
+constexpr int kGemvMinTokens = 8;  // from this many tokens the grouped GEMV runs (default)
 std::atomic<int> g_gemv_min{kGemvMinTokens};  // moe_set_gemv_min_tokens
 
 constexpr int kMaxGrid = 1024;  // largest persistent decode grid
@@ -94,12 +94,14 @@ Layout layout(const moe_config& c, int64_t T) {
   L.x16 = o;      o += up(np * c.hidden * 2);
   L.hhi = o;      o += up(np * imax * 2);
   L.hlo = o;      o += up(np * imax * 2);
-  const size_t nq = c.inter / (32 * moe::kGvUPI) > 0 ? c.inter / (32 * moe::kGvUPI) : 1;
+  const int upi = moe::gemv_units_per_item(static_cast<int>(T), c.top_k, c.num_experts, c.inter, c.shared_inter);
+  const size_t nq = c.inter / (32 * upi) > 0 ? c.inter / (32 * upi) : 1;
   L.o = o;        o += up(nq * np * c.hidden * 4);
   L.xsx = o;      o += up(np * (c.hidden / 64 + 1) * 4);
   L.xsh = o;      o += up(np * (imax / 64 + 1) * 4 * 4);
   {
-    const size_t ps = 128 / c.bits, nsg = c.hidden / ps, qsp = 3 * (ps / 4) + 1;
+    const size_t ps = 128 / c.bits, nsg = c.hidden / ps;
+    const size_t qsp = c.bits == 4 ? moe::xq_stride<4>() : moe::xq_stride<8>();
     L.gxq = o;    o += up(static_cast<size_t>(T) * nsg * qsp * 4);
     L.gxsc = o;   o += up(static_cast<size_t>(T) * 4);
   }
@@ -470,9 +472,10 @@ moe_status gemv_ffn(const moe_config& c, const moe_layer_weights& wt, const uint
   gp->I = I;
   gp->group = c.group;
   gp->npairs = np;
+  gp->upi = moe::gemv_units_per_item(T, k, E, I, c.shared_inter);
   gp->hdr = v.hdr;
   if ((e = moe::launch_grouped_gemv(*gp, c.bits, sms, st)) != cudaSuccess) return cuda_fail(e, "grouped GEMV launch");
-  const int nq = I / (32 * moe::kGvUPI);
+  const int nq = I / (32 * gp->upi);
   if ((e = moe::launch_gv_combine(o, w, v.sgate, T, k, H, c.shared_inter, nq, np, y, sms * 4, st)) != cudaSuccess)
     return cuda_fail(e, "combine launch");
   return MOE_OK;

@@ -12,6 +12,17 @@ namespace moe {
 
 constexpr int kRouteTokTile = 8;  // tokens per router CTA tile (one counter each)
 
+struct SortParams {
+  const int32_t* idx;    // [T][k]
+  int T, k, E, with_shared;
+  int32_t* perm;         // [T*k (+T)]
+  int32_t* offsets;      // [E+1 (+1)]
+  int32_t* chunks;       // optional [max][3]: expert, first sorted position, pair count (<= chunk_tokens)
+  int32_t* nchunks;      // optional scalar
+  int chunk_tokens;
+  WsHeader* hdr;
+};
+
 struct RouteParams {
   const uint16_t* x;     // bf16 [T][H]
   const uint16_t* wr;    // bf16 [E][H]
@@ -51,16 +62,6 @@ struct GlueParams {
   float eps;
 };
 
-struct SortParams {
-  const int32_t* idx;    // [T][k]
-  int T, k, E, with_shared;
-  int32_t* perm;         // [T*k (+T)]
-  int32_t* offsets;      // [E+1 (+1)]
-  int32_t* chunks;       // optional [max][3]: expert, first sorted position, pair count (<= chunk_tokens)
-  int32_t* nchunks;      // optional scalar
-  int chunk_tokens;
-  WsHeader* hdr;
-};
 
 constexpr int kChunkTokens = 32;  // pairs per GEMM chunk (the MMA N dimension)
 
@@ -151,9 +152,31 @@ struct DecodeParams {
 };
 
 // Grouped GEMV (csrc/grouped_gemv.cu): the batched path on the CUDA cores for a few tokens per
-// expert. A work item is (chunk of <= kGvTPI pairs of one expert, group of kGvUPI 32-column units).
+// expert. A work item is (chunk of <= kGvTPI pairs of one expert, group of upi 32-column units);
+// upi (1, 2 or kGvUPI) is gemv_units_per_item's choice for the batch size.
 constexpr int kGvTPI = 4;  // pairs per chunk
-constexpr int kGvUPI = 4;  // units per item
+
+// Words per 16-byte code segment in the per-token quad table of the grouped GEMV (xq_token): the
+// 3 * 32 / BITS quad words and the segment's sum, padded to 4 m words with m odd, so that each
+// segment starts on 16 bytes and the 16-byte loads of 8 consecutive segments (one shared-memory
+// phase) hit distinct banks.
+template <int BITS>
+__host__ __device__ constexpr int xq_stride() {
+  return 4 * ((((3 * (32 / BITS) + 1) + 3) / 4) | 1);
+}
+constexpr int kGvUPI = 4;  // most units per item
+constexpr int kGvItemsTarget = 128;  // work items wanted per launch: about one per SM of a 148-SM part
+
+// Units per work item for T tokens: the largest of 4, 2, 1 whose item count reaches
+// kGvItemsTarget with one chunk per distinct expert (fewer units per item split the experts of a
+// small batch over more CTAs, at the cost of more partial outputs to combine).
+inline int gemv_units_per_item(int T, int k, int E, int I, int Is) {
+  const long np = static_cast<long>(T) * k + (Is > 0 ? T : 0);
+  const long est = np < E + (Is > 0 ? 1 : 0) ? np : E + (Is > 0 ? 1 : 0);
+  for (int u = kGvUPI; u > 1; u >>= 1)
+    if (est * (I / (32 * u)) >= kGvItemsTarget) return u;
+  return 1;
+}
 struct GemvParams {
   const int32_t* chunks;   // [nchunks][3]: expert (E = shared), first sorted position, pair count
   const int32_t* nchunks;
@@ -166,8 +189,8 @@ struct GemvParams {
   const uint16_t* dsb;     // group-major down scales and biases (moe_prepare_down_sb) or null
   const uint16_t* sdsb;
   CUtensorMap tm_dn, tm_sdn;  // canonical down codes (when dcu / sdcu are null)
-  float* o;                // [I / (32 kGvUPI)][npairs][H] partial expert outputs by pair id
-  int T, k, H, E, I, group, npairs;
+  float* o;                // [I / (32 upi)][npairs][H] partial expert outputs by pair id
+  int T, k, H, E, I, group, npairs, upi;
   WsHeader* hdr;
 };
 bool grouped_gemv_supported(int H, int I, int Is, int group, int bits, size_t smem_limit);

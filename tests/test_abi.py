@@ -161,13 +161,23 @@ def test_stack_and_sort_validation_errors():
 
 
 def test_batched_threshold_knob():
-    """moe_set_batched_min_tokens returns the previous threshold; T < 1 restores the default 8."""
+    """moe_set_batched_min_tokens returns the previous threshold; T < 1 restores the default 128."""
     lib = moe.lib()
-    assert lib.moe_set_batched_min_tokens(3) == 8
+    assert lib.moe_set_batched_min_tokens(3) == 128
     assert lib.moe_set_batched_min_tokens(100) == 3
     assert lib.moe_set_batched_min_tokens(0) == 100
-    assert lib.moe_set_batched_min_tokens(-5) == 8
-    assert lib.moe_set_batched_min_tokens(0) == 8
+    assert lib.moe_set_batched_min_tokens(-5) == 128
+    assert lib.moe_set_batched_min_tokens(0) == 128
+
+
+def test_gemv_threshold_knob():
+    """moe_set_gemv_min_tokens returns the previous threshold; T < 1 restores the default 8."""
+    lib = moe.lib()
+    assert lib.moe_set_gemv_min_tokens(3) == 8
+    assert lib.moe_set_gemv_min_tokens(100) == 3
+    assert lib.moe_set_gemv_min_tokens(0) == 100
+    assert lib.moe_set_gemv_min_tokens(-5) == 8
+    assert lib.moe_set_gemv_min_tokens(0) == 8
 
 
 def test_prepare_calls_validate_before_the_device():

@@ -1,8 +1,11 @@
 """GPU parity of the batched tensor-core path (token-by-expert grouping,
 tcgen05 grouped dequant-GEMMs, combine) against the CPU oracle.
 
-The library takes this path from 8 tokens up (moe_expert_ffn,
-moe_layer_forward, moe_stack_forward); below that, tokens run one at a time.
+By default the library takes this path from 128 tokens up (moe_expert_ffn,
+moe_layer_forward, moe_stack_forward), the grouped GEMV from 8 and the
+per-token kernels below that. These tests move the tensor-core threshold
+down to 8 tokens (moe_set_batched_min_tokens), so that 8 to 127 tokens are
+covered on this path too.
 """
 
 import numpy as np
@@ -17,6 +20,13 @@ from parity import (DeviceLayer, ParityStats, Y_MAX_ABS, Y_REL_L2, bits, check_t
 pytestmark = pytest.mark.gpu
 
 S35 = synth.SHAPES["35b"]
+
+
+@pytest.fixture(autouse=True)
+def tensor_core_from_8_tokens():
+    pb = moe.moe_set_batched_min_tokens(8)
+    yield
+    moe.moe_set_batched_min_tokens(pb)
 
 
 def layer_call(shape, lw, x):
@@ -43,9 +53,9 @@ def test_batched_path_is_taken(key):
     """With the thresholds at 8 (batched) and 2 (grouped GEMV), the workloads'
     shapes run on the tensor-core path from 8 tokens up (route, sort, gather,
     two GEMMs, combine, glue: 7 kernels a layer), on the grouped GEMV from 2
-    to 7 tokens (route, quantise x, sort, GEMV, combine, glue: 6 a layer; 4-bit
-    shapes only), and on the token-at-a-time kernels (4 a layer) when the GEMV
-    is switched off."""
+    to 7 tokens (route, sort, fixed-point x, GEMV, combine, glue: 6 a layer;
+    4-bit shapes only), and on the token-at-a-time kernels (route, gate/up,
+    down, glue: 4 a layer) when the GEMV is switched off."""
     cfg = moe.make_config(synth.SHAPES[key])
     pb, pg = moe.moe_set_batched_min_tokens(8), moe.moe_set_gemv_min_tokens(2)
     try:

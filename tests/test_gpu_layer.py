@@ -91,16 +91,16 @@ def test_batch_equals_single_token_calls(tiny):
 
 def test_grouped_gemv_is_batch_invariant(tiny):
     """On the grouped GEMV a token's output depends on its own x alone (its own fixed-point scale,
-    partial sums combined in a fixed order): the same bits in a batch of 13 as in a batch of two
-    copies of it."""
+    partial sums combined in a fixed order, for a given number of units per work item, which
+    depends on the batch size): the same bits in a batch of 13 as in a batch of 13 copies of it."""
     lw, host, x = tiny
     pg, pb = moe.moe_set_gemv_min_tokens(2), moe.moe_set_batched_min_tokens(1 << 30)
     try:
         assert moe.moe_stack_path_name(moe.make_config(TINY), 13, 1) == "grouped_gemv"
         idx, w, y = _run_layer(TINY, lw, x[:13])
         for t in range(13):
-            i2, w2, y2 = _run_layer(TINY, lw, x[t:t + 1].repeat(2, 1))
-            for r in range(2):
+            i2, w2, y2 = _run_layer(TINY, lw, x[t:t + 1].repeat(13, 1))
+            for r in (0, 6, 12):
                 assert np.array_equal(i2[r], idx[t]) and np.array_equal(w2[r], w[t]) and np.array_equal(y2[r], y[t])
     finally:
         moe.moe_set_gemv_min_tokens(pg)

@@ -82,13 +82,22 @@ def test_decode_stack_parity(key):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("key", ["35b_t64", "35b_t512"])
-def test_batched_stack_parity(key):
+@pytest.mark.parametrize("key,path", [("35b_t64", "grouped_gemv"), ("35b_t64", "batched"), ("35b_t512", "batched")])
+def test_batched_stack_parity(key, path):
+    """The batched stacks on the path the library picks for them by default (grouped GEMV at 64
+    tokens, tensor cores at 512) and, at 64 tokens, on the tensor-core path as well."""
     shape = synth.SHAPES[key]
     T = shape.tokens
+    cfg = moe.make_config(shape)
     layers = [synth.make_layer(shape, l, "cuda") for l in range(shape.layers)]
     x0 = synth.make_batch(shape, T, 0, "cuda")
-    tx, ti, tw, ty, xo = run_stack(shape, layers, x0)
+    forced = path != moe.moe_stack_path_name(cfg, T, shape.layers)
+    pb = moe.moe_set_batched_min_tokens(1 if forced else 0)  # 0: the default threshold
+    try:
+        assert moe.moe_stack_path_name(cfg, T, shape.layers) == path
+        tx, ti, tw, ty, xo = run_stack(shape, layers, x0)
+    finally:
+        moe.moe_set_batched_min_tokens(pb)
     total = ParityStats()
     rng = np.random.default_rng(T)
     # every token of every layer at T=64; at T=512 every token of the first two, a middle and the
@@ -102,7 +111,7 @@ def test_batched_stack_parity(key):
     flips = check_glue(bits(x0), tx, ty, xo)
     want = len(full) * T + (shape.layers - len(full)) * 8
     assert total.checked == want
-    print(f"{key}: {total.checked} (token, layer) pairs checked (every token on {len(full)} of {shape.layers} "
+    print(f"{key} on {path}: {total.checked} (token, layer) pairs checked (every token on {len(full)} of {shape.layers} "
           f"layers), {total.excluded} gap-excluded, max-abs {total.max_abs:.2e}, rel-L2 {total.max_rel_l2:.2e}, "
           f"glue flips {flips}")
     assert total.excluded <= max(2, total.checked // 50)
