@@ -44,7 +44,9 @@ NOMINAL_HBM_GBS = 8000.0
 # Keyed by the workload and a hash of the kernel's source files: a capture of another revision of
 # the kernel is not reported (traffic null).
 KERNEL_SOURCES = ("stack_split.cu", "decode_common.cuh", "moe_common.cuh", "moe_launch.h")
-DECODE_TRAFFIC_PER_LAYER = {}
+# dram__bytes_read.sum + dram__bytes_write.sum per layer of decode_split_kernel from the 4-layer
+# capture in profiles/decode_split_kernel_35b_l4_full.md, keyed by workload and kernel source hash
+DECODE_TRAFFIC_PER_LAYER = {("35b", "c85cf996acf27956"): (68_030_464 + 1_740_544) / 4}
 
 
 def kernel_source_hash() -> str:
@@ -496,7 +498,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true", help="skip the other workloads' block")
     ap.add_argument("--sweep", action="store_true",
-                    help="time the per-token path against the batched path for T = 1..64 tokens and exit")
+                    help="time the per-token kernels, the grouped GEMV and the tensor-core path for "
+                         "T = 1..512 tokens and exit")
+    ap.add_argument("--path", default=None, choices=["per_layer", "grouped_gemv", "batched"],
+                    help="pin the multi-token path (moe_set_gemv_min_tokens / moe_set_batched_min_tokens); "
+                         "the default is the library's choice for the token count")
     ap.add_argument("--layers", type=int, default=0,
                     help="profile a shorter stack (small ncu case); the default is the full stack")
     ap.add_argument("--workload", default=SHAPE_KEY, choices=sorted(synth.SHAPES),
@@ -511,6 +517,10 @@ def main():
     if args.sweep:
         dispatch_sweep(key=args.workload)
         return
+    if args.path is not None:  # process-wide dispatch thresholds
+        gthr, bthr = {"per_layer": (1 << 30, 1 << 30), "grouped_gemv": (2, 1 << 30), "batched": (1 << 30, 2)}[args.path]
+        moe.moe_set_gemv_min_tokens(gthr)
+        moe.moe_set_batched_min_tokens(bthr)
     dist, rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
     key = args.workload
