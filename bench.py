@@ -317,10 +317,11 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
-def workload_config(shape):
+def workload_config(shape, stock=False):
+    layout = "stock gate/up (separate gate and up tensors)" if stock else "packed gate/up"
     return {"workload": f"{shape.name}: T={shape.tokens} through {shape.layers} stacked MoE layers "
                         f"(H={shape.hidden}, E={shape.num_experts}, top-{shape.top_k}, I=Is={shape.inter}, "
-                        f"{shape.bits}-bit affine g{shape.group}, bf16 scale/bias, packed gate/up)",
+                        f"{shape.bits}-bit affine g{shape.group}, bf16 scale/bias, {layout})",
             "tokens_per_step": shape.tokens, "layers": shape.layers,
             "l2": f"inputs larger than L2: {shape.layers * shape.num_experts * shape.expert_bytes() / 1e9:.1f} GB "
                   "resident expert stack, a new token (new experts) every step"}
@@ -347,8 +348,9 @@ class Workload:
     """One workload's stack on the device, ready to step: weights (with their decode-ready
     copies), a workspace and the tokens of `nsteps` steps."""
 
-    def __init__(self, key, nsteps, rank=0, layers=0):
+    def __init__(self, key, nsteps, rank=0, layers=0, stock=False):
         self.key = key
+        self.stock = stock
         shape = synth.SHAPES[key]
         if layers:
             import dataclasses
@@ -357,6 +359,9 @@ class Workload:
         self.cfg = moe.make_config(shape)
         sid = synth.SHAPE_SEED_ID[key]
         self.layers = [synth.make_layer(shape, l, "cuda", seed_id=sid) for l in range(shape.layers)]
+        if stock:  # the stock gate/up layout: separate gate and up tensors (the packed copies freed)
+            self.layers = [synth.stock_layer(lw) for lw in self.layers]
+            torch.cuda.empty_cache()
         self.arr = moe.make_layer_array([moe.make_layer_weights(lw, self.cfg) for lw in self.layers])
         self.T = shape.tokens
         self.ws = moe.Workspace(self.cfg, self.T, L=shape.layers)
@@ -372,10 +377,13 @@ class Workload:
         moe.moe_stack_forward(self.cfg, self.arr, self.tokens[i * T:(i + 1) * T], self.xout, self.ws, stream=stream)
 
     def path(self):
-        return moe.moe_stack_path_name(self.cfg, self.T, self.shape.layers)
+        p = moe.moe_stack_path_name(self.cfg, self.T, self.shape.layers)
+        return "grouped_gemv" if (self.stock and p == "batched") else p  # the tensor cores read packed only
 
     def launches(self):
-        return moe.moe_stack_kernel_launches(self.cfg, self.T, self.shape.layers)
+        n = moe.moe_stack_kernel_launches(self.cfg, self.T, self.shape.layers)
+        return 1 + 6 * self.shape.layers if (self.stock and self.path() != moe.moe_stack_path_name(
+            self.cfg, self.T, self.shape.layers)) else n
 
     def bytes_per_step(self, warmup, steps):
         if self.T == 1:
@@ -500,6 +508,9 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="time the per-token kernels, the grouped GEMV and the tensor-core path for "
                          "T = 1..512 tokens and exit")
+    ap.add_argument("--stock", action="store_true",
+                    help="the stock (unpacked) gate/up layout: each expert's gate and up rows in separate "
+                         "tensors, the A/B baseline of the packed layout")
     ap.add_argument("--path", default=None, choices=["per_layer", "grouped_gemv", "batched"],
                     help="pin the multi-token path (moe_set_gemv_min_tokens / moe_set_batched_min_tokens); "
                          "the default is the library's choice for the token count")
@@ -526,7 +537,7 @@ def main():
     key = args.workload
     nsteps = args.warmup + args.steps
     # each rank its own tokens (independent replicas); a step is one batch of T tokens
-    wl = Workload(key, nsteps, rank, args.layers)
+    wl = Workload(key, nsteps, rank, args.layers, stock=args.stock)
     shape, T = wl.shape, wl.T
     stream = torch.cuda.current_stream()
 
@@ -583,7 +594,8 @@ def main():
     peak, peak_src = peaks()
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and T == 1:
+    # (the stock layout is an A/B variant of the same workload: its line carries no oracle leg)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.stock and T == 1:
         cores = os.cpu_count() or 1
         threads = min(cores, shape.top_k + 1)  # one expert per thread
         v, evals, dt, par = cpu_oracle_leg(shape, wl.cfg, wl.arr, wl.ws, wl.layers, wl.tokens[:4], threads)
@@ -598,7 +610,7 @@ def main():
     if persistent and (key, src_hash) in DECODE_TRAFFIC_PER_LAYER:
         traffic = DECODE_TRAFFIC_PER_LAYER[(key, src_hash)] * shape.layers
     sec = None
-    if world == 1 and not args.no_secondary and not args.layers and key == SHAPE_KEY:
+    if world == 1 and not args.no_secondary and not args.layers and not args.stock and key == SHAPE_KEY:
         del wl
         torch.cuda.empty_cache()
         sec = secondary([k for k in ("80b", "35b8", "35b_t64", "35b_t512") if k != key], 32, args.warmup, peak)
@@ -609,7 +621,7 @@ def main():
             "vs_baseline": None, "dtype": "f32", "weights": f"u{shape.bits} affine g{shape.group}, bf16 scale/bias",
             "arithmetic": "exact integer byte dot products (dp4a) of the codes with a 22-bit fixed-point copy of the "
                           "activations, fp32 scale/bias and sums" if path == "decode_split_kernel" else "fp32",
-            "data": "synthetic", "config": workload_config(shape),
+            "data": "synthetic", "config": workload_config(shape, args.stock),
             "hbm_gbs": gbs, "hbm_frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm",
                          "kernel": (f"{path} (the whole stack, one launch per step)" if persistent

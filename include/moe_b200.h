@@ -127,6 +127,18 @@ typedef struct {
   const uint16_t* shared_down_sb;
   const uint8_t* down_units;
   const uint8_t* shared_down_units;
+  /* Optional stock (unpacked) gate/up layout, the A/B baseline of the packed
+   * routed gate/up (Runnel README, "Streaming CLI": --stock-mlp). When
+   * up.q is non-NULL, gate_up holds only the gate rows, E matrices [I][H],
+   * and up the up rows, E matrices [I][H], with the same expert strides as
+   * gate_up (codes, and scales/biases); likewise shared_up / shared_gate_up
+   * for the shared expert (shared_up.q non-NULL exactly when up.q is; a
+   * mismatch, or strides that differ, is MOE_ERR_INVALID_ARG). Results are
+   * the same as with the packed layout.
+   * The tensor-core path reads the packed layout only: a call with stock
+   * weights runs the grouped GEMV where it would run the tensor cores. */
+  moe_qtensor up;
+  moe_qtensor shared_up;
 } moe_layer_weights;
 
 /* Per-layer record of a stack run; any member may be NULL (not recorded). */

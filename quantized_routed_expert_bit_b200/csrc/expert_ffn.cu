@@ -88,12 +88,11 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int per_tok = p.k * blk_r + blk_s;
   const int t = blockIdx.x / per_tok;
   const int r = blockIdx.x % per_tok;
-  int j, rb, Ij, e = 0;
+  int j, rb, e = 0;
   QMat m;
   if (r < p.k * blk_r) {
     j = r / blk_r;
     rb = r % blk_r;
-    Ij = p.I;
     m = p.gate_up;
     e = p.idx[static_cast<size_t>(t) * p.k + j];
     if (e < 0 || e >= p.E) {
@@ -103,7 +102,6 @@ __global__ void __launch_bounds__(kWarps * 32)
   } else {
     j = p.k;
     rb = r - p.k * blk_r;
-    Ij = p.Is;
     m = p.sh_gate_up;
     if (rb == 0 && threadIdx.x < 32) {
       // The shared expert's gate, sigmoid(x . w_sg), for phase 2.
@@ -141,9 +139,9 @@ __global__ void __launch_bounds__(kWarps * 32)
     fence_mbar_init();
     mbar_arrive_expect_tx(&bar, 4 * sb_bytes);
     bulk_g2s(sb + 0 * sb_elems, sbase + static_cast<size_t>(i0) * ng, sb_bytes, &bar);
-    bulk_g2s(sb + 1 * sb_elems, sbase + static_cast<size_t>(Ij + i0) * ng, sb_bytes, &bar);
+    bulk_g2s(sb + 1 * sb_elems, sbase + m.up_s + static_cast<size_t>(i0) * ng, sb_bytes, &bar);
     bulk_g2s(sb + 2 * sb_elems, bbase + static_cast<size_t>(i0) * ng, sb_bytes, &bar);
-    bulk_g2s(sb + 3 * sb_elems, bbase + static_cast<size_t>(Ij + i0) * ng, sb_bytes, &bar);
+    bulk_g2s(sb + 3 * sb_elems, bbase + m.up_b + static_cast<size_t>(i0) * ng, sb_bytes, &bar);
   }
 
   const uint16_t* xt = p.x + static_cast<size_t>(t) * H;
@@ -165,7 +163,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     for (int rr = 0; rr < kRowsPerWarp; ++rr) {
       const int i = i0 + warp * kRowsPerWarp + rr;
       const uint8_t* qg = qbase + static_cast<size_t>(i) * row_bytes;
-      const uint8_t* qu = qbase + static_cast<size_t>(Ij + i) * row_bytes;
+      const uint8_t* qu = qbase + m.up_q + static_cast<size_t>(i) * row_bytes;
 #pragma unroll
       for (int c = 0; c < kChunkGU; ++c) {
         const int s = c0 + 32 * c + lane;

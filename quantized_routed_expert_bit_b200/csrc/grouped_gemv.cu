@@ -157,11 +157,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
       mbar_arrive_expect_tx(&bar_gc[b][bt], 2 * cb + (bt == 0 ? 4 * sbb : 0u));
       for (int gu = 0; gu < 2; ++gu)
         bulk_g2s(base + static_cast<size_t>(gu * kUnit + bt * kBatch) * rowb,
-                 qb + static_cast<size_t>(gu * I + u.i0 + bt * kBatch) * rowb, cb, &bar_gc[b][bt]);
+                 qb + (gu ? mq.up_q : 0) + static_cast<size_t>(u.i0 + bt * kBatch) * rowb, cb, &bar_gc[b][bt]);
       if (bt == 0)
         for (int kind = 0; kind < 4; ++kind)  // gate sc, up sc, gate bi, up bi
           bulk_g2s(gsb + static_cast<size_t>(kind * kUnit) * ng,
-                   ((kind & 2) ? bb : sb) + static_cast<size_t>((kind & 1) * I + u.i0) * ng, sbb, &bar_gc[b][bt]);
+                   ((kind & 2) ? bb : sb) + ((kind & 1) ? ((kind & 2) ? mq.up_b : mq.up_s) : 0) +
+                       static_cast<size_t>(u.i0) * ng, sbb,
+                   &bar_gc[b][bt]);
     }
     s_pend_gc[b] = par;
   };

@@ -165,15 +165,35 @@ moe_status check_qt(const moe_qtensor& q, int64_t rows, int64_t K, int bits, int
   return MOE_OK;
 }
 
+// The stock (unpacked) gate/up layout: separate gate and up tensors (moe_layer_weights.up).
+bool stock_layout(const moe_layer_weights& w) { return w.up.q != nullptr; }
+
+// The up tensor of the stock layout against its gate tensor: the same expert strides.
+moe_status check_up(const moe_qtensor& g, const moe_qtensor& u, int64_t n, const char* what) {
+  if (n > 1 && (u.q_expert_stride != g.q_expert_stride || u.sb_expert_stride != g.sb_expert_stride))
+    return fail(MOE_ERR_INVALID_ARG, "%s: expert strides differ from the gate tensor's", what);
+  return MOE_OK;
+}
+
 moe_status check_weights(const moe_config& c, const moe_layer_weights* w, bool need_router) {
   if (!w) return fail(MOE_ERR_INVALID_ARG, "weights is NULL");
   moe_status s;
   if (need_router && (s = check_ptr(w->router_w, 16, "router_w"))) return s;
   if (w->router_bias && !aligned(w->router_bias, 4)) return fail(MOE_ERR_INVALID_ARG, "router_bias misaligned");
-  if ((s = check_qt(w->gate_up, 2LL * c.inter, c.hidden, c.bits, c.group, c.num_experts, "gate_up"))) return s;
+  const bool stock = stock_layout(*w);
+  const int64_t gu_rows = stock ? 1 : 2;  // gate_up rows per intermediate index
+  if ((s = check_qt(w->gate_up, gu_rows * c.inter, c.hidden, c.bits, c.group, c.num_experts, "gate_up"))) return s;
+  if (stock && ((s = check_qt(w->up, c.inter, c.hidden, c.bits, c.group, c.num_experts, "up")) ||
+                (s = check_up(w->gate_up, w->up, c.num_experts, "up"))))
+    return s;
   if ((s = check_qt(w->down, c.hidden, c.inter, c.bits, c.group, c.num_experts, "down"))) return s;
   if (c.shared_inter > 0) {
-    if ((s = check_qt(w->shared_gate_up, 2LL * c.shared_inter, c.hidden, c.bits, c.group, 1, "shared_gate_up")))
+    if ((s = check_qt(w->shared_gate_up, gu_rows * c.shared_inter, c.hidden, c.bits, c.group, 1, "shared_gate_up")))
+      return s;
+    if (stock != (w->shared_up.q != nullptr))
+      return fail(MOE_ERR_INVALID_ARG, "shared_up.q must be set exactly when up.q is");
+    if (stock && ((s = check_qt(w->shared_up, c.shared_inter, c.hidden, c.bits, c.group, 1, "shared_up")) ||
+                  (s = check_up(w->shared_gate_up, w->shared_up, 1, "shared_up"))))
       return s;
     if ((s = check_qt(w->shared_down, c.hidden, c.shared_inter, c.bits, c.group, 1, "shared_down"))) return s;
     if ((s = check_ptr(w->shared_gate_w, 16, "shared_gate_w"))) return s;
@@ -198,7 +218,22 @@ moe_status check_ws(const moe_config& c, void* ws, size_t ws_bytes, int64_t T, L
 }
 
 moe::QMat qmat(const moe_qtensor& q) {
-  return moe::QMat{q.q, q.scales, q.biases, q.q_expert_stride, q.sb_expert_stride};
+  return moe::QMat{q.q, q.scales, q.biases, q.q_expert_stride, q.sb_expert_stride, 0, 0, 0};
+}
+
+// A gate/up matrix set with the offsets of its up rows: I rows on in the packed layout, the up
+// tensor in the stock layout.
+moe::QMat qmat_gu(const moe_config& c, const moe_qtensor& gu, const moe_qtensor& up, bool stock, int I) {
+  moe::QMat m = qmat(gu);
+  if (stock) {
+    m.up_q = static_cast<int64_t>(reinterpret_cast<uintptr_t>(up.q) - reinterpret_cast<uintptr_t>(gu.q));
+    m.up_s = static_cast<int64_t>(reinterpret_cast<uintptr_t>(up.scales) - reinterpret_cast<uintptr_t>(gu.scales)) / 2;
+    m.up_b = static_cast<int64_t>(reinterpret_cast<uintptr_t>(up.biases) - reinterpret_cast<uintptr_t>(gu.biases)) / 2;
+  } else {
+    m.up_q = static_cast<int64_t>(I) * c.hidden * c.bits / 8;
+    m.up_s = m.up_b = static_cast<int64_t>(I) * (c.hidden / c.group);
+  }
+  return m;
 }
 
 moe_status route(const moe_config& c, const uint16_t* x, int T, const uint16_t* wr, const float* rbias,
@@ -215,10 +250,11 @@ moe_status ffn(const moe_config& c, const moe_layer_weights& wt, const uint16_t*
   p.idx = idx;
   p.w = w;
   p.y = y;
-  p.gate_up = qmat(wt.gate_up);
+  const bool stock = stock_layout(wt);
+  p.gate_up = qmat_gu(c, wt.gate_up, wt.up, stock, c.inter);
   p.down = qmat(wt.down);
   if (c.shared_inter > 0) {
-    p.sh_gate_up = qmat(wt.shared_gate_up);
+    p.sh_gate_up = qmat_gu(c, wt.shared_gate_up, wt.shared_up, stock, c.shared_inter);
     p.sh_down = qmat(wt.shared_down);
     p.wsg = wt.shared_gate_w;
   }
@@ -300,6 +336,7 @@ bool batched_eligible(const moe_config& c, int T) {
 // Experts' gate/up and down for T tokens given their selection, on the tensor cores.
 moe_status batched_ffn(const moe_config& c, const moe_layer_weights& wt, const uint16_t* x, int T, const int32_t* idx,
                        const float* w, uint16_t* y, void* ws, const Layout& Ly, cudaStream_t st) {
+  if (stock_layout(wt)) return fail(MOE_ERR_UNSUPPORTED, "the tensor-core path reads the packed gate/up layout");
   char* b = static_cast<char*>(ws);
   const moe::WsView v = view(ws, Ly);
   const int H = c.hidden, I = c.inter, k = c.top_k, E = c.num_experts;
@@ -410,9 +447,11 @@ int device_smem_optin() {
 // Whether T tokens take the grouped GEMV (a few tokens per expert, CUDA cores): from
 // moe_set_gemv_min_tokens tokens up, below the batched tensor-core path's threshold (or where that
 // path does not apply), for shapes whose units of 32 columns come in whole groups of kGvUPI.
-bool gemv_eligible(const moe_config& c, int T) {
+// stock: the layer is in the stock gate/up layout, which the tensor-core path does not read; the
+// grouped GEMV then also takes the token counts the tensor cores would.
+bool gemv_eligible(const moe_config& c, int T, bool stock = false) {
   if (T < g_gemv_min.load(std::memory_order_relaxed)) return false;
-  if (batched_eligible(c, T)) return false;
+  if (!stock && batched_eligible(c, T)) return false;
   if (!encode_fn()) return false;
   const int optin = device_smem_optin();
   if (optin < 1024) return false;
@@ -448,9 +487,10 @@ moe_status gemv_ffn(const moe_config& c, const moe_layer_weights& wt, const uint
   gp->perm = perm;
   gp->xq = xq;
   gp->xsc = xsc;
-  gp->gu = qmat(wt.gate_up);
+  const bool stock = stock_layout(wt);
+  gp->gu = qmat_gu(c, wt.gate_up, wt.up, stock, I);
   gp->dn = qmat(wt.down);
-  gp->sgu = qmat(shared ? wt.shared_gate_up : wt.gate_up);
+  gp->sgu = shared ? qmat_gu(c, wt.shared_gate_up, wt.shared_up, stock, c.shared_inter) : gp->gu;
   gp->sdn = qmat(shared ? wt.shared_down : wt.down);
   gp->dcu = wt.down_units;
   gp->dsb = wt.down_sb;
@@ -532,14 +572,15 @@ bool decode_eligible(const moe_config& c, int L, int* grid, bool* split = nullpt
   return true;
 }
 
-moe::LayerDesc layer_desc(const moe_layer_weights& w) {
+moe::LayerDesc layer_desc(const moe_config& c, const moe_layer_weights& w) {
   moe::LayerDesc d{};
   d.wr = w.router_w;
   d.rbias = w.router_bias;
   d.wsg = w.shared_gate_w;
-  d.gu = qmat(w.gate_up);
+  const bool stock = stock_layout(w);
+  d.gu = qmat_gu(c, w.gate_up, w.up, stock, c.inter);
   d.dn = qmat(w.down);
-  d.sgu = qmat(w.shared_gate_up);
+  d.sgu = qmat_gu(c, w.shared_gate_up, w.shared_up, stock, c.shared_inter);
   d.sdn = qmat(w.shared_down);
   d.dsb = w.down_sb;
   d.sdsb = w.shared_down_sb;
@@ -590,7 +631,7 @@ moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, in
     P->r_in = (l0 == 0) ? nullptr : rmid;
     P->out = last ? x_out : xmid;
     P->r_out = last ? nullptr : rmid;
-    for (int i = 0; i < n; ++i) P->layers[i] = layer_desc(layers[l0 + i]);
+    for (int i = 0; i < n; ++i) P->layers[i] = layer_desc(c, layers[l0 + i]);
     if (split) {
       // down codes as (row bytes, H rows, experts), one unit's 32 columns x 256 rows per copy
       const int64_t rb = static_cast<int64_t>(c.inter) * c.bits / 8;
@@ -683,9 +724,10 @@ moe_status moe_expert_ffn(const moe_config* cfg, const moe_layer_weights* w, con
     return s;
   Layout L;
   if ((s = check_ws(*cfg, ws, ws_bytes, T, &L))) return s;
-  if (batched_eligible(*cfg, T))
+  const bool stock = stock_layout(*w);
+  if (!stock && batched_eligible(*cfg, T))
     return batched_ffn(*cfg, *w, x, T, topk_idx, topk_w, y, ws, L, reinterpret_cast<cudaStream_t>(stream));
-  if (gemv_eligible(*cfg, T))
+  if (gemv_eligible(*cfg, T, stock))
     return gemv_ffn(*cfg, *w, x, T, topk_idx, topk_w, y, ws, L, reinterpret_cast<cudaStream_t>(stream));
   return ffn(*cfg, *w, x, T, topk_idx, topk_w, y, view(ws, L), reinterpret_cast<cudaStream_t>(stream));
 }
@@ -709,8 +751,9 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, 
   const moe::WsView v = view(ws, L);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if ((s = route(*cfg, x, T, w->router_w, w->router_bias, idx, wt, v, st))) return s;
-  if (batched_eligible(*cfg, T)) return batched_ffn(*cfg, *w, x, T, idx, wt, y, ws, L, st);
-  if (gemv_eligible(*cfg, T)) return gemv_ffn(*cfg, *w, x, T, idx, wt, y, ws, L, st);
+  const bool stock = stock_layout(*w);
+  if (!stock && batched_eligible(*cfg, T)) return batched_ffn(*cfg, *w, x, T, idx, wt, y, ws, L, st);
+  if (gemv_eligible(*cfg, T, stock)) return gemv_ffn(*cfg, *w, x, T, idx, wt, y, ws, L, st);
   return ffn(*cfg, *w, x, T, idx, wt, y, v, st);
 }
 
@@ -738,8 +781,10 @@ moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weights* lay
   int split_late = 0, split_two = 0;
   if (T == 1 && decode_eligible(*cfg, L, &grid, &split, &split_late, &split_two))
     return stack_decode(*cfg, layers, L, x0, x_out, trace, ws, Ly, grid, split, split_late, split_two, st);
-  const bool batched = batched_eligible(*cfg, T);
-  const bool gemv = !batched && gemv_eligible(*cfg, T);
+  bool stock = false;  // any layer in the stock gate/up layout keeps the stack off the tensor cores
+  for (int l = 0; l < L; ++l) stock = stock || stock_layout(layers[l]);
+  const bool batched = !stock && batched_eligible(*cfg, T);
+  const bool gemv = !batched && gemv_eligible(*cfg, T, stock);
   const size_t TH = static_cast<size_t>(T) * cfg->hidden;
   const size_t Tk = static_cast<size_t>(T) * cfg->top_k;
   float* r = reinterpret_cast<float*>(b + Ly.r);

@@ -40,6 +40,12 @@ struct QMat {
   const uint16_t* b;
   int64_t q_stride;   // bytes per expert
   int64_t sb_stride;  // elements per expert
+  // gate/up matrices: where an expert's up rows start, from its gate rows (codes in bytes, scales
+  // and biases in elements): I rows further on in the packed layout, the distance to the separate
+  // up tensors in the stock layout (moe_layer_weights.up); 0 for the down matrices
+  int64_t up_q;
+  int64_t up_s;
+  int64_t up_b;
 };
 
 struct FfnParams {

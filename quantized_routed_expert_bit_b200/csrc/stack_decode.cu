@@ -408,10 +408,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         const int j = jA + sg;
         const bool routed = j < k;
         const QMat& m = routed ? Ld.gu : Ld.sgu;
-        const int Ij = routed ? I : Is;
         const int row = (sg == 0 ? iA : -nA) + lo;
-        const uint8_t* src = m.q + static_cast<size_t>(routed ? s_idx[j] : 0) * m.q_stride +
-                             static_cast<size_t>(gu * Ij + row) * rowb;
+        const uint8_t* src = m.q + static_cast<size_t>(routed ? s_idx[j] : 0) * m.q_stride + (gu ? m.up_q : 0) +
+                             static_cast<size_t>(row) * rowb;
         copy_tx(dbuf + static_cast<size_t>(gu * cv.npc_max + lo) * rowb, src, static_cast<uint32_t>((hi - lo) * rowb),
                 &bar_gc[b]);
       }
@@ -436,10 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         const int j = jA + sg;
         const bool routed = j < k;
         const QMat& m = routed ? Ld.gu : Ld.sgu;
-        const int Ij = routed ? I : Is;
         const int row = sg == 0 ? iA + pair : pair - nA;
         const uint16_t* src = ((kind & 2) ? m.b : m.s) + static_cast<size_t>(routed ? s_idx[j] : 0) * m.sb_stride +
-                              static_cast<size_t>((kind & 1) * Ij + row) * ng + part * 8;
+                              ((kind & 1) ? ((kind & 2) ? m.up_b : m.up_s) : 0) + static_cast<size_t>(row) * ng +
+                              part * 8;
         *reinterpret_cast<uint4*>(gsb + static_cast<size_t>(kind * cv.npc_max + pair) * ng + part * 8) =
             __ldg(reinterpret_cast<const uint4*>(src));
       }

@@ -423,7 +423,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
   auto issue_unit = [&](const LayerDesc& Ld, int l, const Unit& U, int e, int gpar, int db) {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     const QMat& mq = U.routed ? Ld.gu : Ld.sgu;
-    const int Ij = U.routed ? I : Is;
     const int iA = U.i0;
     const uint8_t* qb = mq.q + static_cast<size_t>(e) * mq.q_stride;
     const uint16_t* sb = mq.s + static_cast<size_t>(e) * mq.sb_stride;
@@ -431,17 +430,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
     const uint32_t cb = static_cast<uint32_t>(kBatch) * rowb, sbb = static_cast<uint32_t>(kUnit) * ng * 2;
 #pragma unroll 1
     for (int b = 0; b < kNB; ++b) {
-      const int r0 = iA + b * kBatch;  // first gate row of the batch; its up row is Ij + r0
+      const int r0 = iA + b * kBatch;  // first gate row of the batch; its up row r0 starts at up_q
       if (lane == 0) mbar_arrive_expect_tx(&bar_gc[b], 2 * cb + (b == 0 ? 4 * sbb : 0u));
       __syncwarp();
       if (lane < (b == 0 ? 6 : 2)) {
         const int gu = lane & 1, kind = lane >> 1;  // kind 0 codes, 1 scales, 2 biases
         if (kind == 0)
           bulk_g2s(gcd + static_cast<size_t>(gu * kUnit + b * kBatch) * rowb,
-                   qb + static_cast<size_t>(gu * Ij + r0) * rowb, cb, &bar_gc[b]);
+                   qb + (gu ? mq.up_q : 0) + static_cast<size_t>(r0) * rowb, cb, &bar_gc[b]);
         else
           bulk_g2s(gsb + static_cast<size_t>(((kind - 1) * 2 + gu) * kUnit) * ng,
-                   (kind == 1 ? sb : bb) + static_cast<size_t>(gu * Ij + iA) * ng, sbb, &bar_gc[b]);
+                   (kind == 1 ? sb + (gu ? mq.up_s : 0) : bb + (gu ? mq.up_b : 0)) + static_cast<size_t>(iA) * ng, sbb, &bar_gc[b]);
       }
     }
     if (lane == 0) {

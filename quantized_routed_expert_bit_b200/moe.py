@@ -45,7 +45,8 @@ class QTensor(ctypes.Structure):
 class LayerWeights(ctypes.Structure):
     _fields_ = [("router_w", P), ("router_bias", P), ("gate_up", QTensor), ("down", QTensor),
                 ("shared_gate_up", QTensor), ("shared_down", QTensor), ("shared_gate_w", P),
-                ("down_sb", P), ("shared_down_sb", P), ("down_units", P), ("shared_down_units", P)]
+                ("down_sb", P), ("shared_down_sb", P), ("down_units", P), ("shared_down_units", P),
+                ("up", QTensor), ("shared_up", QTensor)]
 
 
 class Trace(ctypes.Structure):
@@ -195,9 +196,11 @@ def make_layer_weights(lw, cfg: Optional[Config] = None) -> LayerWeights:
     dsb = sdsb = dcu = sdcu = None
     if cfg is not None and lw.down.q.is_cuda and split_decode(cfg):
         dsb, sdsb, dcu, sdcu = prepare_layer(cfg, lw)
+    up = getattr(lw, "up", None)  # the stock gate/up layout (synth.stock_layer)
+    shared_up = getattr(lw, "shared_up", None)
     return LayerWeights(lw.router_w.data_ptr(), _p(lw.router_bias), _qtensor(lw.gate_up), _qtensor(lw.down),
                         _qtensor(lw.shared_gate_up), _qtensor(lw.shared_down), _p(lw.shared_gate_w),
-                        _p(dsb), _p(sdsb), _p(dcu), _p(sdcu))
+                        _p(dsb), _p(sdsb), _p(dcu), _p(sdcu), _qtensor(up), _qtensor(shared_up))
 
 
 def split_decode(cfg: Config) -> bool:

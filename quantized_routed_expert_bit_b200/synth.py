@@ -160,6 +160,10 @@ class LayerWeights:
     shared_gate_up: Optional[QTensor]  # [1][2Is][H]
     shared_down: Optional[QTensor]     # [1][H][Is]
     shared_gate_w: Optional[torch.Tensor]  # bf16 [H]
+    # The stock (unpacked) gate/up layout: when set, gate_up holds only the gate rows [E][I][H]
+    # and up the up rows [E][I][H] (stock_layer); None in the packed layout.
+    up: Optional[QTensor] = None
+    shared_up: Optional[QTensor] = None
 
 
 def _quantized_stack(n: int, rows: int, K: int, bits: int, group: int, seed: int, device,
@@ -177,6 +181,22 @@ def _quantized_stack(n: int, rows: int, K: int, bits: int, group: int, seed: int
         b[e0:e1] = bb.reshape(e1 - e0, rows, -1)
         del w, qq, ss, bb
     return QTensor(q, s, b, rows, K)
+
+
+def _split_rows(qt: QTensor, half: int) -> QTensor:
+    """Rows [half*R/2, (half+1)*R/2) of every matrix of qt, as contiguous tensors of their own."""
+    r = qt.rows // 2
+    sl = slice(half * r, (half + 1) * r)
+    return QTensor(qt.q[:, sl].contiguous(), qt.scales[:, sl].contiguous(), qt.biases[:, sl].contiguous(), r, qt.K)
+
+
+def stock_layer(lw: LayerWeights) -> LayerWeights:
+    """The same layer in the stock gate/up layout: the packed [2I][H] matrices split into
+    separate gate [I][H] and up [I][H] tensors (new allocations; same codes, scales, biases)."""
+    sg = lw.shared_gate_up
+    return dataclasses.replace(lw, gate_up=_split_rows(lw.gate_up, 0), up=_split_rows(lw.gate_up, 1),
+                               shared_gate_up=None if sg is None else _split_rows(sg, 0),
+                               shared_up=None if sg is None else _split_rows(sg, 1))
 
 
 def make_layer(shape: MoEShape, layer: int, device="cpu", seed_id: Optional[int] = None) -> LayerWeights:

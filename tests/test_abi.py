@@ -140,6 +140,31 @@ def test_expert_ffn_validation_errors():
     assert call_ffn(c0, w0, T=0) == moe.MOE_OK
 
 
+def test_stock_layout_validation_errors():
+    """The stock gate/up layout (separate gate and up tensors) is checked before the device: the up
+    tensors need the gate tensors' expert strides, and shared_up is set exactly when up is."""
+    c = cfg35()
+    H, I, b, g = c.hidden, c.inter, c.bits, c.group
+    half_q, half_sb = I * H * b // 8, I * H // g
+
+    def stock(**over):
+        w = fake_weights(c, gate_up=fake_qt(half_q, half_sb), up=fake_qt(half_q, half_sb),
+                         shared_gate_up=fake_qt(0, 0), shared_up=fake_qt(0, 0))
+        for k, v in over.items():
+            setattr(w, k, v)
+        return w
+
+    assert call_ffn(c, stock(), T=0) == moe.MOE_OK
+    assert call_ffn(c, stock(up=fake_qt(half_q + 16, half_sb))) == moe.MOE_ERR_INVALID_ARG
+    assert b"strides" in moe.lib().moe_last_error_string()
+    assert call_ffn(c, stock(up=fake_qt(half_q, half_sb + 8))) == moe.MOE_ERR_INVALID_ARG
+    assert call_ffn(c, stock(shared_up=moe.QTensor(None, None, None, 0, 0))) == moe.MOE_ERR_INVALID_ARG
+    assert b"shared_up" in moe.lib().moe_last_error_string()
+    assert call_ffn(c, stock(up=fake_qt(half_q, half_sb - 8))) == moe.MOE_ERR_INVALID_ARG  # too short for I rows
+    # packed weights with a shared_up tensor: inconsistent
+    assert call_ffn(c, fake_weights(c, shared_up=fake_qt(0, 0))) == moe.MOE_ERR_INVALID_ARG
+
+
 def test_stack_and_sort_validation_errors():
     c = cfg35()
     lib = moe.lib()
