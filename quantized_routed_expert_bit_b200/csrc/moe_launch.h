@@ -11,6 +11,7 @@
 namespace moe {
 
 constexpr int kRouteTokTile = 8;  // tokens per router CTA tile (one counter each)
+constexpr int kRouteMmaMinTokens = 64;  // from this many tokens the router runs on the tensor cores
 
 struct SortParams {
   const int32_t* idx;    // [T][k]

@@ -167,6 +167,118 @@ __global__ void __launch_bounds__(WPC * 32) route_topk_kernel(const __grid_const
   if (threadIdx.x == 0) p.ws.counters[tile] = 0u;  // ready for the next call
 }
 
+// ---------------------------------------------------------------- tensor-core router (many tokens)
+//
+// From kRouteMmaMinTokens tokens the router is a GEMM worth the tensor cores: logits[t][e] =
+// x[t] . Wr[e] with mma.sync m16n8k16 (bf16 products exact, fp32 accumulation), CTA tile 16 tokens
+// x 64 experts (4 warps, 16 experts each), K in chunks of kMmaK through double-buffered shared
+// memory (16-byte cp.async; rows padded to kMmaLd elements so the fragment loads hit 32 distinct
+// banks), then softmax + top-k by a second kernel, one warp per token. The logits come out of a
+// different summation order than the CUDA-core kernel's, so selections agree with it wherever the
+// k-th/(k+1)-th gap is not within the last bits of fp32.
+
+constexpr int kMmaK = 128;          // K per shared-memory chunk
+constexpr int kMmaLd = kMmaK + 8;   // row stride of the chunks (elements): 68 words, rows 4 banks apart
+constexpr int kMmaTokens = 16;
+constexpr int kMmaExperts = 64;
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(128) route_mma_kernel(const __grid_constant__ RouteParams p) {
+  __shared__ __align__(16) uint16_t sx[2][kMmaTokens * kMmaLd];
+  __shared__ __align__(16) uint16_t sw[2][kMmaExperts * kMmaLd];
+  const int t0 = blockIdx.y * kMmaTokens, e0 = blockIdx.x * kMmaExperts;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, q = lane & 3;
+  const int nch = (p.H + kMmaK - 1) / kMmaK;
+  // one K chunk of the tile's x rows and router rows into buffer b (rows past T or E, and K past H,
+  // read as zeros: their products are never stored)
+  auto load = [&](int ch, int b) {
+    const int k0 = ch * kMmaK;
+    for (int i = tid; i < (kMmaTokens + kMmaExperts) * (kMmaK / 8); i += 128) {
+      const int row = i / (kMmaK / 8), seg = i % (kMmaK / 8);
+      const int k = k0 + seg * 8;
+      const bool isx = row < kMmaTokens;
+      const int r = isx ? row : row - kMmaTokens;
+      uint16_t* dst = isx ? &sx[b][r * kMmaLd + seg * 8] : &sw[b][r * kMmaLd + seg * 8];
+      const int grow = isx ? t0 + r : e0 + r;
+      const bool ok = k < p.H && grow < (isx ? p.T : p.E);
+      if (ok) {
+        const uint16_t* src = isx ? p.x + static_cast<size_t>(grow) * p.H + k : p.wr + static_cast<size_t>(grow) * p.H + k;
+        cp_async16(dst, src);
+      } else {
+        *reinterpret_cast<uint4*>(dst) = uint4{};
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  float acc[2][4];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
+  load(0, 0);
+  for (int ch = 0; ch < nch; ++ch) {
+    const int b = ch & 1;
+    if (ch + 1 < nch) {
+      load(ch + 1, b ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();
+    const uint16_t* xa = sx[b];
+    const uint16_t* wb = sw[b] + warp * 16 * kMmaLd;
+#pragma unroll
+    for (int kk = 0; kk < kMmaK; kk += 16) {
+      const uint32_t a0 = *reinterpret_cast<const uint32_t*>(&xa[g * kMmaLd + kk + 2 * q]);
+      const uint32_t a1 = *reinterpret_cast<const uint32_t*>(&xa[(g + 8) * kMmaLd + kk + 2 * q]);
+      const uint32_t a2 = *reinterpret_cast<const uint32_t*>(&xa[g * kMmaLd + kk + 8 + 2 * q]);
+      const uint32_t a3 = *reinterpret_cast<const uint32_t*>(&xa[(g + 8) * kMmaLd + kk + 8 + 2 * q]);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint16_t* wr = wb + (j * 8 + g) * kMmaLd + kk + 2 * q;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(wr);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(wr + 8);
+        mma_bf16_16816(acc[j], a0, a1, a2, a3, b0, b1);
+      }
+    }
+    __syncthreads();  // the buffer is refilled by the next iteration's load
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int e = e0 + warp * 16 + j * 8 + 2 * q;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int t = t0 + g + 8 * h;
+      if (t >= p.T) continue;
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+        if (e + c < p.E)
+          p.ws.logits[static_cast<size_t>(t) * p.E + e + c] = acc[j][2 * h + c] + (p.rbias ? p.rbias[e + c] : 0.f);
+    }
+  }
+}
+
+// Softmax + top-k of every token from the logits, one warp per token.
+__global__ void __launch_bounds__(256) topk_kernel(const __grid_constant__ RouteParams p) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= p.T) return;
+  const int lane = threadIdx.x & 31;
+  const size_t tok = static_cast<size_t>(t);
+  if (p.E <= 256) topk_token<8>(p.ws.logits + tok * p.E, p.E, p.k, p.renorm, p.idx_out + tok * p.k, p.w_out + tok * p.k,
+                                lane);
+  else topk_token<16>(p.ws.logits + tok * p.E, p.E, p.k, p.renorm, p.idx_out + tok * p.k, p.w_out + tok * p.k,
+                      lane);
+}
+
 template <int TT, int WPC, int R>
 cudaError_t launch_t(const RouteParams& p, cudaStream_t stream) {
   constexpr int kRowsPerCta = WPC * R;
@@ -185,6 +297,14 @@ cudaError_t launch_t(const RouteParams& p, cudaStream_t stream) {
 
 cudaError_t launch_route_topk(const RouteParams& p, cudaStream_t stream) {
   static_assert(kRouteTokTile == 8, "the arrival counters are sized for 8-token tiles (a superset for 16)");
+  if (p.T >= kRouteMmaMinTokens) {  // tensor cores, then top-k
+    dim3 grid((p.E + kMmaExperts - 1) / kMmaExperts, (p.T + kMmaTokens - 1) / kMmaTokens);
+    route_mma_kernel<<<grid, 128, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    topk_kernel<<<(p.T + 7) / 8, 256, 0, stream>>>(p);
+    return cudaGetLastError();
+  }
   // 16-token tiles stage 16 rows of x (at most 128 KB); two rows per warp once the FMAs, not the
   // row loads, dominate and there are tiles enough to fill the GPU with half the row blocks
   if (p.T >= 256 && p.H <= 4096) return launch_t<16, 8, 2>(p, stream);
