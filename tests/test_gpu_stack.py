@@ -148,6 +148,8 @@ SMALL_STACKS = {
     "top8-e64": (1024, 64, 8, 128, 128, 4, 32, 6, False),
     # (5 * 1024 + 1024) / 32 = 192 units: more than one per SM, some CTAs take two
     "two-units": (256, 16, 5, 1024, 1024, 4, 32, 4, False),
+    # (7 * 1024 + 1024) / 32 = 256 units: 108 CTAs take a second unit
+    "two-units-k7": (256, 16, 7, 1024, 1024, 4, 32, 3, False),
 }
 
 
