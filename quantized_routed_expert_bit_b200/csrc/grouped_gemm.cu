@@ -566,25 +566,35 @@ __global__ void __launch_bounds__(256) gather_kernel(BatchParams p) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   const int npairs = p.T * p.k + (p.Is > 0 ? p.T : 0);
+  constexpr int kRun = 8;  // segments of a row loaded by a lane before any is converted
   for (int pos = warp; pos < npairs; pos += nwarps) {
     const int pid = p.perm[pos];
     const int t = (pid < p.T * p.k) ? pid / p.k : pid - p.T * p.k;
     const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t) * p.H);
     uint4* dst = reinterpret_cast<uint4*>(p.x16 + static_cast<size_t>(pos) * p.H);
-    for (int s = lane; s < p.H / 8; s += 32) {  // H % 256 == 0: every lane has a segment
-      const uint4 v = xr[s];
-      const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                          bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-      __half o[8];
+    for (int s0 = lane; s0 < p.H / 8; s0 += 32 * kRun) {  // H % 256 == 0: every lane has a segment
+      uint4 v[kRun];
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) o[p.perm8 ? perm8_pos(kk) : kk] = __float2half_rn(f[kk]);
-      dst[s] = *reinterpret_cast<const uint4*>(o);
-      // sum of each group of 64 (8 segments, 8 consecutive lanes)
-      float g = ((f[0] + f[1]) + (f[2] + f[3])) + ((f[4] + f[5]) + (f[6] + f[7]));
-      g += __shfl_xor_sync(0xffffffffu, g, 1);
-      g += __shfl_xor_sync(0xffffffffu, g, 2);
-      g += __shfl_xor_sync(0xffffffffu, g, 4);
-      if ((lane & 7) == 0) p.xs[static_cast<size_t>(pos) * (p.H / 64) + s / 8] = g;
+      for (int u = 0; u < kRun; ++u)
+        if (s0 + 32 * u < p.H / 8) v[u] = __ldg(xr + s0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < kRun; ++u) {
+        const int s = s0 + 32 * u;
+        if (s < p.H / 8) {  // the same for all lanes of the warp (H / 8 is a multiple of 32)
+          const float f[8] = {bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y),
+                              bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w)};
+          __half o[8];
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) o[p.perm8 ? perm8_pos(kk) : kk] = __float2half_rn(f[kk]);
+          dst[s] = *reinterpret_cast<const uint4*>(o);
+          // sum of each group of 64 (8 segments, 8 consecutive lanes)
+          float g = ((f[0] + f[1]) + (f[2] + f[3])) + ((f[4] + f[5]) + (f[6] + f[7]));
+          g += __shfl_xor_sync(0xffffffffu, g, 1);
+          g += __shfl_xor_sync(0xffffffffu, g, 2);
+          g += __shfl_xor_sync(0xffffffffu, g, 4);
+          if ((lane & 7) == 0) p.xs[static_cast<size_t>(pos) * (p.H / 64) + s / 8] = g;
+        }
+      }
     }
   }
   if (p.Is > 0) {
@@ -610,16 +620,36 @@ __global__ void __launch_bounds__(256) gather_kernel(BatchParams p) {
 }
 
 // y[t][r] = bf16( sum_j w[t][j] * O[t*k+j][r] + gate[t] * O[T*k+t][r] ), rank order, shared last.
+// Each thread four consecutive rows of one token (16-byte loads), all k (+1) pair rows loaded before
+// the first multiply; the sum in rank order, the shared expert last, as one fma chain per row.
 __global__ void __launch_bounds__(256) combine_kernel(BatchParams p) {
-  const size_t n = static_cast<size_t>(p.T) * p.H;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+  constexpr int kMaxSlots = 17;  // k <= 16, plus the shared expert
+  const size_t n4 = static_cast<size_t>(p.T) * p.H / 4;
+  const int ns = p.k + (p.Is > 0 ? 1 : 0);
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const int t = static_cast<int>(i / p.H), r = static_cast<int>(i % p.H);
-    float acc = 0.f;
-    for (int j = 0; j < p.k; ++j)
-      acc = fmaf(p.w[static_cast<size_t>(t) * p.k + j], p.o[(static_cast<size_t>(t) * p.k + j) * p.H + r], acc);
-    if (p.Is > 0) acc = fmaf(p.sgate[t], p.o[(static_cast<size_t>(p.T) * p.k + t) * p.H + r], acc);
-    p.y[i] = f32_to_bf16(acc);
+    const int t = static_cast<int>((4 * i) / p.H), r = static_cast<int>((4 * i) % p.H);
+    float4 v[kMaxSlots];
+#pragma unroll
+    for (int j = 0; j < kMaxSlots; ++j)
+      if (j < ns) {
+        const size_t pid = j < p.k ? static_cast<size_t>(t) * p.k + j : static_cast<size_t>(p.T) * p.k + t;
+        v[j] = __ldg(reinterpret_cast<const float4*>(p.o + pid * p.H + r));
+      }
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < kMaxSlots; ++j)
+      if (j < ns) {
+        const float c = j < p.k ? p.w[static_cast<size_t>(t) * p.k + j] : p.sgate[t];
+        acc.x = fmaf(c, v[j].x, acc.x);
+        acc.y = fmaf(c, v[j].y, acc.y);
+        acc.z = fmaf(c, v[j].z, acc.z);
+        acc.w = fmaf(c, v[j].w, acc.w);
+      }
+    uint2 packed;
+    packed.x = static_cast<uint32_t>(f32_to_bf16(acc.x)) | (static_cast<uint32_t>(f32_to_bf16(acc.y)) << 16);
+    packed.y = static_cast<uint32_t>(f32_to_bf16(acc.z)) | (static_cast<uint32_t>(f32_to_bf16(acc.w)) << 16);
+    *reinterpret_cast<uint2*>(p.y + 4 * i) = packed;
   }
 }
 
