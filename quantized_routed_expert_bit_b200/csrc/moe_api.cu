@@ -59,6 +59,23 @@ std::atomic<int> g_gemv_min{kGemvMinTokens};  // moe_set_gemv_min_tokens
 
 constexpr int kMaxGrid = 1024;  // largest persistent decode grid
 
+// Partial-output rows (planes x pairs, each H floats) the grouped GEMV needs for any call of up to T
+// tokens: the units per item grow with the batch, so a smaller batch can need more planes than a
+// larger one. Up to the batch size where the units per item reach kGvUPI every size is a candidate;
+// from there the plane count is fixed and the rows grow with T.
+long gemv_partial_rows(int T, int k, int E, int I, int Is) {
+  auto rows = [&](int t) {
+    const long np = static_cast<long>(t) * k + (Is > 0 ? t : 0);
+    return static_cast<long>(I / (32 * moe::gemv_units_per_item(t, k, E, I, Is))) * np;
+  };
+  long best = rows(T);
+  for (int t = 1; t < T; ++t) {
+    if (rows(t) > best) best = rows(t);
+    if (moe::gemv_units_per_item(t, k, E, I, Is) == moe::kGvUPI) break;
+  }
+  return best;
+}
+
 Layout layout(const moe_config& c, int64_t T) {
   Layout L{};
   const int64_t imax = c.inter > c.shared_inter ? c.inter : c.shared_inter;
@@ -94,9 +111,11 @@ Layout layout(const moe_config& c, int64_t T) {
   L.x16 = o;      o += up(np * c.hidden * 2);
   L.hhi = o;      o += up(np * imax * 2);
   L.hlo = o;      o += up(np * imax * 2);
-  const int upi = moe::gemv_units_per_item(static_cast<int>(T), c.top_k, c.num_experts, c.inter, c.shared_inter);
-  const size_t nq = c.inter / (32 * upi) > 0 ? c.inter / (32 * upi) : 1;
-  L.o = o;        o += up(nq * np * c.hidden * 4);
+  // the partial outputs of the grouped GEMV for any call of up to T tokens (at least one plane: the
+  // tensor-core path's outputs)
+  const size_t orow = std::max<size_t>(
+      np, gemv_partial_rows(static_cast<int>(T), c.top_k, c.num_experts, c.inter, c.shared_inter));
+  L.o = o;        o += up(orow * c.hidden * 4);
   L.xsx = o;      o += up(np * (c.hidden / 64 + 1) * 4);
   L.xsh = o;      o += up(np * (imax / 64 + 1) * 4 * 4);
   {

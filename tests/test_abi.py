@@ -74,6 +74,16 @@ def test_workspace_size_rejects_unsupported_configs(bad):
     assert moe.lib().moe_workspace_size(ctypes.byref(cfg35(**bad)), 1, 1) == 0
 
 
+@pytest.mark.parametrize("shape", ["tiny", "35b", "80b", "35b8"])
+def test_workspace_for_t_tokens_serves_every_smaller_call(shape):
+    """A workspace sized for T tokens is large enough for every call of fewer tokens (the grouped
+    GEMV's partial outputs need more planes at some small sizes than at larger ones)."""
+    from quantized_routed_expert_bit_b200 import synth
+    c = moe.make_config(synth.SHAPES[shape])
+    sizes = [moe.lib().moe_workspace_size(ctypes.byref(c), T, 1) for T in range(1, 300)]
+    assert all(b >= a for a, b in zip(sizes, sizes[1:]))
+
+
 def test_workspace_size_grows_with_tokens():
     lib = moe.lib()
     a = lib.moe_workspace_size(ctypes.byref(cfg35()), 1, 40)
