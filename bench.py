@@ -46,7 +46,7 @@ NOMINAL_HBM_GBS = 8000.0
 KERNEL_SOURCES = ("stack_split.cu", "decode_common.cuh", "moe_common.cuh", "moe_launch.h")
 # dram__bytes_read.sum + dram__bytes_write.sum per layer of decode_split_kernel from the 4-layer
 # capture in profiles/decode_split_kernel_35b_l4_full.md, keyed by workload and kernel source hash
-DECODE_TRAFFIC_PER_LAYER = {("35b", "c33a9706c1c47e02"): (68_040_960 + 690_176) / 4}
+DECODE_TRAFFIC_PER_LAYER = {("35b", "e67515cd65af64d5"): (68_040_960 + 893_184) / 4}
 
 
 def kernel_source_hash() -> str:
@@ -446,10 +446,11 @@ def secondary(keys, steps, warmup, peak, budget_s=150.0):
 
 
 def dispatch_sweep(steps=8, warmup=3, Ts=(1, 2, 3, 4, 6, 8, 12, 16, 24, 32, 48, 64, 96, 128, 192, 256, 512), key=None):
-    """The three multi-token paths for T tokens through a stack (the per-token kernels, the grouped
-    GEMV, the batched tensor-core path; moe_set_gemv_min_tokens / moe_set_batched_min_tokens pick
-    one; one token through a stack always runs the persistent decode kernel): one JSON line per
-    (T, path) with its device time per step, then the fastest path per T."""
+    """The multi-token paths for T tokens through a stack (the persistent decode kernel a token at a
+    time, up to 16 tokens; the per-token kernels; the grouped GEMV; the batched tensor-core path;
+    moe_set_decode_max_tokens / moe_set_gemv_min_tokens / moe_set_batched_min_tokens pick one; one
+    token through a stack always runs the persistent decode kernel): one JSON line per (T, path)
+    with its device time per step, then the fastest path per T."""
     key = key or SHAPE_KEY
     shape = synth.SHAPES[key]
     cfg = moe.make_config(shape)
@@ -458,19 +459,22 @@ def dispatch_sweep(steps=8, warmup=3, Ts=(1, 2, 3, 4, 6, 8, 12, 16, 24, 32, 48, 
     arr = moe.make_layer_array([moe.make_layer_weights(lw, cfg) for lw in layers])
     stream = torch.cuda.current_stream()
     best = {}
-    paths = (("per_layer", 1 << 30, 1 << 30), ("grouped_gemv", 1, 1 << 30), ("batched", 1 << 30, 1))
+    # (path, GEMV threshold, tensor-core threshold, decode threshold)
+    paths = (("decode_split_kernel", 1 << 30, 1 << 30, 1 << 30), ("per_layer", 1 << 30, 1 << 30, 1),
+             ("grouped_gemv", 1, 1 << 30, 1), ("batched", 1 << 30, 1, 1))
     for T in Ts:
         x = [synth.make_tokens(shape, [i], "cuda", seed_id=sid) if T == 1 else
              synth.make_batch(shape, T, i, "cuda", seed_id=sid) for i in range(warmup + steps)]
         xo = torch.empty(T, shape.hidden, dtype=torch.bfloat16, device="cuda")
         ws = moe.Workspace(cfg, T, L=shape.layers)
-        for path, gthr, bthr in paths:
+        for path, gthr, bthr, dthr in paths:
             pg, pb = moe.moe_set_gemv_min_tokens(gthr), moe.moe_set_batched_min_tokens(bthr)
+            pd = moe.moe_set_decode_max_tokens(dthr)
             try:
                 name = moe.moe_stack_path_name(cfg, T, shape.layers)
                 launches = moe.moe_stack_kernel_launches(cfg, T, shape.layers)
-                if T > 1 and name != path:
-                    continue
+                if T > 1 and (name != path or (path.startswith("decode") and T > 16)):
+                    continue  # (a token at a time on the decode kernel is timed up to 16 tokens)
                 for i in range(warmup):
                     moe.moe_stack_forward(cfg, arr, x[i], xo, ws, stream=stream)
                 torch.cuda.synchronize()
@@ -483,6 +487,7 @@ def dispatch_sweep(steps=8, warmup=3, Ts=(1, 2, 3, 4, 6, 8, 12, 16, 24, 32, 48, 
             finally:
                 moe.moe_set_gemv_min_tokens(pg)
                 moe.moe_set_batched_min_tokens(pb)
+                moe.moe_set_decode_max_tokens(pd)
             assert moe.moe_get_device_status(ws) == moe.MOE_OK
             ms = e0.elapsed_time(e1) / steps
             rec = {"sweep": "dispatch", "workload": shape.name, "T": T, "path": name, "ms_per_step": ms,
@@ -511,7 +516,7 @@ def main():
     ap.add_argument("--stock", action="store_true",
                     help="the stock (unpacked) gate/up layout: each expert's gate and up rows in separate "
                          "tensors, the A/B baseline of the packed layout")
-    ap.add_argument("--path", default=None, choices=["per_layer", "grouped_gemv", "batched"],
+    ap.add_argument("--path", default=None, choices=["decode", "per_layer", "grouped_gemv", "batched"],
                     help="pin the multi-token path (moe_set_gemv_min_tokens / moe_set_batched_min_tokens); "
                          "the default is the library's choice for the token count")
     ap.add_argument("--layers", type=int, default=0,
@@ -529,9 +534,11 @@ def main():
         dispatch_sweep(key=args.workload)
         return
     if args.path is not None:  # process-wide dispatch thresholds
-        gthr, bthr = {"per_layer": (1 << 30, 1 << 30), "grouped_gemv": (2, 1 << 30), "batched": (1 << 30, 2)}[args.path]
+        gthr, bthr, dthr = {"decode": (1 << 30, 1 << 30, 1 << 30), "per_layer": (1 << 30, 1 << 30, 1),
+                            "grouped_gemv": (2, 1 << 30, 1), "batched": (1 << 30, 2, 1)}[args.path]
         moe.moe_set_gemv_min_tokens(gthr)
         moe.moe_set_batched_min_tokens(bthr)
+        moe.moe_set_decode_max_tokens(dthr)
     dist, rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
     key = args.workload

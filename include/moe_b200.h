@@ -199,8 +199,9 @@ MOE_API moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weig
                              moe_stream_t stream);
 
 /* Number of kernel launches moe_stack_forward makes for T tokens and L
- * layers on the current device: a single token runs the whole stack as one
- * persistent kernel (one launch per 48 layers) when the shape fits it; from
+ * layers on the current device: up to the decode threshold
+ * (moe_set_decode_max_tokens) each token runs the whole stack as one
+ * persistent kernel (T launches per 48 layers) when the shape fits it; from
  * the batched threshold up (moe_set_batched_min_tokens) the batched path
  * (1 + 7*L) where it applies; from the GEMV threshold up
  * (moe_set_gemv_min_tokens) the grouped GEMV (1 + 6*L) where it applies;
@@ -209,7 +210,7 @@ MOE_API int32_t moe_stack_kernel_launches(const moe_config* cfg, int32_t T, int3
 
 /* Name of the path moe_stack_forward takes for T tokens and L layers on the
  * current device (a static string): "decode_split_kernel" or
- * "decode_stack_kernel" (one token, the persistent kernels), "batched" (the
+ * "decode_stack_kernel" (the persistent kernels, a token at a time), "batched" (the
  * grouped tensor-core path), "grouped_gemv" (a few tokens per expert, CUDA
  * cores), "per_layer" (four kernels per layer), "none"
  * (T or L is 0); NULL on a bad configuration. */
@@ -231,6 +232,14 @@ MOE_API int32_t moe_set_batched_min_tokens(int32_t T);
  * default (8). Returns the previous value. Process-wide, as above. Not on
  * the pages. */
 MOE_API int32_t moe_set_gemv_min_tokens(int32_t T);
+
+/* Sets the token count up to which moe_stack_forward runs its tokens one
+ * at a time through the single-token persistent kernel (one launch per
+ * token and 48 layers; each token's result as if it were called alone),
+ * where the shape has that kernel; 1 keeps it to single tokens, T < 1
+ * restores the default (7). Takes precedence over the two thresholds
+ * above. Process-wide, as above. Not on the pages. */
+MOE_API int32_t moe_set_decode_max_tokens(int32_t T);
 
 /* The batched path's grouping step on its own: the T*k (token, slot) pairs
  * of topk_idx [T][k] grouped by expert, stable in (token, slot) order, with

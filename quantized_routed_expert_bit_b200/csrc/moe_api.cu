@@ -56,6 +56,13 @@ constexpr int kBatchMinTokens = 128;  // from this many tokens the grouped tenso
 std::atomic<int> g_batch_min{kBatchMinTokens};  // moe_set_batched_min_tokens
 constexpr int kGemvMinTokens = 8;  // from this many tokens the grouped GEMV runs (default)
 std::atomic<int> g_gemv_min{kGemvMinTokens};  // moe_set_gemv_min_tokens
+// Up to this many tokens moe_stack_forward runs the single-token persistent kernel once per token
+// (where the shape has one): below the GEMV threshold it beats the per-token kernels at every
+// measured batch size (default)
+constexpr int kDecodeMaxTokens = 7;
+std::atomic<int> g_decode_max{kDecodeMaxTokens};  // moe_set_decode_max_tokens
+
+bool decode_tokens(int T) { return T == 1 || (T >= 1 && T <= g_decode_max.load(std::memory_order_relaxed)); }
 
 constexpr int kMaxGrid = 1024;  // largest persistent decode grid
 
@@ -608,7 +615,9 @@ moe::LayerDesc layer_desc(const moe_config& c, const moe_layer_weights& w) {
   return d;
 }
 
-moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, int L, const uint16_t* x0,
+// One token at a time through the stack on the persistent kernel: T launches (per 48 layers), token t
+// from row t of x0 into row t of x_out, its trace in row t of each layer's [T] rows.
+moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, int L, int T, const uint16_t* x0,
                         uint16_t* x_out, const moe_trace* trace, void* ws, const Layout& Ly, int grid, bool split,
                         int split_late, int split_two, cudaStream_t st) {
   char* b = static_cast<char*>(ws);
@@ -621,11 +630,7 @@ moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, in
   P->group = c.group;
   P->renorm = c.renorm;
   P->eps = 1e-6f;
-  P->tr_x = trace ? trace->x : nullptr;
-  P->tr_idx = trace ? trace->idx : nullptr;
-  P->tr_w = trace ? trace->w : nullptr;
-  P->tr_y = trace ? trace->y : nullptr;
-  P->tr_t = trace ? trace->t : nullptr;
+  P->tr_rows = T;
   P->logits = reinterpret_cast<uint32_t*>(b + Ly.dlogits);
   P->hbuf = reinterpret_cast<uint32_t*>(b + Ly.dh);
   P->ybuf = reinterpret_cast<uint32_t*>(b + Ly.dy);
@@ -641,15 +646,24 @@ moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, in
   P->hdr = reinterpret_cast<moe::WsHeader*>(b + Ly.hdr);
   uint16_t* xmid = reinterpret_cast<uint16_t*>(b + Ly.dx);
   float* rmid = reinterpret_cast<float*>(b + Ly.dr);
+  const size_t H = static_cast<size_t>(c.hidden), k = static_cast<size_t>(c.top_k);
+  const bool one_launch = L <= moe::kMaxDecodeLayers;  // the layer descriptors are built once
+  for (int t = 0; t < T; ++t)
   for (int l0 = 0; l0 < L; l0 += moe::kMaxDecodeLayers) {
     const int n = (L - l0 < moe::kMaxDecodeLayers) ? L - l0 : moe::kMaxDecodeLayers;
     const bool last = (l0 + n == L);
     P->L = n;
     P->l0 = l0;
-    P->x0 = (l0 == 0) ? x0 : xmid;
+    P->x0 = (l0 == 0) ? x0 + t * H : xmid;
     P->r_in = (l0 == 0) ? nullptr : rmid;
-    P->out = last ? x_out : xmid;
+    P->out = last ? x_out + t * H : xmid;
     P->r_out = last ? nullptr : rmid;
+    P->tr_x = (trace && trace->x) ? trace->x + t * H : nullptr;
+    P->tr_idx = (trace && trace->idx) ? trace->idx + t * k : nullptr;
+    P->tr_w = (trace && trace->w) ? trace->w + t * k : nullptr;
+    P->tr_y = (trace && trace->y) ? trace->y + t * H : nullptr;
+    P->tr_t = (trace && t == 0) ? trace->t : nullptr;  // phase timestamps: the first token's
+    if (t == 0 || !one_launch) {  // else the previous token's launch had the same layers
     for (int i = 0; i < n; ++i) P->layers[i] = layer_desc(c, layers[l0 + i]);
     if (split) {
       // down codes as (row bytes, H rows, experts), one unit's 32 columns x 256 rows per copy
@@ -665,6 +679,7 @@ moe_status stack_decode(const moe_config& c, const moe_layer_weights* layers, in
                     rb * c.hidden, ub, 256))
           return fail(MOE_ERR_CUDA, "tensor map of layer %d's shared down codes", l0 + i);
       }
+    }
     }
     cudaError_t e = cudaMemsetAsync(b + Ly.dlogits, 0, Ly.dr - Ly.dlogits, st);
     if (e != cudaSuccess) return cuda_fail(e, "exchange word reset");
@@ -682,8 +697,8 @@ int32_t moe_stack_kernel_launches(const moe_config* cfg, int32_t T, int32_t L) {
   if (check_cfg(cfg) != MOE_OK || T < 0 || L < 0) return -1;
   if (T == 0 || L == 0) return 0;
   int grid = 0;
-  if (T == 1 && decode_eligible(*cfg, L, &grid))
-    return (L + moe::kMaxDecodeLayers - 1) / moe::kMaxDecodeLayers;
+  if (decode_tokens(T) && decode_eligible(*cfg, L, &grid))
+    return T * ((L + moe::kMaxDecodeLayers - 1) / moe::kMaxDecodeLayers);
   if (batched_eligible(*cfg, T)) return 1 + 7 * L;  // route, sort, gather, 2 GEMMs, combine, glue
   if (gemv_eligible(*cfg, T)) return 1 + 6 * L;     // route, sort, xquant, GEMV, combine, glue
   return 1 + 4 * L;
@@ -694,7 +709,8 @@ const char* moe_stack_path_name(const moe_config* cfg, int32_t T, int32_t L) {
   if (T == 0 || L == 0) return "none";
   int grid = 0;
   bool split = false;
-  if (T == 1 && decode_eligible(*cfg, L, &grid, &split)) return split ? "decode_split_kernel" : "decode_stack_kernel";
+  if (decode_tokens(T) && decode_eligible(*cfg, L, &grid, &split))
+    return split ? "decode_split_kernel" : "decode_stack_kernel";
   if (batched_eligible(*cfg, T)) return "batched";
   if (gemv_eligible(*cfg, T)) return "grouped_gemv";
   return "per_layer";
@@ -798,8 +814,8 @@ moe_status moe_stack_forward(const moe_config* cfg, const moe_layer_weights* lay
   int grid = 0;
   bool split = false;
   int split_late = 0, split_two = 0;
-  if (T == 1 && decode_eligible(*cfg, L, &grid, &split, &split_late, &split_two))
-    return stack_decode(*cfg, layers, L, x0, x_out, trace, ws, Ly, grid, split, split_late, split_two, st);
+  if (decode_tokens(T) && decode_eligible(*cfg, L, &grid, &split, &split_late, &split_two))
+    return stack_decode(*cfg, layers, L, T, x0, x_out, trace, ws, Ly, grid, split, split_late, split_two, st);
   bool stock = false;  // any layer in the stock gate/up layout keeps the stack off the tensor cores
   for (int l = 0; l < L; ++l) stock = stock || stock_layout(layers[l]);
   const bool batched = !stock && batched_eligible(*cfg, T);
@@ -901,6 +917,10 @@ int32_t moe_set_batched_min_tokens(int32_t T) {
 
 int32_t moe_set_gemv_min_tokens(int32_t T) {
   return g_gemv_min.exchange(T < 1 ? kGemvMinTokens : T);
+}
+
+int32_t moe_set_decode_max_tokens(int32_t T) {
+  return g_decode_max.exchange(T < 1 ? kDecodeMaxTokens : T);
 }
 
 moe_status moe_check_wait_limit(void* ws, size_t ws_bytes, int32_t* gave_up, moe_stream_t stream) {

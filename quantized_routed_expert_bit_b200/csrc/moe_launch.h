@@ -136,6 +136,7 @@ struct DecodeParams {
   float* tr_w;           // [layers][k] or null
   uint16_t* tr_y;        // bf16 [layers][H] or null
   uint64_t* tr_t;        // [layers][8] phase timestamps of CTA 0, or null
+  int tr_rows;           // trace rows per layer (the call's tokens, run one launch each; 1 for one token)
   // exchange words between CTAs (workspace), zero at launch; each written to
   // kDecodeReplicas copies (`*_rep` words apart), CTA c reads copy c % kDecodeReplicas
   uint32_t* logits;      // [E+1] fp32 logits, last mantissa bit = layer parity

@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         const float v = bf16_to_f32(p.x0[i]);
         xn[i] = v;
         rr[i] = p.r_in ? p.r_in[i] : v;
-        if (c == 0 && p.tr_x) p.tr_x[static_cast<size_t>(p.l0) * H + i] = p.x0[i];
+        if (c == 0 && p.tr_x) p.tr_x[static_cast<size_t>(p.l0) * p.tr_rows * H + i] = p.x0[i];
       }
     } else {
       // y of the previous layer: 4 rows per thread
@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
       for (int i = tid; i < H; i += kThreads) {
         const uint16_t xb = f32_to_bf16(rr[i] * inv);
         xn[i] = bf16_to_f32(xb);
-        if (c == 0 && p.tr_x) p.tr_x[static_cast<size_t>(lg) * H + i] = xb;
+        if (c == 0 && p.tr_x) p.tr_x[static_cast<size_t>(lg) * p.tr_rows * H + i] = xb;
       }
     }
     __syncthreads();
@@ -383,8 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
         s_idx[lane] = my_e;
         s_w[lane] = ex / den;
         if (c == 0) {
-          if (p.tr_idx) p.tr_idx[static_cast<size_t>(lg) * k + lane] = my_e;
-          if (p.tr_w) p.tr_w[static_cast<size_t>(lg) * k + lane] = ex / den;
+          if (p.tr_idx) p.tr_idx[static_cast<size_t>(lg) * p.tr_rows * k + lane] = my_e;
+          if (p.tr_w) p.tr_w[static_cast<size_t>(lg) * p.tr_rows * k + lane] = ex / den;
         }
       }
       if (lane == 0) s_sg = (Is > 0) ? 1.f / (1.f + expf(-__uint_as_float(wsg))) : 0.f;
@@ -655,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stack_kernel(const __grid_
 #pragma unroll
       for (int r = 0; r < kDecodeReplicas; ++r)
         st_word(p.ybuf + r * p.y_rep + row, (static_cast<uint32_t>(yb) << 16) | (tag & 0xffffu));
-      if (p.tr_y) p.tr_y[static_cast<size_t>(lg) * H + row] = yb;
+      if (p.tr_y) p.tr_y[static_cast<size_t>(lg) * p.tr_rows * H + row] = yb;
     }
     stamp(6);
   }

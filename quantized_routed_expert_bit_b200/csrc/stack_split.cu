@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
           rr4[u] = p.r_in ? p.r_in[4 * tid + u] : xv[u];
           mx = fmaxf(mx, fabsf(xv[u]));
         }
-        if (c == 0 && p.tr_x) *reinterpret_cast<uint2*>(p.tr_x + static_cast<size_t>(p.l0) * H + 4 * tid) = w;
+        if (c == 0 && p.tr_x) *reinterpret_cast<uint2*>(p.tr_x + static_cast<size_t>(p.l0) * p.tr_rows * H + 4 * tid) = w;
       }
       float unused;
       block_sum_max(0.f, mx, unused, m);
@@ -498,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
           mx = fmaxf(mx, fabsf(rr4[u]));
         }
         if (c == 0 && p.tr_y)
-          *reinterpret_cast<uint2*>(p.tr_y + static_cast<size_t>(lg - 1) * H + 4 * tid) =
+          *reinterpret_cast<uint2*>(p.tr_y + static_cast<size_t>(lg - 1) * p.tr_rows * H + 4 * tid) =
               make_uint2(yb[0] | (static_cast<uint32_t>(yb[1]) << 16), yb[2] | (static_cast<uint32_t>(yb[3]) << 16));
       }
       float tot;
@@ -514,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
           xv[u] = bf16_to_f32(xb[u]);
         }
         if (c == 0 && p.tr_x)
-          *reinterpret_cast<uint2*>(p.tr_x + static_cast<size_t>(lg) * H + 4 * tid) =
+          *reinterpret_cast<uint2*>(p.tr_x + static_cast<size_t>(lg) * p.tr_rows * H + 4 * tid) =
               make_uint2(xb[0] | (static_cast<uint32_t>(xb[1]) << 16), xb[2] | (static_cast<uint32_t>(xb[3]) << 16));
       }
     }
@@ -646,8 +646,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
         s_idx[lane] = my_e;
         s_w[lane] = ex / den;
         if (c == 0) {
-          if (p.tr_idx) p.tr_idx[static_cast<size_t>(lg) * k + lane] = my_e;
-          if (p.tr_w) p.tr_w[static_cast<size_t>(lg) * k + lane] = ex / den;
+          if (p.tr_idx) p.tr_idx[static_cast<size_t>(lg) * p.tr_rows * k + lane] = my_e;
+          if (p.tr_w) p.tr_w[static_cast<size_t>(lg) * p.tr_rows * k + lane] = ex / den;
         }
       }
       if (lane == 0) s_sg = (Is > 0) ? 1.f / (1.f + expf(-__uint_as_float(wsg))) : 0.f;
@@ -846,7 +846,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
         const uint16_t yb = f32_to_bf16(y[u]);
         rr4[u] += bf16_to_f32(yb);
         ss = fmaf(rr4[u], rr4[u], ss);
-        if (p.tr_y) p.tr_y[static_cast<size_t>(p.l0 + p.L - 1) * H + 4 * tid + u] = yb;
+        if (p.tr_y) p.tr_y[static_cast<size_t>(p.l0 + p.L - 1) * p.tr_rows * H + 4 * tid + u] = yb;
       }
     }
     float tot, unused;

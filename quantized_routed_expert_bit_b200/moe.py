@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.moe_set_batched_min_tokens.restype = I32
         L.moe_set_gemv_min_tokens.argtypes = [I32]
         L.moe_set_gemv_min_tokens.restype = I32
+        L.moe_set_decode_max_tokens.argtypes = [I32]
+        L.moe_set_decode_max_tokens.restype = I32
         L.moe_stack_kernel_launches.argtypes = [CP, I32, I32]
         L.moe_stack_kernel_launches.restype = I32
         L.moe_stack_path_name.argtypes = [CP, I32, I32]
@@ -310,6 +312,13 @@ def moe_set_gemv_min_tokens(T: int) -> int:
     """Token count from which the grouped GEMV path runs (process-wide); T < 1 restores the
     default. Returns the previous value."""
     return int(lib().moe_set_gemv_min_tokens(int(T)))
+
+
+def moe_set_decode_max_tokens(T: int) -> int:
+    """Token count up to which moe_stack_forward runs its tokens one at a time through the
+    single-token persistent kernel (process-wide); T < 1 restores the default. Returns the
+    previous value."""
+    return int(lib().moe_set_decode_max_tokens(int(T)))
 
 
 def moe_stack_path_name(cfg: Config, T: int, L: int) -> Optional[str]:

@@ -205,6 +205,14 @@ def test_batched_threshold_knob():
     assert lib.moe_set_batched_min_tokens(0) == 128
 
 
+def test_decode_threshold_knob():
+    """moe_set_decode_max_tokens returns the previous threshold; T < 1 restores the default 7."""
+    lib = moe.lib()
+    assert lib.moe_set_decode_max_tokens(3) == 7
+    assert lib.moe_set_decode_max_tokens(0) == 3
+    assert lib.moe_set_decode_max_tokens(-1) == 7
+
+
 def test_gemv_threshold_knob():
     """moe_set_gemv_min_tokens returns the previous threshold; T < 1 restores the default 8."""
     lib = moe.lib()

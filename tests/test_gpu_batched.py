@@ -57,7 +57,11 @@ def test_batched_path_is_taken(key):
     4-bit shapes only), and on the token-at-a-time kernels (route, gate/up,
     down, glue: 4 a layer) when the GEMV is switched off."""
     cfg = moe.make_config(synth.SHAPES[key])
+    # by default up to 7 tokens through a stack run one at a time on the decode kernel
+    assert moe.moe_stack_path_name(cfg, 7, 3) == "decode_split_kernel"
+    assert moe.moe_stack_kernel_launches(cfg, 7, 3) == 7
     pb, pg = moe.moe_set_batched_min_tokens(8), moe.moe_set_gemv_min_tokens(2)
+    pd = moe.moe_set_decode_max_tokens(1)
     try:
         assert moe.moe_stack_kernel_launches(cfg, 8, 3) == 1 + 7 * 3
         assert moe.moe_stack_kernel_launches(cfg, 512, 3) == 1 + 7 * 3
@@ -73,6 +77,7 @@ def test_batched_path_is_taken(key):
     finally:
         moe.moe_set_batched_min_tokens(pb)
         moe.moe_set_gemv_min_tokens(pg)
+        moe.moe_set_decode_max_tokens(pd)
 
 
 @pytest.mark.parametrize("T", [7, 8, 16])

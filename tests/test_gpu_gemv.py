@@ -18,12 +18,15 @@ pytestmark = pytest.mark.gpu
 
 @pytest.fixture(autouse=True)
 def gemv_path():
-    """Grouped GEMV from 2 tokens up, never the tensor-core path; defaults restored after."""
+    """Grouped GEMV from 2 tokens up, never the tensor-core path, and stacks of a few tokens not a
+    token at a time on the decode kernel; defaults restored after."""
     pg = moe.moe_set_gemv_min_tokens(2)
     pb = moe.moe_set_batched_min_tokens(1 << 30)
+    pd = moe.moe_set_decode_max_tokens(1)
     yield
     moe.moe_set_gemv_min_tokens(pg)
     moe.moe_set_batched_min_tokens(pb)
+    moe.moe_set_decode_max_tokens(pd)
 
 
 def layer_call(shape, lw, x, prepared=True):

@@ -12,6 +12,8 @@ differences do not compound through later routing. The residual/RMSNorm
 glue between layers is checked separately (within one bf16 ulp).
 """
 
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -173,6 +175,26 @@ def test_small_decode_stacks(name, prepared):
     assert total.excluded <= 2
 
 
+@pytest.mark.parametrize("key,T,L", [("35b", 3, 4), ("80b", 2, 3)])
+def test_small_batch_runs_a_token_at_a_time(key, T, L):
+    """Up to 7 tokens through a stack run one after another on the persistent decode kernel (T
+    launches), each token's trace in its row of every layer: every (token, layer) teacher-forced
+    against the oracle, and the glue."""
+    shape = dataclasses.replace(synth.SHAPES[key], layers=L)
+    cfg = moe.make_config(shape)
+    assert moe.moe_stack_path_name(cfg, T, L) == "decode_split_kernel"
+    assert moe.moe_stack_kernel_launches(cfg, T, L) == T
+    layers = [synth.make_layer(shape, l, "cuda", seed_id=60) for l in range(L)]
+    x0 = synth.make_batch(shape, T, 2, "cuda", seed_id=60)
+    tx, ti, tw, ty, xo = run_stack(shape, layers, x0)
+    total = ParityStats()
+    for l in range(L):
+        total.merge(check_tokens(DeviceLayer(shape, layers[l]), tx[l], ti[l], tw[l], ty[l], range(T), f"{key} {l}"))
+    check_glue(bits(x0), tx, ty, xo)
+    assert total.checked == T * L
+    print(f"{key} T={T}: {total.checked} pairs, max-abs {total.max_abs:.2e} rel-L2 {total.max_rel_l2:.2e}")
+
+
 def test_single_token_path_matches_multi_kernel_path():
     """One token through the persistent kernel against the same token run
     twice in a batch of two through the multi-kernel path, layer by layer on
@@ -191,11 +213,13 @@ def test_single_token_path_matches_multi_kernel_path():
     tx, ti, tw, ty, _ = run_stack(shape, layers, x1)
     ws = moe.Workspace(cfg, 2)
     pg = moe.moe_set_gemv_min_tokens(1 << 30)  # the four-kernel per-token path for T=2
+    pd = moe.moe_set_decode_max_tokens(1)
     try:
         assert moe.moe_stack_kernel_launches(cfg, 2, 4) == 17
         _compare_with_per_layer(shape, cfg, layers, tx, ti, tw, ty, ws)
     finally:
         moe.moe_set_gemv_min_tokens(pg)
+        moe.moe_set_decode_max_tokens(pd)
 
 
 def _compare_with_per_layer(shape, cfg, layers, tx, ti, tw, ty, ws):
