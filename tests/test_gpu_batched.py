@@ -107,6 +107,29 @@ def test_batched_layer_parity(key, T):
     print(f"{key} T={T}: {st.checked} tokens, max-abs {st.max_abs:.2e} rel-L2 {st.max_rel_l2:.2e}")
 
 
+def test_large_batch_layer(layer35):
+    """3,000 tokens through one layer on the default path (tensor cores, router on the tensor
+    cores): the sort's selection no longer fits its shared-memory copy (27,000 pairs) and is read
+    through L2, the GEMMs run ~5,000 chunks; sampled tokens against the oracle, and every token's
+    selection a valid set."""
+    lw, host = layer35
+    T = 3000
+    x = synth.make_batch(S35, T, 5, "cuda", seed_id=2)
+    pb = moe.moe_set_batched_min_tokens(0)  # the library's default threshold
+    try:
+        assert moe.moe_stack_path_name(moe.make_config(S35), T, 1) == "batched"
+        idx, w, y = layer_call(S35, lw, x)
+    finally:
+        moe.moe_set_batched_min_tokens(pb)
+    s = np.sort(idx, axis=1)
+    assert np.all((s >= 0) & (s < S35.num_experts)) and np.all(s[:, 1:] != s[:, :-1])
+    assert np.allclose(w.sum(axis=1), 1.0, atol=1e-5)
+    toks = [0, 1, 15, 16, 1023, 1024, 2047, 2048, 2999]
+    st = check_tokens(host, bits(x), idx, w, y, toks, "T=3000")
+    assert st.checked == len(toks)
+    print(f"T={T}: {st.checked} sampled tokens, max-abs {st.max_abs:.2e} rel-L2 {st.max_rel_l2:.2e}")
+
+
 def test_expert_with_hundreds_of_tokens(layer35):
     """Expert 3 is every token's first choice: 300 tokens for one expert (three
     GEMM chunks of <= 128), besides the shared expert's three chunks."""
