@@ -608,6 +608,7 @@ cudaError_t launch_grouped_gemv(const GemvParams& p, int bits, int grid, cudaStr
   if (bits == 4) return ch == 1 ? launch_gv<4, 1>(p, grid, st) : launch_gv<4, 2>(p, grid, st);
   if (ch == 1) return launch_gv<8, 1>(p, grid, st);
   if (ch == 2) return launch_gv<8, 2>(p, grid, st);
+  if (ch == 3) return launch_gv<8, 3>(p, grid, st);  // 1536-wide 8-bit rows
   return launch_gv<8, 4>(p, grid, st);
 }
 

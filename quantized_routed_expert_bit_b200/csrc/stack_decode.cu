@@ -778,6 +778,7 @@ cudaError_t launch_decode_stack(const DecodeParams& p, int bits, int grid, cudaS
   }
   if (ch == 1) return launch_t<8, 1>(p, smem, grid, stream);
   if (ch == 2) return launch_t<8, 2>(p, smem, grid, stream);
+  if (ch == 3) return launch_t<8, 3>(p, smem, grid, stream);  // 1536-wide 8-bit rows
   return launch_t<8, 4>(p, smem, grid, stream);
 }
 

@@ -920,6 +920,7 @@ cudaError_t launch_decode_split(const DecodeParams& p, int bits, int grid, cudaS
     }
     if (ch == 1) return launch_t<8, 1, true>(p, smem, grid, stream);
     if (ch == 2) return launch_t<8, 2, true>(p, smem, grid, stream);
+    if (ch == 3) return launch_t<8, 3, true>(p, smem, grid, stream);
     return launch_t<8, 4, true>(p, smem, grid, stream);
   }
   if (bits == 4) {
@@ -928,6 +929,7 @@ cudaError_t launch_decode_split(const DecodeParams& p, int bits, int grid, cudaS
   }
   if (ch == 1) return launch_t<8, 1, false>(p, smem, grid, stream);
   if (ch == 2) return launch_t<8, 2, false>(p, smem, grid, stream);
+  if (ch == 3) return launch_t<8, 3, false>(p, smem, grid, stream);  // 1536-wide 8-bit rows
   return launch_t<8, 4, false>(p, smem, grid, stream);
 }
 

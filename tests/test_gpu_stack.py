@@ -145,6 +145,8 @@ def test_decode_stack_longer_than_one_launch():
 SMALL_STACKS = {
     # name: (H, E, k, I, Is, bits, group, layers, router bias)
     "8bit": (256, 16, 2, 128, 128, 8, 32, 6, True),
+    # 1536-wide 8-bit rows: 96 code segments, three per lane
+    "8bit-h1536": (1536, 16, 2, 128, 128, 8, 32, 3, False),
     "no-shared": (256, 16, 2, 128, 0, 4, 32, 6, False),
     "top1-g64": (512, 32, 1, 256, 256, 4, 64, 6, False),
     "top8-e64": (1024, 64, 8, 128, 128, 4, 32, 6, False),
@@ -173,6 +175,28 @@ def test_small_decode_stacks(name, prepared):
             total.merge(check_tokens(DeviceLayer(shape, layers[l]), tx[l], ti[l], tw[l], ty[l], [0], f"{name} {l}"))
         check_glue(bits(x0), tx, ty, xo)
     assert total.excluded <= 2
+
+
+def test_exchange_kernel_stack():
+    """A shape the split kernel's plan does not take (8-bit, 1536 wide, top-9 of 256: 160 units
+    need a second unit on some CTAs, and two units' 8-bit rows do not fit in its shared memory)
+    runs on decode_stack_kernel; two tokens, every layer teacher-forced against the oracle, and
+    the glue."""
+    shape = synth.MoEShape("stack-8bit-h1536-top9", 1536, 256, 9, 512, 512, 8, 64, 2, False, 1)
+    cfg = moe.make_config(shape)
+    assert moe.moe_stack_path_name(cfg, 1, shape.layers) == "decode_stack_kernel"
+    layers = [synth.make_layer(shape, l, "cuda", seed_id=70) for l in range(shape.layers)]
+    total = ParityStats()
+    for tok in (0, 1):
+        x0 = synth.make_tokens(shape, [tok], "cuda", seed_id=70)
+        tx, ti, tw, ty, xo = run_stack(shape, layers, x0)
+        for l in range(shape.layers):
+            total.merge(check_tokens(DeviceLayer(shape, layers[l]), tx[l], ti[l], tw[l], ty[l], [0], f"layer {l}"))
+        check_glue(bits(x0), tx, ty, xo)
+    assert total.checked == 2 * shape.layers
+    print(f"exchange kernel: max-abs {total.max_abs:.2e} rel-L2 {total.max_rel_l2:.2e}")
+    del layers
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("key,T,L", [("35b", 3, 4), ("80b", 2, 3)])
