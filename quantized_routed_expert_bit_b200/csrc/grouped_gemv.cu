@@ -5,8 +5,9 @@
 // the intermediate (a unit) at a time:
 //
 //   xquant   every token's x as the fixed-point quads of the integer dot
-//            products (decode_common.cuh: X = rint(x * 2^S), three bytes),
-//            per token its own S; also the shared expert's sigmoid gate;
+//            products (X = rint(x * 2^S) in 16 bits, two byte planes: see
+//            fix_exp16), per token its own S; also the shared expert's
+//            sigmoid gate;
 //   gemv     per work item (chunk, group of upi units, upi = 1, 2 or 4 as
 //            gemv_units_per_item picks for the batch size): the item's
 //            tokens' quads (bulk copies, issued while the previous item's
@@ -48,6 +49,47 @@ constexpr int kBoxRows = 256;        // down rows per tensor copy (canonical dow
 
 __host__ __device__ constexpr uint32_t al128(uint32_t v) { return (v + 127u) & ~127u; }
 
+// x in 16-bit fixed point. With one to four tokens per chunk the kernel is bound by its integer
+// instruction issue, one dp4a per byte plane per four codes and token, and the gate/up rows carry
+// two thirds of the codes: so x is held in two byte planes (X = 256 X1 + X0, X1 signed) instead of
+// the decode kernel's three, X = rint(x 2^S) with S from the token's largest |x|. Elements within
+// 7 binades of the largest are exact (bf16 has 8 significant bits); smaller ones are rounded to
+// 2^-S, an error below 2^-15 of the largest element, which enters the gate/up outputs as
+// sum_i w_i e_i (w the dequantised weights). A CPU emulation of this rounding on 400 tokens of a
+// 256-wide top-2 layer and 24 of the 2048-wide one puts the bf16 outputs within rel-L2 7.2e-4 and
+// 4.2e-4 of the exact ones (bound 1e-3). The unit's h keeps three planes (a unit's 32 h values are
+// few and heavy-tailed: in two planes the same emulation exceeds the bound on 13 of 400 tokens).
+// The largest bf16 below 2^(e+1), times 2^(14-e), is 32640 < 2^15: no overflow.
+__device__ __forceinline__ int fix_exp16(float m) {
+  if (!(m > 0.f)) return 0;
+  int e = ((__float_as_uint(m) >> 23) & 0xFF) - 127;  // floor(log2 m) for normal m
+  if (e < -100) e = -100;
+  return 14 - e;
+}
+
+// sum over one 16-byte segment of codes of q * X for X in two byte planes (q1[.] the signed high
+// bytes, q0[.] the low bytes, laid out as for seg_dot): two exact integer sums, one fp32 rounding
+template <int BITS>
+__device__ __forceinline__ float seg_dot2(const uint4& c, const uint32_t* q1, const uint32_t* q0) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  int a1 = 0;
+  uint32_t a0 = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if constexpr (BITS == 4) {
+      const uint32_t lo = w[i] & 0x0F0F0F0Fu, hi = (w[i] >> 4) & 0x0F0F0F0Fu;
+      a1 = dp4a_us(lo, q1[2 * i], a1);
+      a1 = dp4a_us(hi, q1[2 * i + 1], a1);
+      a0 = dp4a_uu(lo, q0[2 * i], a0);
+      a0 = dp4a_uu(hi, q0[2 * i + 1], a0);
+    } else {
+      a1 = dp4a_us(w[i], q1[i], a1);
+      a0 = dp4a_uu(w[i], q0[i], a0);
+    }
+  }
+  return fmaf(static_cast<float>(a1), 256.f, static_cast<float>(a0));
+}
+
 // Shared-memory carve-up; identical on host (sizing) and device.
 struct GvCarve {
   int PS, nsg, QS, QSP, ng, ngd, rowb, UB;
@@ -59,7 +101,7 @@ __host__ __device__ inline GvCarve gv_carve(int H, int I, int group, int bits) {
   GvCarve c{};
   c.PS = 128 / bits;
   c.nsg = H / c.PS;
-  c.QS = 3 * (c.PS / 4);
+  c.QS = 2 * (c.PS / 4);
   c.QSP = bits == 4 ? xq_stride<4>() : xq_stride<8>();  // quads + sum, padded for 16-byte loads
   c.ng = H / group;
   c.ngd = I / group;
@@ -298,9 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
 #pragma unroll
             for (int ch = 0; ch < CH; ++ch) {
               const int s = gs0 + 32 * ch;
-              uint32_t xr[3 * QW];
+              uint32_t xr[2 * QW];
 #pragma unroll
-              for (int w = 0; w < 3 * QW; w += 4) {
+              for (int w = 0; w < 2 * QW; w += 4) {
                 const uint4 v4 = *reinterpret_cast<const uint4*>(xt + s * cv.QSP + w);
                 xr[w] = v4.x;
                 xr[w + 1] = v4.y;
@@ -310,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
               const float xsm = __uint_as_float(xt[s * cv.QSP + cv.QS]);
 #pragma unroll
               for (int r2 = 0; r2 < 2; ++r2) {
-                const float d = seg_dot<BITS>(cd[r2][ch], xr + 2 * QW, xr + QW, xr);
+                const float d = seg_dot2<BITS>(cd[r2][ch], xr + QW, xr);
                 a2[r2] = fmaf(scv[r2][ch], d, fmaf(biv[r2][ch], xsm, a2[r2]));
               }
             }
@@ -435,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const __grid_
 }
 
 // Every token's x as the fixed-point quads the gate/up dot products read ([T][nsg][QSP] words,
-// QSP = xq_stride: per segment the three byte planes' quads, the segment's sum of X, padding), its
+// QSP = xq_stride: per segment the two byte planes' quads, the segment's sum of X, padding), its
 // 2^-S, and the shared expert's sigmoid gate. One CTA per token, H/4 threads, each thread 4
 // consecutive elements (element group g = thread g: its partner group g ^ 1 is the neighbouring
 // lane, the PS / 4 groups of a segment are consecutive lanes).
@@ -468,7 +510,7 @@ __global__ void xquant_kernel(const uint16_t* __restrict__ x, const uint16_t* __
     m = fmaxf(m, s_red[0][w]);
     sg += s_red[1][w];
   }
-  const int S = fix_exp(m);
+  const int S = fix_exp16(m);
   const float sx = pow2f(S);
   int X[4];
 #pragma unroll
@@ -495,12 +537,12 @@ __global__ void xquant_kernel(const uint16_t* __restrict__ x, const uint16_t* __
   }
   uint32_t* dst = xq + static_cast<size_t>(t) * nsg * QSP;
 #pragma unroll
-  for (int j = 0; j < 3; ++j)
+  for (int j = 0; j < 2; ++j)
     dst[sgi * QSP + j * QW + qi] =
         xbyte(e[0], j) | (xbyte(e[1], j) << 8) | (xbyte(e[2], j) << 16) | (xbyte(e[3], j) << 24);
 #pragma unroll
   for (int o = 1; o < PS / 4; o <<= 1) xs += __shfl_xor_sync(0xffffffffu, xs, o);
-  if ((tid & (PS / 4 - 1)) == 0) dst[sgi * QSP + 3 * QW] = __float_as_uint(static_cast<float>(xs));
+  if ((tid & (PS / 4 - 1)) == 0) dst[sgi * QSP + 2 * QW] = __float_as_uint(static_cast<float>(xs));
   if (tid == 0) {
     xsc[t] = pow2f(-S);
     if (Is > 0) sgate[t] = 1.f / (1.f + expf(-sg));

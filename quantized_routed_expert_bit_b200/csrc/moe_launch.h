@@ -165,12 +165,12 @@ struct DecodeParams {
 constexpr int kGvTPI = 4;  // pairs per chunk
 
 // Words per 16-byte code segment in the per-token quad table of the grouped GEMV (xq_token): the
-// 3 * 32 / BITS quad words and the segment's sum, padded to 4 m words with m odd, so that each
-// segment starts on 16 bytes and the 16-byte loads of 8 consecutive segments (one shared-memory
-// phase) hit distinct banks.
+// 2 * 32 / BITS quad words (two byte planes of 16-bit fixed point) and the segment's sum, padded
+// to 4 m words with m odd, so that each segment starts on 16 bytes and the 16-byte loads of 8
+// consecutive segments (one shared-memory phase) hit distinct banks.
 template <int BITS>
 __host__ __device__ constexpr int xq_stride() {
-  return 4 * ((((3 * (32 / BITS) + 1) + 3) / 4) | 1);
+  return 4 * ((((2 * (32 / BITS) + 1) + 3) / 4) | 1);
 }
 constexpr int kGvUPI = 4;  // most units per item
 constexpr int kGvItemsTarget = 128;  // work items wanted per launch: about one per SM of a 148-SM part
