@@ -46,7 +46,7 @@ NOMINAL_HBM_GBS = 8000.0
 KERNEL_SOURCES = ("stack_split.cu", "decode_common.cuh", "moe_common.cuh", "moe_launch.h")
 # dram__bytes_read.sum + dram__bytes_write.sum per layer of decode_split_kernel from the 4-layer
 # capture in profiles/decode_split_kernel_35b_l4_full.md, keyed by workload and kernel source hash
-DECODE_TRAFFIC_PER_LAYER = {("35b", "f0d18f39ff601895"): (68_041_984 + 969_216) / 4}
+DECODE_TRAFFIC_PER_LAYER = {("35b", "afa65bc43f7fbf78"): (68_041_728 + 1_808_384) / 4}
 
 
 def kernel_source_hash() -> str:
