@@ -55,10 +55,11 @@ __host__ __device__ constexpr uint32_t al128(uint32_t v) { return (v + 127u) & ~
 // the decode kernel's three, X = rint(x 2^S) with S from the token's largest |x|. Elements within
 // 7 binades of the largest are exact (bf16 has 8 significant bits); smaller ones are rounded to
 // 2^-S, an error below 2^-15 of the largest element, which enters the gate/up outputs as
-// sum_i w_i e_i (w the dequantised weights). A CPU emulation of this rounding on 400 tokens of a
-// 256-wide top-2 layer and 24 of the 2048-wide one puts the bf16 outputs within rel-L2 7.2e-4 and
-// 4.2e-4 of the exact ones (bound 1e-3). The unit's h keeps three planes (a unit's 32 h values are
-// few and heavy-tailed: in two planes the same emulation exceeds the bound on 13 of 400 tokens).
+// sum_i w_i e_i (w the dequantised weights). tests/test_fixed_point_reading.py emulates this
+// rounding around the oracle: on 400 tokens of the 256-wide top-2 layer the bf16 outputs stay
+// within rel-L2 9.2e-4 of the oracle's (6.2e-4 with x exact: one-ulp flips of a few outputs
+// dominate at that width), under the bound of 1e-3. The unit's h keeps three planes (a unit's 32
+// h values are few and heavy-tailed: in two planes as well, 12 of the 400 tokens exceed the bound).
 // The largest bf16 below 2^(e+1), times 2^(14-e), is 32640 < 2^15: no overflow.
 __device__ __forceinline__ int fix_exp16(float m) {
   if (!(m > 0.f)) return 0;
