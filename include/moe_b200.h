@@ -227,10 +227,11 @@ MOE_API int32_t moe_set_batched_min_tokens(int32_t T);
 
 /* Sets the token count from which those calls take the grouped GEMV path
  * (a few tokens per expert: each selected expert's weights read once for
- * all of its tokens, dot products on the CUDA cores) instead of the
- * per-token kernels, below the batched threshold; T < 1 restores the
- * default (8). Returns the previous value. Process-wide, as above. Not on
- * the pages. */
+ * all of its tokens, dot products on the CUDA cores, each token's x rounded
+ * to 16-bit fixed point: within the same tolerance as the other paths, not
+ * bit-identical to them) instead of the per-token kernels, below the batched
+ * threshold; T < 1 restores the default (8). Returns the previous value.
+ * Process-wide, as above. Not on the pages. */
 MOE_API int32_t moe_set_gemv_min_tokens(int32_t T);
 
 /* Sets the token count up to which moe_stack_forward runs its tokens one
