@@ -1,4 +1,4 @@
-"""The fixed-point reading of the grouped GEMV (x in 16 bits, h in 24), checked on the CPU.
+"""The fixed-point readings of the integer dot products, checked on the CPU.
 
 The grouped GEMV holds each token's x as X = rint(x * 2^S) in two byte planes
 (S from the token's largest |x|: 2^S * max|x| < 2^15) and each unit's h in three
@@ -7,7 +7,9 @@ rounding alone (up to fp32 summation order). Emulating that rounding in
 float64 around the oracle's dequantised weights, 400 seeded tokens of the
 256-wide top-2 layer must keep their bf16 outputs within the parity bound
 (rel-L2 1e-3 against the oracle's bf16 output); rounding h to 16 bits as well
-must not (which is why h keeps three planes). The routing is the oracle's.
+must not (which is why h keeps three planes). The decode and per-token kernels
+hold x and h in three planes (2^S * max < 2^22): the same emulation must keep
+the same bound. The routing is the oracle's.
 """
 
 import numpy as np
@@ -73,3 +75,8 @@ def test_sixteen_bit_x_keeps_the_bound():
 def test_sixteen_bit_h_would_not():
     rel = _rel_l2_per_token(x_top=14, h_top=13)
     assert (rel > REL_L2).sum() > 0, f"worst rel-L2 {rel.max():.3e}"
+
+
+def test_decode_fixed_point_keeps_the_bound():
+    rel = _rel_l2_per_token(x_top=21, h_top=21)
+    assert rel.max() < REL_L2, f"worst rel-L2 {rel.max():.3e}"
