@@ -7,9 +7,9 @@ rounding alone (up to fp32 summation order). Emulating that rounding in
 float64 around the oracle's dequantised weights, 400 seeded tokens of the
 256-wide top-2 layer must keep their bf16 outputs within the parity bound
 (rel-L2 1e-3 against the oracle's bf16 output); rounding h to 16 bits as well
-must not (which is why h keeps three planes). The decode and per-token kernels
-hold x and h in three planes (2^S * max < 2^22): the same emulation must keep
-the same bound. The routing is the oracle's.
+must not (which is why h keeps three planes). The split decode kernel holds x
+and h in three planes (2^S * max < 2^22): the same emulation must keep the
+same bound. The routing is the oracle's.
 """
 
 import numpy as np
